@@ -1,0 +1,162 @@
+/*
+ * kiattn -- K-interval attention (quantized softmax in attention), forward
+ * and backward, on NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * The operator is the one defined in "Pretraining Transformers with
+ * Quantized Softmax in Attention" (Zhu, Hu, Kozlowski; arXiv 2609.33591):
+ *   section 3 (operator family, calibration, reconstruction, calibration
+ *   gradients, surrogate placement), Appendix A (operator definitions and
+ *   edge cases) and Appendix B (gradient derivations).
+ *
+ * For one (batch, head) and query row i with visible keys J_i (j <= i when
+ * causal, all keys otherwise):
+ *   s_j = q_i . k_j                     (no 1/sqrt(d): the caller scales Q)
+ *   m = max s, n = min s                (arg-extrema: lowest index on ties)
+ *   h = (m - n)/K  (MinMax)   or   tau/K  (FWM)
+ *   u_j = (m - s_j)/h,  k_j = min(floor u_j, K-1),  t_j = u_j - k_j
+ *   G_k = e^{-k h}, k = 0..K            (the K+1 grid values)
+ *   LERP     w_j = G_k + t_j (G_{k+1} - G_k)
+ *   Nearest  w_j = G_{k + [t_j >= 1/2]}
+ *   FWM: w_j = 0 when u_j > K (the tail below m - tau)
+ *   MinMax rows with span m - n < 1e-12: w_j = 1 (degenerate branch)
+ *   P = w / sum(w),  O_i = sum_j P_j v_j
+ * Backward, with the normalisation Jacobian at the surrogate's point (LERP
+ * and Prob-STE at the LERP weights, Weight-STE at the hard weights), the LERP
+ * scalar derivatives, and the calibration derivatives through m (and n)
+ * filtered by the gradient mode (full, detach, max-only, min-only, zero-sum
+ * projection).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are device pointers to fp32, contiguous [B, H, T, d], 16-byte
+ *     aligned.  Keys are stored like Q (not transposed); the argument is
+ *     called Kt only to keep it apart from the interval count K.
+ *   - The caller owns and allocates every buffer (outputs, stats,
+ *     workspace).  The library allocates nothing, never synchronises, and
+ *     enqueues all work on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Return 0 on success or a negative KIA_ERR_* code; nothing is launched
+ *     when an argument check fails.  kiattn_strerror() names the code.
+ *   - Supported: d in {64, 128}; T >= 1 (any T, ragged tails included);
+ *     1 <= K <= 64; tau > 0 (FWM); B*H*T <= 2^30.
+ */
+#ifndef KIATTN_H_
+#define KIATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* calibration (section 3, Calibration) */
+#define KIA_CAL_MINMAX 0 /* h = row span / K */
+#define KIA_CAL_FWM 1    /* window [m - tau, m], h = tau / K, zero tail */
+/* reconstruction (section 3, Reconstruction) */
+#define KIA_REC_LERP 0
+#define KIA_REC_NEAREST 1
+/* surrogate placement for Nearest (section 3, Surrogate placement; Figure 1) */
+#define KIA_STE_WEIGHT 0 /* straight-through before normalisation */
+#define KIA_STE_PROB 1   /* straight-through after normalisation */
+/* gradient mode (section 3, Calibration gradients; Appendix B; section 5.1) */
+#define KIA_GRAD_FULL 0
+#define KIA_GRAD_DETACH 1
+#define KIA_GRAD_MAX_ONLY 2
+#define KIA_GRAD_MIN_ONLY 3
+#define KIA_GRAD_PROJECT 4
+/* contraction arithmetic (Appendix C.1: TF32 products in training) */
+#define KIA_GEMM_TF32 0 /* tcgen05 TF32 tensor-core products, fp32 accumulation */
+#define KIA_GEMM_FP32 1 /* exact fp32 products on the CUDA cores (checking mode) */
+/* operator */
+#define KIA_OP_KINTERVAL 0
+#define KIA_OP_SOFTMAX 1 /* exact softmax attention (Appendix G reference row) */
+
+/* error codes */
+#define KIA_OK 0
+#define KIA_ERR_INVALID_ARG -1  /* null pointer, bad size, bad enum, misalignment */
+#define KIA_ERR_UNSUPPORTED -2  /* valid but not implemented (e.g. d not 64/128) */
+#define KIA_ERR_CUDA -3         /* a CUDA launch or driver call failed */
+#define KIA_ERR_TIMEOUT -4      /* a bounded device-side wait gave up */
+#define KIA_ERR_STATS_MISMATCH -5 /* stats buffer written by another shape/config */
+#define KIA_ERR_CAPACITY -6     /* size beyond a fixed-capacity entry point's limit */
+
+typedef struct {
+  int n_intervals; /* K >= 1 */
+  int cal;         /* KIA_CAL_* */
+  float tau;       /* FWM window width in nats (6 in the paper) */
+  int rec;         /* KIA_REC_* */
+  int ste;         /* KIA_STE_* (ignored for LERP) */
+  int grad;        /* KIA_GRAD_* (backward only) */
+  int causal;      /* 1: key j visible to query i iff j <= i */
+  int gemm;        /* KIA_GEMM_* */
+  int op;          /* KIA_OP_* */
+} kia_config;
+
+/* Bytes of the per-row statistics buffer that kiattn_fwd writes and
+ * kiattn_bwd reads: row max/min and their indices, 1/h, the normalisers,
+ * the per-row grid (MinMax), and for Prob-STE the LERP-point output O_L.
+ * Returns 0 for invalid arguments. */
+size_t kiattn_stats_bytes(int B, int H, int T, int d, const kia_config* cfg);
+
+/* Bytes of device scratch kiattn_bwd needs (per-row centering D, the row
+ * sums A and C of the calibration terms, the calibration coefficients).
+ * Returns 0 for invalid arguments. */
+size_t kiattn_workspace_bytes(int B, int H, int T, int d, const kia_config* cfg);
+
+/* Forward (section 3; Appendix A).  Q, Kt, V: inputs [B,H,T,d].  O: output
+ * [B,H,T,d].  stats: kiattn_stats_bytes() bytes, written here and read by
+ * kiattn_bwd (keep it unchanged between the two calls).  The forward does
+ * not depend on cfg->grad, so one forward serves every gradient mode.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+int kiattn_fwd(const float* Q, const float* Kt, const float* V, float* O, void* stats, int B,
+               int H, int T, int d, const kia_config* cfg, void* stream);
+
+/* Backward (section 3, Calibration gradients and Surrogate placement;
+ * Appendix B).  Inputs Q, Kt, V, O (the forward output), dO [B,H,T,d] and
+ * the stats written by kiattn_fwd with the same shape and config (cfg->grad
+ * may differ).  Outputs dQ, dK, dV [B,H,T,d] (overwritten).  dS_dbg, when
+ * not NULL, receives the score gradient [B,H,T,T] (invisible entries 0) for
+ * checking.  workspace: kiattn_workspace_bytes() bytes of device scratch,
+ * contents on entry irrelevant.
+ * Errors: INVALID_ARG, UNSUPPORTED, STATS_MISMATCH, CUDA. */
+int kiattn_bwd(const float* Q, const float* Kt, const float* V, const float* O, const float* dO,
+               const void* stats, float* dQ, float* dK, float* dV, float* dS_dbg, int B, int H,
+               int T, int d, const kia_config* cfg, void* workspace, void* stream);
+
+/* The fp32 weight stage alone on given scores (section 3, Reconstruction;
+ * Appendix A), for bit-exact checking.  S: device fp32 [rows, cols]; row i
+ * sees keys 0..row_len[i]-1 (device int32 [rows], 1..cols).  Outputs
+ * (device, [rows, cols]; t, bin, row_m, row_n nullable): w the weight, bin
+ * the interval index k (LERP) or node r (Nearest), -1 for FWM tail or
+ * invisible keys, t the in-interval position; row_m / row_n [rows] the
+ * row extrema.  Degenerate MinMax rows give w = 1, bin = 0, t = 0.
+ * Errors: INVALID_ARG, CUDA. */
+int kiattn_weights_from_S(const float* S, int rows, int cols, const int* row_len,
+                          const kia_config* cfg, float* w, int* bin, float* t, float* row_m,
+                          float* row_n, void* stream);
+
+/* The score contraction of the forward alone, S = Q Kt^T per (batch, head),
+ * with the same tile path and arithmetic as kiattn_fwd (cfg->gemm).  S:
+ * device fp32 [B,H,T,T]; entries outside the visible set are set to 0.
+ * For checking the TF32 operand rounding against the oracle.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T, int d,
+                  const kia_config* cfg, void* stream);
+
+/* Error word raised by device code since the last reset: KIA_ERR_TIMEOUT
+ * when a bounded wait inside a kernel gave up, KIA_ERR_STATS_MISMATCH when
+ * kiattn_bwd was handed stats written for another shape or config (the
+ * backward kernels then skip their work), 0 otherwise.  Synchronous: it
+ * copies the word from the device (and clears it when reset != 0). */
+int kiattn_device_error(int reset);
+
+/* Human-readable name of a KIA_* return code (static string). */
+const char* kiattn_strerror(int code);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int kiattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIATTN_H_ */

@@ -1,0 +1,163 @@
+// Backward row passes around the main backward kernels:
+//   prep   - centering D_i = dO_i . O_bar_i (O_bar = O, or O_L for Prob-STE),
+//            clears the A / C accumulators (and dQ for the atomic path),
+//            checks the stats header against the call;
+//   calib  - calibration coefficients per row from A, C and the gradient mode
+//            (section 3 Calibration gradients; Appendix B), applied as the
+//            2-sparse update at the argmax / argmin keys;
+//   scan   - the zero-sum projection's common-mode shift c_i, which adds
+//            c_i to every visible score gradient of row i: dQ_i += c_i sum_J k_j
+//            and dK_j += sum_{i sees j} c_i q_i (prefix / suffix sums).
+// All are O(B H T d) and bandwidth-bound.
+#pragma once
+#include "kia_elem.cuh"
+#include "kia_stats.cuh"
+
+namespace kia {
+
+constexpr int kRowWarps = 8;  // warps (rows) per block in the row passes
+
+template <int D>
+__global__ void __launch_bounds__(32 * kRowWarps)
+bwd_prep_kernel(const float* __restrict__ O, const float* __restrict__ dO, StatsView st, WorkView wk,
+                float* __restrict__ dQ_zero, OpParams p, int B, int H, int T) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long rows = (long long)B * H * T;
+  const long long row = (long long)blockIdx.x * kRowWarps + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    const bool ok = header_matches(st.header, B, H, T, D, p);
+    *wk.status = ok ? 0 : 1;
+    if (!ok) atomicExch(&g_kia_device_error, KIA_ERR_STATS_MISMATCH);
+  }
+  if (row >= rows) return;
+  const float* ob = (st.OL ? st.OL : O) + row * D;
+  const float* g = dO + row * D;
+  float acc = 0.0f;
+#pragma unroll
+  for (int c = lane; c < D; c += 32) acc = fmaf(g[c], ob[c], acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    wk.D[row] = acc;
+    wk.A[row] = 0.0f;
+    wk.C[row] = 0.0f;
+    wk.gm[row] = 0.0f;
+    wk.gn[row] = 0.0f;
+  }
+  if (dQ_zero) {
+#pragma unroll
+    for (int c = lane; c < D; c += 32) dQ_zero[row * D + c] = 0.0f;
+  }
+}
+
+// Calibration coefficients (Appendix B):
+//   MinMax: g_m = A / h + C / K,  g_n = -C / K;   FWM: g_m = A / h, g_n = 0.
+// full: both; detach: none; max-only: g_m; min-only: g_n; projection: the
+// shift c = A / (h |J_i|) on every visible key (applied by the scan pass).
+template <int D>
+__global__ void __launch_bounds__(32 * kRowWarps)
+bwd_calib_kernel(const float* __restrict__ Q, const float* __restrict__ Kt, StatsView st,
+                 WorkView wk, float* __restrict__ dQ, float* __restrict__ dK,
+                 float* __restrict__ dS_dbg, OpParams p, int B, int H, int T) {
+  if (*wk.status != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long rows = (long long)B * H * T;
+  const long long row = (long long)blockIdx.x * kRowWarps + warp;
+  if (row >= rows || p.softmax || p.grad == KIA_GRAD_DETACH) return;
+  const int i = (int)(row % T);
+  const long long bh = row / T;
+  const float rh = st.rh[row];
+  if (rh == 0.0f) return;  // degenerate row: no calibration term
+  const float A = wk.A[row], C = wk.C[row];
+  const int L = p.causal ? i + 1 : T;
+  if (p.grad == KIA_GRAD_PROJECT) {
+    const float c = A * rh / (float)L;
+    if (lane == 0) wk.gm[row] = c;
+    if (dS_dbg) {
+      float* ds = dS_dbg + row * (long long)T;
+      for (int j = lane; j < L; j += 32) ds[j] += c;
+    }
+    return;
+  }
+  float gm = 0.0f, gn = 0.0f;
+  const float gm_full = (p.cal == KIA_CAL_MINMAX) ? A * rh + C / p.Kf : A * rh;
+  const float gn_full = (p.cal == KIA_CAL_MINMAX) ? -C / p.Kf : 0.0f;
+  if (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY) gm = gm_full;
+  if (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MIN_ONLY) gn = gn_full;
+  const int am = st.am[row], an = st.an[row];
+  if (lane == 0) {
+    wk.gm[row] = gm;
+    wk.gn[row] = gn;
+    if (dS_dbg) {
+      float* ds = dS_dbg + row * (long long)T;
+      ds[am] += gm;
+      ds[an] += gn;
+    }
+  }
+  const size_t base = (size_t)bh * T * D;
+  const float* q = Q + row * D;
+  const float* ka = Kt + base + (size_t)am * D;
+  const float* kn = Kt + base + (size_t)an * D;
+#pragma unroll
+  for (int c = lane; c < D; c += 32) {
+    dQ[row * D + c] += gm * ka[c] + gn * kn[c];
+    if (gm != 0.0f) atomicAdd(dK + base + (size_t)am * D + c, gm * q[c]);
+    if (gn != 0.0f) atomicAdd(dK + base + (size_t)an * D + c, gn * q[c]);
+  }
+}
+
+// Zero-sum projection, common-mode part.  Block = (bh, 32-column chunk);
+// 8 groups of 32 threads split the T rows into contiguous ranges; fp64
+// running sums.
+constexpr int kScanGroups = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kScanGroups)
+bwd_project_scan_kernel(const float* __restrict__ Q, const float* __restrict__ Kt, WorkView wk,
+                        float* __restrict__ dQ, float* __restrict__ dK, OpParams p, int T) {
+  if (*wk.status != 0) return;
+  __shared__ double sK[kScanGroups][32];
+  __shared__ double sQ[kScanGroups][32];
+  const int bh = blockIdx.x;
+  const int col = blockIdx.y * 32 + (threadIdx.x & 31);
+  const int grp = threadIdx.x >> 5;
+  const int per = (T + kScanGroups - 1) / kScanGroups;
+  const int r0 = grp * per, r1 = min(T, r0 + per);
+  const size_t base = (size_t)bh * T * D;
+  const float* cc = wk.gm + (size_t)bh * T;
+  double sk = 0.0, sq = 0.0;
+  for (int r = r0; r < r1; ++r) {
+    sk += (double)Kt[base + (size_t)r * D + col];
+    sq += (double)cc[r] * (double)Q[base + (size_t)r * D + col];
+  }
+  sK[grp][threadIdx.x & 31] = sk;
+  sQ[grp][threadIdx.x & 31] = sq;
+  __syncthreads();
+  double allK = 0.0, allQ = 0.0, preK = 0.0, sufQ = 0.0;
+  for (int g = 0; g < kScanGroups; ++g) {
+    allK += sK[g][threadIdx.x & 31];
+    allQ += sQ[g][threadIdx.x & 31];
+    if (g < grp) preK += sK[g][threadIdx.x & 31];
+    if (g > grp) sufQ += sQ[g][threadIdx.x & 31];
+  }
+  if (!p.causal) {
+    for (int r = r0; r < r1; ++r) {
+      dQ[base + (size_t)r * D + col] += (float)((double)cc[r] * allK);
+      dK[base + (size_t)r * D + col] += (float)allQ;
+    }
+    return;
+  }
+  // prefix over keys for dQ (j <= i), suffix over queries for dK (i >= j)
+  double runK = preK;
+  for (int r = r0; r < r1; ++r) {
+    runK += (double)Kt[base + (size_t)r * D + col];
+    dQ[base + (size_t)r * D + col] += (float)((double)cc[r] * runK);
+  }
+  double runQ = sufQ;
+  for (int r = r1 - 1; r >= r0; --r) {
+    runQ += (double)cc[r] * (double)Q[base + (size_t)r * D + col];
+    dK[base + (size_t)r * D + col] += (float)runQ;
+  }
+}
+
+}  // namespace kia

@@ -1,0 +1,219 @@
+// Tensor-core (tcgen05, kind::tf32) path: host-side tensor maps and the
+// score-tile kernel behind kiattn_scores.  The fused forward and backward
+// kernels are in kia_tc_fwd.cuh / kia_tc_bwd.cuh.
+//
+// Shared-memory operand tiles: a [128 rows x d] fp32 tile is stored as d/32
+// column blocks of [128 rows x 32 fp32] (128 B per row, 16 KB per block).
+// Two swizzles, both written by TMA from the same [B*H, T, d] tensor:
+//  * K-major (the contraction runs over d, rows are M or N): 128-byte
+//    swizzle of 16-byte atoms, 8-row groups 1024 B apart;
+//  * MN-major (the contraction runs over the rows): tf32 operands must use
+//    the 128-byte swizzle of 32-byte atoms, 4-row groups 512 B apart, column
+//    blocks 16 KB apart.
+// A tile used both ways (Q, dO, K in the backward) is loaded once per layout.
+#pragma once
+#include <cuda.h>
+
+#include "kia_elem.cuh"
+#include "kia_stats.cuh"
+
+namespace kia {
+
+constexpr uint32_t kBlockBytes = KIA_TILE * 128;  // one [128 x 32] fp32 column block
+
+// ------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [BH, T, d] fp32 tensor; box = 32 columns x 128 rows x 1, 128-byte swizzle
+// (16-byte atoms for K-major use, 32-byte atoms for MN-major use),
+// out-of-range rows read as zero.
+inline bool make_tmap(CUtensorMap* m, const float* base, int BH, int T, int d,
+                      bool mn_major = false) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)T * d * 4};
+  cuuint32_t box[3] = {32, KIA_TILE, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------ descriptor helpers
+
+// K-major operand, 8-element (32-byte) K step ks of a tile at smem address
+// `tile`: column block ks / 4, byte offset (ks % 4) * 32 inside the 128-byte
+// swizzle row.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int ks) {
+  return smem_desc(tile + (uint32_t)(ks >> 2) * kBlockBytes + (uint32_t)(ks & 3) * 32u, 16u, 1024u,
+                   kLayoutSW128);
+}
+// MN-major operand (32-byte-atom swizzle), K step ks = rows 8ks..8ks+7
+// (1024 B); two 4-row groups 512 B apart, column blocks 16 KB apart.
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int ks) {
+  return smem_desc(tile + (uint32_t)ks * 1024u, kBlockBytes, 512u, kLayoutSW128Atom32);
+}
+
+// ------------------------------------------------------ score tile kernel
+
+template <int D>
+struct ScoresSmem {
+  float q[D * KIA_TILE];
+  float k[D * KIA_TILE];
+  uint64_t bar_tma;
+  uint64_t bar_mma;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// One 128 x 128 score tile per CTA (4 warps).  Thread t of the CTA owns
+// TMEM lane t = query row t of the tile.
+template <int D>
+__global__ void __launch_bounds__(128)
+tc_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 float* __restrict__ S, OpParams p, int T) {
+  extern __shared__ __align__(1024) uint8_t smraw[];
+  ScoresSmem<D>& sm = *reinterpret_cast<ScoresSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  const int qt = blockIdx.x, kt = blockIdx.y, bh = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = qt * KIA_TILE + threadIdx.x;
+  const bool skip = p.causal && kt > qt;
+  if (skip) {
+    if (row < T) {
+      float* dst = S + ((size_t)bh * T + row) * T + (size_t)kt * KIA_TILE;
+      for (int c = 0; c < KIA_TILE && kt * KIA_TILE + c < T; ++c) dst[c] = 0.0f;
+    }
+    return;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_tma, 1);
+    mbar_init(&sm.bar_mma, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    mbar_arrive_expect_tx(&sm.bar_tma, 2u * D * KIA_TILE * 4u);
+#pragma unroll
+    for (int b = 0; b < D / 32; ++b) {
+      tma_load_3d(sm.q + b * 32 * KIA_TILE, &tmQ, &sm.bar_tma, b * 32, qt * KIA_TILE, bh);
+      tma_load_3d(sm.k + b * 32 * KIA_TILE, &tmK, &sm.bar_tma, b * 32, kt * KIA_TILE, bh);
+    }
+    if (mbar_wait(&sm.bar_tma, 0, abort)) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_tf32(128, 128, 0, 0);
+      const uint32_t qa = smem_u32(sm.q), ka = smem_u32(sm.k);
+#pragma unroll
+      for (int ks = 0; ks < D / 8; ++ks)
+        mma_tf32_ss(tmem, desc_kmajor(qa, ks), desc_kmajor(ka, ks), idesc, ks > 0 ? 1u : 0u);
+      tc_commit(&sm.bar_mma);
+    }
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_mma, 0, abort));
+  tc_fence_after();
+  if (ok) {
+    float v[32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32), v);
+      tmem_ld_wait();
+      if (row < T) {
+        float* dst = S + ((size_t)bh * T + row) * T;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int key = kt * KIA_TILE + c * 32 + i;
+          if (key < T) dst[key] = (p.causal && key > row) ? 0.0f : v[i];
+        }
+      }
+    }
+  } else {
+    drain_in_flight();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+template <int D>
+int tc_scores(const float* Q, const float* Kt, float* S, int B, int H, int T, const OpParams& p,
+              cudaStream_t s) {
+  CUtensorMap tq, tk;
+  if (!make_tmap(&tq, Q, B * H, T, D) || !make_tmap(&tk, Kt, B * H, T, D)) return KIA_ERR_CUDA;
+  const size_t smem = sizeof(ScoresSmem<D>) + 1024;
+  if (cudaFuncSetAttribute(tc_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return KIA_ERR_CUDA;
+  const int nt = (T + KIA_TILE - 1) / KIA_TILE;
+  dim3 grid(nt, nt, B * H);
+  tc_scores_kernel<D><<<grid, 128, smem, s>>>(tq, tk, S, p, T);
+  return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
+}
+
+// Exact-fp32 scores (same dot-product order as the exact path's kernels).
+template <int D>
+__global__ void simt_scores_kernel(const float* __restrict__ Q, const float* __restrict__ Kt,
+                                   float* __restrict__ S, OpParams p, int T) {
+  const int bh = blockIdx.y;
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)T * T) return;
+  const int i = (int)(e / T), j = (int)(e % T);
+  const float* q = Q + ((size_t)bh * T + i) * D;
+  const float* k = Kt + ((size_t)bh * T + j) * D;
+  float s = 0.0f;
+  for (int c = 0; c < D; ++c) s = fmaf(q[c], k[c], s);
+  S[(size_t)bh * T * T + e] = (p.causal && j > i) ? 0.0f : s;
+}
+
+template <int D>
+int simt_scores(const float* Q, const float* Kt, float* S, int B, int H, int T, const OpParams& p,
+                cudaStream_t s) {
+  dim3 grid((unsigned)(((long long)T * T + 255) / 256), B * H);
+  simt_scores_kernel<D><<<grid, 256, 0, s>>>(Q, Kt, S, p, T);
+  return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
+}
+
+// Fused kernels: filled in by kia_tc_fwd.cuh / kia_tc_bwd.cuh.
+template <int D>
+int tc_forward(const float* Q, const float* Kt, const float* V, float* O, void* stats, int B,
+               int H, int T, const OpParams& p, cudaStream_t s);
+template <int D>
+int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO,
+                const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
+                float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s);
+
+}  // namespace kia
+
+#include "kia_tc_bwd.cuh"
+#include "kia_tc_fwd.cuh"

@@ -1,0 +1,380 @@
+// Fused tensor-core forward of K-interval attention (sm_100a).
+//
+// One CTA per (batch*head, 128-query tile), heaviest causal tiles first.
+// Two sweeps over the key tiles, because the grid of a row is anchored at
+// its final extrema (section 3, Calibration): no weight exists before the
+// row max (and min) are known, so there is no online rescaling.
+//   sweep 1: S = Q K^T (tcgen05 kind::tf32, accumulator in TMEM) -> row
+//            max / min and their lowest indices;
+//   calibration: h, 1/h, and the grid G_k = e^{-k h} (per row under MinMax,
+//            one shared table under FWM) into shared memory;
+//   sweep 2: S recomputed -> weights from the grid (LERP or Nearest, FWM
+//            tail) -> written back into the same TMEM columns as the A
+//            operand of O += P V (and P_L for Prob-STE, O_L += P_L V);
+//   epilogue: O = O_acc / W (and O_L = O_L_acc / W_L), per-row statistics.
+//
+// Warp roles (6 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
+// 2..5 = element warps; element thread r owns TMEM lane r = query row r of
+// the tile (warp w reaches lanes 32*(w%4)..32*(w%4)+31).
+#pragma once
+#include "kia_tc.cuh"
+
+namespace kia {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kStages = (D == 64) ? 2 : 1;      // K and V ring depth
+  static constexpr uint32_t kTileBytes = D * KIA_TILE * 4;
+  static constexpr int kThreads = 192;
+};
+
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2];    // S tile ready in TMEM buffer b (tcgen05.commit)
+  uint64_t s_free[2];    // sweep 1: element warps done reading buffer b (128 arrivals)
+  uint64_t p_ready[2];   // sweep 2: P written into buffer b (128 arrivals)
+  uint64_t pv_done[2];   // sweep 2: P V of buffer b finished (tcgen05.commit)
+  uint64_t pl_free;      // P_L consumed by O_L += P_L V (tcgen05.commit)
+  uint64_t o_full;       // all P V done
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
+tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, StatsView st,
+              OpParams p, int B, int H, int T, int nsb) {
+  using Cfg = FwdCfg<D>;
+  constexpr int NS = Cfg::kStages;
+  extern __shared__ uint8_t smraw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
+                                             ~uintptr_t(1023));
+  float* sQ = reinterpret_cast<float*>(base);
+  float* sK = reinterpret_cast<float*>(base + Cfg::kTileBytes);
+  float* sV = reinterpret_cast<float*>(base + (1 + NS) * Cfg::kTileBytes);
+  float* sTab = reinterpret_cast<float*>(base + (1 + 2 * NS) * Cfg::kTileBytes);
+  const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
+  const int tab_floats = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : (p.K + 1));
+  FwdBars& bar = *reinterpret_cast<FwdBars*>(sTab + ((tab_floats + 31) & ~31));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int nt = (T + KIA_TILE - 1) / KIA_TILE;
+  const int qt = nt - 1 - blockIdx.y;
+  const int nkt = p.causal ? qt + 1 : nt;
+  const bool prob = needs_OL(p);
+  // TMEM columns: S buffers [0, 128*nsb), P_L, O, O_L
+  const uint32_t col_pl = 128u * nsb;
+  const uint32_t col_o = col_pl + (prob ? 128u : 0u);
+  const uint32_t col_ol = col_o + D;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.k_empty[s], 1);
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
+      mbar_init(&bar.s_full[s], 1);
+      mbar_init(&bar.s_free[s], 128);
+      mbar_init(&bar.p_ready[s], 128);
+      mbar_init(&bar.pv_done[s], 1);
+    }
+    mbar_init(&bar.pl_free, 1);
+    mbar_init(&bar.o_full, 1);
+    bar.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  volatile int* abort = &bar.abort;
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bar.q_full, Cfg::kTileBytes);
+      for (int b = 0; b < D / 32; ++b)
+        tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.q_full, b * 32, qt * KIA_TILE, bh);
+      int kc = 0, vc = 0;
+      for (int sweep = 0; sweep < 2 && !failed; ++sweep) {
+        for (int j = 0; j < nkt; ++j) {
+          {
+            const int s = kc % NS, n = kc / NS;
+            if (!mbar_wait(&bar.k_empty[s], (n & 1) ^ 1, abort)) { failed = true; break; }
+            mbar_arrive_expect_tx(&bar.k_full[s], Cfg::kTileBytes);
+            float* dst = sK + s * (Cfg::kTileBytes / 4);
+            for (int b = 0; b < D / 32; ++b)
+              tma_load_3d(dst + b * 32 * KIA_TILE, &tmK, &bar.k_full[s], b * 32, j * KIA_TILE, bh);
+            ++kc;
+          }
+          if (sweep == 1) {
+            const int s = vc % NS, n = vc / NS;
+            if (!mbar_wait(&bar.v_empty[s], (n & 1) ^ 1, abort)) { failed = true; break; }
+            mbar_arrive_expect_tx(&bar.v_full[s], Cfg::kTileBytes);
+            float* dst = sV + s * (Cfg::kTileBytes / 4);
+            for (int b = 0; b < D / 32; ++b)
+              tma_load_3d(dst + b * 32 * KIA_TILE, &tmV, &bar.v_full[s], b * 32, j * KIA_TILE, bh);
+            ++vc;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_tf32(128, 128, 0, 0);
+      const uint32_t idesc_o = idesc_tf32(128, D, 0, 1);
+      const uint32_t qa = smem_u32(sQ);
+      int kc = 0, vc = 0;
+      int use1[2] = {0, 0};   // sweep-1 uses of each S buffer
+      int use2[2] = {0, 0};   // sweep-2 uses of each S buffer
+      failed = !mbar_wait(&bar.q_full, 0, abort);
+      // issue S = Q K_j^T into buffer b
+      auto issue_s = [&](int sweep, int j) -> bool {
+        const int b = j % nsb;
+        if (sweep == 0) {
+          if (use1[b] > 0 && !mbar_wait(&bar.s_free[b], (use1[b] - 1) & 1, abort)) return false;
+          ++use1[b];
+        } else {
+          if (use2[b] == 0) {
+            if (use1[b] > 0 && !mbar_wait(&bar.s_free[b], (use1[b] - 1) & 1, abort)) return false;
+          } else if (!mbar_wait(&bar.pv_done[b], (use2[b] - 1) & 1, abort)) {
+            return false;
+          }
+          ++use2[b];
+        }
+        const int s = kc % NS, n = kc / NS;
+        if (!mbar_wait(&bar.k_full[s], n & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sK + s * (Cfg::kTileBytes / 4));
+#pragma unroll
+        for (int ks = 0; ks < D / 8; ++ks)
+          mma_tf32_ss(tmem + 128u * b, desc_kmajor(qa, ks), desc_kmajor(ka, ks), idesc_s,
+                      ks > 0 ? 1u : 0u);
+        tc_commit(&bar.s_full[b]);
+        tc_commit(&bar.k_empty[s]);
+        ++kc;
+        return true;
+      };
+      if (!failed) {
+        for (int j = 0; j < nkt; ++j)
+          if (!issue_s(0, j)) { failed = true; break; }
+      }
+      if (!failed) {
+        int pr[2] = {0, 0};
+        if (!issue_s(1, 0)) failed = true;
+        for (int j = 0; j < nkt && !failed; ++j) {
+          // two S buffers: the next S overlaps this tile's weights and P V;
+          // one buffer: the next S must wait until P V has read P
+          if (nsb == 2 && j + 1 < nkt && !issue_s(1, j + 1)) { failed = true; break; }
+          const int b = j % nsb;
+          if (!mbar_wait(&bar.p_ready[b], pr[b] & 1, abort)) { failed = true; break; }
+          ++pr[b];
+          const int s = vc % NS, n = vc / NS;
+          if (!mbar_wait(&bar.v_full[s], n & 1, abort)) { failed = true; break; }
+          tc_fence_after();
+          const uint32_t va = smem_u32(sV + s * (Cfg::kTileBytes / 4));
+#pragma unroll
+          for (int ks = 0; ks < KIA_TILE / 8; ++ks)
+            mma_tf32_ts(tmem + col_o, tmem + 128u * b + 8u * ks, desc_mnmajor(va, ks), idesc_o,
+                        (j > 0 || ks > 0) ? 1u : 0u);
+          if (prob) {
+#pragma unroll
+            for (int ks = 0; ks < KIA_TILE / 8; ++ks)
+              mma_tf32_ts(tmem + col_ol, tmem + col_pl + 8u * ks, desc_mnmajor(va, ks), idesc_o,
+                          (j > 0 || ks > 0) ? 1u : 0u);
+            tc_commit(&bar.pl_free);
+          }
+          tc_commit(&bar.v_empty[s]);
+          tc_commit(&bar.pv_done[b]);
+          ++vc;
+          if (nsb == 1 && j + 1 < nkt && !issue_s(1, j + 1)) { failed = true; break; }
+        }
+        if (!failed) tc_commit(&bar.o_full);
+      }
+    }
+  } else {
+    // ------------------------------------------------------ element warps
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qrow = qt * KIA_TILE + r;
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    int sf[2] = {0, 0};  // completed phases of s_full per buffer
+    float m = -INFINITY, n = INFINITY;
+    int am = 0, an = 0;
+    float v[32];
+    // sweep 1: statistics
+    for (int j = 0; j < nkt; ++j) {
+      const int b = j % nsb;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
+      ++sf[b];
+      tc_fence_after();
+      const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tmem + lane_addr + 128u * b + 32u * c, v);
+        tmem_ld_wait();
+        const int key0 = j * KIA_TILE + c * 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int key = key0 + i;
+          const bool ok = !edge || (key < T && (!p.causal || key <= qrow));
+          if (ok) {
+            if (v[i] > m) { m = v[i]; am = key; }
+            if (v[i] < n) { n = v[i]; an = key; }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar.s_free[b]);
+    }
+    // calibration (section 3) and the grid
+    const RowState rs = make_row_state(p, m, n);
+    const int ts = minmax_tab ? KIA_TILE : 1;
+    const float* tab = minmax_tab ? sTab + r : sTab;
+    const long long grow = (long long)bh * T + qrow;
+    if (!p.softmax) {
+      if (minmax_tab) {
+        for (int k = 0; k <= p.K; ++k) {
+          const float G = rs.degen ? 1.0f : grid_value(k, rs.cal.h);
+          sTab[k * KIA_TILE + r] = G;
+          if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
+        }
+      } else if (r <= p.K) {
+        const float G = grid_value(r, p.fwm_h);
+        sTab[r] = G;
+        if (bh == 0 && qt == nt - 1) st.table[r] = G;
+      }
+    }
+    named_bar_sync(1, 128);
+    // sweep 2: weights -> P (and P_L) in TMEM, normalisers
+    float W = 0.0f, WL = 0.0f;
+    for (int j = 0; j < nkt && !failed; ++j) {
+      const int b = j % nsb;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
+      ++sf[b];
+      if (prob && j > 0 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bar.pl_free, (j - 1) & 1, abort))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tmem + lane_addr + 128u * b + 32u * c, v);
+        tmem_ld_wait();
+        float vl[32];
+        const int key0 = j * KIA_TILE + c * 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int key = key0 + i;
+          const bool ok = !edge || (key < T && (!p.causal || key <= qrow));
+          ElemFwd e = elem_forward(p, rs, tab, ts, v[i]);
+          if (!ok) { e.wf = 0.0f; e.wl = 0.0f; }
+          W += e.wf;
+          WL += e.wl;
+          v[i] = e.wf;
+          vl[i] = e.wl;
+        }
+        tmem_st32(tmem + lane_addr + 128u * b + 32u * c, v);
+        if (prob) tmem_st32(tmem + lane_addr + col_pl + 32u * c, vl);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bar.p_ready[b]);
+    }
+    // epilogue
+    if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.o_full, 0, abort))) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        tmem_ld32(tmem + lane_addr + col_o + 32u * c, v);
+        tmem_ld_wait();
+        if (qrow < T) {
+          float4* o4 = reinterpret_cast<float4*>(O + grow * D + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            o4[i] = make_float4(__fdiv_rn(v[4 * i], W), __fdiv_rn(v[4 * i + 1], W),
+                                __fdiv_rn(v[4 * i + 2], W), __fdiv_rn(v[4 * i + 3], W));
+        }
+        if (prob) {
+          tmem_ld32(tmem + lane_addr + col_ol + 32u * c, v);
+          tmem_ld_wait();
+          if (qrow < T) {
+            float4* o4 = reinterpret_cast<float4*>(st.OL + grow * D + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              o4[i] = make_float4(__fdiv_rn(v[4 * i], WL), __fdiv_rn(v[4 * i + 1], WL),
+                                  __fdiv_rn(v[4 * i + 2], WL), __fdiv_rn(v[4 * i + 3], WL));
+          }
+        }
+      }
+      if (qrow < T) {
+        st.m[grow] = m;
+        st.n[grow] = n;
+        st.am[grow] = am;
+        st.an[grow] = an;
+        st.rh[grow] = rs.degen ? 0.0f : rs.cal.rh;
+        st.h[grow] = rs.degen ? 0.0f : rs.cal.h;
+        st.Wf[grow] = W;
+        st.Wb[grow] = (!p.softmax && lerp_normpoint(p)) ? WL : W;
+      }
+      if (bh == 0 && qt == nt - 1 && r == 0) write_header(st.header, B, H, T, D, p);
+    } else {
+      failed = true;
+    }
+  }
+  if (failed || *abort) drain_in_flight();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+size_t tc_fwd_smem(const OpParams& p) {
+  constexpr int NS = FwdCfg<D>::kStages;
+  const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
+  const int tab = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : (p.K + 1));
+  return 1024 + (size_t)(1 + 2 * NS) * FwdCfg<D>::kTileBytes + (size_t)((tab + 31) & ~31) * 4 +
+         sizeof(FwdBars);
+}
+
+template <int D>
+int tc_forward(const float* Q, const float* Kt, const float* V, float* O, void* stats, int B,
+               int H, int T, const OpParams& p, cudaStream_t s) {
+  const long long rows = (long long)B * H * T;
+  StatsView st = stats_view(stats, rows, D, p);
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, Q, B * H, T, D) || !make_tmap(&tk, Kt, B * H, T, D) ||
+      !make_tmap(&tv, V, B * H, T, D, /*mn_major=*/true))
+    return KIA_ERR_CUDA;
+  const size_t smem = tc_fwd_smem<D>(p);
+  if (smem > 232448) return KIA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(tc_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return KIA_ERR_CUDA;
+  // TMEM: S buffers (128 columns each), P_L (128, Prob-STE), O and O_L (D each)
+  const bool prob = needs_OL(p);
+  int nsb = 2;
+  if (256 + (prob ? 128 + 2 * D : D) > 512) nsb = 1;
+  const int nt = (T + KIA_TILE - 1) / KIA_TILE;
+  dim3 grid(B * H, nt);
+  tc_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, smem, s>>>(tq, tk, tv, O, st, p, B, H, T, nsb);
+  return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
+}
+
+}  // namespace kia

@@ -1,0 +1,281 @@
+// kiattn C ABI: argument checks, launch configuration and the order of the
+// kernels for K-interval attention forward and backward on sm_100a.
+// One translation unit: the kernels live in the headers included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/kiattn.h"
+#include "kia_common.cuh"
+#include "kia_elem.cuh"
+#include "kia_epilogue.cuh"
+#include "kia_simt.cuh"
+#include "kia_stats.cuh"
+#include "kia_tc.cuh"
+#include "kia_weights.cuh"
+
+using namespace kia;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_config(const kia_config* cfg) {
+  if (!cfg) return KIA_ERR_INVALID_ARG;
+  if (cfg->n_intervals < 1 || cfg->n_intervals > KIA_MAX_K) return KIA_ERR_UNSUPPORTED;
+  if (cfg->cal != KIA_CAL_MINMAX && cfg->cal != KIA_CAL_FWM) return KIA_ERR_INVALID_ARG;
+  if (cfg->rec != KIA_REC_LERP && cfg->rec != KIA_REC_NEAREST) return KIA_ERR_INVALID_ARG;
+  if (cfg->ste != KIA_STE_WEIGHT && cfg->ste != KIA_STE_PROB) return KIA_ERR_INVALID_ARG;
+  if (cfg->grad < KIA_GRAD_FULL || cfg->grad > KIA_GRAD_PROJECT) return KIA_ERR_INVALID_ARG;
+  if (cfg->gemm != KIA_GEMM_TF32 && cfg->gemm != KIA_GEMM_FP32) return KIA_ERR_INVALID_ARG;
+  if (cfg->op != KIA_OP_KINTERVAL && cfg->op != KIA_OP_SOFTMAX) return KIA_ERR_INVALID_ARG;
+  if (cfg->causal != 0 && cfg->causal != 1) return KIA_ERR_INVALID_ARG;
+  if (cfg->cal == KIA_CAL_FWM && !(cfg->tau > 0.0f && cfg->tau < 1e30f)) return KIA_ERR_INVALID_ARG;
+  return KIA_OK;
+}
+
+int check_shape(int B, int H, int T, int d) {
+  if (B < 1 || H < 1 || T < 1) return KIA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KIA_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * H * T;
+  if (rows > (1ll << 30) || (long long)B * H > 65535ll * 1024) return KIA_ERR_UNSUPPORTED;
+  if (rows * (long long)d > (1ll << 40)) return KIA_ERR_UNSUPPORTED;
+  return KIA_OK;
+}
+
+OpParams make_params(const kia_config* cfg) {
+  OpParams p;
+  p.K = cfg->n_intervals;
+  p.Kf = (float)p.K;
+  p.cal = cfg->cal;
+  p.rec = cfg->rec;
+  p.ste = (cfg->rec == KIA_REC_LERP) ? KIA_STE_WEIGHT : cfg->ste;
+  p.grad = cfg->grad;
+  p.causal = cfg->causal;
+  p.softmax = cfg->op == KIA_OP_SOFTMAX;
+  p.tau = cfg->tau;
+  p.fwm_h = (cfg->cal == KIA_CAL_FWM) ? cfg->tau / p.Kf : 0.0f;
+  p.fwm_rh = (cfg->cal == KIA_CAL_FWM) ? p.Kf / cfg->tau : 0.0f;
+  p.tf32_ops = 0;
+  if (p.softmax) {  // the softmax row has no grid: normalise the unused axes
+    p.cal = KIA_CAL_MINMAX;
+    p.rec = KIA_REC_LERP;
+    p.ste = KIA_STE_WEIGHT;
+    p.K = 1;
+    p.Kf = 1.0f;
+    p.tau = 0.0f;
+    p.fwm_h = p.fwm_rh = 0.0f;
+  }
+  return p;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
+}
+
+template <typename Kern>
+int set_smem(Kern k, size_t bytes) {
+  if (bytes > 48 * 1024) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+      return KIA_ERR_CUDA;
+  }
+  return KIA_OK;
+}
+
+size_t simt_tab_floats(const OpParams& p, int rowsPerTab) {
+  if (p.softmax) return 0;
+  return (p.cal == KIA_CAL_MINMAX) ? (size_t)(p.K + 1) * rowsPerTab : (size_t)(p.K + 1);
+}
+
+template <int D>
+int simt_forward(const float* Q, const float* Kt, const float* V, float* O, void* stats, int B,
+                 int H, int T, const OpParams& p, cudaStream_t s) {
+  const long long rows = (long long)B * H * T;
+  StatsView st = stats_view(stats, rows, D, p);
+  const size_t smem =
+      (kSimtRows * (D + 1) + 2 * kSimtKeys * D + simt_tab_floats(p, kSimtRows)) * sizeof(float);
+  if (set_smem(simt_fwd_kernel<D>, smem)) return KIA_ERR_CUDA;
+  dim3 grid((T + kSimtRows - 1) / kSimtRows, B * H);
+  simt_fwd_kernel<D><<<grid, kSimtRows, smem, s>>>(Q, Kt, V, O, st, p, B, H, T);
+  return launch_status();
+}
+
+template <int D>
+int simt_backward(const float* Q, const float* Kt, const float* V, const float* dO,
+                  const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
+                  float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s) {
+  dim3 grid((T + kSimtRows - 1) / kSimtRows, B * H);
+  const size_t smq = (2 * kSimtRows * (D + 1) + 2 * kSimtKeys * D + simt_tab_floats(p, kSimtRows)) *
+                     sizeof(float);
+  if (set_smem(simt_bwd_q_kernel<D>, smq)) return KIA_ERR_CUDA;
+  simt_bwd_q_kernel<D><<<grid, kSimtRows, smq, s>>>(Q, Kt, V, dO, st, wk, dQ, dS_dbg, p, T);
+  if (launch_status()) return KIA_ERR_CUDA;
+  const size_t smkv = (2 * kSimtRows * (D + 1) + 2 * kSimtKeys * D + kSimtKeys * 6 +
+                       simt_tab_floats(p, kSimtKeys)) *
+                      sizeof(float);
+  if (set_smem(simt_bwd_kv_kernel<D>, smkv)) return KIA_ERR_CUDA;
+  simt_bwd_kv_kernel<D><<<grid, kSimtRows, smkv, s>>>(Q, Kt, V, dO, st, wk, dK, dV, p, T);
+  return launch_status();
+}
+
+template <int D>
+int backward_rows(const float* Q, const float* Kt, const float* O, const float* dO,
+                  const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dS_dbg,
+                  int B, int H, int T, const OpParams& p, cudaStream_t s, bool prep,
+                  float* dQ_zero) {
+  const long long rows = (long long)B * H * T;
+  const unsigned nb = (unsigned)((rows + kRowWarps - 1) / kRowWarps);
+  if (prep) {
+    bwd_prep_kernel<D><<<nb, 32 * kRowWarps, 0, s>>>(O, dO, st, wk, dQ_zero, p, B, H, T);
+    return launch_status();
+  }
+  bwd_calib_kernel<D><<<nb, 32 * kRowWarps, 0, s>>>(Q, Kt, st, wk, dQ, dK, dS_dbg, p, B, H, T);
+  if (launch_status()) return KIA_ERR_CUDA;
+  if (!p.softmax && p.grad == KIA_GRAD_PROJECT) {
+    dim3 g(B * H, D / 32);
+    bwd_project_scan_kernel<D><<<g, 32 * kScanGroups, 0, s>>>(Q, Kt, wk, dQ, dK, p, T);
+    if (launch_status()) return KIA_ERR_CUDA;
+  }
+  return KIA_OK;
+}
+
+template <int D>
+int backward(const float* Q, const float* Kt, const float* V, const float* O, const float* dO,
+             const void* stats, float* dQ, float* dK, float* dV, float* dS_dbg, int B, int H,
+             int T, const OpParams& p, int gemm, void* workspace, cudaStream_t s) {
+  const long long rows = (long long)B * H * T;
+  StatsView st = stats_view(const_cast<void*>(stats), rows, D, p);
+  WorkView wk = work_view(workspace, rows);
+  if (dS_dbg) {
+    if (cudaMemsetAsync(dS_dbg, 0, (size_t)rows * T * sizeof(float), s) != cudaSuccess)
+      return KIA_ERR_CUDA;
+  }
+  const bool tc = gemm == KIA_GEMM_TF32;
+  int rc = backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, true, nullptr);
+  if (rc) return rc;
+  if (tc && D == 64) {
+    rc = tc_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s);
+  } else {
+    // d = 128 in TF32 mode: CUDA-core kernels with the tensor cores' operand
+    // truncation, so the backward sees the arithmetic of the TF32 forward
+    OpParams q = p;
+    q.tf32_ops = tc ? 1 : 0;
+    rc = simt_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, q, s);
+  }
+  if (rc) return rc;
+  return backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, false, nullptr);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kiattn_stats_bytes(int B, int H, int T, int d, const kia_config* cfg) {
+  if (check_config(cfg) || check_shape(B, H, T, d)) return 0;
+  const OpParams p = make_params(cfg);
+  return stats_layout((long long)B * H * T, d, p).total;
+}
+
+size_t kiattn_workspace_bytes(int B, int H, int T, int d, const kia_config* cfg) {
+  if (check_config(cfg) || check_shape(B, H, T, d)) return 0;
+  return work_bytes((long long)B * H * T);
+}
+
+int kiattn_fwd(const float* Q, const float* Kt, const float* V, float* O, void* stats, int B,
+               int H, int T, int d, const kia_config* cfg, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_shape(B, H, T, d))) return rc;
+  if (!Q || !Kt || !V || !O || !stats) return KIA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(Kt) || !aligned16(V) || !aligned16(O) || !aligned16(stats))
+    return KIA_ERR_INVALID_ARG;
+  const OpParams p = make_params(cfg);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->gemm == KIA_GEMM_FP32) {
+    return d == 64 ? simt_forward<64>(Q, Kt, V, O, stats, B, H, T, p, s)
+                   : simt_forward<128>(Q, Kt, V, O, stats, B, H, T, p, s);
+  }
+  return d == 64 ? tc_forward<64>(Q, Kt, V, O, stats, B, H, T, p, s)
+                 : tc_forward<128>(Q, Kt, V, O, stats, B, H, T, p, s);
+}
+
+int kiattn_bwd(const float* Q, const float* Kt, const float* V, const float* O, const float* dO,
+               const void* stats, float* dQ, float* dK, float* dV, float* dS_dbg, int B, int H,
+               int T, int d, const kia_config* cfg, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_shape(B, H, T, d))) return rc;
+  if (!Q || !Kt || !V || !O || !dO || !stats || !dQ || !dK || !dV || !workspace)
+    return KIA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(Kt) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
+      !aligned16(stats) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
+      !aligned16(workspace) || (dS_dbg && !aligned16(dS_dbg)))
+    return KIA_ERR_INVALID_ARG;
+  const OpParams p = make_params(cfg);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? backward<64>(Q, Kt, V, O, dO, stats, dQ, dK, dV, dS_dbg, B, H, T, p, cfg->gemm,
+                                workspace, s)
+                 : backward<128>(Q, Kt, V, O, dO, stats, dQ, dK, dV, dS_dbg, B, H, T, p,
+                                 cfg->gemm, workspace, s);
+}
+
+int kiattn_weights_from_S(const float* S, int rows, int cols, const int* row_len,
+                          const kia_config* cfg, float* w, int* bin, float* t, float* row_m,
+                          float* row_n, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!S || !row_len || !w || rows < 1 || cols < 1) return KIA_ERR_INVALID_ARG;
+  if ((long long)rows * cols > (1ll << 40)) return KIA_ERR_UNSUPPORTED;
+  if (cfg->op != KIA_OP_KINTERVAL) return KIA_ERR_INVALID_ARG;
+  const OpParams p = make_params(cfg);
+  const unsigned nb = (unsigned)((rows + kWeightsWarps - 1) / kWeightsWarps);
+  weights_from_S_kernel<<<nb, 32 * kWeightsWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+      S, rows, cols, row_len, p, w, bin, t, row_m, row_n);
+  return launch_status();
+}
+
+int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T, int d,
+                  const kia_config* cfg, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_shape(B, H, T, d))) return rc;
+  if (!Q || !Kt || !S || !aligned16(Q) || !aligned16(Kt) || !aligned16(S))
+    return KIA_ERR_INVALID_ARG;
+  const OpParams p = make_params(cfg);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->gemm == KIA_GEMM_FP32) {
+    return d == 64 ? simt_scores<64>(Q, Kt, S, B, H, T, p, s)
+                   : simt_scores<128>(Q, Kt, S, B, H, T, p, s);
+  }
+  return d == 64 ? tc_scores<64>(Q, Kt, S, B, H, T, p, s) : tc_scores<128>(Q, Kt, S, B, H, T, p, s);
+}
+
+const char* kiattn_strerror(int code) {
+  switch (code) {
+    case KIA_OK: return "ok";
+    case KIA_ERR_INVALID_ARG: return "invalid argument";
+    case KIA_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case KIA_ERR_CUDA: return "CUDA launch or driver error";
+    case KIA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case KIA_ERR_STATS_MISMATCH: return "stats buffer was written for another shape or config";
+    case KIA_ERR_CAPACITY: return "size exceeds the fixed scratch capacity";
+    default: return "unknown error";
+  }
+}
+
+int kiattn_version(void) { return 10000; }
+
+int kiattn_device_error(int reset) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_kia_device_error, sizeof(int)) != cudaSuccess) return KIA_ERR_CUDA;
+  if (reset) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(g_kia_device_error, &z, sizeof(int)) != cudaSuccess) return KIA_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

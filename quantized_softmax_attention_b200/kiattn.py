@@ -1,0 +1,204 @@
+"""Python binding of the kiattn C ABI (argument marshalling only).
+
+Every function here has the name of a C entry point in ``include/kiattn.h``
+and forwards torch CUDA tensors' device pointers plus the current CUDA
+stream.  All arithmetic runs in the CUDA library ``libkiattn.so``; there is
+no Python, PyTorch or CPU implementation of the operator behind these calls.
+If the library is missing the import fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkiattn.so")
+
+CAL_MINMAX, CAL_FWM = 0, 1
+REC_LERP, REC_NEAREST = 0, 1
+STE_WEIGHT, STE_PROB = 0, 1
+GRAD_FULL, GRAD_DETACH, GRAD_MAX_ONLY, GRAD_MIN_ONLY, GRAD_PROJECT = 0, 1, 2, 3, 4
+GEMM_TF32, GEMM_FP32 = 0, 1
+OP_KINTERVAL, OP_SOFTMAX = 0, 1
+
+ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error", -4: "timeout",
+          -5: "stats mismatch", -6: "capacity exceeded"}
+
+SYMBOLS = ("kiattn_stats_bytes", "kiattn_workspace_bytes", "kiattn_fwd", "kiattn_bwd",
+           "kiattn_weights_from_S", "kiattn_scores", "kiattn_strerror", "kiattn_version",
+           "kiattn_device_error")
+
+
+class KiattnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({ERRORS.get(code, 'unknown')})")
+        self.code = code
+
+
+class kia_config(ctypes.Structure):
+    _fields_ = [("n_intervals", ctypes.c_int), ("cal", ctypes.c_int), ("tau", ctypes.c_float),
+                ("rec", ctypes.c_int), ("ste", ctypes.c_int), ("grad", ctypes.c_int),
+                ("causal", ctypes.c_int), ("gemm", ctypes.c_int), ("op", ctypes.c_int)]
+
+
+@dataclass(frozen=True)
+class Config:
+    """The operator's axes (section 3): K, calibration, reconstruction,
+    surrogate, gradient mode; plus causal mask, contraction arithmetic and
+    operator (K-interval or exact softmax)."""
+
+    K: int = 4
+    cal: int = CAL_MINMAX
+    tau: float = 6.0
+    rec: int = REC_LERP
+    ste: int = STE_WEIGHT
+    grad: int = GRAD_FULL
+    causal: bool = True
+    gemm: int = GEMM_TF32
+    op: int = OP_KINTERVAL
+
+    def c(self) -> kia_config:
+        return kia_config(int(self.K), int(self.cal), float(self.tau), int(self.rec),
+                          int(self.ste), int(self.grad), int(bool(self.causal)), int(self.gemm),
+                          int(self.op))
+
+    def replace(self, **kw) -> "Config":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return Config(**d)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"kiattn CUDA library not built: {LIB_PATH} is missing "
+                          "(run python -m quantized_softmax_attention_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, cp, i = ctypes.c_void_p, ctypes.POINTER(kia_config), ctypes.c_int
+    lib.kiattn_stats_bytes.argtypes = [i, i, i, i, cp]
+    lib.kiattn_stats_bytes.restype = ctypes.c_size_t
+    lib.kiattn_workspace_bytes.argtypes = [i, i, i, i, cp]
+    lib.kiattn_workspace_bytes.restype = ctypes.c_size_t
+    lib.kiattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, cp, vp]
+    lib.kiattn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, cp, vp, vp]
+    lib.kiattn_weights_from_S.argtypes = [vp, i, i, vp, cp, vp, vp, vp, vp, vp, vp]
+    lib.kiattn_scores.argtypes = [vp, vp, vp, i, i, i, i, cp, vp]
+    lib.kiattn_strerror.argtypes = [i]
+    lib.kiattn_strerror.restype = ctypes.c_char_p
+    lib.kiattn_version.restype = i
+    lib.kiattn_device_error.argtypes = [i]
+    for name in ("kiattn_fwd", "kiattn_bwd", "kiattn_weights_from_S", "kiattn_scores",
+                 "kiattn_device_error"):
+        getattr(lib, name).restype = i
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("kiattn takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("kiattn takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise KiattnError(fn, rc)
+
+
+def kiattn_stats_bytes(B, H, T, d, cfg: Config) -> int:
+    return int(_lib.kiattn_stats_bytes(B, H, T, d, ctypes.byref(cfg.c())))
+
+
+def kiattn_workspace_bytes(B, H, T, d, cfg: Config) -> int:
+    return int(_lib.kiattn_workspace_bytes(B, H, T, d, ctypes.byref(cfg.c())))
+
+
+def kiattn_fwd(Q, K, V, O, stats, cfg: Config, stream=None):
+    B, H, T, d = Q.shape
+    _check("kiattn_fwd", _lib.kiattn_fwd(_p(Q), _p(K), _p(V), _p(O), _p(stats), B, H, T, d,
+                                         ctypes.byref(cfg.c()), _stream(stream)))
+
+
+def kiattn_bwd(Q, K, V, O, dO, stats, dQ, dK, dV, workspace, cfg: Config, dS_dbg=None,
+               stream=None):
+    B, H, T, d = Q.shape
+    _check("kiattn_bwd", _lib.kiattn_bwd(_p(Q), _p(K), _p(V), _p(O), _p(dO), _p(stats), _p(dQ),
+                                         _p(dK), _p(dV), _p(dS_dbg), B, H, T, d,
+                                         ctypes.byref(cfg.c()), _p(workspace), _stream(stream)))
+
+
+def kiattn_weights_from_S(S, row_len, cfg: Config, w, bin=None, t=None, row_m=None, row_n=None,
+                          stream=None):
+    rows, cols = S.shape
+    _check("kiattn_weights_from_S",
+           _lib.kiattn_weights_from_S(_p(S), rows, cols, _p(row_len), ctypes.byref(cfg.c()), _p(w),
+                                      _p(bin), _p(t), _p(row_m), _p(row_n), _stream(stream)))
+
+
+def kiattn_scores(Q, K, S, cfg: Config, stream=None):
+    B, H, T, d = Q.shape
+    _check("kiattn_scores", _lib.kiattn_scores(_p(Q), _p(K), _p(S), B, H, T, d,
+                                               ctypes.byref(cfg.c()), _stream(stream)))
+
+
+def kiattn_strerror(code: int) -> str:
+    return _lib.kiattn_strerror(code).decode()
+
+
+def kiattn_version() -> int:
+    return int(_lib.kiattn_version())
+
+
+def kiattn_device_error(reset: bool = True) -> int:
+    return int(_lib.kiattn_device_error(1 if reset else 0))
+
+
+# ------------------------------------------------------------ conveniences
+
+class Buffers:
+    """Device buffers for one shape/config: outputs, stats and workspace,
+    allocated once with torch (the library itself allocates nothing)."""
+
+    def __init__(self, B, H, T, d, cfg: Config, device="cuda"):
+        self.shape = (B, H, T, d)
+        f = dict(dtype=torch.float32, device=device)
+        self.O = torch.empty(self.shape, **f)
+        self.dQ = torch.empty(self.shape, **f)
+        self.dK = torch.empty(self.shape, **f)
+        self.dV = torch.empty(self.shape, **f)
+        sb = kiattn_stats_bytes(B, H, T, d, cfg)
+        wb = kiattn_workspace_bytes(B, H, T, d, cfg)
+        if sb == 0 or wb == 0:
+            raise KiattnError("kiattn_stats_bytes", -1)
+        self.stats = torch.empty(sb, dtype=torch.uint8, device=device)
+        self.work = torch.empty(wb, dtype=torch.uint8, device=device)
+
+
+def forward(Q, K, V, cfg: Config, bufs: Buffers | None = None, stream=None):
+    bufs = bufs or Buffers(*Q.shape, cfg, device=Q.device)
+    kiattn_fwd(Q, K, V, bufs.O, bufs.stats, cfg, stream)
+    return bufs
+
+
+def backward(Q, K, V, dO, cfg: Config, bufs: Buffers, dS_dbg=None, stream=None):
+    kiattn_bwd(Q, K, V, bufs.O, dO, bufs.stats, bufs.dQ, bufs.dK, bufs.dV, bufs.work, cfg,
+               dS_dbg=dS_dbg, stream=stream)
+    return bufs

@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds for
+sm_100a, loads, exports every entry point that include/kiattn.h declares,
+sizes its buffers, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def K():
+    from quantized_softmax_attention_b200 import build
+    build.build()
+    from quantized_softmax_attention_b200 import kiattn
+    return kiattn
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kiattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kiattn_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol(K):
+    lib = ctypes.CDLL(K.LIB_PATH)
+    names = _declared()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(K.SYMBOLS)
+
+
+def test_version_and_strerror(K):
+    assert K.kiattn_version() >= 10000
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert K.kiattn_strerror(code) != "unknown error"
+    assert K.kiattn_strerror(-99) == "unknown error"
+
+
+def test_buffer_sizes(K):
+    cfg = K.Config(K=4, cal=K.CAL_MINMAX)
+    B, H, T, d = 2, 3, 300, 64
+    rows = B * H * T
+    sb = K.kiattn_stats_bytes(B, H, T, d, cfg)
+    # 8 per-row words + per-row grid of K+1 values, plus header and padding
+    assert sb >= rows * (8 + 5) * 4
+    assert sb < rows * (8 + 5) * 4 + 64 * 1024
+    fwm = K.kiattn_stats_bytes(B, H, T, d, cfg.replace(cal=K.CAL_FWM))
+    assert fwm < sb
+    prob = K.kiattn_stats_bytes(B, H, T, d, cfg.replace(rec=K.REC_NEAREST, ste=K.STE_PROB))
+    assert prob >= sb + rows * d * 4          # O_L for Prob-STE
+    wb = K.kiattn_workspace_bytes(B, H, T, d, cfg)
+    assert rows * 5 * 4 <= wb < rows * 5 * 4 + 4096
+    assert K.kiattn_stats_bytes(B, H, T, 96, cfg) == 0      # d unsupported
+    assert K.kiattn_stats_bytes(B, H, T, d, cfg.replace(K=0)) == 0
+    assert K.kiattn_stats_bytes(B, H, T, d, cfg.replace(K=65)) == 0
+    assert K.kiattn_stats_bytes(B, H, T, d, cfg.replace(cal=K.CAL_FWM, tau=0.0)) == 0
+
+
+def test_bad_arguments_rejected_without_launch(K):
+    lib = K.lib()
+    c = K.Config().c()
+    fake = ctypes.c_void_p(1 << 20)          # never dereferenced: checks fail first
+    # null pointers
+    assert lib.kiattn_fwd(None, fake, fake, fake, fake, 1, 1, 128, 64, ctypes.byref(c), None) == -1
+    # unsupported head size
+    assert lib.kiattn_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 96, ctypes.byref(c), None) == -2
+    # misaligned pointer
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.kiattn_fwd(odd, fake, fake, fake, fake, 1, 1, 128, 64, ctypes.byref(c), None) == -1
+    # bad enum / K
+    bad = K.Config(grad=7).c()
+    assert lib.kiattn_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, ctypes.byref(bad), None) == -1
+    bad = K.Config(K=100).c()
+    assert lib.kiattn_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, ctypes.byref(bad), None) == -2
+    # empty shapes
+    assert lib.kiattn_fwd(fake, fake, fake, fake, fake, 1, 1, 0, 64, ctypes.byref(c), None) == -1
+    assert lib.kiattn_bwd(fake, fake, fake, fake, fake, fake, fake, fake, fake, None, 0, 1, 16, 64,
+                          ctypes.byref(c), fake, None) == -1
+    assert lib.kiattn_bwd(fake, fake, fake, fake, None, fake, fake, fake, fake, None, 1, 1, 16, 64,
+                          ctypes.byref(c), fake, None) == -1
+    assert lib.kiattn_weights_from_S(fake, 0, 8, fake, ctypes.byref(c), fake, None, None, None,
+                                     None, None) == -1
+    assert lib.kiattn_scores(fake, fake, None, 1, 1, 8, 64, ctypes.byref(c), None) == -1
+    assert lib.kiattn_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, None, None) == -1
+
+
+def test_product_path_does_not_import_the_oracle():
+    """The binding and the CUDA sources never reference the oracle."""
+    pkg = os.path.join(ROOT, "quantized_softmax_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "kiattn_ref" not in txt, f

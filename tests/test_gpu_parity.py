@@ -1,0 +1,223 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Sizes span several 128-row tiles and a ragged tail; tolerances are the ones
+the operator's checking protocol fixes: bit-exact weight stage on the same
+scores, relative L2 <= 1e-5 in exact-fp32 mode and <= 2e-3 in TF32 mode,
+per-row |sum_j dS_j| <= 1e-5 ||dS_i|| for the zero-sum gradient modes.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as ref
+
+pytestmark = pytest.mark.gpu
+
+K = pytest.importorskip("quantized_softmax_attention_b200.kiattn")
+from parity_util import compare, flag_rows, oracle_scores, rel_l2  # noqa: E402
+
+RECSTE = [(K.REC_LERP, K.STE_WEIGHT), (K.REC_NEAREST, K.STE_WEIGHT), (K.REC_NEAREST, K.STE_PROB)]
+MODES = [K.GRAD_FULL, K.GRAD_DETACH, K.GRAD_MAX_ONLY, K.GRAD_MIN_ONLY, K.GRAD_PROJECT]
+# operand rounding of the tcgen05 kind::tf32 MMA, measured by
+# test_tc_scores_operand_rounding below
+TF32_RULE = ref.ROUND_TRUNC
+
+
+def _inputs(B, H, T, d, seed, qscale=None, kscale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    sh = (B, H, T, d)
+    q = torch.randn(sh, generator=g) * (qscale if qscale is not None else d ** -0.5)
+    k = torch.randn(sh, generator=g) * kscale
+    v = torch.randn(sh, generator=g)
+    do = torch.randn(sh, generator=g)
+    return [x.numpy().astype(np.float32) for x in (q, k, v, do)]
+
+
+# ------------------------------------------------------------ weight stage
+
+def _weight_rows(rng, rows, cols):
+    S = rng.standard_normal((rows, cols)).astype(np.float32) * rng.uniform(0.5, 12, (rows, 1)).astype(np.float32)
+    L = rng.integers(1, cols + 1, rows).astype(np.int32)
+    # crafted rows: constant (degenerate), two values, scores on grid nodes,
+    # a huge span (subnormal / zero grid values), a near-degenerate span
+    S[0] = 1.25
+    S[1, :] = 0.0
+    S[1, ::2] = -3.0
+    S[2] = -1.5 * rng.integers(0, 5, cols).astype(np.float32)
+    S[3] = np.linspace(0, -400, cols).astype(np.float32)
+    S[4] = (1.0 + rng.integers(0, 2, cols) * 1e-6).astype(np.float32)
+    L[:5] = cols
+    return S, L
+
+
+@pytest.mark.parametrize("cal", [K.CAL_MINMAX, K.CAL_FWM])
+@pytest.mark.parametrize("rec", [K.REC_LERP, K.REC_NEAREST])
+@pytest.mark.parametrize("Kint", [1, 2, 4, 16, 64])
+def test_weight_stage_bit_exact(cal, rec, Kint):
+    """Bin indices, t, row extrema and weights equal the oracle's fp32
+    definition bit for bit on the same scores."""
+    rng = np.random.default_rng(1000 + 10 * cal + rec + Kint)
+    S, L = _weight_rows(rng, 300, 517)
+    cfg = K.Config(K=Kint, cal=cal, rec=rec, tau=6.0)
+    exp = ref.weights_fp32(S, L, ref.RefConfig(K=Kint, cal=cal, rec=rec, tau=6.0))
+    dev = "cuda"
+    s = torch.from_numpy(S).to(dev)
+    l = torch.from_numpy(L).to(dev)
+    w = torch.empty_like(s)
+    t = torch.empty_like(s)
+    b = torch.empty(S.shape, dtype=torch.int32, device=dev)
+    m = torch.empty(S.shape[0], device=dev)
+    n = torch.empty(S.shape[0], device=dev)
+    K.kiattn_weights_from_S(s, l, cfg, w, b, t, m, n)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(m.cpu().numpy().view(np.uint32), exp["m"].view(np.uint32))
+    np.testing.assert_array_equal(n.cpu().numpy().view(np.uint32), exp["n"].view(np.uint32))
+    np.testing.assert_array_equal(b.cpu().numpy(), exp["bin"])
+    np.testing.assert_array_equal(t.cpu().numpy().view(np.uint32), exp["t"].view(np.uint32))
+    np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), exp["w"].view(np.uint32))
+
+
+# ------------------------------------------------------------------ scores
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp32_scores_exact(d):
+    Q, Kt, _, _ = _inputs(1, 2, 200, d, 5)
+    cfg = K.Config(gemm=K.GEMM_FP32)
+    q, k = torch.from_numpy(Q).cuda(), torch.from_numpy(Kt).cuda()
+    S = torch.empty((1, 2, 200, 200), device="cuda")
+    K.kiattn_scores(q, k, S, cfg)
+    exp = np.tril(oracle_scores(Q, Kt, ref.ROUND_NONE))
+    assert rel_l2(S.cpu().numpy(), exp) < 1e-6
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [128, 300])
+def test_tc_scores_operand_rounding(d, T):
+    """The tcgen05 TF32 scores match the oracle's S with operands rounded by
+    TF32_RULE to fp32 accumulation accuracy (and the other rules do not)."""
+    Q, Kt, _, _ = _inputs(2, 2, T, d, 6, qscale=1.0)
+    q, k = torch.from_numpy(Q).cuda(), torch.from_numpy(Kt).cuda()
+    S = torch.empty((2, 2, T, T), device="cuda")
+    for causal in (True, False):
+        K.kiattn_scores(q, k, S, K.Config(causal=causal))
+        got = S.cpu().numpy()
+        errs = {}
+        for rule in (ref.ROUND_TRUNC, ref.ROUND_RNA, ref.ROUND_RNE, ref.ROUND_NONE):
+            exp = oracle_scores(Q, Kt, rule)
+            if causal:
+                exp = np.tril(exp)
+            errs[rule] = rel_l2(got, exp)
+        print("tf32 rounding rule errors", errs)
+        assert errs[TF32_RULE] < 2e-6, errs
+        assert min(v for r, v in errs.items() if r != TF32_RULE) > 10 * errs[TF32_RULE], errs
+
+
+# ------------------------------------------------- exact-fp32 operator path
+
+SMALL = [(1, 2, 128, 64), (1, 2, 200, 64), (1, 1, 160, 128)]
+
+
+@pytest.mark.parametrize("shape", SMALL)
+@pytest.mark.parametrize("cal", [K.CAL_MINMAX, K.CAL_FWM])
+@pytest.mark.parametrize("rec,ste", RECSTE)
+def test_fp32_path_matches_oracle_all_modes(shape, cal, rec, ste):
+    B, H, T, d = shape
+    Q, Kt, V, dO = _inputs(B, H, T, d, 7 + T + d + cal, qscale=0.5)
+    for grad in MODES:
+        cfg = K.Config(K=4, cal=cal, rec=rec, ste=ste, grad=grad, gemm=K.GEMM_FP32)
+        errs, gpu, _ = compare(Q, Kt, V, dO, cfg, ref.ROUND_NONE, 1e-5, 1e-4)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 1e-5, (grad, errs)
+        if grad in (K.GRAD_FULL, K.GRAD_PROJECT):
+            assert errs["zero_sum"] < 1e-5, errs
+        assert errs["flagged"] < errs["rows"] // 4
+
+
+def test_fp32_path_softmax_and_noncausal():
+    Q, Kt, V, dO = _inputs(1, 2, 192, 64, 11)
+    for causal, op in itertools.product((True, False), (K.OP_SOFTMAX, K.OP_KINTERVAL)):
+        cfg = K.Config(K=16, cal=K.CAL_MINMAX, rec=K.REC_LERP, causal=causal, op=op,
+                       gemm=K.GEMM_FP32)
+        errs, _, _ = compare(Q, Kt, V, dO, cfg, ref.ROUND_NONE, 1e-5, 1e-4)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 1e-5, (causal, op, errs)
+
+
+def test_fp32_forward_bitwise_identical_across_modes_and_surrogates():
+    Q, Kt, V, dO = _inputs(1, 2, 256, 64, 12, qscale=0.7)
+    from parity_util import run_gpu
+    for cal in (K.CAL_MINMAX, K.CAL_FWM):
+        outs = []
+        for grad, ste in itertools.product(MODES, (K.STE_WEIGHT, K.STE_PROB)):
+            cfg = K.Config(K=4, cal=cal, rec=K.REC_NEAREST, ste=ste, grad=grad, gemm=K.GEMM_FP32)
+            outs.append(run_gpu(Q, Kt, V, dO, cfg, bwd=False)["O"])
+        for o in outs[1:]:
+            np.testing.assert_array_equal(o.view(np.uint32), outs[0].view(np.uint32))
+
+
+# ------------------------------------------------- tensor-core (TF32) path
+
+TC_SHAPES = [(1, 2, 128, 64), (1, 2, 200, 64), (2, 1, 384, 64)]
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES)
+@pytest.mark.parametrize("cal", [K.CAL_MINMAX, K.CAL_FWM])
+@pytest.mark.parametrize("rec,ste", RECSTE)
+def test_tc_path_matches_oracle_all_modes(shape, cal, rec, ste):
+    """tcgen05 TF32 forward + backward against the oracle with TF32 operand
+    rounding, every gradient mode, tolerance 2e-3 relative L2."""
+    B, H, T, d = shape
+    Q, Kt, V, dO = _inputs(B, H, T, d, 21 + T + cal, qscale=0.5)
+    for grad in MODES:
+        cfg = K.Config(K=4, cal=cal, rec=rec, ste=ste, grad=grad)
+        errs, _, _ = compare(Q, Kt, V, dO, cfg, TF32_RULE, 2e-3, 1e-4)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 2e-3, (grad, errs)
+        if grad in (K.GRAD_FULL, K.GRAD_PROJECT):
+            assert errs["zero_sum"] < 1e-5, errs
+        assert errs["flagged"] < errs["rows"] // 4
+
+
+@pytest.mark.parametrize("Kint", [1, 2, 16, 32, 64])
+@pytest.mark.parametrize("cal", [K.CAL_MINMAX, K.CAL_FWM])
+def test_tc_path_interval_counts(Kint, cal):
+    Q, Kt, V, dO = _inputs(1, 2, 256, 64, 31 + Kint, qscale=0.5)
+    for rec, ste in RECSTE:
+        cfg = K.Config(K=Kint, cal=cal, rec=rec, ste=ste)
+        errs, _, _ = compare(Q, Kt, V, dO, cfg, TF32_RULE, 2e-3, 1e-4)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 2e-3, (rec, ste, errs)
+
+
+def test_tc_path_softmax_and_noncausal():
+    Q, Kt, V, dO = _inputs(1, 2, 320, 64, 41)
+    for causal, op in itertools.product((True, False), (K.OP_SOFTMAX, K.OP_KINTERVAL)):
+        cfg = K.Config(K=16, cal=K.CAL_MINMAX, rec=K.REC_LERP, causal=causal, op=op)
+        errs, _, _ = compare(Q, Kt, V, dO, cfg, TF32_RULE, 2e-3, 1e-4)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 2e-3, (causal, op, errs)
+
+
+def test_tc_forward_bitwise_identical_across_modes_and_surrogates():
+    Q, Kt, V, dO = _inputs(2, 2, 256, 64, 42, qscale=0.7)
+    from parity_util import run_gpu
+    for cal in (K.CAL_MINMAX, K.CAL_FWM):
+        outs = []
+        for grad, ste in itertools.product(MODES, (K.STE_WEIGHT, K.STE_PROB)):
+            cfg = K.Config(K=4, cal=cal, rec=K.REC_NEAREST, ste=ste, grad=grad)
+            outs.append(run_gpu(Q, Kt, V, dO, cfg, bwd=False)["O"])
+        for o in outs[1:]:
+            np.testing.assert_array_equal(o.view(np.uint32), outs[0].view(np.uint32))
+
+
+def test_tc_d128_forward_and_backward():
+    Q, Kt, V, dO = _inputs(1, 2, 256, 128, 43)
+    for cal, (rec, ste) in itertools.product((K.CAL_MINMAX, K.CAL_FWM), RECSTE):
+        cfg = K.Config(K=32, cal=cal, rec=rec, ste=ste)
+        errs, _, _ = compare(Q, Kt, V, dO, cfg, TF32_RULE, 2e-3, 1e-4)
+        assert errs["O"] < 2e-3, errs
+        # the d = 128 backward runs the exact-fp32 kernels on the TF32 forward
+        for name in ("dQ", "dK", "dV"):
+            assert errs[name] < 2e-3, (cal, rec, ste, errs)
