@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark: K-interval attention forward + backward on B200.
+
+Default workload: the GPT-2-124M attention shape B8 H12 T1024 d64, causal,
+FWM (tau = 6, h = 1.5), Nearest reconstruction with Prob-STE, K = 4, full
+calibration gradients -- synthetic inputs with per-head score spans of 8-40
+nats.  One step = kiattn_fwd + kiattn_bwd over that batch.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  Throughput is algorithmic TFLOP/s: causal
+GEMM units U = B*H*T^2*d; forward 3U (+1U for Prob-STE's P_L V), backward 5U.
+With N GPUs (torchrun) every rank runs its own batch (weak scaling, no
+collective on the data path); value = all ranks' flops / max-over-ranks time.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+# roofline denominators: MEASURED_PEAKS.json (bf16 dense burst) scaled by the
+# nominal dense TF32 / BF16 ratio of B200 (1.1 / 2.25 PFLOP/s)
+TF32_OVER_BF16 = 1.1 / 2.25
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gpt2_fwm",
+                    choices=["gpt2_fwm", "gpt2_heavy", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def workload(name):
+    from quantized_softmax_attention_b200 import workloads as W
+    return {"gpt2_fwm": W.gpt2_fwm, "gpt2_heavy": W.gpt2_heavy, "tiny": W.tiny}[name]()
+
+
+def gemm_units(w):
+    return w.B * w.H * w.T * w.T * w.d
+
+
+def algorithmic_flops(w):
+    """Forward 3U (+1U with Prob-STE) and backward 5U, U = B H T^2 d
+    (2 flops per multiply-add over the causal half counts T^2 d per GEMM)."""
+    prob = w.rec == 1 and w.ste == 1
+    return (8 + (1 if prob else 0)) * gemm_units(w)
+
+
+def config_dict(w, n):
+    names = {0: "MinMax", 1: "FWM"}
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "K": w.K,
+            "calibration": names[w.cal], "tau": w.tau if w.cal == 1 else None,
+            "reconstruction": "LERP" if w.rec == 0 else "Nearest",
+            "surrogate": None if w.rec == 0 else ("Prob-STE" if w.ste else "Weight-STE"),
+            "grad": "full", "causal": w.causal, "parallelism": f"dp{n}",
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+        return float(mp["bf16_tflops"]), float(mp["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, enabled: bool = True):
+        self.index = index
+        self.proc = None
+        self.path = None
+        if not enabled:
+            return
+        fd, self.path = tempfile.mkstemp(prefix="kia_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9 or parts[0] != str(self.index):
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU side
+
+def cpu_oracle_rate(w, target_s=10.0, max_reps=20):
+    """fp64 CPU oracle (test infrastructure) on the full workload, repeated
+    until ~target_s of work; returns (TFLOP/s, seconds, reps, cores)."""
+    import oracle as ref
+    from quantized_softmax_attention_b200 import workloads as W
+    q, k, v, g = (x.numpy() for x in W.make_inputs(w))
+    cfg = ref.RefConfig(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
+                        causal=w.causal)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        ref.attention(q, k, v, g, cfg)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= target_s or reps >= max_reps:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return algorithmic_flops(w) * reps / el / 1e12, el, reps, cores
+
+
+def reference_arm(args):
+    """The oracle timed as the reference implementation: each step is the
+    fp64 CPU operator on a bounded sample (the first heads of batch 0)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as ref
+    from quantized_softmax_attention_b200 import workloads as W
+    w = workload(args.workload)
+    heads = min(w.H, 4)
+    q, k, v, g = (x.numpy() for x in W.make_inputs(w, B=1, H=heads))
+    cfg = ref.RefConfig(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
+                        causal=w.causal)
+    flops = algorithmic_flops(w) * heads / (w.B * w.H)
+    for _ in range(args.warmup):
+        ref.attention(q, k, v, g, cfg)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        ref.attention(q, k, v, g, cfg)
+    el = time.perf_counter() - t0
+    val = flops * args.steps / el / 1e12
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = f"batch 0, heads 0..{heads - 1} of {w.name} per step (fp64, OpenMP)"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w, 1),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "K-interval attn fwd+bwd TFLOP/s at B8·H12·T1024·d64; % TF32 roofline"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "quantized_softmax_attention_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    ent = rec.get("kernels", {}).get(kernel)
+    if not ent or rec.get("source_digest") != source_digest():
+        return None
+    return ent.get("bytes_per_launch_full_size")
+
+
+# ------------------------------------------------------------------ GPU side
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from quantized_softmax_attention_b200 import kiattn as K
+    from quantized_softmax_attention_b200 import workloads as W
+
+    w = workload(args.workload)
+    cfg = K.Config(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
+                   causal=w.causal, gemm=K.GEMM_TF32)
+    w_rank = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    host = [x.pin_memory() for x in W.make_inputs(w_rank)]
+    dev = [x.cuda() for x in host]
+    q, k, v, g = dev
+    bufs = K.Buffers(w.B, w.H, w.T, w.d, cfg)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        K.kiattn_fwd(q, k, v, bufs.O, bufs.stats, cfg)
+        K.kiattn_bwd(q, k, v, bufs.O, g, bufs.stats, bufs.dQ, bufs.dK, bufs.dV, bufs.work, cfg)
+
+    launches_per_step = 1 + 4 + (1 if w.grad == K.GRAD_PROJECT else 0)
+    K.kiattn_profile_enable(True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    err = K.kiattn_device_error(True)
+    if err != 0:
+        raise RuntimeError(f"device error word {err}")
+
+    sampler = ClockSampler(local, enabled=not args.no_clocks)
+    time.sleep(0.3 if sampler.proc else 0.0)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    phase_tot = {}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+        ph = K.kiattn_profile_read()          # synchronises on this step
+        for kk, vv in ph.items():
+            phase_tot[kk] = phase_tot.get(kk, 0.0) + vv
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = float(t.item()) / args.steps
+    flops = algorithmic_flops(w)
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        hout = [torch.empty(bufs.O.shape, dtype=torch.float32).pin_memory() for _ in range(4)]
+        nrep = max(3, min(args.steps, 50))
+        for _ in range(2):
+            for hd, dd in zip(host, dev):
+                dd.copy_(hd, non_blocking=True)
+            step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(nrep):
+            for hd, dd in zip(host, dev):
+                dd.copy_(hd, non_blocking=True)
+            step()
+            for ho, dd in zip(hout, (bufs.O, bufs.dQ, bufs.dK, bufs.dV)):
+                ho.copy_(dd, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / nrep], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        nbytes = sum(x.numel() * 4 for x in host)
+        e2e = {"value": world * flops / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": 4 * bufs.O.numel() * 4,
+               "ms_per_step": float(te.item())}
+    K.kiattn_profile_enable(False)
+
+    # roofline of the dominant kernel (tensor-core bound: TF32 contraction)
+    U = gemm_units(w)
+    prob = w.rec == 1 and w.ste == 1
+    kernel_flops = {"fwd": (3 + (1 if prob else 0)) * U, "bwd_query_pass": 3 * U,
+                    "bwd_key_pass": 4 * U}
+    kernel_names = {"fwd": "tc_fwd_kernel", "bwd_query_pass": "tc_bwd_q_kernel",
+                    "bwd_key_pass": "tc_bwd_kv_kernel"}
+    dom = max(kernel_flops, key=lambda kk: phase_tot.get(kk, 0.0))
+    dom_ms = phase_tot[dom] / args.steps
+    bf16, _, src = peaks()
+    peak = bf16 * TF32_OVER_BF16
+    achieved = kernel_flops[dom] / (dom_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": kernel_names[dom], "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": ncu_traffic(kernel_names[dom]),
+            "peak_source": f"{src} bf16 dense x {TF32_OVER_BF16:.4f} (nominal TF32/BF16)",
+            "flops_per_launch": kernel_flops[dom],
+            "phase_ms": {kk: vv / args.steps for kk, vv in phase_tot.items()}}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32",
+            "data": "synthetic", "config": config_dict(w, world), "roofline": roof,
+            "frac_of_tf32_roofline": value / world / peak,
+            "gpu_launches": launches_per_step * args.steps}
+    if e2e:
+        line["e2e"] = e2e
+    if clocks:
+        line["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, secs, reps, cores = cpu_oracle_rate(w)
+        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": f"full {w.name} batch x{reps} ({secs:.1f} s, fp64)"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -149,6 +149,17 @@ int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T
  * copies the word from the device (and clears it when reset != 0). */
 int kiattn_device_error(int reset);
 
+/* Phase timing for profiling.  kiattn_profile_enable(1) makes kiattn_fwd
+ * and kiattn_bwd record CUDA events on their stream around each internal
+ * kernel (the library creates its events once; no device memory).
+ * kiattn_profile_read() synchronises on the last recorded event and writes
+ * the milliseconds of the most recent calls' phases into ms[0..n-1] in this
+ * order: forward kernel, backward row prep, backward query pass, backward
+ * key pass, backward calibration rows; it returns the number written or a
+ * negative KIA_ERR_* code.  Not thread-safe; meant for benchmarks. */
+int kiattn_profile_enable(int on);
+int kiattn_profile_read(float* ms, int n);
+
 /* Human-readable name of a KIA_* return code (static string). */
 const char* kiattn_strerror(int code);
 

@@ -142,6 +142,9 @@ __device__ __forceinline__ GridPos grid_position(const OpParams& p, const RowCal
   }
   int k = (int)floorf(u);
   k = k > p.K - 1 ? p.K - 1 : k;
+  // u >= 0 whenever s is the score the row max came from; a score
+  // recomputed by a different contraction order can exceed m by an ulp
+  k = k < 0 ? 0 : k;
   g.k = k;
   g.u = u;
   g.t = __fsub_rn(u, (float)k);

@@ -211,7 +211,8 @@ int tc_forward(const float* Q, const float* Kt, const float* V, float* O, void* 
 template <int D>
 int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO,
                 const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
-                float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s);
+                float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
+                void (*mark)(int, cudaStream_t));
 
 }  // namespace kia
 

@@ -503,7 +503,8 @@ size_t tc_bwd_kv_smem(const OpParams& p) {
 template <int D>
 int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO,
                 const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
-                float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s) {
+                float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
+                void (*mark)(int, cudaStream_t)) {
   if constexpr (D != 64) {
     return KIA_ERR_UNSUPPORTED;
   } else {
@@ -526,8 +527,10 @@ int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO
     tc_bwd_q_kernel<D><<<grid, kBwdThreads, smq, s>>>(tq, tg, tk, tkm, tv, st, wk, dQ, dS_dbg, p,
                                                       T);
     if (cudaGetLastError() != cudaSuccess) return KIA_ERR_CUDA;
+    mark(4, s);
     tc_bwd_kv_kernel<D><<<grid, kBwdThreads, smk, s>>>(tq, tqm, tg, tgm, tk, tv, st, wk, dK, dV,
                                                        p, T);
+    mark(5, s);
     return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
   }
 }

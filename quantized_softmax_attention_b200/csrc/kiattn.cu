@@ -21,6 +21,18 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// ------------------------------------------------------ phase profiling
+// Events: 0 fwd start, 1 fwd end, 2 bwd start, 3 after prep, 4 after the
+// query pass, 5 after the key pass, 6 after the calibration rows.
+constexpr int kProfEvents = 7;
+bool g_prof_on = false;
+bool g_prof_created = false;
+cudaEvent_t g_prof_ev[kProfEvents];
+
+void prof_mark(int i, cudaStream_t s) {
+  if (g_prof_on) cudaEventRecord(g_prof_ev[i], s);
+}
+
 int check_config(const kia_config* cfg) {
   if (!cfg) return KIA_ERR_INVALID_ARG;
   if (cfg->n_intervals < 1 || cfg->n_intervals > KIA_MAX_K) return KIA_ERR_UNSUPPORTED;
@@ -154,19 +166,25 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
       return KIA_ERR_CUDA;
   }
   const bool tc = gemm == KIA_GEMM_TF32;
+  prof_mark(2, s);
   int rc = backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, true, nullptr);
   if (rc) return rc;
+  prof_mark(3, s);
   if (tc && D == 64) {
-    rc = tc_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s);
+    rc = tc_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s, prof_mark);
   } else {
     // d = 128 in TF32 mode: CUDA-core kernels with the tensor cores' operand
     // truncation, so the backward sees the arithmetic of the TF32 forward
     OpParams q = p;
     q.tf32_ops = tc ? 1 : 0;
     rc = simt_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, q, s);
+    prof_mark(4, s);
+    prof_mark(5, s);
   }
   if (rc) return rc;
-  return backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, false, nullptr);
+  rc = backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, false, nullptr);
+  prof_mark(6, s);
+  return rc;
 }
 
 }  // namespace
@@ -194,12 +212,16 @@ int kiattn_fwd(const float* Q, const float* Kt, const float* V, float* O, void* 
     return KIA_ERR_INVALID_ARG;
   const OpParams p = make_params(cfg);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  prof_mark(0, s);
   if (cfg->gemm == KIA_GEMM_FP32) {
-    return d == 64 ? simt_forward<64>(Q, Kt, V, O, stats, B, H, T, p, s)
-                   : simt_forward<128>(Q, Kt, V, O, stats, B, H, T, p, s);
-  }
-  return d == 64 ? tc_forward<64>(Q, Kt, V, O, stats, B, H, T, p, s)
+    rc = d == 64 ? simt_forward<64>(Q, Kt, V, O, stats, B, H, T, p, s)
+                 : simt_forward<128>(Q, Kt, V, O, stats, B, H, T, p, s);
+  } else {
+    rc = d == 64 ? tc_forward<64>(Q, Kt, V, O, stats, B, H, T, p, s)
                  : tc_forward<128>(Q, Kt, V, O, stats, B, H, T, p, s);
+  }
+  prof_mark(1, s);
+  return rc;
 }
 
 int kiattn_bwd(const float* Q, const float* Kt, const float* V, const float* O, const float* dO,
@@ -267,6 +289,33 @@ const char* kiattn_strerror(int code) {
 }
 
 int kiattn_version(void) { return 10000; }
+
+int kiattn_profile_enable(int on) {
+  if (on && !g_prof_created) {
+    for (int i = 0; i < kProfEvents; ++i)
+      if (cudaEventCreate(&g_prof_ev[i]) != cudaSuccess) return KIA_ERR_CUDA;
+    g_prof_created = true;
+  }
+  g_prof_on = on != 0;
+  return KIA_OK;
+}
+
+int kiattn_profile_read(float* ms, int n) {
+  if (!ms || n < 0) return KIA_ERR_INVALID_ARG;
+  if (!g_prof_created) return KIA_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(g_prof_ev[kProfEvents - 1]) != cudaSuccess ||
+      cudaEventSynchronize(g_prof_ev[1]) != cudaSuccess)
+    return KIA_ERR_CUDA;
+  const int pairs[5][2] = {{0, 1}, {2, 3}, {3, 4}, {4, 5}, {5, 6}};
+  int w = 0;
+  for (int i = 0; i < 5 && w < n; ++i, ++w) {
+    float t = 0.0f;
+    if (cudaEventElapsedTime(&t, g_prof_ev[pairs[i][0]], g_prof_ev[pairs[i][1]]) != cudaSuccess)
+      t = -1.0f;
+    ms[w] = t;
+  }
+  return w;
+}
 
 int kiattn_device_error(int reset) {
   int v = 0;

@@ -29,7 +29,8 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error", 
 
 SYMBOLS = ("kiattn_stats_bytes", "kiattn_workspace_bytes", "kiattn_fwd", "kiattn_bwd",
            "kiattn_weights_from_S", "kiattn_scores", "kiattn_strerror", "kiattn_version",
-           "kiattn_device_error")
+           "kiattn_device_error", "kiattn_profile_enable", "kiattn_profile_read")
+PHASES = ("fwd", "bwd_prep", "bwd_query_pass", "bwd_key_pass", "bwd_calibration")
 
 
 class KiattnError(RuntimeError):
@@ -89,6 +90,10 @@ def _load():
     lib.kiattn_strerror.restype = ctypes.c_char_p
     lib.kiattn_version.restype = i
     lib.kiattn_device_error.argtypes = [i]
+    lib.kiattn_profile_enable.argtypes = [i]
+    lib.kiattn_profile_enable.restype = i
+    lib.kiattn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), i]
+    lib.kiattn_profile_read.restype = i
     for name in ("kiattn_fwd", "kiattn_bwd", "kiattn_weights_from_S", "kiattn_scores",
                  "kiattn_device_error"):
         getattr(lib, name).restype = i
@@ -169,6 +174,18 @@ def kiattn_version() -> int:
 
 def kiattn_device_error(reset: bool = True) -> int:
     return int(_lib.kiattn_device_error(1 if reset else 0))
+
+
+def kiattn_profile_enable(on: bool = True):
+    _check("kiattn_profile_enable", _lib.kiattn_profile_enable(1 if on else 0))
+
+
+def kiattn_profile_read() -> dict:
+    buf = (ctypes.c_float * len(PHASES))()
+    n = _lib.kiattn_profile_read(buf, len(PHASES))
+    if n < 0:
+        raise KiattnError("kiattn_profile_read", n)
+    return {PHASES[i]: float(buf[i]) for i in range(n)}
 
 
 # ------------------------------------------------------------ conveniences
