@@ -122,6 +122,30 @@ int kiattn_bwd(const float* Q, const float* Kt, const float* V, const float* O, 
                const void* stats, float* dQ, float* dK, float* dV, float* dS_dbg, int B, int H,
                int T, int d, const kia_config* cfg, void* workspace, void* stream);
 
+/* Backward for callers that cannot allocate device memory.  Some callers
+ * can't call cudaMalloc: a plugin inside a host engine that owns all device
+ * memory and forbids allocation once it has started, or a latency-bound
+ * loop where an allocation would synchronise the device.  This entry point
+ * takes the same arguments as kiattn_bwd minus the workspace and uses a
+ * scratch array that the library itself declares (no counterpart in the
+ * paper: it only changes where the backward's scratch lives).
+ *   - Capacity: B*H*T <= KIA_NOALLOC_MAX_ROWS rows; larger calls return
+ *     KIA_ERR_CAPACITY and launch nothing.  Every GPU that loads the
+ *     library holds the scratch (about 20 MiB) until the process exits.
+ *   - The first call on a device, with that device current, looks up the
+ *     scratch's device address; make that first call before any stream
+ *     capture.
+ *   - It calls no cudaMalloc / cudaFree.  Each call clears the scratch
+ *     fields that must start at zero; the scratch keeps the last call's
+ *     contents otherwise.
+ *   - All calls share one scratch per device: calls that overlap on the GPU
+ *     (several streams, several host threads) race; serialise them. */
+#define KIA_NOALLOC_MAX_ROWS (1 << 20)
+int kiattn_bwd_noalloc(const float* Q, const float* Kt, const float* V, const float* O,
+                       const float* dO, const void* stats, float* dQ, float* dK, float* dV,
+                       float* dS_dbg, int B, int H, int T, int d, const kia_config* cfg,
+                       void* stream);
+
 /* The fp32 weight stage alone on given scores (section 3, Reconstruction;
  * Appendix A), for bit-exact checking.  S: device fp32 [rows, cols]; row i
  * sees keys 0..row_len[i]-1 (device int32 [rows], 1..cols).  Outputs

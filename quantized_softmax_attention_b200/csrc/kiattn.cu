@@ -6,6 +6,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/kiattn.h"
 #include "kia_common.cuh"
 #include "kia_elem.cuh"
@@ -187,6 +189,16 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
   return rc;
 }
 
+// Scratch of kiattn_bwd_noalloc: the backward's workspace for up to
+// KIA_NOALLOC_MAX_ROWS rows, declared by the library so that the caller
+// allocates nothing.  Host code only ever uses its device address, looked up
+// once per device.
+constexpr size_t kNoallocScratchBytes = 5 * ((size_t)KIA_NOALLOC_MAX_ROWS * 4) + 256;
+static __device__ __align__(256) unsigned char g_kia_noalloc_scratch[kNoallocScratchBytes];
+constexpr int kMaxDevices = 64;
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
 }  // namespace
 
 extern "C" {
@@ -242,6 +254,34 @@ int kiattn_bwd(const float* Q, const float* Kt, const float* V, const float* O, 
                                 workspace, s)
                  : backward<128>(Q, Kt, V, O, dO, stats, dQ, dK, dV, dS_dbg, B, H, T, p,
                                  cfg->gemm, workspace, s);
+}
+
+int kiattn_bwd_noalloc(const float* Q, const float* Kt, const float* V, const float* O,
+                       const float* dO, const void* stats, float* dQ, float* dK, float* dV,
+                       float* dS_dbg, int B, int H, int T, int d, const kia_config* cfg,
+                       void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_shape(B, H, T, d))) return rc;
+  const long long rows = (long long)B * H * T;
+  if (rows > KIA_NOALLOC_MAX_ROWS || work_bytes(rows) > kNoallocScratchBytes)
+    return KIA_ERR_CAPACITY;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KIA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KIA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_kia_noalloc_scratch) != cudaSuccess || !p)
+        return KIA_ERR_CUDA;
+      g_noalloc_addr[dev] = p;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  return kiattn_bwd(Q, Kt, V, O, dO, stats, dQ, dK, dV, dS_dbg, B, H, T, d, cfg, scratch,
+                    stream);
 }
 
 int kiattn_weights_from_S(const float* S, int rows, int cols, const int* row_len,

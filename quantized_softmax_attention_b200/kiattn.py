@@ -29,7 +29,9 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error", 
 
 SYMBOLS = ("kiattn_stats_bytes", "kiattn_workspace_bytes", "kiattn_fwd", "kiattn_bwd",
            "kiattn_weights_from_S", "kiattn_scores", "kiattn_strerror", "kiattn_version",
-           "kiattn_device_error", "kiattn_profile_enable", "kiattn_profile_read")
+           "kiattn_device_error", "kiattn_profile_enable", "kiattn_profile_read",
+           "kiattn_bwd_noalloc")
+NOALLOC_MAX_ROWS = 1 << 20
 PHASES = ("fwd", "bwd_prep", "bwd_query_pass", "bwd_key_pass", "bwd_calibration")
 
 
@@ -84,6 +86,9 @@ def _load():
     lib.kiattn_workspace_bytes.restype = ctypes.c_size_t
     lib.kiattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, cp, vp]
     lib.kiattn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, cp, vp, vp]
+    lib.kiattn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, cp,
+                                       vp]
+    lib.kiattn_bwd_noalloc.restype = i
     lib.kiattn_weights_from_S.argtypes = [vp, i, i, vp, cp, vp, vp, vp, vp, vp, vp]
     lib.kiattn_scores.argtypes = [vp, vp, vp, i, i, i, i, cp, vp]
     lib.kiattn_strerror.argtypes = [i]
@@ -148,6 +153,17 @@ def kiattn_bwd(Q, K, V, O, dO, stats, dQ, dK, dV, workspace, cfg: Config, dS_dbg
     _check("kiattn_bwd", _lib.kiattn_bwd(_p(Q), _p(K), _p(V), _p(O), _p(dO), _p(stats), _p(dQ),
                                          _p(dK), _p(dV), _p(dS_dbg), B, H, T, d,
                                          ctypes.byref(cfg.c()), _p(workspace), _stream(stream)))
+
+
+def kiattn_bwd_noalloc(Q, K, V, O, dO, stats, dQ, dK, dV, cfg: Config, dS_dbg=None,
+                       stream=None):
+    """Backward with the library's own fixed scratch (no workspace argument),
+    for callers that cannot allocate device memory; B*H*T <= NOALLOC_MAX_ROWS."""
+    B, H, T, d = Q.shape
+    _check("kiattn_bwd_noalloc",
+           _lib.kiattn_bwd_noalloc(_p(Q), _p(K), _p(V), _p(O), _p(dO), _p(stats), _p(dQ), _p(dK),
+                                   _p(dV), _p(dS_dbg), B, H, T, d, ctypes.byref(cfg.c()),
+                                   _stream(stream)))
 
 
 def kiattn_weights_from_S(S, row_len, cfg: Config, w, bin=None, t=None, row_m=None, row_n=None,
