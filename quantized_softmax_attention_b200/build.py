@@ -40,7 +40,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         if all(os.path.getmtime(s) <= t for s in _sources()):
             return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--fmad=true", "-shared",
+    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++20", "--fmad=true", "-shared",
            "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-o", tmp, SRC]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")

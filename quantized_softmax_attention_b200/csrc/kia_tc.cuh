@@ -216,5 +216,5 @@ int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO
 
 }  // namespace kia
 
-#include "kia_tc_bwd.cuh"
 #include "kia_tc_fwd.cuh"
+#include "kia_tc_bwd.cuh"

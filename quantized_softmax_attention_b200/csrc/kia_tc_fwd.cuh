@@ -13,19 +13,24 @@
 //            operand of O += P V (and P_L for Prob-STE, O_L += P_L V);
 //   epilogue: O = O_acc / W (and O_L = O_L_acc / W_L), per-row statistics.
 //
-// Warp roles (6 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
-// 2..5 = element warps; element thread r owns TMEM lane r = query row r of
-// the tile (warp w reaches lanes 32*(w%4)..32*(w%4)+31).
+// Warp roles (10 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
+// 2..9 = element warps.  Element warp w reaches TMEM lanes 32*(w%4)..+31
+// (query rows); warps w and w+4 share those rows and split each 128-column
+// tile into halves, so each query row is served by two threads whose row
+// statistics are merged through shared memory.
 #pragma once
+#include "kia_fast.cuh"
 #include "kia_tc.cuh"
 
 namespace kia {
+
+constexpr int kElemThreads = 256;   // 8 element warps
+constexpr int kTcThreads = 320;     // + producer + MMA warp
 
 template <int D>
 struct FwdCfg {
   static constexpr int kStages = (D == 64) ? 2 : 1;      // K and V ring depth
   static constexpr uint32_t kTileBytes = D * KIA_TILE * 4;
-  static constexpr int kThreads = 192;
 };
 
 struct FwdBars {
@@ -33,31 +38,44 @@ struct FwdBars {
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2];    // S tile ready in TMEM buffer b (tcgen05.commit)
-  uint64_t s_free[2];    // sweep 1: element warps done reading buffer b (128 arrivals)
-  uint64_t p_ready[2];   // sweep 2: P written into buffer b (128 arrivals)
+  uint64_t s_free[2];    // sweep 1: element warps done reading buffer b (256 arrivals)
+  uint64_t p_ready[2];   // sweep 2: P written into buffer b (256 arrivals)
   uint64_t pv_done[2];   // sweep 2: P V of buffer b finished (tcgen05.commit)
   uint64_t pl_free;      // P_L consumed by O_L += P_L V (tcgen05.commit)
   uint64_t o_full;       // all P V done
+  uint64_t row_sync;     // element-thread rendezvous (256 arrivals), used 3 times
   uint32_t tmem_base;
   int abort;
 };
 
-template <int D>
-__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
+// Shared-memory scratch of the element warps: per-half row statistics.
+struct FwdRowX {
+  float m[2][KIA_TILE];
+  float n[2][KIA_TILE];
+  int am[2][KIA_TILE];
+  int an[2][KIA_TILE];
+  float W[2][KIA_TILE];
+  float WL[2][KIA_TILE];
+};
+
+template <int D, class V>
+__global__ void __launch_bounds__(kTcThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, StatsView st,
-              OpParams p, int B, int H, int T, int nsb) {
+              OpParams p, int B, int H, int T, int nsb, int tab_in_smem) {
   using Cfg = FwdCfg<D>;
   constexpr int NS = Cfg::kStages;
+  constexpr bool PROB = V::PROB;
   extern __shared__ uint8_t smraw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
   float* sQ = reinterpret_cast<float*>(base);
   float* sK = reinterpret_cast<float*>(base + Cfg::kTileBytes);
   float* sV = reinterpret_cast<float*>(base + (1 + NS) * Cfg::kTileBytes);
-  float* sTab = reinterpret_cast<float*>(base + (1 + 2 * NS) * Cfg::kTileBytes);
-  const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
-  const int tab_floats = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : (p.K + 1));
+  FwdRowX& rx = *reinterpret_cast<FwdRowX*>(base + (1 + 2 * NS) * Cfg::kTileBytes);
+  float* sTab = reinterpret_cast<float*>(&rx + 1);
+  const int tab_floats =
+      V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : (p.K + 1));
   FwdBars& bar = *reinterpret_cast<FwdBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -65,10 +83,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   const int qt = nt - 1 - blockIdx.y;
   const int nkt = p.causal ? qt + 1 : nt;
-  const bool prob = needs_OL(p);
   // TMEM columns: S buffers [0, 128*nsb), P_L, O, O_L
   const uint32_t col_pl = 128u * nsb;
-  const uint32_t col_o = col_pl + (prob ? 128u : 0u);
+  const uint32_t col_o = col_pl + (PROB ? 128u : 0u);
   const uint32_t col_ol = col_o + D;
 
   if (threadIdx.x == 0) {
@@ -79,12 +96,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(&bar.v_full[s], 1);
       mbar_init(&bar.v_empty[s], 1);
       mbar_init(&bar.s_full[s], 1);
-      mbar_init(&bar.s_free[s], 128);
-      mbar_init(&bar.p_ready[s], 128);
+      mbar_init(&bar.s_free[s], kElemThreads);
+      mbar_init(&bar.p_ready[s], kElemThreads);
       mbar_init(&bar.pv_done[s], 1);
     }
     mbar_init(&bar.pl_free, 1);
     mbar_init(&bar.o_full, 1);
+    mbar_init(&bar.row_sync, kElemThreads);
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -142,7 +160,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       int use1[2] = {0, 0};   // sweep-1 uses of each S buffer
       int use2[2] = {0, 0};   // sweep-2 uses of each S buffer
       failed = !mbar_wait(&bar.q_full, 0, abort);
-      // issue S = Q K_j^T into buffer b
+      // issue S = Q K_j^T into buffer j % nsb
       auto issue_s = [&](int sweep, int j) -> bool {
         const int b = j % nsb;
         if (sweep == 0) {
@@ -191,7 +209,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           for (int ks = 0; ks < KIA_TILE / 8; ++ks)
             mma_tf32_ts(tmem + col_o, tmem + 128u * b + 8u * ks, desc_mnmajor(va, ks), idesc_o,
                         (j > 0 || ks > 0) ? 1u : 0u);
-          if (prob) {
+          if constexpr (PROB) {
 #pragma unroll
             for (int ks = 0; ks < KIA_TILE / 8; ++ks)
               mma_tf32_ts(tmem + col_ol, tmem + col_pl + 8u * ks, desc_mnmajor(va, ks), idesc_o,
@@ -209,64 +227,103 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   } else {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
+    const int half = (warp - 2) >> 2;          // which 64 columns of a tile
+    const int r = quad * 32 + lane;            // query row in the tile
     const int qrow = qt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const uint32_t col0 = 64u * half;
+    const long long grow = (long long)bh * T + (qrow < T ? qrow : T - 1);
     int sf[2] = {0, 0};  // completed phases of s_full per buffer
     float m = -INFINITY, n = INFINITY;
     int am = 0, an = 0;
     float v[32];
-    // sweep 1: statistics
+    // sweep 1: statistics of this thread's 64 columns of each tile
     for (int j = 0; j < nkt; ++j) {
       const int b = j % nsb;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
       ++sf[b];
       tc_fence_after();
       const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_addr + 128u * b + 32u * c, v);
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(tmem + lane_addr + 128u * b + col0 + 32u * c, v);
         tmem_ld_wait();
-        const int key0 = j * KIA_TILE + c * 32;
+        const int key0 = j * KIA_TILE + (int)col0 + c * 32;
+        if (!edge) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = key0 + i;
-          const bool ok = !edge || (key < T && (!p.causal || key <= qrow));
-          if (ok) {
-            if (v[i] > m) { m = v[i]; am = key; }
-            if (v[i] < n) { n = v[i]; an = key; }
+          for (int i = 0; i < 32; ++i) {
+            if (v[i] > m) { m = v[i]; am = key0 + i; }
+            if (v[i] < n) { n = v[i]; an = key0 + i; }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = key0 + i;
+            if (key < T && (!p.causal || key <= qrow)) {
+              if (v[i] > m) { m = v[i]; am = key; }
+              if (v[i] < n) { n = v[i]; an = key; }
+            }
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&bar.s_free[b]);
     }
+    // merge the two halves of the row (lowest index on ties)
+    rx.m[half][r] = m;
+    rx.n[half][r] = n;
+    rx.am[half][r] = am;
+    rx.an[half][r] = an;
+    mbar_arrive(&bar.row_sync);
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
+    {
+      const float m0 = rx.m[0][r], m1 = rx.m[1][r], n0 = rx.n[0][r], n1 = rx.n[1][r];
+      const int a0 = rx.am[0][r], a1 = rx.am[1][r], b0 = rx.an[0][r], b1 = rx.an[1][r];
+      m = fmaxf(m0, m1);
+      am = (m0 > m1) ? a0 : (m1 > m0 ? a1 : min(a0, a1));
+      n = fminf(n0, n1);
+      an = (n0 < n1) ? b0 : (n1 < n0 ? b1 : min(b0, b1));
+    }
     // calibration (section 3) and the grid
-    const RowState rs = make_row_state(p, m, n);
-    const int ts = minmax_tab ? KIA_TILE : 1;
-    const float* tab = minmax_tab ? sTab + r : sTab;
-    const long long grow = (long long)bh * T + qrow;
-    if (!p.softmax) {
-      if (minmax_tab) {
-        for (int k = 0; k <= p.K; ++k) {
-          const float G = rs.degen ? 1.0f : grid_value(k, rs.cal.h);
+    const RowCal rc = row_calibration(p, m, n);
+    const bool degen = V::MINMAX && rc.h == 0.0f;
+    const float* tab = sTab;
+    int ts = 1;
+    if constexpr (V::MINMAX) {
+      if (tab_in_smem) {
+        for (int k = half; k <= p.K; k += 2) {
+          const float G = degen ? 1.0f : grid_value(k, rc.h);
           sTab[k * KIA_TILE + r] = G;
           if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
         }
-      } else if (r <= p.K) {
-        const float G = grid_value(r, p.fwm_h);
-        sTab[r] = G;
-        if (bh == 0 && qt == nt - 1) st.table[r] = G;
+        tab = sTab + r;
+        ts = KIA_TILE;
+      } else {
+        for (int k = half; k <= p.K; k += 2) {
+          const float G = degen ? 1.0f : grid_value(k, rc.h);
+          if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
+        }
+        __threadfence_block();
+        tab = st.table + grow * (p.K + 1);
+      }
+    } else if constexpr (!V::SOFTMAX) {
+      const int k = (int)threadIdx.x - 64;
+      if (k >= 0 && k <= p.K) {
+        const float G = grid_value(k, p.fwm_h);
+        sTab[k] = G;
+        if (bh == 0 && qt == nt - 1) st.table[k] = G;
       }
     }
-    named_bar_sync(1, 128);
+    mbar_arrive(&bar.row_sync);
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 1, abort))) failed = true;
+    const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     // sweep 2: weights -> P (and P_L) in TMEM, normalisers
     float W = 0.0f, WL = 0.0f;
     for (int j = 0; j < nkt && !failed; ++j) {
       const int b = j % nsb;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
       ++sf[b];
-      if (prob && j > 0 &&
+      if (PROB && j > 0 &&
           !__all_sync(0xffffffffu, mbar_wait(&bar.pl_free, (j - 1) & 1, abort))) {
         failed = true;
         break;
@@ -274,48 +331,61 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_after();
       const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_addr + 128u * b + 32u * c, v);
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t col = col0 + 32u * c;
+        tmem_ld32(tmem + lane_addr + 128u * b + col, v);
         tmem_ld_wait();
         float vl[32];
-        const int key0 = j * KIA_TILE + c * 32;
+        const int key0 = j * KIA_TILE + (int)col;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int key = key0 + i;
-          const bool ok = !edge || (key < T && (!p.causal || key <= qrow));
-          ElemFwd e = elem_forward(p, rs, tab, ts, v[i]);
-          if (!ok) { e.wf = 0.0f; e.wl = 0.0f; }
-          W += e.wf;
-          WL += e.wl;
-          v[i] = e.wf;
-          vl[i] = e.wl;
+          float wf, wl;
+          fwd_weights<V>(tab, ts, rc.m, rc.rh, Kf, Km1f, v[i], wf, wl);
+          if (edge) {
+            const int key = key0 + i;
+            if (!(key < T && (!p.causal || key <= qrow))) { wf = 0.0f; wl = 0.0f; }
+          }
+          W += wf;
+          v[i] = wf;
+          if constexpr (PROB) {
+            WL += wl;
+            vl[i] = wl;
+          }
         }
-        tmem_st32(tmem + lane_addr + 128u * b + 32u * c, v);
-        if (prob) tmem_st32(tmem + lane_addr + col_pl + 32u * c, vl);
+        tmem_st32(tmem + lane_addr + 128u * b + col, v);
+        if constexpr (PROB) tmem_st32(tmem + lane_addr + col_pl + col, vl);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar.p_ready[b]);
     }
-    // epilogue
+    // normalisers of the whole row
+    rx.W[half][r] = W;
+    rx.WL[half][r] = WL;
+    mbar_arrive(&bar.row_sync);
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
+    W = rx.W[0][r] + rx.W[1][r];
+    WL = PROB ? rx.WL[0][r] + rx.WL[1][r] : W;
+    // epilogue: this thread writes D/2 columns of its row
     if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.o_full, 0, abort))) {
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        tmem_ld32(tmem + lane_addr + col_o + 32u * c, v);
+      for (int c = 0; c < D / 64; ++c) {
+        const uint32_t col = (uint32_t)(half * (D / 2) + 32 * c);
+        tmem_ld32(tmem + lane_addr + col_o + col, v);
         tmem_ld_wait();
         if (qrow < T) {
-          float4* o4 = reinterpret_cast<float4*>(O + grow * D + c * 32);
+          float4* o4 = reinterpret_cast<float4*>(O + grow * D + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             o4[i] = make_float4(__fdiv_rn(v[4 * i], W), __fdiv_rn(v[4 * i + 1], W),
                                 __fdiv_rn(v[4 * i + 2], W), __fdiv_rn(v[4 * i + 3], W));
         }
-        if (prob) {
-          tmem_ld32(tmem + lane_addr + col_ol + 32u * c, v);
+        if constexpr (PROB) {
+          tmem_ld32(tmem + lane_addr + col_ol + col, v);
           tmem_ld_wait();
           if (qrow < T) {
-            float4* o4 = reinterpret_cast<float4*>(st.OL + grow * D + c * 32);
+            float4* o4 = reinterpret_cast<float4*>(st.OL + grow * D + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               o4[i] = make_float4(__fdiv_rn(v[4 * i], WL), __fdiv_rn(v[4 * i + 1], WL),
@@ -323,17 +393,17 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
         }
       }
-      if (qrow < T) {
+      if (qrow < T && half == 0) {
         st.m[grow] = m;
         st.n[grow] = n;
         st.am[grow] = am;
         st.an[grow] = an;
-        st.rh[grow] = rs.degen ? 0.0f : rs.cal.rh;
-        st.h[grow] = rs.degen ? 0.0f : rs.cal.h;
+        st.rh[grow] = degen ? 0.0f : rc.rh;
+        st.h[grow] = degen ? 0.0f : rc.h;
         st.Wf[grow] = W;
-        st.Wb[grow] = (!p.softmax && lerp_normpoint(p)) ? WL : W;
+        st.Wb[grow] = (!V::SOFTMAX && lerp_normpoint(p)) ? WL : W;
       }
-      if (bh == 0 && qt == nt - 1 && r == 0) write_header(st.header, B, H, T, D, p);
+      if (bh == 0 && qt == nt - 1 && threadIdx.x == 64) write_header(st.header, B, H, T, D, p);
     } else {
       failed = true;
     }
@@ -345,12 +415,53 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 }
 
 template <int D>
-size_t tc_fwd_smem(const OpParams& p) {
+size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem) {
   constexpr int NS = FwdCfg<D>::kStages;
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
-  const int tab = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : (p.K + 1));
-  return 1024 + (size_t)(1 + 2 * NS) * FwdCfg<D>::kTileBytes + (size_t)((tab + 31) & ~31) * 4 +
-         sizeof(FwdBars);
+  const int tab =
+      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : (p.K + 1));
+  return 1024 + (size_t)(1 + 2 * NS) * FwdCfg<D>::kTileBytes + sizeof(FwdRowX) +
+         (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
+}
+
+template <int D, class V>
+int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, float* O,
+                 const StatsView& st, int B, int H, int T, const OpParams& p, cudaStream_t s) {
+  bool tab_in_smem = true;
+  size_t smem = tc_fwd_smem<D>(p, true);
+  if (smem > 232448) {
+    tab_in_smem = false;
+    smem = tc_fwd_smem<D>(p, false);
+  }
+  if (smem > 232448) return KIA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(tc_fwd_kernel<D, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return KIA_ERR_CUDA;
+  // TMEM: S buffers (128 columns each), P_L (128, Prob-STE), O and O_L (D each)
+  int nsb = 2;
+  if (256 + (V::PROB ? 128 + 2 * D : D) > 512) nsb = 1;
+  const int nt = (T + KIA_TILE - 1) / KIA_TILE;
+  dim3 grid(B * H, nt);
+  tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, O, st, p, B, H, T, nsb,
+                                                     tab_in_smem ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
+}
+
+// Calls f.template operator()<V>() with the compile-time variant of p.
+template <class F>
+int dispatch_variant(const OpParams& p, F&& f) {
+  if (p.softmax) return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_LERP, false, true>>();
+  const bool prob = p.rec == KIA_REC_NEAREST && p.ste == KIA_STE_PROB;
+  if (p.cal == KIA_CAL_MINMAX) {
+    if (p.rec == KIA_REC_LERP)
+      return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_LERP, false, false>>();
+    if (prob) return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_NEAREST, true, false>>();
+    return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_NEAREST, false, false>>();
+  }
+  if (p.rec == KIA_REC_LERP)
+    return f.template operator()<Var<KIA_CAL_FWM, KIA_REC_LERP, false, false>>();
+  if (prob) return f.template operator()<Var<KIA_CAL_FWM, KIA_REC_NEAREST, true, false>>();
+  return f.template operator()<Var<KIA_CAL_FWM, KIA_REC_NEAREST, false, false>>();
 }
 
 template <int D>
@@ -362,19 +473,9 @@ int tc_forward(const float* Q, const float* Kt, const float* V, float* O, void* 
   if (!make_tmap(&tq, Q, B * H, T, D) || !make_tmap(&tk, Kt, B * H, T, D) ||
       !make_tmap(&tv, V, B * H, T, D, /*mn_major=*/true))
     return KIA_ERR_CUDA;
-  const size_t smem = tc_fwd_smem<D>(p);
-  if (smem > 232448) return KIA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(tc_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return KIA_ERR_CUDA;
-  // TMEM: S buffers (128 columns each), P_L (128, Prob-STE), O and O_L (D each)
-  const bool prob = needs_OL(p);
-  int nsb = 2;
-  if (256 + (prob ? 128 + 2 * D : D) > 512) nsb = 1;
-  const int nt = (T + KIA_TILE - 1) / KIA_TILE;
-  dim3 grid(B * H, nt);
-  tc_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, smem, s>>>(tq, tk, tv, O, st, p, B, H, T, nsb);
-  return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
+  return dispatch_variant(p, [&]<class Vt>() {
+    return tc_forward_v<D, Vt>(tq, tk, tv, O, st, B, H, T, p, s);
+  });
 }
 
 }  // namespace kia
