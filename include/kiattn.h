@@ -131,7 +131,7 @@ int kiattn_bwd(const float* Q, const float* Kt, const float* V, const float* O, 
  * paper: it only changes where the backward's scratch lives).
  *   - Capacity: B*H*T <= KIA_NOALLOC_MAX_ROWS rows; larger calls return
  *     KIA_ERR_CAPACITY and launch nothing.  Every GPU that loads the
- *     library holds the scratch (about 20 MiB) until the process exits.
+ *     library holds the scratch (about 28 MiB) until the process exits.
  *   - The first call on a device, with that device current, looks up the
  *     scratch's device address; make that first call before any stream
  *     capture.

@@ -6,6 +6,7 @@
 //   LERP w = fma(t, G_{k+1} - G_k, G_k),  Nearest w = G_{k + [t >= 1/2]}.
 // floor(u) for 0 <= u <= K-1 is taken as (u + 1.5*2^23 rounded down) -
 // 1.5*2^23, which is exact and yields the integer index from the same bits.
+// Both weights of a row read the pair (G_k, G_{k+1}); Nearest selects from it.
 //
 // Degenerate MinMax rows (span < 1e-12) need no branch: their grid is all
 // ones and rh = 0, so u = 0, w = 1 (uniform P), a_k = 0, and the backward
@@ -29,6 +30,20 @@ struct Var {
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
+// Grid of one row: G_k at p[k * ts] (float table), or the pair
+// (G_k, G_{k+1}) at q[k] (pair table, one 8-byte load).
+struct GridF {
+  const float* p;
+  int ts;
+  __device__ __forceinline__ float2 pair(int k) const {
+    return make_float2(p[k * ts], p[(k + 1) * ts]);
+  }
+};
+struct GridP {
+  const float2* q;
+  __device__ __forceinline__ float2 pair(int k) const { return q[k]; }
+};
+
 struct Pos {
   float u;   // grid coordinate (MinMax: clamped to K)
   float t;   // position inside the interval
@@ -36,13 +51,16 @@ struct Pos {
   int k;     // interval index
 };
 
-template <class V>
+// CLAMP0: the score may exceed the row max by an ulp (recomputed by another
+// contraction order), so clamp u at 0 before taking the interval index.
+template <class V, bool CLAMP0>
 __device__ __forceinline__ Pos grid_pos(float m, float rh, float Kf, float Km1f, float s) {
   Pos p;
   float u = __fmul_rn(__fsub_rn(m, s), rh);
   if constexpr (V::MINMAX) u = fminf(u, Kf);
   p.u = u;
-  const float uc = fminf(fmaxf(u, 0.0f), Km1f);
+  float uc = fminf(u, Km1f);
+  if constexpr (CLAMP0) uc = fmaxf(uc, 0.0f);
   const float tmp = __fadd_rd(uc, kMagic);
   p.kf = __fsub_rn(tmp, kMagic);
   p.k = __float_as_int(tmp) - kMagicBits;
@@ -50,67 +68,137 @@ __device__ __forceinline__ Pos grid_pos(float m, float rh, float Kf, float Km1f,
   return p;
 }
 
-// Forward weights: wf (forward probabilities' numerator) and wl (LERP weight,
-// kept for Prob-STE).  tab[k * ts] = G_k.
-template <class V>
-__device__ __forceinline__ void fwd_weights(const float* tab, int ts, float m, float rh, float Kf,
+// ------------------------------------------------ packed pairs (f32x2)
+// sm_100 issues two fp32 adds / muls / fmas as one instruction; each half is
+// an ordinary IEEE round-to-nearest (or round-down) operation, so results are
+// bit-identical to the scalar sequence.
+__device__ __forceinline__ unsigned long long pk(float2 a) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+__device__ __forceinline__ float2 upk(unsigned long long r) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+  return a;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+__device__ __forceinline__ float2 add2_rd(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)), "l"(pk(c)));
+  return upk(r);
+}
+
+// Forward weights of two neighbouring scores at once (same arithmetic as
+// fwd_weights, paired).  wf2 / wl2 as in fwd_weights.
+template <class V, bool CLAMP0, class G>
+__device__ __forceinline__ void fwd_weights2(const G& grid, float m, float rh, float Kf,
+                                             float Km1f, float s0, float s1, float2& wf2,
+                                             float2& wl2) {
+  if constexpr (V::SOFTMAX) {
+    wf2 = make_float2(__expf(s0 - m), __expf(s1 - m));
+    wl2 = wf2;
+  } else {
+    float2 u = mul2(sub2(make_float2(m, m), make_float2(s0, s1)), make_float2(rh, rh));
+    if constexpr (V::MINMAX) u = make_float2(fminf(u.x, Kf), fminf(u.y, Kf));
+    float2 uc = make_float2(fminf(u.x, Km1f), fminf(u.y, Km1f));
+    if constexpr (CLAMP0) uc = make_float2(fmaxf(uc.x, 0.0f), fmaxf(uc.y, 0.0f));
+    const float2 mg = make_float2(kMagic, kMagic);
+    const float2 tmp = add2_rd(uc, mg);
+    const float2 kf = sub2(tmp, mg);
+    const float2 t = sub2(u, kf);
+    const float2 g0 = grid.pair(__float_as_int(tmp.x) - kMagicBits);
+    const float2 g1 = grid.pair(__float_as_int(tmp.y) - kMagicBits);
+    const float2 lo = make_float2(g0.x, g1.x), hi = make_float2(g0.y, g1.y);
+    const float2 lerp = fma2(t, sub2(hi, lo), lo);
+    if constexpr (V::NEAREST) {
+      wf2 = make_float2(t.x >= 0.5f ? hi.x : lo.x, t.y >= 0.5f ? hi.y : lo.y);
+      wl2 = V::PROB ? lerp : wf2;
+    } else {
+      wf2 = lerp;
+      wl2 = lerp;
+    }
+    if constexpr (V::FWM) {
+      const bool t0 = u.x > Kf, t1 = u.y > Kf;
+      wf2 = make_float2(t0 ? 0.0f : wf2.x, t1 ? 0.0f : wf2.y);
+      wl2 = make_float2(t0 ? 0.0f : wl2.x, t1 ? 0.0f : wl2.y);
+    }
+  }
+}
+
+// Forward weights: wf (forward probabilities' numerator) and wl (LERP
+// weight, used by Prob-STE's normalisation point).  CLAMP0 for tiles that
+// hold masked scores (which may lie above the row max).
+template <class V, bool CLAMP0, class G>
+__device__ __forceinline__ void fwd_weights(const G& grid, float m, float rh, float Kf,
                                             float Km1f, float s, float& wf, float& wl) {
   if constexpr (V::SOFTMAX) {
     wf = __expf(s - m);
     wl = wf;
   } else {
-    const Pos p = grid_pos<V>(m, rh, Kf, Km1f, s);
+    const Pos p = grid_pos<V, CLAMP0>(m, rh, Kf, Km1f, s);
+    const float2 g = grid.pair(p.k);
+    const float lerp = __fmaf_rn(p.t, __fsub_rn(g.y, g.x), g.x);
     if constexpr (V::NEAREST) {
-      const int r = p.k + (p.t >= 0.5f ? 1 : 0);
-      wf = tab[r * ts];
-      if constexpr (V::PROB) {
-        const float g0 = tab[p.k * ts], g1 = tab[(p.k + 1) * ts];
-        wl = __fmaf_rn(p.t, __fsub_rn(g1, g0), g0);
-      } else {
-        wl = wf;
-      }
+      wf = (p.t >= 0.5f) ? g.y : g.x;
+      wl = V::PROB ? lerp : wf;
     } else {
-      const float g0 = tab[p.k * ts], g1 = tab[(p.k + 1) * ts];
-      wf = __fmaf_rn(p.t, __fsub_rn(g1, g0), g0);
-      wl = wf;
+      wf = lerp;
+      wl = lerp;
     }
     if constexpr (V::FWM) {
-      if (p.u > Kf) {
-        wf = 0.0f;
-        wl = 0.0f;
-      }
+      const bool tail = p.u > Kf;
+      wf = tail ? 0.0f : wf;
+      wl = tail ? 0.0f : wl;
     }
   }
 }
 
-// Backward of one element (normalisation Jacobian already applied: dw =
-// (dP - D) / W_bar).  Returns dS; accumulates A += dw a_k and, when NEED_C,
-// C += dw (b - a_k u / h) with b = -(1-t) k G_k - t (k+1) G_{k+1}.
-// nrh = -rh; dg = 1 on degenerate rows, else 0.
-template <class V, bool NEED_C>
-__device__ __forceinline__ float bwd_delta(const float* tab, int ts, float m, float rh, float nrh,
-                                           float dg, float Kf, float Km1f, float s, float dw,
-                                           float& A, float& C) {
+// Backward of one element in the query pass (dw = (dP - D) / W_bar, the
+// normalisation Jacobian at the surrogate's point).  Returns the detached
+// dS; accumulates A += dw a_k and, when NEED_C, C += dw (b - a_k u / h) with
+// b = -(1-t) k G_k - t (k+1) G_{k+1}.  nrh = -rh; dg = 1 on degenerate rows.
+template <class V, bool NEED_C, class G>
+__device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, float nrh, float dg,
+                                           float Kf, float Km1f, float s, float dw, float& A,
+                                           float& C) {
   if constexpr (V::SOFTMAX) {
     return __expf(s - m) * dw;
   } else {
-    const Pos p = grid_pos<V>(m, rh, Kf, Km1f, s);
-    float g0 = tab[p.k * ts], g1 = tab[(p.k + 1) * ts];
+    const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
+    float2 g = grid.pair(p.k);
     if constexpr (V::FWM) {
-      if (p.u > Kf) {
-        g0 = 0.0f;
-        g1 = 0.0f;
-      }
+      const bool tail = p.u > Kf;
+      g.x = tail ? 0.0f : g.x;
+      g.y = tail ? 0.0f : g.y;
     }
-    const float a = __fsub_rn(g1, g0);
-    const float da = dw * a;
+    const float da = dw * __fsub_rn(g.y, g.x);
     A += da;
     float delta;
     if constexpr (V::MINMAX) {
       delta = fmaf(dw, dg, da * nrh);
       if constexpr (NEED_C) {
-        const float kg0 = p.kf * g0;
-        const float bpos = fmaf(p.t, fmaf(p.kf + 1.0f, g1, -kg0), kg0);  // -b
+        const float kg0 = p.kf * g.x;
+        const float bpos = fmaf(p.t, fmaf(p.kf + 1.0f, g.y, -kg0), kg0);  // -b
         C = fmaf(delta, p.u, fmaf(-dw, bpos, C));
       }
     } else {
@@ -120,49 +208,54 @@ __device__ __forceinline__ float bwd_delta(const float* tab, int ts, float m, fl
   }
 }
 
-// The forward probability numerator in the key pass (thread = key row).
-template <class V>
-__device__ __forceinline__ float fwd_weight_only(const float* tab, int ts, float m, float rh,
-                                                 float Kf, float Km1f, float s) {
-  float wf, wl;
-  fwd_weights<V>(tab, ts, m, rh, Kf, Km1f, s, wf, wl);
-  return wf;
-}
-
 // Backward of one element in the key pass: the forward probability P (for
-// dV) and dS (for dK), with the grid position computed once.
-template <class V>
-__device__ __forceinline__ void kv_elem(const float* tab, int ts, float m, float rh, float nrh,
-                                        float dg, float rWf, float Kf, float Km1f, float s,
-                                        float dw, float& P, float& dS) {
+// dV) and the detached dS (for dK), from one grid position.
+template <class V, class G>
+__device__ __forceinline__ void kv_elem(const G& grid, float m, float rh, float dg, float rWf,
+                                        float Kf, float Km1f, float s, float dw, float& P,
+                                        float& dS) {
   if constexpr (V::SOFTMAX) {
     const float w = __expf(s - m);
     P = w * rWf;
     dS = w * dw;
   } else {
-    const Pos p = grid_pos<V>(m, rh, Kf, Km1f, s);
-    float g0 = tab[p.k * ts], g1 = tab[(p.k + 1) * ts];
-    float wf;
-    if constexpr (V::NEAREST) {
-      wf = (p.t >= 0.5f) ? g1 : g0;
-    } else {
-      wf = __fmaf_rn(p.t, __fsub_rn(g1, g0), g0);
-    }
+    const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
+    float2 g = grid.pair(p.k);
+    float wf = V::NEAREST ? ((p.t >= 0.5f) ? g.y : g.x) : __fmaf_rn(p.t, __fsub_rn(g.y, g.x), g.x);
     if constexpr (V::FWM) {
-      if (p.u > Kf) {
-        g0 = 0.0f;
-        g1 = 0.0f;
-        wf = 0.0f;
-      }
+      const bool tail = p.u > Kf;
+      g.x = tail ? 0.0f : g.x;
+      g.y = tail ? 0.0f : g.y;
+      wf = tail ? 0.0f : wf;
     }
     P = wf * rWf;
-    const float da = dw * __fsub_rn(g1, g0);
+    const float da = dw * __fsub_rn(g.y, g.x);
     if constexpr (V::MINMAX) {
-      dS = fmaf(dw, dg, da * nrh);
+      dS = fmaf(dw, dg, -(da * rh));
     } else {
-      dS = da * nrh;
+      dS = -(da * rh);
     }
   }
+}
+
+// Calibration coefficients of one row from its row sums (Appendix B):
+//   MinMax: g_m = A / h + C / K,  g_n = -C / K;   FWM: g_m = A / h, g_n = 0,
+// filtered by the gradient mode; the zero-sum projection instead returns its
+// common-mode shift c = A / (h |J_i|) in gm (gn = 0).  Degenerate and
+// softmax rows have none.
+__device__ __forceinline__ void calibration_coeffs(const OpParams& p, float A, float C, float rh,
+                                                   int L, float& gm, float& gn) {
+  gm = 0.0f;
+  gn = 0.0f;
+  if (p.softmax || rh == 0.0f || p.grad == KIA_GRAD_DETACH) return;
+  if (p.grad == KIA_GRAD_PROJECT) {
+    gm = A * rh / (float)L;
+    return;
+  }
+  const float gm_full = (p.cal == KIA_CAL_MINMAX) ? A * rh + C / p.Kf : A * rh;
+  const float gn_full = (p.cal == KIA_CAL_MINMAX) ? -C / p.Kf : 0.0f;
+  if (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY) gm = gm_full;
+  if (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MIN_ONLY) gn = gn_full;
 }
 
 }  // namespace kia

@@ -219,6 +219,8 @@ simt_bwd_q_kernel(const float* __restrict__ Q, const float* __restrict__ Kt,
   for (int c = 0; c < D; ++c) dq[c] = acc[c];
   wk.A[row] = A;
   wk.C[row] = C;
+  wk.am[row] = st.am[row];
+  wk.an[row] = st.an[row];
 }
 
 // dK / dV side: one thread per key row, queries streamed through shared

@@ -32,6 +32,8 @@ struct WorkView {
   float* C;     // row sum of dw * (b - a_k u / h)
   float* gm;    // calibration coefficient added at the argmax key (or the projection shift)
   float* gn;    // calibration coefficient added at the argmin key
+  int* am;      // argmax key of the row (the calibration target)
+  int* an;      // argmin key of the row
   int* status;  // 0 = stats header matched the call, 1 = mismatch (kernels skip)
 };
 
@@ -83,9 +85,11 @@ __host__ __device__ inline StatsView stats_view(void* base, long long rows, int 
   return v;
 }
 
-__host__ __device__ inline size_t work_bytes(long long rows) {
-  return 5 * align256((size_t)rows * 4) + 256;
+constexpr int kWorkArrays = 7;
+__host__ __device__ constexpr size_t work_bytes_c(long long rows) {
+  return kWorkArrays * (((size_t)rows * 4 + 255) & ~size_t(255)) + 256;
 }
+__host__ __device__ inline size_t work_bytes(long long rows) { return work_bytes_c(rows); }
 
 __host__ __device__ inline WorkView work_view(void* base, long long rows) {
   char* b = static_cast<char*>(base);
@@ -96,7 +100,9 @@ __host__ __device__ inline WorkView work_view(void* base, long long rows) {
   w.C = reinterpret_cast<float*>(b + 2 * r4);
   w.gm = reinterpret_cast<float*>(b + 3 * r4);
   w.gn = reinterpret_cast<float*>(b + 4 * r4);
-  w.status = reinterpret_cast<int*>(b + 5 * r4);
+  w.am = reinterpret_cast<int*>(b + 5 * r4);
+  w.an = reinterpret_cast<int*>(b + 6 * r4);
+  w.status = reinterpret_cast<int*>(b + 7 * r4);
   return w;
 }
 

@@ -209,7 +209,7 @@ template <int D>
 int tc_forward(const float* Q, const float* Kt, const float* V, float* O, void* stats, int B,
                int H, int T, const OpParams& p, cudaStream_t s);
 template <int D>
-int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO,
+int tc_backward(const float* Q, const float* Kt, const float* V, const float* O, const float* dO,
                 const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
                 float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
                 void (*mark)(int, cudaStream_t));

@@ -15,13 +15,17 @@
 // Both passes stream the other side in half tiles of 64 rows through two
 // TMEM buffers, so the MMAs of the next half tile run while the element
 // warps work on the current one.  Each output row is owned by one CTA and
-// written once: no atomics.  The calibration terms (section 3, Calibration
-// gradients; Appendix B) are added afterwards from A and C by the row passes
-// in kia_epilogue.cuh.
-// Warp roles (10 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
-// 2..9 = element warps (warp w reaches TMEM lanes 32*(w%4)..+31; warps w and
-// w+4 split each half tile's 64 columns).
+// written once: no atomics.  The query pass also computes the centering D
+// of its rows and, once its row sums are complete, the calibration terms
+// (section 3, Calibration gradients; Appendix B): g_m at the argmax key and
+// g_n at the argmin key (or the zero-sum projection's shift), added to dQ
+// there and folded into dS^T by the key pass before its dK contraction.
+// Warp roles (18 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
+// 2..17 = element warps (warp w reaches TMEM lanes 32*(w%4)..+31; the four
+// warps sharing those lanes split each half tile's 64 columns).
 #pragma once
+#include <type_traits>
+
 #include "kia_fast.cuh"
 #include "kia_tc.cuh"
 
@@ -34,10 +38,10 @@ struct BwdQBars {
   uint64_t kv_full, kv_empty;     // K_j, V_j K-major (for S, dP)
   uint64_t kmn_full, kmn_empty;   // K_j MN-major (for dQ)
   uint64_t sp_full[2];            // S and dP of a half tile in TMEM buffer b
-  uint64_t elem_done[2];          // dS written into buffer b (256 arrivals)
+  uint64_t elem_done[2];          // dS written into buffer b
   uint64_t st_free[2];            // dQ MMA of buffer b done
   uint64_t dq_full;               // all dQ MMAs done
-  uint64_t row_sync;              // element-thread rendezvous (256 arrivals)
+  uint64_t row_sync;              // element-thread rendezvous
   uint32_t tmem_base;
   int abort;
 };
@@ -47,8 +51,8 @@ struct BwdKBars {
   uint64_t qd_full, qd_empty;     // Q_i, dO_i K-major (for S^T, dP^T)
   uint64_t mn_full, mn_empty;     // Q_i, dO_i MN-major (for dK, dV)
   uint64_t sp_full[2];            // S^T and dP^T of a half tile in TMEM buffer b
-  uint64_t qc_ready;              // per-query constants of a tile loaded (256 arrivals)
-  uint64_t elem_done[2];          // P^T, dS^T written into buffer b (256 arrivals)
+  uint64_t qc_ready;              // per-query constants of a tile loaded
+  uint64_t elem_done[2];          // P^T, dS^T written into buffer b
   uint64_t st_free[2];            // dV, dK MMAs of buffer b done
   uint64_t acc_full;              // all dV, dK MMAs done
   uint32_t tmem_base;
@@ -61,11 +65,22 @@ template <int D, class V, bool NEED_C>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKmn,
-                const __grid_constant__ CUtensorMap tmV, StatsView st, WorkView wk,
-                float* __restrict__ dQ, float* __restrict__ dS_dbg, OpParams p, int T) {
+                const __grid_constant__ CUtensorMap tmV, const float* __restrict__ Kt,
+                const float* __restrict__ O, const float* __restrict__ dO, StatsView st,
+                WorkView wk, float* __restrict__ dQ, float* __restrict__ dS_dbg, OpParams p, int B,
+                int H, int T) {
   static_assert(D == 64, "tensor-core backward tiles are laid out for d = 64");
   constexpr uint32_t kTile = D * KIA_TILE * 4;
-  if (*wk.status != 0) return;
+  // the stats must come from a forward of this shape and configuration
+  __shared__ int s_hdr_ok;
+  if (threadIdx.x == 0) {
+    const bool ok = header_matches(st.header, B, H, T, D, p);
+    s_hdr_ok = ok ? 1 : 0;
+    if (blockIdx.x == 0 && blockIdx.y == 0) *wk.status = ok ? 0 : 1;
+    if (!ok) atomicExch(&g_kia_device_error, KIA_ERR_STATS_MISMATCH);
+  }
+  __syncthreads();
+  if (!s_hdr_ok) return;
   extern __shared__ uint8_t smraw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
@@ -74,9 +89,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   float* sK = reinterpret_cast<float*>(base + 2 * kTile);
   float* sKmn = reinterpret_cast<float*>(base + 3 * kTile);
   float* sV = reinterpret_cast<float*>(base + 4 * kTile);
-  float* sAC = reinterpret_cast<float*>(base + 5 * kTile);   // [2 halves][2][128]
-  float* sTab = sAC + 4 * KIA_TILE;
-  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (p.K + 1) * KIA_TILE : (p.K + 1));
+  float* sAC = reinterpret_cast<float*>(base + 5 * kTile);   // [kRowSplit][2][128]
+  float* sTab = sAC + 2 * kRowSplit * KIA_TILE;
+  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (p.K + 1) * KIA_TILE : 2 * (p.K + 1));
   BwdQBars& bar = *reinterpret_cast<BwdQBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,7 +201,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;       // which 16 columns of a half tile
     const int r = quad * 32 + lane;
     const int q = qt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
@@ -194,80 +209,150 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const long long qr = rowbase + (q < T ? q : T - 1);
     // this row's calibration and centering (written by the forward and prep)
     const float m = st.m[qr];
+    const float n = st.n[qr];
+    const int am = st.am[qr], an = V::MINMAX ? st.an[qr] : am;
     const float rh = st.rh[qr];
     const float nrh = -rh;
     const float dg = (V::MINMAX && rh == 0.0f) ? 1.0f : 0.0f;
     const int L = p.causal ? q + 1 : T;
     // a one-key row has P = 1 whatever its score: zero gradient
     const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]);
-    const float Dc = wk.D[qr];
+    // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE)
+    float Dc = 0.0f;
+    {
+      const float4* g4 = reinterpret_cast<const float4*>(dO + qr * D);
+      const float4* o4 = reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qr * D);
+#pragma unroll 4
+      for (int c = 0; c < D / 4; ++c) {
+        const float4 a = g4[c], b4 = o4[c];
+        Dc = fmaf(a.x, b4.x, Dc);
+        Dc = fmaf(a.y, b4.y, Dc);
+        Dc = fmaf(a.z, b4.z, Dc);
+        Dc = fmaf(a.w, b4.w, Dc);
+      }
+      if (part == 0 && q < T) wk.D[qr] = Dc;
+    }
+
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
-    const float* tab = sTab;
-    int ts = 1;
+    float2* sPair = reinterpret_cast<float2*>(sTab);
     if constexpr (V::MINMAX) {
-      for (int k = half; k <= p.K; k += 2) sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
-      tab = sTab + r;
-      ts = KIA_TILE;
+      for (int k = part; k <= p.K; k += kRowSplit) sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
     } else if constexpr (!V::SOFTMAX) {
       const int k = (int)threadIdx.x - 64;
-      if (k >= 0 && k <= p.K) sTab[k] = st.table[k];
+      if (k >= 0 && k < p.K) sPair[k] = make_float2(st.table[k], st.table[k + 1]);
     }
+    using Grid = std::conditional_t<V::MINMAX, GridF, GridP>;
+    Grid grid;
+    if constexpr (V::MINMAX) grid = GridF{sTab + r, KIA_TILE};
+    else grid = GridP{sPair};
     mbar_arrive(&bar.row_sync);
     if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
     float A = 0.0f, C = 0.0f;
-    float v[32], g[32];
+    float v[16], g[16];
     for (int u = 0; u < nunits && !failed; ++u) {
       const int b = u & 1, j = u >> 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[b], (u >> 1) & 1, abort))) { failed = true; break; }
       tc_fence_after();
-      const uint32_t cs = 128u * b + 32u * half;       // this thread's 32 columns of S
-      tmem_ld32(tmem + lane_addr + cs, v);
-      tmem_ld32(tmem + lane_addr + cs + 64u, g);
+      const uint32_t cs = 128u * b + 16u * part;       // this thread's 16 columns of S
+      tmem_ld16(tmem + lane_addr + cs, v);
+      tmem_ld16(tmem + lane_addr + cs + 64u, g);
       tmem_ld_wait();
-      const int key0 = j * KIA_TILE + 64 * b + 32 * half;
+      const int key0 = j * KIA_TILE + 64 * b + 16 * part;
       const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
+      if (!edge) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float dw = (g[i] - Dc) * rWb;
-        if (edge) {
-          const int key = key0 + i;
-          if (!(key < T && (!p.causal || key <= q))) dw = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+          const float dw = (g[i] - Dc) * rWb;
+          v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
         }
-        v[i] = bwd_delta<V, NEED_C>(tab, ts, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int key = key0 + i;
+          const bool ok = key < T && (!p.causal || key <= q);
+          const float dw = ok ? (g[i] - Dc) * rWb : 0.0f;
+          v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+        }
       }
-      tmem_st32(tmem + lane_addr + cs, v);
+      tmem_st16(tmem + lane_addr + cs, v);
       if (dS_dbg && q < T) {
         float* dst = dS_dbg + (rowbase + q) * T + key0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 16; ++i)
           if (key0 + i < T) dst[i] = v[i];
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar.elem_done[b]);
     }
-    // row sums of both halves
-    sAC[(half * 2 + 0) * KIA_TILE + r] = A;
-    sAC[(half * 2 + 1) * KIA_TILE + r] = C;
+    // row sums of the four column groups
+    sAC[(part * 2 + 0) * KIA_TILE + r] = A;
+    sAC[(part * 2 + 1) * KIA_TILE + r] = C;
     mbar_arrive(&bar.row_sync);
     if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 1, abort))) failed = true;
     if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.dq_full, 0, abort))) {
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        const uint32_t col = (uint32_t)(half * (D / 2) + 32 * c);
-        tmem_ld32(tmem + lane_addr + kColDQ + col, v);
+      // calibration terms of this row (section 3, Calibration gradients;
+      // Appendix B): dS gains g_m at the argmax key and g_n at the argmin key
+      const float Arow = (sAC[0 * KIA_TILE + r] + sAC[2 * KIA_TILE + r]) +
+                         (sAC[4 * KIA_TILE + r] + sAC[6 * KIA_TILE + r]);
+      const float Crow = (sAC[1 * KIA_TILE + r] + sAC[3 * KIA_TILE + r]) +
+                         (sAC[5 * KIA_TILE + r] + sAC[7 * KIA_TILE + r]);
+      float gm, gn;
+      calibration_coeffs(p, Arow, Crow, rh, L, gm, gn);
+      const bool proj = p.grad == KIA_GRAD_PROJECT;
+      const float gmq = proj ? 0.0f : gm;   // the projection shift is applied by the scan pass
+      const float* ka = Kt + (rowbase + am) * D;
+      const float* kn = Kt + (rowbase + an) * D;
+      {
+        constexpr int kCols = D / kRowSplit;   // 16
+        const uint32_t col = (uint32_t)(part * kCols);
+        float o[kCols];
+        tmem_ld16(tmem + lane_addr + kColDQ + col, o);
         tmem_ld_wait();
         if (q < T) {
+          if (gmq != 0.0f) {
+            const float4* k4 = reinterpret_cast<const float4*>(ka + col);
+#pragma unroll
+            for (int i = 0; i < kCols / 4; ++i) {
+              const float4 kk = k4[i];
+              o[4 * i] = fmaf(gmq, kk.x, o[4 * i]);
+              o[4 * i + 1] = fmaf(gmq, kk.y, o[4 * i + 1]);
+              o[4 * i + 2] = fmaf(gmq, kk.z, o[4 * i + 2]);
+              o[4 * i + 3] = fmaf(gmq, kk.w, o[4 * i + 3]);
+            }
+          }
+          if (V::MINMAX && gn != 0.0f) {
+            const float4* k4 = reinterpret_cast<const float4*>(kn + col);
+#pragma unroll
+            for (int i = 0; i < kCols / 4; ++i) {
+              const float4 kk = k4[i];
+              o[4 * i] = fmaf(gn, kk.x, o[4 * i]);
+              o[4 * i + 1] = fmaf(gn, kk.y, o[4 * i + 1]);
+              o[4 * i + 2] = fmaf(gn, kk.z, o[4 * i + 2]);
+              o[4 * i + 3] = fmaf(gn, kk.w, o[4 * i + 3]);
+            }
+          }
           float4* o4 = reinterpret_cast<float4*>(dQ + (rowbase + q) * D + col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < kCols / 4; ++i)
+            o4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
       }
-      if (q < T && half == 0) {
-        wk.A[rowbase + q] = sAC[0 * KIA_TILE + r] + sAC[2 * KIA_TILE + r];
-        wk.C[rowbase + q] = sAC[1 * KIA_TILE + r] + sAC[3 * KIA_TILE + r];
+      if (q < T && part == 0) {
+        wk.gm[rowbase + q] = gm;
+        wk.gn[rowbase + q] = gn;
+        wk.am[rowbase + q] = am;
+        wk.an[rowbase + q] = an;
+        if (dS_dbg) {
+          float* ds = dS_dbg + (rowbase + q) * T;
+          if (proj) {
+            for (int jj = 0; jj < L; ++jj) ds[jj] += gm;
+          } else {
+            ds[am] += gm;
+            ds[an] += gn;
+          }
+        }
       }
     } else {
       failed = true;
@@ -281,7 +366,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
 // ------------------------------------------------------------------ key pass
 
-template <int D, class V>
+template <int D, class V, bool PROJ>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQmn,
                  const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmGmn,
@@ -300,11 +385,12 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float* sG = reinterpret_cast<float*>(base + 3 * kTile);
   float* sQmn = reinterpret_cast<float*>(base + 4 * kTile);
   float* sGmn = reinterpret_cast<float*>(base + 5 * kTile);
-  float4* sC4 = reinterpret_cast<float4*>(base + 6 * kTile);       // (m, rh, D, rWb) per query
-  float2* sC2 = reinterpret_cast<float2*>(sC4 + KIA_TILE);         // (rWf, dg) per query
-  float* sTab = reinterpret_cast<float*>(sC2 + KIA_TILE);
+  float4* sC4 = reinterpret_cast<float4*>(base + 6 * kTile);  // (m, rh, D, rWb) per query
+  float4* sCA = sC4 + KIA_TILE;                               // (rWf, dg, g_m or c, g_n)
+  int2* sCI = reinterpret_cast<int2*>(sCA + KIA_TILE);         // argmax, argmin keys - tile start
+  float* sTab = reinterpret_cast<float*>(sCI + KIA_TILE);
   const int K1 = p.K + 1;
-  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? K1 * KIA_TILE : 0) : K1);
+  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? K1 * KIA_TILE : 0) : 2 * K1);
   BwdKBars& bar = *reinterpret_cast<BwdKBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -423,15 +509,16 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;        // which 16 query columns of a half tile
     const int r = quad * 32 + lane;
-    const int e = (int)threadIdx.x - 64;          // 0..255
+    const int e = (int)threadIdx.x - 64;     // 0..kElemThreads-1
     const int kj = kt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const long long rowbase = (long long)bh * T;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
-    if (!V::SOFTMAX && !V::MINMAX && e < K1) sTab[e] = st.table[e];
-    float v[32], g[32];
+    if (!V::SOFTMAX && !V::MINMAX && e < p.K)
+      reinterpret_cast<float2*>(sTab)[e] = make_float2(st.table[e], st.table[e + 1]);
+    float v[16], g[16];
     for (int u = 0; u < nunits && !failed; ++u) {
       const int b = u & 1, s = u >> 1;
       const int qi = q0 + s;
@@ -450,8 +537,14 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           const int Lq = p.causal ? q + 1 : T;
           sC4[e] = make_float4(st.m[qr], rhq, wk.D[qr],
                                Lq == 1 ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]));
-          sC2[e] = make_float2(__fdiv_rn(1.0f, st.Wf[qr]),
-                               (V::MINMAX && rhq == 0.0f) ? 1.0f : 0.0f);
+          // calibration terms of the query's row, added to dS^T before dK:
+          // g_m at the argmax key, g_n at the argmin key, or the projection
+          // shift c on every visible key
+          const bool live = q < T;
+          sCA[e] = make_float4(__fdiv_rn(1.0f, st.Wf[qr]), (V::MINMAX && rhq == 0.0f) ? 1.0f : 0.0f,
+                               live ? wk.gm[qr] : 0.0f, live ? wk.gn[qr] : 0.0f);
+          sCI[e] = make_int2(PROJ ? -1 : wk.am[qr] - kt * KIA_TILE,
+                             PROJ ? -1 : wk.an[qr] - kt * KIA_TILE);
           if (V::MINMAX && tab_in_smem)
             for (int k = 0; k < K1; ++k) sTab[e * K1 + k] = st.table[qr * K1 + k];
         }
@@ -460,29 +553,36 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[b], (u >> 1) & 1, abort))) { failed = true; break; }
       tc_fence_after();
-      const uint32_t cs = 128u * b + 32u * half;
-      tmem_ld32(tmem + lane_addr + cs, v);
-      tmem_ld32(tmem + lane_addr + cs + 64u, g);
+      const uint32_t cs = 128u * b + 16u * part;
+      tmem_ld16(tmem + lane_addr + cs, v);
+      tmem_ld16(tmem + lane_addr + cs + 64u, g);
       tmem_ld_wait();
-      const int ql0 = 64 * b + 32 * half;              // first query (in the tile) of the chunk
+      const int ql0 = 64 * b + 16 * part;              // first query (in the tile) of the chunk
       const bool edge =
           (p.causal && qi == kt) || (qi + 1) * KIA_TILE > T || (kt + 1) * KIA_TILE > T;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const int ql = ql0 + i;
         const float4 c4 = sC4[ql];
-        const float2 c2 = sC2[ql];
-        const float* tab;
-        int ts = 1;
-        if constexpr (V::MINMAX) {
-          tab = tab_in_smem ? sTab + ql * K1
-                            : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1;
-        } else {
-          tab = sTab;
-        }
-        float dw = (g[i] - c4.z) * c4.w;
+        const float4 ca = sCA[ql];
+        const float dw = (g[i] - c4.z) * c4.w;
         float P, dS;
-        kv_elem<V>(tab, ts, c4.x, c4.y, -c4.y, c2.y, c2.x, Kf, Km1f, v[i], dw, P, dS);
+        if constexpr (V::MINMAX) {
+          const GridF grid{tab_in_smem ? sTab + ql * K1
+                                       : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
+                           1};
+          kv_elem<V>(grid, c4.x, c4.y, ca.y, ca.x, Kf, Km1f, v[i], dw, P, dS);
+        } else {
+          kv_elem<V>(GridP{reinterpret_cast<const float2*>(sTab)}, c4.x, c4.y, ca.y, ca.x, Kf,
+                     Km1f, v[i], dw, P, dS);
+        }
+        if constexpr (PROJ) {
+          dS += ca.z;
+        } else if constexpr (!V::SOFTMAX) {
+          const int2 ci = sCI[ql];
+          dS += (ci.x == r) ? ca.z : 0.0f;
+          if constexpr (V::MINMAX) dS += (ci.y == r) ? ca.w : 0.0f;
+        }
         if (edge) {
           const int q = qi * KIA_TILE + ql;
           if (!(kj < T && q < T && (!p.causal || kj <= q))) {
@@ -493,28 +593,26 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         v[i] = P;
         g[i] = dS;
       }
-      tmem_st32(tmem + lane_addr + cs, v);
-      tmem_st32(tmem + lane_addr + cs + 64u, g);
+      tmem_st16(tmem + lane_addr + cs, v);
+      tmem_st16(tmem + lane_addr + cs + 64u, g);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar.elem_done[b]);
     }
     if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.acc_full, 0, abort))) {
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        const uint32_t col = (uint32_t)(half * (D / 2) + 32 * c);
-        tmem_ld32(tmem + lane_addr + kColDV + col, v);
-        tmem_ld32(tmem + lane_addr + kColDK + col, g);
-        tmem_ld_wait();
-        if (kj < T) {
-          float4* dv4 = reinterpret_cast<float4*>(dV + (rowbase + kj) * D + col);
-          float4* dk4 = reinterpret_cast<float4*>(dK + (rowbase + kj) * D + col);
+      constexpr int kCols = D / kRowSplit;   // 16
+      const uint32_t col = (uint32_t)(part * kCols);
+      tmem_ld16(tmem + lane_addr + kColDV + col, v);
+      tmem_ld16(tmem + lane_addr + kColDK + col, g);
+      tmem_ld_wait();
+      if (kj < T) {
+        float4* dv4 = reinterpret_cast<float4*>(dV + (rowbase + kj) * D + col);
+        float4* dk4 = reinterpret_cast<float4*>(dK + (rowbase + kj) * D + col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            dv4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            dk4[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
-          }
+        for (int i = 0; i < kCols / 4; ++i) {
+          dv4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          dk4[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
         }
       }
     } else {
@@ -530,24 +628,24 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 template <int D>
 size_t tc_bwd_q_smem(const OpParams& p) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
-  const int tab = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : (p.K + 1));
-  return 1024 + 5 * (size_t)D * KIA_TILE * 4 + 4 * KIA_TILE * 4 + (size_t)((tab + 31) & ~31) * 4 +
-         sizeof(BwdQBars);
+  const int tab = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : 2 * (p.K + 1));
+  return 1024 + 5 * (size_t)D * KIA_TILE * 4 + 2 * kRowSplit * KIA_TILE * 4 +
+         (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdQBars);
 }
 
 template <int D>
 size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
-      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : (p.K + 1));
-  return 1024 + 6 * (size_t)D * KIA_TILE * 4 + KIA_TILE * (16 + 8) +
+      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
+  return 1024 + 6 * (size_t)D * KIA_TILE * 4 + KIA_TILE * (16 + 16 + 8) +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdKBars);
 }
 
 template <int D, class V>
-int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float* dO,
-                  const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
-                  float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
+int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float* O,
+                  const float* dO, const StatsView& st, const WorkView& wk, float* dQ, float* dK,
+                  float* dV, float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
                   void (*mark)(int, cudaStream_t)) {
   const int BH = B * H;
   CUtensorMap tq, tqm, tg, tgm, tk, tkm, tv;
@@ -568,28 +666,34 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
-    tc_bwd_q_kernel<D, V, true><<<grid, kTcThreads, smq, s>>>(tq, tg, tk, tkm, tv, st, wk, dQ,
-                                                              dS_dbg, p, T);
+    tc_bwd_q_kernel<D, V, true><<<grid, kTcThreads, smq, s>>>(tq, tg, tk, tkm, tv, Kt, O, dO, st,
+                                                              wk, dQ, dS_dbg, p, B, H, T);
   } else {
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
-    tc_bwd_q_kernel<D, V, false><<<grid, kTcThreads, smq, s>>>(tq, tg, tk, tkm, tv, st, wk, dQ,
-                                                               dS_dbg, p, T);
+    tc_bwd_q_kernel<D, V, false><<<grid, kTcThreads, smq, s>>>(tq, tg, tk, tkm, tv, Kt, O, dO,
+                                                               st, wk, dQ, dS_dbg, p, B, H, T);
   }
   if (cudaGetLastError() != cudaSuccess) return KIA_ERR_CUDA;
   mark(4, s);
-  if (cudaFuncSetAttribute(tc_bwd_kv_kernel<D, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smk) != cudaSuccess)
+  auto launch_kv = [&](auto kern) -> int {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk) !=
+        cudaSuccess)
+      return KIA_ERR_CUDA;
+    kern<<<grid, kTcThreads, smk, s>>>(tq, tqm, tg, tgm, tk, tv, st, wk, dK, dV, p, T,
+                                       kv_tab_smem ? 1 : 0);
+    return KIA_OK;
+  };
+  const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;
+  if ((proj ? launch_kv(tc_bwd_kv_kernel<D, V, true>) : launch_kv(tc_bwd_kv_kernel<D, V, false>)))
     return KIA_ERR_CUDA;
-  tc_bwd_kv_kernel<D, V><<<grid, kTcThreads, smk, s>>>(tq, tqm, tg, tgm, tk, tv, st, wk, dK, dV, p,
-                                                       T, kv_tab_smem ? 1 : 0);
   mark(5, s);
   return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
 }
 
 template <int D>
-int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO,
+int tc_backward(const float* Q, const float* Kt, const float* V, const float* O, const float* dO,
                 const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
                 float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
                 void (*mark)(int, cudaStream_t)) {
@@ -597,7 +701,8 @@ int tc_backward(const float* Q, const float* Kt, const float* V, const float* dO
     return KIA_ERR_UNSUPPORTED;
   } else {
     return dispatch_variant(p, [&]<class Vt>() {
-      return tc_backward_v<D, Vt>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s, mark);
+      return tc_backward_v<D, Vt>(Q, Kt, V, O, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s,
+                                  mark);
     });
   }
 }

@@ -13,19 +13,20 @@
 //            operand of O += P V (and P_L for Prob-STE, O_L += P_L V);
 //   epilogue: O = O_acc / W (and O_L = O_L_acc / W_L), per-row statistics.
 //
-// Warp roles (10 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
-// 2..9 = element warps.  Element warp w reaches TMEM lanes 32*(w%4)..+31
-// (query rows); warps w and w+4 share those rows and split each 128-column
-// tile into halves, so each query row is served by two threads whose row
-// statistics are merged through shared memory.
+// Warp roles (18 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
+// 2..17 = element warps.  Element warp w reaches TMEM lanes 32*(w%4)..+31
+// (query rows); the four warps that share those rows split each 128-column
+// tile into 32-column groups, so each query row is served by four threads
+// whose row statistics are merged through shared memory.
 #pragma once
 #include "kia_fast.cuh"
 #include "kia_tc.cuh"
 
 namespace kia {
 
-constexpr int kElemThreads = 256;   // 8 element warps
-constexpr int kTcThreads = 320;     // + producer + MMA warp
+constexpr int kRowSplit = 4;        // element threads per TMEM lane (row)
+constexpr int kElemThreads = 128 * kRowSplit;   // 16 element warps
+constexpr int kTcThreads = kElemThreads + 64;   // + producer + MMA warp
 
 template <int D>
 struct FwdCfg {
@@ -38,24 +39,24 @@ struct FwdBars {
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2];    // S tile ready in TMEM buffer b (tcgen05.commit)
-  uint64_t s_free[2];    // sweep 1: element warps done reading buffer b (256 arrivals)
-  uint64_t p_ready[2];   // sweep 2: P written into buffer b (256 arrivals)
+  uint64_t s_free[2];    // sweep 1: element warps done reading buffer b
+  uint64_t p_ready[2];   // sweep 2: P written into buffer b
   uint64_t pv_done[2];   // sweep 2: P V of buffer b finished (tcgen05.commit)
   uint64_t pl_free;      // P_L consumed by O_L += P_L V (tcgen05.commit)
   uint64_t o_full;       // all P V done
-  uint64_t row_sync;     // element-thread rendezvous (256 arrivals), used 3 times
+  uint64_t row_sync;     // element-thread rendezvous, used 3 times
   uint32_t tmem_base;
   int abort;
 };
 
-// Shared-memory scratch of the element warps: per-half row statistics.
+// Shared-memory scratch of the element warps: per-column-group row statistics.
 struct FwdRowX {
-  float m[2][KIA_TILE];
-  float n[2][KIA_TILE];
-  int am[2][KIA_TILE];
-  int an[2][KIA_TILE];
-  float W[2][KIA_TILE];
-  float WL[2][KIA_TILE];
+  float m[kRowSplit][KIA_TILE];
+  float n[kRowSplit][KIA_TILE];
+  int am[kRowSplit][KIA_TILE];
+  int an[kRowSplit][KIA_TILE];
+  float W[kRowSplit][KIA_TILE];
+  float WL[kRowSplit][KIA_TILE];
 };
 
 template <int D, class V>
@@ -75,7 +76,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   FwdRowX& rx = *reinterpret_cast<FwdRowX*>(base + (1 + 2 * NS) * Cfg::kTileBytes);
   float* sTab = reinterpret_cast<float*>(&rx + 1);
   const int tab_floats =
-      V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : (p.K + 1));
+      V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   FwdBars& bar = *reinterpret_cast<FwdBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -227,91 +228,108 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   } else {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;          // which 64 columns of a tile
+    const int part = (warp - 2) >> 2;          // which 32 columns of a tile
     const int r = quad * 32 + lane;            // query row in the tile
     const int qrow = qt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const uint32_t col0 = 64u * half;
+    const uint32_t col0 = 32u * part;
     const long long grow = (long long)bh * T + (qrow < T ? qrow : T - 1);
     int sf[2] = {0, 0};  // completed phases of s_full per buffer
+    // row extrema and the keys of their first occurrences
     float m = -INFINITY, n = INFINITY;
     int am = 0, an = 0;
     float v[32];
-    // sweep 1: statistics of this thread's 64 columns of each tile
+    // sweep 1: statistics of this thread's 32 columns of each tile
     for (int j = 0; j < nkt; ++j) {
       const int b = j % nsb;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
       ++sf[b];
       tc_fence_after();
       const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(tmem + lane_addr + 128u * b + col0 + 32u * c, v);
-        tmem_ld_wait();
-        const int key0 = j * KIA_TILE + (int)col0 + c * 32;
-        if (!edge) {
+      tmem_ld32(tmem + lane_addr + 128u * b + col0, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bar.s_free[b]);
+      const int key0 = j * KIA_TILE + (int)col0;
+      if (!edge) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (v[i] > m) { m = v[i]; am = key0 + i; }
-            if (v[i] < n) { n = v[i]; an = key0 + i; }
+        for (int i = 0; i < 32; ++i) {
+          // strict comparisons keep the lowest index on ties
+          if (v[i] > m) am = key0 + i;
+          m = fmaxf(m, v[i]);
+          if constexpr (V::MINMAX) {
+            if (v[i] < n) an = key0 + i;
+            n = fminf(n, v[i]);
           }
-        } else {
+        }
+      } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int key = key0 + i;
-            if (key < T && (!p.causal || key <= qrow)) {
-              if (v[i] > m) { m = v[i]; am = key; }
-              if (v[i] < n) { n = v[i]; an = key; }
-            }
+        for (int i = 0; i < 32; ++i) {
+          const int key = key0 + i;
+          const bool ok = key < T && (!p.causal || key <= qrow);
+          const float vx = ok ? v[i] : -INFINITY;
+          if (vx > m) am = key;
+          m = fmaxf(m, vx);
+          if constexpr (V::MINMAX) {
+            const float vn = ok ? v[i] : INFINITY;
+            if (vn < n) an = key;
+            n = fminf(n, vn);
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bar.s_free[b]);
     }
-    // merge the two halves of the row (lowest index on ties)
-    rx.m[half][r] = m;
-    rx.n[half][r] = n;
-    rx.am[half][r] = am;
-    rx.an[half][r] = an;
+    // merge the four column groups of the row (lowest index on ties)
+    rx.m[part][r] = m;
+    rx.n[part][r] = n;
+    rx.am[part][r] = am;
+    rx.an[part][r] = an;
     mbar_arrive(&bar.row_sync);
     if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
-    {
-      const float m0 = rx.m[0][r], m1 = rx.m[1][r], n0 = rx.n[0][r], n1 = rx.n[1][r];
-      const int a0 = rx.am[0][r], a1 = rx.am[1][r], b0 = rx.an[0][r], b1 = rx.an[1][r];
-      m = fmaxf(m0, m1);
-      am = (m0 > m1) ? a0 : (m1 > m0 ? a1 : min(a0, a1));
-      n = fminf(n0, n1);
-      an = (n0 < n1) ? b0 : (n1 < n0 ? b1 : min(b0, b1));
+    m = rx.m[0][r];
+    am = rx.am[0][r];
+    n = rx.n[0][r];
+    an = rx.an[0][r];
+#pragma unroll
+    for (int h = 1; h < kRowSplit; ++h) {
+      const float mh = rx.m[h][r], nh = rx.n[h][r];
+      const int ah = rx.am[h][r], bh2 = rx.an[h][r];
+      am = (mh > m) ? ah : (mh == m ? min(am, ah) : am);
+      m = fmaxf(m, mh);
+      an = (nh < n) ? bh2 : (nh == n ? min(an, bh2) : an);
+      n = fminf(n, nh);
+    }
+    if constexpr (!V::MINMAX) {
+      n = m;   // FWM and softmax do not use the row minimum
+      an = am;
     }
     // calibration (section 3) and the grid
     const RowCal rc = row_calibration(p, m, n);
     const bool degen = V::MINMAX && rc.h == 0.0f;
-    const float* tab = sTab;
-    int ts = 1;
+    float2* sPair = reinterpret_cast<float2*>(sTab);
     if constexpr (V::MINMAX) {
       if (tab_in_smem) {
-        for (int k = half; k <= p.K; k += 2) {
+        for (int k = part; k <= p.K; k += kRowSplit) {
           const float G = degen ? 1.0f : grid_value(k, rc.h);
           sTab[k * KIA_TILE + r] = G;
           if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
         }
-        tab = sTab + r;
-        ts = KIA_TILE;
       } else {
-        for (int k = half; k <= p.K; k += 2) {
+        for (int k = part; k <= p.K; k += kRowSplit) {
           const float G = degen ? 1.0f : grid_value(k, rc.h);
           if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
         }
         __threadfence_block();
-        tab = st.table + grow * (p.K + 1);
       }
     } else if constexpr (!V::SOFTMAX) {
+      // one grid for every row: pairs (G_k, G_{k+1}), k = 0..K-1
       const int k = (int)threadIdx.x - 64;
-      if (k >= 0 && k <= p.K) {
-        const float G = grid_value(k, p.fwm_h);
-        sTab[k] = G;
-        if (bh == 0 && qt == nt - 1) st.table[k] = G;
+      if (k >= 0 && k < p.K) {
+        const float G0 = grid_value(k, p.fwm_h), G1 = grid_value(k + 1, p.fwm_h);
+        sPair[k] = make_float2(G0, G1);
+        if (bh == 0 && qt == nt - 1) {
+          st.table[k] = G0;
+          if (k == p.K - 1) st.table[k + 1] = G1;
+        }
       }
     }
     mbar_arrive(&bar.row_sync);
@@ -319,89 +337,105 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     // sweep 2: weights -> P (and P_L) in TMEM, normalisers
     float W = 0.0f, WL = 0.0f;
-    for (int j = 0; j < nkt && !failed; ++j) {
-      const int b = j % nsb;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
-      ++sf[b];
-      if (PROB && j > 0 &&
-          !__all_sync(0xffffffffu, mbar_wait(&bar.pl_free, (j - 1) & 1, abort))) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-      const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        const uint32_t col = col0 + 32u * c;
-        tmem_ld32(tmem + lane_addr + 128u * b + col, v);
-        tmem_ld_wait();
-        float vl[32];
-        const int key0 = j * KIA_TILE + (int)col;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float wf, wl;
-          fwd_weights<V>(tab, ts, rc.m, rc.rh, Kf, Km1f, v[i], wf, wl);
-          if (edge) {
-            const int key = key0 + i;
-            if (!(key < T && (!p.causal || key <= qrow))) { wf = 0.0f; wl = 0.0f; }
-          }
-          W += wf;
-          v[i] = wf;
-          if constexpr (PROB) {
-            WL += wl;
-            vl[i] = wl;
-          }
+    auto sweep2 = [&](auto grid) {
+      for (int j = 0; j < nkt && !failed; ++j) {
+        const int b = j % nsb;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
+        ++sf[b];
+        if (PROB && j > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(&bar.pl_free, (j - 1) & 1, abort))) {
+          failed = true;
+          break;
         }
-        tmem_st32(tmem + lane_addr + 128u * b + col, v);
-        if constexpr (PROB) tmem_st32(tmem + lane_addr + col_pl + col, vl);
+        tc_fence_after();
+        const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t col = col0 + 16u * c;
+          float w16[16], vl[16];
+          tmem_ld16(tmem + lane_addr + 128u * b + col, w16);
+          tmem_ld_wait();
+          const int key0 = j * KIA_TILE + (int)col;
+          if (!edge) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float wf, wl;
+              fwd_weights<V, false>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
+              W += wf;
+              w16[i] = wf;
+              if constexpr (PROB) {
+                WL += wl;
+                vl[i] = wl;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float wf, wl;
+              fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
+              const int key = key0 + i;
+              const bool ok = key < T && (!p.causal || key <= qrow);
+              wf = ok ? wf : 0.0f;
+              wl = ok ? wl : 0.0f;
+              W += wf;
+              w16[i] = wf;
+              if constexpr (PROB) {
+                WL += wl;
+                vl[i] = wl;
+              }
+            }
+          }
+          tmem_st16(tmem + lane_addr + 128u * b + col, w16);
+          if constexpr (PROB) tmem_st16(tmem + lane_addr + col_pl + col, vl);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar.p_ready[b]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bar.p_ready[b]);
+    };
+    if constexpr (V::MINMAX) {
+      if (tab_in_smem) sweep2(GridF{sTab + r, KIA_TILE});
+      else sweep2(GridF{st.table + grow * (p.K + 1), 1});
+    } else {
+      sweep2(GridP{sPair});
     }
     // normalisers of the whole row
-    rx.W[half][r] = W;
-    rx.WL[half][r] = WL;
+    rx.W[part][r] = W;
+    rx.WL[part][r] = WL;
     mbar_arrive(&bar.row_sync);
     if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
-    W = rx.W[0][r] + rx.W[1][r];
-    WL = PROB ? rx.WL[0][r] + rx.WL[1][r] : W;
-    // epilogue: this thread writes D/2 columns of its row
+    const float Wrow = (rx.W[0][r] + rx.W[1][r]) + (rx.W[2][r] + rx.W[3][r]);
+    const float WLrow =
+        PROB ? (rx.WL[0][r] + rx.WL[1][r]) + (rx.WL[2][r] + rx.WL[3][r]) : Wrow;
+    // epilogue: this thread writes D/4 columns of its row
     if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.o_full, 0, abort))) {
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        const uint32_t col = (uint32_t)(half * (D / 2) + 32 * c);
-        tmem_ld32(tmem + lane_addr + col_o + col, v);
+      constexpr int kCols = D / kRowSplit;     // 16 or 32
+      const uint32_t col = (uint32_t)(part * kCols);
+      float o[kCols];
+      auto write_row = [&](uint32_t tcol, float* dst, float w) {
+        if constexpr (kCols == 16) tmem_ld16(tmem + lane_addr + tcol + col, o);
+        else tmem_ld32(tmem + lane_addr + tcol + col, o);
         tmem_ld_wait();
         if (qrow < T) {
-          float4* o4 = reinterpret_cast<float4*>(O + grow * D + col);
+          float4* o4 = reinterpret_cast<float4*>(dst + grow * D + col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o4[i] = make_float4(__fdiv_rn(v[4 * i], W), __fdiv_rn(v[4 * i + 1], W),
-                                __fdiv_rn(v[4 * i + 2], W), __fdiv_rn(v[4 * i + 3], W));
+          for (int i = 0; i < kCols / 4; ++i)
+            o4[i] = make_float4(__fdiv_rn(o[4 * i], w), __fdiv_rn(o[4 * i + 1], w),
+                                __fdiv_rn(o[4 * i + 2], w), __fdiv_rn(o[4 * i + 3], w));
         }
-        if constexpr (PROB) {
-          tmem_ld32(tmem + lane_addr + col_ol + col, v);
-          tmem_ld_wait();
-          if (qrow < T) {
-            float4* o4 = reinterpret_cast<float4*>(st.OL + grow * D + col);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              o4[i] = make_float4(__fdiv_rn(v[4 * i], WL), __fdiv_rn(v[4 * i + 1], WL),
-                                  __fdiv_rn(v[4 * i + 2], WL), __fdiv_rn(v[4 * i + 3], WL));
-          }
-        }
-      }
-      if (qrow < T && half == 0) {
+      };
+      write_row(col_o, O, Wrow);
+      if constexpr (PROB) write_row(col_ol, st.OL, WLrow);
+      if (qrow < T && part == 0) {
         st.m[grow] = m;
         st.n[grow] = n;
         st.am[grow] = am;
         st.an[grow] = an;
         st.rh[grow] = degen ? 0.0f : rc.rh;
         st.h[grow] = degen ? 0.0f : rc.h;
-        st.Wf[grow] = W;
-        st.Wb[grow] = (!V::SOFTMAX && lerp_normpoint(p)) ? WL : W;
+        st.Wf[grow] = Wrow;
+        st.Wb[grow] = (!V::SOFTMAX && lerp_normpoint(p)) ? WLrow : Wrow;
       }
       if (bh == 0 && qt == nt - 1 && threadIdx.x == 64) write_header(st.header, B, H, T, D, p);
     } else {
@@ -419,7 +453,7 @@ size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem) {
   constexpr int NS = FwdCfg<D>::kStages;
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
-      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : (p.K + 1));
+      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   return 1024 + (size_t)(1 + 2 * NS) * FwdCfg<D>::kTileBytes + sizeof(FwdRowX) +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
 }

@@ -150,7 +150,7 @@ int backward_rows(const float* Q, const float* Kt, const float* O, const float* 
   if (launch_status()) return KIA_ERR_CUDA;
   if (!p.softmax && p.grad == KIA_GRAD_PROJECT) {
     dim3 g(B * H, D / 32);
-    bwd_project_scan_kernel<D><<<g, 32 * kScanGroups, 0, s>>>(Q, Kt, wk, dQ, dK, p, T);
+    bwd_project_scan_kernel<D><<<g, 32 * kScanGroups, 0, s>>>(Q, Kt, wk, dQ, dK, p, T, 1);
     if (launch_status()) return KIA_ERR_CUDA;
   }
   return KIA_OK;
@@ -169,21 +169,33 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
   }
   const bool tc = gemm == KIA_GEMM_TF32;
   prof_mark(2, s);
-  int rc = backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, true, nullptr);
+  int rc;
+  if (tc && D == 64) {
+    // query pass (checks the stats, centering, dQ with its calibration terms),
+    // key pass (dK with the calibration terms folded into dS, dV)
+    prof_mark(3, s);
+    rc = tc_backward<D>(Q, Kt, V, O, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s, prof_mark);
+    if (rc) return rc;
+    if (!p.softmax && p.grad == KIA_GRAD_PROJECT) {
+      // the key pass already folded the projection shift into dK
+      dim3 g(B * H, D / 32);
+      bwd_project_scan_kernel<D><<<g, 32 * kScanGroups, 0, s>>>(Q, Kt, wk, dQ, dK, p, T, 0);
+      if (launch_status()) return KIA_ERR_CUDA;
+    }
+    prof_mark(6, s);
+    return KIA_OK;
+  }
+  // exact-fp32 kernels (and the d = 128 backward in TF32 mode, with the
+  // tensor cores' operand truncation so it sees the TF32 forward's arithmetic)
+  rc = backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, true, nullptr);
   if (rc) return rc;
   prof_mark(3, s);
-  if (tc && D == 64) {
-    rc = tc_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s, prof_mark);
-  } else {
-    // d = 128 in TF32 mode: CUDA-core kernels with the tensor cores' operand
-    // truncation, so the backward sees the arithmetic of the TF32 forward
-    OpParams q = p;
-    q.tf32_ops = tc ? 1 : 0;
-    rc = simt_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, q, s);
-    prof_mark(4, s);
-    prof_mark(5, s);
-  }
+  OpParams q = p;
+  q.tf32_ops = tc ? 1 : 0;
+  rc = simt_backward<D>(Q, Kt, V, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, q, s);
   if (rc) return rc;
+  prof_mark(4, s);
+  prof_mark(5, s);
   rc = backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, false, nullptr);
   prof_mark(6, s);
   return rc;
@@ -193,7 +205,7 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
 // KIA_NOALLOC_MAX_ROWS rows, declared by the library so that the caller
 // allocates nothing.  Host code only ever uses its device address, looked up
 // once per device.
-constexpr size_t kNoallocScratchBytes = 5 * ((size_t)KIA_NOALLOC_MAX_ROWS * 4) + 256;
+constexpr size_t kNoallocScratchBytes = work_bytes_c(KIA_NOALLOC_MAX_ROWS);
 static __device__ __align__(256) unsigned char g_kia_noalloc_scratch[kNoallocScratchBytes];
 constexpr int kMaxDevices = 64;
 void* g_noalloc_addr[kMaxDevices] = {};

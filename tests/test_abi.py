@@ -53,7 +53,7 @@ def test_buffer_sizes(K):
     prob = K.kiattn_stats_bytes(B, H, T, d, cfg.replace(rec=K.REC_NEAREST, ste=K.STE_PROB))
     assert prob >= sb + rows * d * 4          # O_L for Prob-STE
     wb = K.kiattn_workspace_bytes(B, H, T, d, cfg)
-    assert rows * 5 * 4 <= wb < rows * 5 * 4 + 4096
+    assert rows * 7 * 4 <= wb < rows * 7 * 4 + 4096
     assert K.kiattn_stats_bytes(B, H, T, 96, cfg) == 0      # d unsupported
     assert K.kiattn_stats_bytes(B, H, T, d, cfg.replace(K=0)) == 0
     assert K.kiattn_stats_bytes(B, H, T, d, cfg.replace(K=65)) == 0
