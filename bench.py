@@ -225,6 +225,25 @@ def ncu_traffic(kernel: str):
     return ent.get("bytes_per_launch_full_size")
 
 
+# ---------------------------------------------------------- multi-rank host
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank processes its own batch each step; the
+    step time is the slowest rank's."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU side
 
 def main():
@@ -291,12 +310,9 @@ def main():
         dist.barrier()
     clocks = sampler.stop()
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = float(t.item()) / args.steps
+    ms_step = max_over_ranks(total_ms, device="cuda") / args.steps
     flops = algorithmic_flops(w)
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = weak_scaling_value(flops, world, ms_step)
 
     # end to end through the public API from pinned host memory
     e2e = None
@@ -321,13 +337,11 @@ def main():
                 ho.copy_(dd, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / nrep], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te = max_over_ranks(e0.elapsed_time(e1) / nrep, device="cuda")
         nbytes = sum(x.numel() * 4 for x in host)
-        e2e = {"value": world * flops / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": weak_scaling_value(flops, world, te), "unit": "TFLOP/s",
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": 4 * bufs.O.numel() * 4,
-               "ms_per_step": float(te.item())}
+               "ms_per_step": te}
     K.kiattn_profile_enable(False)
 
     # roofline of the dominant kernel (tensor-core bound: TF32 contraction)
