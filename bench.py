@@ -279,7 +279,10 @@ def main():
         K.kiattn_fwd(q, k, v, bufs.O, bufs.stats, cfg)
         K.kiattn_bwd(q, k, v, bufs.O, g, bufs.stats, bufs.dQ, bufs.dK, bufs.dV, bufs.work, cfg)
 
-    launches_per_step = 1 + 4 + (1 if w.grad == K.GRAD_PROJECT else 0)
+    # our kernels per step: the forward, then the tensor-core backward's query
+    # and key passes (d = 64) or the exact backward's four row and tile
+    # kernels (d = 128), plus the projection's scan
+    launches_per_step = 1 + (2 if w.d == 64 else 4) + (1 if w.grad == K.GRAD_PROJECT else 0)
     K.kiattn_profile_enable(True)
     for _ in range(args.warmup):
         flush.zero_()

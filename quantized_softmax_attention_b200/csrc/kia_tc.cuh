@@ -74,6 +74,18 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int ks) {
   return smem_desc(tile + (uint32_t)ks * 1024u, kBlockBytes, 512u, kLayoutSW128Atom32);
 }
 
+// The start address sits in the descriptor's low 14 bits in 16-byte units
+// and never carries out of them (shared memory < 256 KB), so a descriptor
+// moves to another operand or K step by adding the byte offset / 16.  The
+// MMA issuer builds one descriptor per tile and steps it with these.
+__host__ __device__ constexpr uint64_t desc_step(uint32_t bytes) { return bytes >> 4; }
+// K-major: K step ks of a tile (column block ks / 4, 32 bytes per step inside it)
+__host__ __device__ constexpr uint64_t kstep_kmajor(int ks) {
+  return desc_step((uint32_t)(ks >> 2) * kBlockBytes + (uint32_t)(ks & 3) * 32u);
+}
+// MN-major: K step ks = rows 8ks..8ks+7
+__host__ __device__ constexpr uint64_t kstep_mnmajor(int ks) { return desc_step((uint32_t)ks * 1024u); }
+
 // ------------------------------------------------------ score tile kernel
 
 template <int D>

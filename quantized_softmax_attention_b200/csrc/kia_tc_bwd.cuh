@@ -20,9 +20,13 @@
 // (section 3, Calibration gradients; Appendix B): g_m at the argmax key and
 // g_n at the argmin key (or the zero-sum projection's shift), added to dQ
 // there and folded into dS^T by the key pass before its dK contraction.
-// Warp roles (18 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
-// 2..17 = element warps (warp w reaches TMEM lanes 32*(w%4)..+31; the four
-// warps sharing those lanes split each half tile's 64 columns).
+// Warp roles (20 warps): 0 = TMA producer, 1 = issuer of the accumulating
+// MMAs (dQ, or dV and dK) and TMEM owner, 18 = issuer of the score MMAs
+// (S and dP), 19 = spare, 2..17 = element warps in two groups of eight: group g works on the half
+// tiles u with u % 2 == g (TMEM buffer g), so the two groups run out of
+// phase and one computes while the other waits for its operands.  Warp w
+// reaches TMEM lanes 32*(w%4)..+31; the two warps of a group that share
+// those lanes split a half tile's 64 columns.
 #pragma once
 #include <type_traits>
 
@@ -32,14 +36,15 @@
 namespace kia {
 
 constexpr int kBwdSmemTabK = 32;  // key pass: per-query grids up to K = 32 in shared memory
+constexpr int kBwdRegions = 3;    // TMEM regions of 128 columns (S | dP) in rotation
 
 struct BwdQBars {
   uint64_t qd_full;               // Q_i, dO_i (K-major), once
   uint64_t kv_full, kv_empty;     // K_j, V_j K-major (for S, dP)
   uint64_t kmn_full, kmn_empty;   // K_j MN-major (for dQ)
-  uint64_t sp_full[2];            // S and dP of a half tile in TMEM buffer b
-  uint64_t elem_done[2];          // dS written into buffer b
-  uint64_t st_free[2];            // dQ MMA of buffer b done
+  uint64_t sp_full[3];            // S and dP of a half tile in TMEM region r
+  uint64_t elem_done[3];          // dS written into region r
+  uint64_t st_free[3];            // dQ MMA of region r done
   uint64_t dq_full;               // all dQ MMAs done
   uint64_t row_sync;              // element-thread rendezvous
   uint32_t tmem_base;
@@ -50,10 +55,11 @@ struct BwdKBars {
   uint64_t kv_full;               // K_j, V_j K-major, once
   uint64_t qd_full, qd_empty;     // Q_i, dO_i K-major (for S^T, dP^T)
   uint64_t mn_full, mn_empty;     // Q_i, dO_i MN-major (for dK, dV)
-  uint64_t sp_full[2];            // S^T and dP^T of a half tile in TMEM buffer b
-  uint64_t qc_ready;              // per-query constants of a tile loaded
-  uint64_t elem_done[2];          // P^T, dS^T written into buffer b
-  uint64_t st_free[2];            // dV, dK MMAs of buffer b done
+  uint64_t sp_full[3];            // S^T and dP^T of a half tile in TMEM region r
+  uint64_t qc_ready[2];           // per-query constants of group g's unit loaded
+  uint64_t qc_free[2];            // group g done with its unit's constants
+  uint64_t elem_done[3];          // P^T, dS^T written into region r
+  uint64_t st_free[3];            // dV, dK MMAs of region r done
   uint64_t acc_full;              // all dV, dK MMAs done
   uint32_t tmem_base;
   int abort;
@@ -90,7 +96,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   float* sKmn = reinterpret_cast<float*>(base + 3 * kTile);
   float* sV = reinterpret_cast<float*>(base + 4 * kTile);
   float* sAC = reinterpret_cast<float*>(base + 5 * kTile);   // [kRowSplit][2][128]
-  float* sTab = sAC + 2 * kRowSplit * KIA_TILE;
+  float* sDc = sAC + 2 * kRowSplit * KIA_TILE;               // [128] centering D
+  float* sTab = sDc + KIA_TILE;
   const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (p.K + 1) * KIA_TILE : 2 * (p.K + 1));
   BwdQBars& bar = *reinterpret_cast<BwdQBars*>(sTab + ((tab_floats + 31) & ~31));
 
@@ -100,7 +107,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int qt = nt - 1 - blockIdx.y;
   const int nkt = p.causal ? qt + 1 : nt;
   const int nunits = 2 * nkt;          // half key tiles
-  constexpr uint32_t kColDQ = 256;
+  constexpr int R = kBwdRegions;
+  constexpr uint32_t kColDQ = 128u * R;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.qd_full, 1);
@@ -108,9 +116,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(&bar.kv_empty, 1);
     mbar_init(&bar.kmn_full, 1);
     mbar_init(&bar.kmn_empty, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&bar.sp_full[b], 1);
-      mbar_init(&bar.elem_done[b], kElemThreads);
+      mbar_init(&bar.elem_done[b], kGroupThreads);
       mbar_init(&bar.st_free[b], 1);
     }
     mbar_init(&bar.dq_full, 1);
@@ -142,66 +150,93 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, qt * KIA_TILE, bh);
         tma_load_3d(sG + b * 32 * KIA_TILE, &tmG, &bar.qd_full, b * 32, qt * KIA_TILE, bh);
       }
-      for (int j = 0; j < nkt; ++j) {
-        if (!mbar_wait(&bar.kv_empty, (j & 1) ^ 1, abort)) { failed = true; break; }
-        mbar_arrive_expect_tx(&bar.kv_full, 2 * kTile);
-        for (int b = 0; b < D / 32; ++b) {
-          tma_load_3d(sK + b * 32 * KIA_TILE, &tmK, &bar.kv_full, b * 32, j * KIA_TILE, bh);
-          tma_load_3d(sV + b * 32 * KIA_TILE, &tmV, &bar.kv_full, b * 32, j * KIA_TILE, bh);
+      // the two rings refill independently, each as soon as its slot is free
+      int jk = 0, jm = 0;                // next K / V tile, next K MN-major tile
+      PollGuard guard;
+      while ((jk < nkt || jm < nkt) && !failed) {
+        bool moved = false;
+        if (jk < nkt && mbar_test(&bar.kv_empty, (jk & 1) ^ 1)) {
+          mbar_arrive_expect_tx(&bar.kv_full, 2 * kTile);
+          for (int b = 0; b < D / 32; ++b) {
+            tma_load_3d(sK + b * 32 * KIA_TILE, &tmK, &bar.kv_full, b * 32, jk * KIA_TILE, bh);
+            tma_load_3d(sV + b * 32 * KIA_TILE, &tmV, &bar.kv_full, b * 32, jk * KIA_TILE, bh);
+          }
+          ++jk;
+          moved = true;
         }
-        if (!mbar_wait(&bar.kmn_empty, (j & 1) ^ 1, abort)) { failed = true; break; }
-        mbar_arrive_expect_tx(&bar.kmn_full, kTile);
-        for (int b = 0; b < D / 32; ++b)
-          tma_load_3d(sKmn + b * 32 * KIA_TILE, &tmKmn, &bar.kmn_full, b * 32, j * KIA_TILE, bh);
+        if (jm < nkt && mbar_test(&bar.kmn_empty, (jm & 1) ^ 1)) {
+          mbar_arrive_expect_tx(&bar.kmn_full, kTile);
+          for (int b = 0; b < D / 32; ++b)
+            tma_load_3d(sKmn + b * 32 * KIA_TILE, &tmKmn, &bar.kmn_full, b * 32, jm * KIA_TILE, bh);
+          ++jm;
+          moved = true;
+        }
+        if (moved) guard.progress();
+        else if (!guard.idle(abort)) failed = true;
+      }
+    }
+  } else if (warp == kScoreWarp) {
+    // ------------------------------------------------- score-MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
+      // descriptors built once; each MMA only adds a constant step
+      const uint64_t dqa = desc_kmajor(smem_u32(sQ), 0), dga = desc_kmajor(smem_u32(sG), 0),
+                     dka = desc_kmajor(smem_u32(sK), 0), dva = desc_kmajor(smem_u32(sV), 0);
+      uint32_t sf_par = 0;                // per-region phase bits of the st_free waits
+      failed = !mbar_wait(&bar.qd_full, 0, abort);
+      // S, dP of half tile u (keys 64 (u % 2).. of tile u / 2) into region
+      // u % R, once the dQ MMA of unit u - R has released the region
+      for (int u = 0; u < nunits && !failed; ++u) {
+        const int r = u % R, j = u >> 1, h = u & 1;
+        if (u >= R) {
+          if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+          sf_par ^= 1u << r;
+        }
+        if (h == 0 && !mbar_wait(&bar.kv_full, j & 1, abort)) { failed = true; break; }
+        tc_fence_after();
+        const uint64_t koff = desc_step((uint32_t)h * 64u * 128u);   // rows 64h.. of the key tile
+        const uint32_t dst = tmem + 128u * r;
+#pragma unroll
+        for (int ks = 0; ks < D / 8; ++ks)
+          mma_tf32_ss(dst, dqa + kstep_kmajor(ks), dka + koff + kstep_kmajor(ks), id_s, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < D / 8; ++ks)
+          mma_tf32_ss(dst + 64u, dga + kstep_kmajor(ks), dva + koff + kstep_kmajor(ks), id_s,
+                      ks > 0);
+        tc_commit(&bar.sp_full[r]);
+        if (h == 1) tc_commit(&bar.kv_empty);
       }
     }
   } else if (warp == 1) {
-    // --------------------------------------------------------- MMA issuer
+    // --------------------------------------------------- dQ-MMA issuer
     if (lane == 0) {
-      const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
       const uint32_t id_dq = idesc_tf32(128, D, 0, 1);
-      const uint32_t qa = smem_u32(sQ), ga = smem_u32(sG), ka = smem_u32(sK),
-                     kma = smem_u32(sKmn), va = smem_u32(sV);
-      // dQ of half tile u: A = dS in TMEM buffer u&1, B = rows 64*(u&1).. of K_j (MN-major)
-      auto issue_dq = [&](int u) -> bool {
-        const int b = u & 1, j = u >> 1;
-        if (!mbar_wait(&bar.elem_done[b], (u >> 1) & 1, abort)) return false;
-        if (b == 0 && !mbar_wait(&bar.kmn_full, j & 1, abort)) return false;
+      const uint64_t dkm = desc_mnmajor(smem_u32(sKmn), 0);
+      uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
+      // dQ of half tile u: A = dS in region u % R, B = rows 64 (u % 2).. of K_j (MN-major)
+      for (int u = 0; u < nunits && !failed; ++u) {
+        const int r = u % R, j = u >> 1, h = u & 1;
+        if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
+        ed_par ^= 1u << r;
+        if (h == 0 && !mbar_wait(&bar.kmn_full, j & 1, abort)) { failed = true; break; }
         tc_fence_after();
+        const uint64_t db = dkm + kstep_mnmajor(8 * h);
+        const uint32_t pa = tmem + 128u * r;
+        const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_tf32_ts(tmem + kColDQ, tmem + 128u * b + 8u * kk, desc_mnmajor(kma, 8 * b + kk),
-                      id_dq, (u > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&bar.st_free[b]);
-        if (b == 1) tc_commit(&bar.kmn_empty);
-        return true;
-      };
-      failed = !mbar_wait(&bar.qd_full, 0, abort);
-      for (int u = 0; u < nunits && !failed; ++u) {
-        const int b = u & 1, j = u >> 1;
-        if (b == 0 && !mbar_wait(&bar.kv_full, j & 1, abort)) { failed = true; break; }
-        if (u >= 2 && !mbar_wait(&bar.st_free[b], ((u >> 1) - 1) & 1, abort)) { failed = true; break; }
-        tc_fence_after();
-        const uint32_t koff = (uint32_t)b * 64u * 128u;     // rows 64b.. of the key tile
-#pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(tmem + 128u * b, desc_kmajor(qa, ks), desc_kmajor(ka + koff, ks), id_s,
-                      ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(tmem + 128u * b + 64u, desc_kmajor(ga, ks), desc_kmajor(va + koff, ks),
-                      id_s, ks > 0);
-        tc_commit(&bar.sp_full[b]);
-        if (b == 1) tc_commit(&bar.kv_empty);
-        if (u >= 1 && !issue_dq(u - 1)) { failed = true; break; }
+          mma_tf32_ts(tmem + kColDQ, pa + 8u * kk, db + kstep_mnmajor(kk), id_dq, kk > 0 ? 1u : acc0);
+        tc_commit(&bar.st_free[r]);
+        if (h == 1) tc_commit(&bar.kmn_empty);
       }
-      if (!failed && !issue_dq(nunits - 1)) failed = true;
       if (!failed) tc_commit(&bar.dq_full);
     }
-  } else {
+  } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;       // which 16 columns of a half tile
+    const int part = (warp - 2) >> 2;       // 0..3: (group, half of a unit)
+    const int grp = part >> 1;              // half tiles u with u % 2 == grp
+    const int sub = part & 1;               // columns 32 sub .. 32 sub + 31 of a unit
     const int r = quad * 32 + lane;
     const int q = qt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
@@ -217,20 +252,32 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int L = p.causal ? q + 1 : T;
     // a one-key row has P = 1 whatever its score: zero gradient
     const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]);
-    // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE)
-    float Dc = 0.0f;
+    // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE): four
+    // consecutive element threads read one row's D values (coalesced), add
+    // their partial sums by shuffles and leave the row's D in shared memory
     {
-      const float4* g4 = reinterpret_cast<const float4*>(dO + qr * D);
-      const float4* o4 = reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qr * D);
-#pragma unroll 4
-      for (int c = 0; c < D / 4; ++c) {
+      const int e = (int)threadIdx.x - 64;
+      const int rr = e >> 2, cc = e & 3;     // row of the tile, quarter of the row
+      const int qq = qt * KIA_TILE + rr;
+      const long long qrr = rowbase + (qq < T ? qq : T - 1);
+      const float4* g4 = reinterpret_cast<const float4*>(dO + qrr * D) + cc * (D / 16);
+      const float4* o4 =
+          reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qrr * D) + cc * (D / 16);
+      float acc = 0.0f;
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
         const float4 a = g4[c], b4 = o4[c];
-        Dc = fmaf(a.x, b4.x, Dc);
-        Dc = fmaf(a.y, b4.y, Dc);
-        Dc = fmaf(a.z, b4.z, Dc);
-        Dc = fmaf(a.w, b4.w, Dc);
+        acc = fmaf(a.x, b4.x, acc);
+        acc = fmaf(a.y, b4.y, acc);
+        acc = fmaf(a.z, b4.z, acc);
+        acc = fmaf(a.w, b4.w, acc);
       }
-      if (part == 0 && q < T) wk.D[qr] = Dc;
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (cc == 0) {
+        sDc[rr] = acc;
+        if (qq < T) wk.D[qrr] = acc;
+      }
     }
 
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
@@ -247,43 +294,47 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     else grid = GridP{sPair};
     mbar_arrive(&bar.row_sync);
     if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
+    const float Dc = sDc[r];
     float A = 0.0f, C = 0.0f;
-    float v[16], g[16];
-    for (int u = 0; u < nunits && !failed; ++u) {
-      const int b = u & 1, j = u >> 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[b], (u >> 1) & 1, abort))) { failed = true; break; }
+    for (int u = grp; u < nunits && !failed; u += 2) {
+      const int j = u >> 1, rg = u % R;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (u / R) & 1, abort))) { failed = true; break; }
       tc_fence_after();
-      const uint32_t cs = 128u * b + 16u * part;       // this thread's 16 columns of S
-      tmem_ld16(tmem + lane_addr + cs, v);
-      tmem_ld16(tmem + lane_addr + cs + 64u, g);
-      tmem_ld_wait();
-      const int key0 = j * KIA_TILE + 64 * b + 16 * part;
       const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
-      if (!edge) {
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float v[16], g[16];
+        const uint32_t cs = 128u * rg + 32u * sub + 16u * c;    // 16 columns of S
+        tmem_ld16(tmem + lane_addr + cs, v);
+        tmem_ld16(tmem + lane_addr + cs + 64u, g);
+        tmem_ld_wait_regs(v, g);
+        const int key0 = j * KIA_TILE + 64 * grp + 32 * sub + 16 * c;
+        if (!edge) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float dw = (g[i] - Dc) * rWb;
-          v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+          for (int i = 0; i < 16; ++i) {
+            const float dw = (g[i] - Dc) * rWb;
+            v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int key = key0 + i;
+            const bool ok = key < T && (!p.causal || key <= q);
+            const float dw = ok ? (g[i] - Dc) * rWb : 0.0f;
+            v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+          }
         }
-      } else {
+        tmem_st16(tmem + lane_addr + cs, v);
+        if (dS_dbg && q < T) {
+          float* dst = dS_dbg + (rowbase + q) * T + key0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int key = key0 + i;
-          const bool ok = key < T && (!p.causal || key <= q);
-          const float dw = ok ? (g[i] - Dc) * rWb : 0.0f;
-          v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+          for (int i = 0; i < 16; ++i)
+            if (key0 + i < T) dst[i] = v[i];
         }
-      }
-      tmem_st16(tmem + lane_addr + cs, v);
-      if (dS_dbg && q < T) {
-        float* dst = dS_dbg + (rowbase + q) * T + key0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (key0 + i < T) dst[i] = v[i];
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar.elem_done[b]);
+      mbar_arrive(&bar.elem_done[rg]);
     }
     // row sums of the four column groups
     sAC[(part * 2 + 0) * KIA_TILE + r] = A;
@@ -390,7 +441,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   int2* sCI = reinterpret_cast<int2*>(sCA + KIA_TILE);         // argmax, argmin keys - tile start
   float* sTab = reinterpret_cast<float*>(sCI + KIA_TILE);
   const int K1 = p.K + 1;
-  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? K1 * KIA_TILE : 0) : 2 * K1);
+  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? K1 * KIA_TILE : 0) : 4 * K1);
   BwdKBars& bar = *reinterpret_cast<BwdKBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -400,7 +451,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int q0 = p.causal ? kt : 0;
   const int ntiles = nt - q0;
   const int nunits = 2 * ntiles;       // half query tiles
-  constexpr uint32_t kColDV = 256, kColDK = 256 + D;
+  constexpr int R = kBwdRegions;
+  constexpr uint32_t kColDV = 128u * R, kColDK = kColDV + D;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.kv_full, 1);
@@ -408,12 +460,15 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     mbar_init(&bar.qd_empty, 1);
     mbar_init(&bar.mn_full, 1);
     mbar_init(&bar.mn_empty, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&bar.sp_full[b], 1);
-      mbar_init(&bar.elem_done[b], kElemThreads);
+      mbar_init(&bar.elem_done[b], kGroupThreads);
       mbar_init(&bar.st_free[b], 1);
     }
-    mbar_init(&bar.qc_ready, kElemThreads);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bar.qc_ready[g], kGroupThreads);
+      mbar_init(&bar.qc_free[g], kGroupThreads);
+    }
     mbar_init(&bar.acc_full, 1);
     bar.abort = 0;
     fence_barrier_init();
@@ -443,169 +498,204 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tma_load_3d(sK + b * 32 * KIA_TILE, &tmK, &bar.kv_full, b * 32, kt * KIA_TILE, bh);
         tma_load_3d(sV + b * 32 * KIA_TILE, &tmV, &bar.kv_full, b * 32, kt * KIA_TILE, bh);
       }
-      for (int s = 0; s < ntiles; ++s) {
-        const int qi = q0 + s;
-        if (!mbar_wait(&bar.qd_empty, (s & 1) ^ 1, abort)) { failed = true; break; }
-        mbar_arrive_expect_tx(&bar.qd_full, 2 * kTile);
-        for (int b = 0; b < D / 32; ++b) {
-          tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, qi * KIA_TILE, bh);
-          tma_load_3d(sG + b * 32 * KIA_TILE, &tmG, &bar.qd_full, b * 32, qi * KIA_TILE, bh);
+      // the two rings refill independently, each as soon as its slot is free
+      int sk = 0, sm = 0;                // next K-major tile, next MN-major tile
+      PollGuard guard;
+      while ((sk < ntiles || sm < ntiles) && !failed) {
+        bool moved = false;
+        if (sk < ntiles && mbar_test(&bar.qd_empty, (sk & 1) ^ 1)) {
+          const int qi = q0 + sk;
+          mbar_arrive_expect_tx(&bar.qd_full, 2 * kTile);
+          for (int b = 0; b < D / 32; ++b) {
+            tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, qi * KIA_TILE, bh);
+            tma_load_3d(sG + b * 32 * KIA_TILE, &tmG, &bar.qd_full, b * 32, qi * KIA_TILE, bh);
+          }
+          ++sk;
+          moved = true;
         }
-        if (!mbar_wait(&bar.mn_empty, (s & 1) ^ 1, abort)) { failed = true; break; }
-        mbar_arrive_expect_tx(&bar.mn_full, 2 * kTile);
-        for (int b = 0; b < D / 32; ++b) {
-          tma_load_3d(sQmn + b * 32 * KIA_TILE, &tmQmn, &bar.mn_full, b * 32, qi * KIA_TILE, bh);
-          tma_load_3d(sGmn + b * 32 * KIA_TILE, &tmGmn, &bar.mn_full, b * 32, qi * KIA_TILE, bh);
+        if (sm < ntiles && mbar_test(&bar.mn_empty, (sm & 1) ^ 1)) {
+          const int qi = q0 + sm;
+          mbar_arrive_expect_tx(&bar.mn_full, 2 * kTile);
+          for (int b = 0; b < D / 32; ++b) {
+            tma_load_3d(sQmn + b * 32 * KIA_TILE, &tmQmn, &bar.mn_full, b * 32, qi * KIA_TILE, bh);
+            tma_load_3d(sGmn + b * 32 * KIA_TILE, &tmGmn, &bar.mn_full, b * 32, qi * KIA_TILE, bh);
+          }
+          ++sm;
+          moved = true;
         }
+        if (moved) guard.progress();
+        else if (!guard.idle(abort)) failed = true;
+      }
+    }
+  } else if (warp == kScoreWarp) {
+    // ------------------------------------------------- score-MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
+      // descriptors built once; each MMA only adds a constant step
+      const uint64_t dka = desc_kmajor(smem_u32(sK), 0), dva = desc_kmajor(smem_u32(sV), 0),
+                     dqa = desc_kmajor(smem_u32(sQ), 0), dga = desc_kmajor(smem_u32(sG), 0);
+      uint32_t sf_par = 0;                // per-region phase bits of the st_free waits
+      failed = !mbar_wait(&bar.kv_full, 0, abort);
+      // S^T, dP^T of half tile u (queries 64 (u % 2).. of tile u / 2) into
+      // region u % R, once the dV / dK MMAs of unit u - R have released it
+      for (int u = 0; u < nunits && !failed; ++u) {
+        const int r = u % R, s = u >> 1, h = u & 1;
+        if (u >= R) {
+          if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+          sf_par ^= 1u << r;
+        }
+        if (h == 0 && !mbar_wait(&bar.qd_full, s & 1, abort)) { failed = true; break; }
+        tc_fence_after();
+        const uint64_t qoff = desc_step((uint32_t)h * 64u * 128u);   // query rows 64h.. of the tile
+        const uint32_t dst = tmem + 128u * r;
+#pragma unroll
+        for (int ks = 0; ks < D / 8; ++ks)
+          mma_tf32_ss(dst, dka + kstep_kmajor(ks), dqa + qoff + kstep_kmajor(ks), id_s, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < D / 8; ++ks)
+          mma_tf32_ss(dst + 64u, dva + kstep_kmajor(ks), dga + qoff + kstep_kmajor(ks), id_s,
+                      ks > 0);
+        tc_commit(&bar.sp_full[r]);
+        if (h == 1) tc_commit(&bar.qd_empty);
       }
     }
   } else if (warp == 1) {
-    // --------------------------------------------------------- MMA issuer
+    // ---------------------------------------------- dV / dK-MMA issuer
     if (lane == 0) {
-      const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
       const uint32_t id_acc = idesc_tf32(128, D, 0, 1);
-      const uint32_t ka = smem_u32(sK), va = smem_u32(sV), qa = smem_u32(sQ), ga = smem_u32(sG),
-                     qma = smem_u32(sQmn), gma = smem_u32(sGmn);
-      // dV += P^T dO, dK += dS^T Q for half tile u (queries 64*(u&1).. of tile u>>1)
-      auto issue_acc = [&](int u) -> bool {
-        const int b = u & 1, s = u >> 1;
-        if (!mbar_wait(&bar.elem_done[b], (u >> 1) & 1, abort)) return false;
-        if (b == 0 && !mbar_wait(&bar.mn_full, s & 1, abort)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_tf32_ts(tmem + kColDV, tmem + 128u * b + 8u * kk, desc_mnmajor(gma, 8 * b + kk),
-                      id_acc, (u > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_tf32_ts(tmem + kColDK, tmem + 128u * b + 64u + 8u * kk,
-                      desc_mnmajor(qma, 8 * b + kk), id_acc, (u > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&bar.st_free[b]);
-        if (b == 1) tc_commit(&bar.mn_empty);
-        return true;
-      };
-      failed = !mbar_wait(&bar.kv_full, 0, abort);
+      const uint64_t dqm = desc_mnmajor(smem_u32(sQmn), 0), dgm = desc_mnmajor(smem_u32(sGmn), 0);
+      uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
+      // dV += P^T dO, dK += dS^T Q for half tile u (A operands in region u % R)
       for (int u = 0; u < nunits && !failed; ++u) {
-        const int b = u & 1, s = u >> 1;
-        if (b == 0 && !mbar_wait(&bar.qd_full, s & 1, abort)) { failed = true; break; }
-        if (u >= 2 && !mbar_wait(&bar.st_free[b], ((u >> 1) - 1) & 1, abort)) { failed = true; break; }
+        const int r = u % R, s = u >> 1, h = u & 1;
+        if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
+        ed_par ^= 1u << r;
+        if (h == 0 && !mbar_wait(&bar.mn_full, s & 1, abort)) { failed = true; break; }
         tc_fence_after();
-        const uint32_t qoff = (uint32_t)b * 64u * 128u;     // query rows 64b.. of the tile
+        const uint64_t hoff = kstep_mnmajor(8 * h);
+        const uint32_t pa = tmem + 128u * r;
+        const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(tmem + 128u * b, desc_kmajor(ka, ks), desc_kmajor(qa + qoff, ks), id_s,
-                      ks > 0);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_tf32_ts(tmem + kColDV, pa + 8u * kk, dgm + hoff + kstep_mnmajor(kk), id_acc,
+                      kk > 0 ? 1u : acc0);
 #pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(tmem + 128u * b + 64u, desc_kmajor(va, ks), desc_kmajor(ga + qoff, ks),
-                      id_s, ks > 0);
-        tc_commit(&bar.sp_full[b]);
-        if (b == 1) tc_commit(&bar.qd_empty);
-        if (u >= 1 && !issue_acc(u - 1)) { failed = true; break; }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_tf32_ts(tmem + kColDK, pa + 64u + 8u * kk, dqm + hoff + kstep_mnmajor(kk), id_acc,
+                      kk > 0 ? 1u : acc0);
+        tc_commit(&bar.st_free[r]);
+        if (h == 1) tc_commit(&bar.mn_empty);
       }
-      if (!failed && !issue_acc(nunits - 1)) failed = true;
       if (!failed) tc_commit(&bar.acc_full);
     }
-  } else {
+  } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;        // which 16 query columns of a half tile
+    const int part = (warp - 2) >> 2;        // 0..3: (group, half of a unit)
+    const int grp = part >> 1;               // half tiles u with u % 2 == grp
+    const int sub = part & 1;                // query columns 32 sub .. 32 sub + 31 of a unit
     const int r = quad * 32 + lane;
-    const int e = (int)threadIdx.x - 64;     // 0..kElemThreads-1
+    const int eg = ((int)threadIdx.x - 64) & (kGroupThreads - 1);   // thread of the group
     const int kj = kt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const long long rowbase = (long long)bh * T;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
-    if (!V::SOFTMAX && !V::MINMAX && e < p.K)
-      reinterpret_cast<float2*>(sTab)[e] = make_float2(st.table[e], st.table[e + 1]);
-    float v[16], g[16];
-    for (int u = 0; u < nunits && !failed; ++u) {
-      const int b = u & 1, s = u >> 1;
+    // FWM: each group keeps its own copy of the shared grid's pairs
+    const float2* sPairG = reinterpret_cast<const float2*>(sTab) + grp * K1;
+    if (!V::SOFTMAX && !V::MINMAX && eg < p.K)
+      reinterpret_cast<float2*>(sTab)[grp * K1 + eg] = make_float2(st.table[eg], st.table[eg + 1]);
+    for (int u = grp; u < nunits && !failed; u += 2) {
+      const int s = u >> 1;
       const int qi = q0 + s;
-      if (b == 0) {
-        // per-query constants of tile qi: every reader of the previous
-        // tile's constants has arrived on that tile's last elem_done
-        if (u >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(&bar.elem_done[1], ((u - 1) >> 1) & 1, abort))) {
-          failed = true;
-          break;
-        }
-        if (e < KIA_TILE) {
-          const int q = qi * KIA_TILE + e;
-          const long long qr = rowbase + (q < T ? q : T - 1);
-          const float rhq = st.rh[qr];
-          const int Lq = p.causal ? q + 1 : T;
-          sC4[e] = make_float4(st.m[qr], rhq, wk.D[qr],
-                               Lq == 1 ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]));
-          // calibration terms of the query's row, added to dS^T before dK:
-          // g_m at the argmax key, g_n at the argmin key, or the projection
-          // shift c on every visible key
-          const bool live = q < T;
-          sCA[e] = make_float4(__fdiv_rn(1.0f, st.Wf[qr]), (V::MINMAX && rhq == 0.0f) ? 1.0f : 0.0f,
-                               live ? wk.gm[qr] : 0.0f, live ? wk.gn[qr] : 0.0f);
-          sCI[e] = make_int2(PROJ ? -1 : wk.am[qr] - kt * KIA_TILE,
-                             PROJ ? -1 : wk.an[qr] - kt * KIA_TILE);
-          if (V::MINMAX && tab_in_smem)
-            for (int k = 0; k < K1; ++k) sTab[e * K1 + k] = st.table[qr * K1 + k];
-        }
-        mbar_arrive(&bar.qc_ready);
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready, s & 1, abort))) { failed = true; break; }
+      const int rg = u % R;
+      // per-query constants of this unit's 64 queries (the group's own half
+      // of the arrays), once every thread of the group is done with its
+      // previous unit
+      if (u >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[grp], (s - 1) & 1, abort))) {
+        failed = true;
+        break;
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[b], (u >> 1) & 1, abort))) { failed = true; break; }
+      if (eg < 64) {
+        const int ql = 64 * grp + eg;
+        const int q = qi * KIA_TILE + ql;
+        const long long qr = rowbase + (q < T ? q : T - 1);
+        const float rhq = st.rh[qr];
+        const int Lq = p.causal ? q + 1 : T;
+        sC4[ql] = make_float4(st.m[qr], rhq, wk.D[qr], Lq == 1 ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]));
+        // calibration terms of the query's row, added to dS^T before dK:
+        // g_m at the argmax key, g_n at the argmin key, or the projection
+        // shift c on every visible key
+        const bool live = q < T;
+        sCA[ql] = make_float4(__fdiv_rn(1.0f, st.Wf[qr]), (V::MINMAX && rhq == 0.0f) ? 1.0f : 0.0f,
+                              live ? wk.gm[qr] : 0.0f, live ? wk.gn[qr] : 0.0f);
+        sCI[ql] = make_int2(PROJ ? -1 : wk.am[qr] - kt * KIA_TILE,
+                            PROJ ? -1 : wk.an[qr] - kt * KIA_TILE);
+        if (V::MINMAX && tab_in_smem)
+          for (int k = 0; k < K1; ++k) sTab[ql * K1 + k] = st.table[qr * K1 + k];
+      }
+      mbar_arrive(&bar.qc_ready[grp]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[grp], s & 1, abort))) { failed = true; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (u / R) & 1, abort))) { failed = true; break; }
       tc_fence_after();
-      const uint32_t cs = 128u * b + 16u * part;
-      tmem_ld16(tmem + lane_addr + cs, v);
-      tmem_ld16(tmem + lane_addr + cs + 64u, g);
-      tmem_ld_wait();
-      const int ql0 = 64 * b + 16 * part;              // first query (in the tile) of the chunk
       const bool edge =
           (p.causal && qi == kt) || (qi + 1) * KIA_TILE > T || (kt + 1) * KIA_TILE > T;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float v[16], g[16];
+        const uint32_t cs = 128u * rg + 32u * sub + 16u * c;
+        tmem_ld16(tmem + lane_addr + cs, v);
+        tmem_ld16(tmem + lane_addr + cs + 64u, g);
+        tmem_ld_wait_regs(v, g);
+        const int ql0 = 64 * grp + 32 * sub + 16 * c;   // first query (in the tile) of the chunk
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int ql = ql0 + i;
-        const float4 c4 = sC4[ql];
-        const float4 ca = sCA[ql];
-        const float dw = (g[i] - c4.z) * c4.w;
-        float P, dS;
-        if constexpr (V::MINMAX) {
-          const GridF grid{tab_in_smem ? sTab + ql * K1
-                                       : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
-                           1};
-          kv_elem<V>(grid, c4.x, c4.y, ca.y, ca.x, Kf, Km1f, v[i], dw, P, dS);
-        } else {
-          kv_elem<V>(GridP{reinterpret_cast<const float2*>(sTab)}, c4.x, c4.y, ca.y, ca.x, Kf,
-                     Km1f, v[i], dw, P, dS);
-        }
-        if constexpr (PROJ) {
-          dS += ca.z;
-        } else if constexpr (!V::SOFTMAX) {
-          const int2 ci = sCI[ql];
-          dS += (ci.x == r) ? ca.z : 0.0f;
-          if constexpr (V::MINMAX) dS += (ci.y == r) ? ca.w : 0.0f;
-        }
-        if (edge) {
-          const int q = qi * KIA_TILE + ql;
-          if (!(kj < T && q < T && (!p.causal || kj <= q))) {
-            P = 0.0f;
-            dS = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+          const int ql = ql0 + i;
+          const float4 c4 = sC4[ql];
+          const float4 ca = sCA[ql];
+          const float dw = (g[i] - c4.z) * c4.w;
+          float P, dS;
+          if constexpr (V::MINMAX) {
+            const GridF grid{tab_in_smem ? sTab + ql * K1
+                                         : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
+                             1};
+            kv_elem<V>(grid, c4.x, c4.y, ca.y, ca.x, Kf, Km1f, v[i], dw, P, dS);
+          } else {
+            kv_elem<V>(GridP{sPairG}, c4.x, c4.y, ca.y, ca.x, Kf, Km1f, v[i], dw, P, dS);
           }
+          if constexpr (PROJ) {
+            dS += ca.z;
+          } else if constexpr (!V::SOFTMAX) {
+            const int2 ci = sCI[ql];
+            dS += (ci.x == r) ? ca.z : 0.0f;
+            if constexpr (V::MINMAX) dS += (ci.y == r) ? ca.w : 0.0f;
+          }
+          if (edge) {
+            const int q = qi * KIA_TILE + ql;
+            if (!(kj < T && q < T && (!p.causal || kj <= q))) {
+              P = 0.0f;
+              dS = 0.0f;
+            }
+          }
+          v[i] = P;
+          g[i] = dS;
         }
-        v[i] = P;
-        g[i] = dS;
+        tmem_st16(tmem + lane_addr + cs, v);
+        tmem_st16(tmem + lane_addr + cs + 64u, g);
       }
-      tmem_st16(tmem + lane_addr + cs, v);
-      tmem_st16(tmem + lane_addr + cs + 64u, g);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar.elem_done[b]);
+      mbar_arrive(&bar.elem_done[rg]);
+      mbar_arrive(&bar.qc_free[grp]);
     }
     if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.acc_full, 0, abort))) {
       tc_fence_after();
       constexpr int kCols = D / kRowSplit;   // 16
       const uint32_t col = (uint32_t)(part * kCols);
+      float v[kCols], g[kCols];
       tmem_ld16(tmem + lane_addr + kColDV + col, v);
       tmem_ld16(tmem + lane_addr + kColDK + col, g);
-      tmem_ld_wait();
+      tmem_ld_wait_regs(v, g);
       if (kj < T) {
         float4* dv4 = reinterpret_cast<float4*>(dV + (rowbase + kj) * D + col);
         float4* dk4 = reinterpret_cast<float4*>(dK + (rowbase + kj) * D + col);
@@ -629,7 +719,7 @@ template <int D>
 size_t tc_bwd_q_smem(const OpParams& p) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : 2 * (p.K + 1));
-  return 1024 + 5 * (size_t)D * KIA_TILE * 4 + 2 * kRowSplit * KIA_TILE * 4 +
+  return 1024 + 5 * (size_t)D * KIA_TILE * 4 + (2 * kRowSplit + 1) * KIA_TILE * 4 +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdQBars);
 }
 
@@ -637,7 +727,7 @@ template <int D>
 size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
-      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
+      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 4 * (p.K + 1));
   return 1024 + 6 * (size_t)D * KIA_TILE * 4 + KIA_TILE * (16 + 16 + 8) +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdKBars);
 }

@@ -1,9 +1,9 @@
 // Fused tensor-core forward of K-interval attention (sm_100a).
 //
 // One CTA per (batch*head, 128-query tile), heaviest causal tiles first.
-// Two sweeps over the key tiles, because the grid of a row is anchored at
-// its final extrema (section 3, Calibration): no weight exists before the
-// row max (and min) are known, so there is no online rescaling.
+// Two sweeps over the keys, because the grid of a row is anchored at its
+// final extrema (section 3, Calibration): no weight exists before the row
+// max (and min) are known, so there is no online rescaling.
 //   sweep 1: S = Q K^T (tcgen05 kind::tf32, accumulator in TMEM) -> row
 //            max / min and their lowest indices;
 //   calibration: h, 1/h, and the grid G_k = e^{-k h} (per row under MinMax,
@@ -13,11 +13,23 @@
 //            operand of O += P V (and P_L for Prob-STE, O_L += P_L V);
 //   epilogue: O = O_acc / W (and O_L = O_L_acc / W_L), per-row statistics.
 //
-// Warp roles (18 warps): 0 = TMA producer, 1 = MMA issuer and TMEM owner,
-// 2..17 = element warps.  Element warp w reaches TMEM lanes 32*(w%4)..+31
-// (query rows); the four warps that share those rows split each 128-column
-// tile into 32-column groups, so each query row is served by four threads
-// whose row statistics are merged through shared memory.
+// Both sweeps walk the keys in units of 64 (half key tiles), numbered
+// across the two sweeps.  Unit U lives in TMEM region U % R (S / P in its
+// first 64 columns, P_L in the next 64; R = 3 regions where the
+// accumulators leave room), so the scores of the next units are computed
+// while the current ones are turned into weights and multiplied into O.
+// Warp roles (20 warps): 0 = TMA producer, 1 = issuer of the accumulating
+// MMAs (O += P V, O_L += P_L V) and TMEM owner, 18 = issuer of the score
+// MMAs (S = Q K^T) -- two issuing threads on different SM sub-partitions,
+// because one thread alone spends more time on commits and waits than the
+// tensor core spends on the MMAs -- 19 = spare, 2..17 = element warps in two
+// groups of eight; group g takes the units with U % 2 == g, so the two
+// groups run half a unit out of phase.  Element warp
+// w reaches TMEM lanes 32*(w%4)..+31 (query rows); in each group two warps
+// share those rows and split a unit's 64 columns, so each query row is
+// served by four threads (two per group) whose row statistics are merged
+// through shared memory.  O and O_L leave through shared memory and TMA
+// stores.
 #pragma once
 #include "kia_fast.cuh"
 #include "kia_tc.cuh"
@@ -25,31 +37,41 @@
 namespace kia {
 
 constexpr int kRowSplit = 4;        // element threads per TMEM lane (row)
-constexpr int kElemThreads = 128 * kRowSplit;   // 16 element warps
-constexpr int kTcThreads = kElemThreads + 64;   // + producer + MMA warp
+constexpr int kElemThreads = 128 * kRowSplit;   // 16 element warps (warps 2..17)
+constexpr int kGroupThreads = kElemThreads / 2; // element threads of one group
+constexpr int kScoreWarp = 2 + kElemThreads / 32;   // warp 18: issues the score MMAs
+// + TMA producer (warp 0), accumulating-MMA issuer (warp 1), score-MMA issuer
+// (warp 18) and one spare warp, so that every SM sub-partition holds five
+// warps (the register budget is set by the busiest sub-partition anyway)
+constexpr int kTcThreads = kElemThreads + 128;
 
-template <int D>
+template <int D, bool PROB>
 struct FwdCfg {
-  static constexpr int kStages = (D == 64) ? 2 : 1;      // K and V ring depth
+  static constexpr int kKStages = (D == 64) ? 3 : 1;     // K ring depth
+  static constexpr int kVStages = (D == 64) ? 2 : 1;     // V ring depth
   static constexpr uint32_t kTileBytes = D * KIA_TILE * 4;
+  // TMEM regions of 128 columns left beside O (and O_L), at most 3
+  static constexpr int kAccCols = PROB ? 2 * D : D;
+  static constexpr int kRegions = (512 - kAccCols) / 128 < 3 ? (512 - kAccCols) / 128 : 3;
+  static_assert(kRegions >= 2, "two TMEM regions at least");
 };
 
 struct FwdBars {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2];
+  uint64_t k_full[3], k_empty[3];
   uint64_t v_full[2], v_empty[2];
-  uint64_t s_full[2];    // S tile ready in TMEM buffer b (tcgen05.commit)
-  uint64_t s_free[2];    // sweep 1: element warps done reading buffer b
-  uint64_t p_ready[2];   // sweep 2: P written into buffer b
-  uint64_t pv_done[2];   // sweep 2: P V of buffer b finished (tcgen05.commit)
-  uint64_t pl_free;      // P_L consumed by O_L += P_L V (tcgen05.commit)
+  uint64_t s_full[3];    // S of a unit ready in region r (tcgen05.commit)
+  uint64_t s_free[3];    // sweep 1: the unit's group done reading region r
+  uint64_t p_ready[3];   // sweep 2: P (and P_L) written into region r
+  uint64_t pv_done[3];   // sweep 2: P V of region r finished (tcgen05.commit)
   uint64_t o_full;       // all P V done
+  uint64_t out_ready;    // O (and O_L) staged in shared memory
   uint64_t row_sync;     // element-thread rendezvous, used 3 times
   uint32_t tmem_base;
   int abort;
 };
 
-// Shared-memory scratch of the element warps: per-column-group row statistics.
+// Shared-memory scratch of the element warps: per-thread row statistics.
 struct FwdRowX {
   float m[kRowSplit][KIA_TILE];
   float n[kRowSplit][KIA_TILE];
@@ -62,18 +84,19 @@ struct FwdRowX {
 template <int D, class V>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, StatsView st,
-              OpParams p, int B, int H, int T, int nsb, int tab_in_smem) {
-  using Cfg = FwdCfg<D>;
-  constexpr int NS = Cfg::kStages;
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const __grid_constant__ CUtensorMap tmOL, StatsView st, OpParams p, int B, int H,
+              int T, int tab_in_smem) {
   constexpr bool PROB = V::PROB;
+  using Cfg = FwdCfg<D, PROB>;
+  constexpr int NSK = Cfg::kKStages, NSV = Cfg::kVStages, R = Cfg::kRegions;
+  constexpr uint32_t kTileF = Cfg::kTileBytes / 4;     // floats per operand tile
   extern __shared__ uint8_t smraw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
   float* sQ = reinterpret_cast<float*>(base);
-  float* sK = reinterpret_cast<float*>(base + Cfg::kTileBytes);
-  float* sV = reinterpret_cast<float*>(base + (1 + NS) * Cfg::kTileBytes);
-  FwdRowX& rx = *reinterpret_cast<FwdRowX*>(base + (1 + 2 * NS) * Cfg::kTileBytes);
+  float* sK = sQ + kTileF;
+  float* sV = sK + NSK * kTileF;
+  FwdRowX& rx = *reinterpret_cast<FwdRowX*>(sV + NSV * kTileF);
   float* sTab = reinterpret_cast<float*>(&rx + 1);
   const int tab_floats =
       V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
@@ -84,25 +107,27 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   const int qt = nt - 1 - blockIdx.y;
   const int nkt = p.causal ? qt + 1 : nt;
-  // TMEM columns: S buffers [0, 128*nsb), P_L, O, O_L
-  const uint32_t col_pl = 128u * nsb;
-  const uint32_t col_o = col_pl + (PROB ? 128u : 0u);
-  const uint32_t col_ol = col_o + D;
+  const int nunits = 2 * nkt;          // half key tiles per sweep
+  // TMEM columns: region r = [128 r, 128 r + 128); then O and O_L (D each)
+  constexpr uint32_t col_o = 128u * R;
+  constexpr uint32_t col_ol = col_o + D;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(&bar.k_full[s], 1);
       mbar_init(&bar.k_empty[s], 1);
-      mbar_init(&bar.v_full[s], 1);
-      mbar_init(&bar.v_empty[s], 1);
       mbar_init(&bar.s_full[s], 1);
-      mbar_init(&bar.s_free[s], kElemThreads);
-      mbar_init(&bar.p_ready[s], kElemThreads);
+      mbar_init(&bar.s_free[s], kGroupThreads);
+      mbar_init(&bar.p_ready[s], kGroupThreads);
       mbar_init(&bar.pv_done[s], 1);
     }
-    mbar_init(&bar.pl_free, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
+    }
     mbar_init(&bar.o_full, 1);
+    mbar_init(&bar.out_ready, kElemThreads);
     mbar_init(&bar.row_sync, kElemThreads);
     bar.abort = 0;
     fence_barrier_init();
@@ -131,19 +156,19 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       for (int sweep = 0; sweep < 2 && !failed; ++sweep) {
         for (int j = 0; j < nkt; ++j) {
           {
-            const int s = kc % NS, n = kc / NS;
+            const int s = kc % NSK, n = kc / NSK;
             if (!mbar_wait(&bar.k_empty[s], (n & 1) ^ 1, abort)) { failed = true; break; }
             mbar_arrive_expect_tx(&bar.k_full[s], Cfg::kTileBytes);
-            float* dst = sK + s * (Cfg::kTileBytes / 4);
+            float* dst = sK + s * kTileF;
             for (int b = 0; b < D / 32; ++b)
               tma_load_3d(dst + b * 32 * KIA_TILE, &tmK, &bar.k_full[s], b * 32, j * KIA_TILE, bh);
             ++kc;
           }
           if (sweep == 1) {
-            const int s = vc % NS, n = vc / NS;
+            const int s = vc % NSV, n = vc / NSV;
             if (!mbar_wait(&bar.v_empty[s], (n & 1) ^ 1, abort)) { failed = true; break; }
             mbar_arrive_expect_tx(&bar.v_full[s], Cfg::kTileBytes);
-            float* dst = sV + s * (Cfg::kTileBytes / 4);
+            float* dst = sV + s * kTileF;
             for (int b = 0; b < D / 32; ++b)
               tma_load_3d(dst + b * 32 * KIA_TILE, &tmV, &bar.v_full[s], b * 32, j * KIA_TILE, bh);
             ++vc;
@@ -151,107 +176,109 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     }
-  } else if (warp == 1) {
-    // --------------------------------------------------------- MMA issuer
+  } else if (warp == kScoreWarp) {
+    // ------------------------------------------------- score-MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_tf32(128, 128, 0, 0);
-      const uint32_t idesc_o = idesc_tf32(128, D, 0, 1);
-      const uint32_t qa = smem_u32(sQ);
-      int kc = 0, vc = 0;
-      int use1[2] = {0, 0};   // sweep-1 uses of each S buffer
-      int use2[2] = {0, 0};   // sweep-2 uses of each S buffer
+      const uint32_t idesc_s = idesc_tf32(128, 64, 0, 0);
+      // descriptors built once; each MMA only adds a constant step
+      const uint64_t dq0 = desc_kmajor(smem_u32(sQ), 0);
+      const uint64_t dk0 = desc_kmajor(smem_u32(sK), 0);
+      int kc = 0;
+      uint32_t pv_par = 0;                // per-region phase bits of the pv_done waits
       failed = !mbar_wait(&bar.q_full, 0, abort);
-      // issue S = Q K_j^T into buffer j % nsb
-      auto issue_s = [&](int sweep, int j) -> bool {
-        const int b = j % nsb;
-        if (sweep == 0) {
-          if (use1[b] > 0 && !mbar_wait(&bar.s_free[b], (use1[b] - 1) & 1, abort)) return false;
-          ++use1[b];
-        } else {
-          if (use2[b] == 0) {
-            if (use1[b] > 0 && !mbar_wait(&bar.s_free[b], (use1[b] - 1) & 1, abort)) return false;
-          } else if (!mbar_wait(&bar.pv_done[b], (use2[b] - 1) & 1, abort)) {
-            return false;
+      // S of unit U (sweep U / nunits, keys 64 (U % nunits) ..) into region
+      // U % R, once the unit R before it has released the region
+      const int total = 2 * nunits;
+      for (int U = 0; U < total && !failed; ++U) {
+        const int r = U % R, prev = U - R;
+        if (prev >= 0) {
+          if (prev < nunits) {
+            if (!mbar_wait(&bar.s_free[r], (prev / R) & 1, abort)) { failed = true; break; }
+          } else {
+            if (!mbar_wait(&bar.pv_done[r], (pv_par >> r) & 1u, abort)) { failed = true; break; }
+            pv_par ^= 1u << r;
           }
-          ++use2[b];
         }
-        const int s = kc % NS, n = kc / NS;
-        if (!mbar_wait(&bar.k_full[s], n & 1, abort)) return false;
+        const int h = U & 1;              // half of the key tile
+        const int s = kc % NSK, n = kc / NSK;
+        if (h == 0 && !mbar_wait(&bar.k_full[s], n & 1, abort)) { failed = true; break; }
         tc_fence_after();
-        const uint32_t ka = smem_u32(sK + s * (Cfg::kTileBytes / 4));
+        const uint64_t dk = dk0 + desc_step((uint32_t)s * Cfg::kTileBytes + (uint32_t)h * 64u * 128u);
+        const uint32_t dst = tmem + 128u * r;
 #pragma unroll
         for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(tmem + 128u * b, desc_kmajor(qa, ks), desc_kmajor(ka, ks), idesc_s,
-                      ks > 0 ? 1u : 0u);
-        tc_commit(&bar.s_full[b]);
-        tc_commit(&bar.k_empty[s]);
-        ++kc;
-        return true;
-      };
-      if (!failed) {
-        for (int j = 0; j < nkt; ++j)
-          if (!issue_s(0, j)) { failed = true; break; }
-      }
-      if (!failed) {
-        int pr[2] = {0, 0};
-        if (!issue_s(1, 0)) failed = true;
-        for (int j = 0; j < nkt && !failed; ++j) {
-          // two S buffers: the next S overlaps this tile's weights and P V;
-          // one buffer: the next S must wait until P V has read P
-          if (nsb == 2 && j + 1 < nkt && !issue_s(1, j + 1)) { failed = true; break; }
-          const int b = j % nsb;
-          if (!mbar_wait(&bar.p_ready[b], pr[b] & 1, abort)) { failed = true; break; }
-          ++pr[b];
-          const int s = vc % NS, n = vc / NS;
-          if (!mbar_wait(&bar.v_full[s], n & 1, abort)) { failed = true; break; }
-          tc_fence_after();
-          const uint32_t va = smem_u32(sV + s * (Cfg::kTileBytes / 4));
-#pragma unroll
-          for (int ks = 0; ks < KIA_TILE / 8; ++ks)
-            mma_tf32_ts(tmem + col_o, tmem + 128u * b + 8u * ks, desc_mnmajor(va, ks), idesc_o,
-                        (j > 0 || ks > 0) ? 1u : 0u);
-          if constexpr (PROB) {
-#pragma unroll
-            for (int ks = 0; ks < KIA_TILE / 8; ++ks)
-              mma_tf32_ts(tmem + col_ol, tmem + col_pl + 8u * ks, desc_mnmajor(va, ks), idesc_o,
-                          (j > 0 || ks > 0) ? 1u : 0u);
-            tc_commit(&bar.pl_free);
-          }
-          tc_commit(&bar.v_empty[s]);
-          tc_commit(&bar.pv_done[b]);
-          ++vc;
-          if (nsb == 1 && j + 1 < nkt && !issue_s(1, j + 1)) { failed = true; break; }
+          mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_s, ks > 0 ? 1u : 0u);
+        tc_commit(&bar.s_full[r]);
+        if (h == 1) {
+          tc_commit(&bar.k_empty[s]);
+          ++kc;
         }
-        if (!failed) tc_commit(&bar.o_full);
       }
     }
-  } else {
+  } else if (warp == 1) {
+    // ------------------------------------------- accumulating-MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_o = idesc_tf32(128, D, 0, 1);
+      const uint64_t dv0 = desc_mnmajor(smem_u32(sV), 0);
+      int vc = 0;
+      uint32_t pr_par = 0;                // per-region phase bits of the p_ready waits
+      for (int u = 0; u < nunits && !failed; ++u) {
+        const int U = nunits + u, r = U % R, h = u & 1;
+        if (!mbar_wait(&bar.p_ready[r], (pr_par >> r) & 1u, abort)) { failed = true; break; }
+        pr_par ^= 1u << r;
+        const int s = vc % NSV, n = vc / NSV;
+        if (h == 0 && !mbar_wait(&bar.v_full[s], n & 1, abort)) { failed = true; break; }
+        tc_fence_after();
+        const uint64_t dv = dv0 + desc_step((uint32_t)s * Cfg::kTileBytes) + kstep_mnmajor(8 * h);
+        const uint32_t pa = tmem + 128u * r;
+        const uint32_t acc0 = u > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_tf32_ts(tmem + col_o, pa + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
+                      kk > 0 ? 1u : acc0);
+        if constexpr (PROB) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_tf32_ts(tmem + col_ol, pa + 64u + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
+                        kk > 0 ? 1u : acc0);
+        }
+        tc_commit(&bar.pv_done[r]);
+        if (h == 1) {
+          tc_commit(&bar.v_empty[s]);
+          ++vc;
+        }
+      }
+      if (!failed) tc_commit(&bar.o_full);
+    }
+  } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;          // which 32 columns of a tile
+    const int part = (warp - 2) >> 2;          // 0..3: (group, half of the unit)
+    const int grp = part >> 1;                 // units U with U % 2 == grp
+    const int sub = part & 1;                  // columns 32 sub .. 32 sub + 31 of a unit
     const int r = quad * 32 + lane;            // query row in the tile
     const int qrow = qt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const uint32_t col0 = 32u * part;
     const long long grow = (long long)bh * T + (qrow < T ? qrow : T - 1);
-    int sf[2] = {0, 0};  // completed phases of s_full per buffer
+    // a unit holds masked keys when it reaches past the first row of the
+    // tile (causal) or past the sequence end
+    const int edge_from = p.causal ? (qt * KIA_TILE) / 64 : nunits;
+    auto is_edge = [&](int u) { return u >= edge_from || (u + 1) * 64 > T; };
     // row extrema and the keys of their first occurrences
     float m = -INFINITY, n = INFINITY;
     int am = 0, an = 0;
-    float v[32];
-    // sweep 1: statistics of this thread's 32 columns of each tile
-    for (int j = 0; j < nkt; ++j) {
-      const int b = j % nsb;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
-      ++sf[b];
+    // sweep 1: statistics of this thread's 32 columns of each of its units
+    for (int U = grp; U < nunits; U += 2) {
+      const int rg = U % R;
+      float v[32];
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[rg], (U / R) & 1, abort))) { failed = true; break; }
       tc_fence_after();
-      const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
-      tmem_ld32(tmem + lane_addr + 128u * b + col0, v);
-      tmem_ld_wait();
+      tmem_ld32(tmem + lane_addr + 128u * rg + 32u * sub, v);
+      tmem_ld_wait_regs(v);
       tc_fence_before();
-      mbar_arrive(&bar.s_free[b]);
-      const int key0 = j * KIA_TILE + (int)col0;
-      if (!edge) {
+      mbar_arrive(&bar.s_free[rg]);
+      const int key0 = 64 * U + 32 * sub;
+      if (!is_edge(U)) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           // strict comparisons keep the lowest index on ties
@@ -278,7 +305,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     }
-    // merge the four column groups of the row (lowest index on ties)
+    // merge the four threads of the row (lowest index on ties)
     rx.m[part][r] = m;
     rx.n[part][r] = n;
     rx.am[part][r] = am;
@@ -338,24 +365,18 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // sweep 2: weights -> P (and P_L) in TMEM, normalisers
     float W = 0.0f, WL = 0.0f;
     auto sweep2 = [&](auto grid) {
-      for (int j = 0; j < nkt && !failed; ++j) {
-        const int b = j % nsb;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], sf[b] & 1, abort))) { failed = true; break; }
-        ++sf[b];
-        if (PROB && j > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait(&bar.pl_free, (j - 1) & 1, abort))) {
-          failed = true;
-          break;
-        }
+      for (int u = grp; u < nunits && !failed; u += 2) {
+        const int U = nunits + u, rg = U % R;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[rg], (U / R) & 1, abort))) { failed = true; break; }
         tc_fence_after();
-        const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
+        const bool edge = is_edge(u);
+        const uint32_t col_s = 128u * rg + 32u * sub;   // this thread's S / P columns
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
-          const uint32_t col = col0 + 16u * c;
           float w16[16], vl[16];
-          tmem_ld16(tmem + lane_addr + 128u * b + col, w16);
-          tmem_ld_wait();
-          const int key0 = j * KIA_TILE + (int)col;
+          tmem_ld16(tmem + lane_addr + col_s + 16u * c, w16);
+          tmem_ld_wait_regs(w16);
+          const int key0 = 64 * u + 32 * sub + 16 * c;
           if (!edge) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -385,12 +406,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               }
             }
           }
-          tmem_st16(tmem + lane_addr + 128u * b + col, w16);
-          if constexpr (PROB) tmem_st16(tmem + lane_addr + col_pl + col, vl);
+          tmem_st16(tmem + lane_addr + col_s + 16u * c, w16);
+          if constexpr (PROB) tmem_st16(tmem + lane_addr + col_s + 64u + 16u * c, vl);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bar.p_ready[b]);
+        mbar_arrive(&bar.p_ready[rg]);
       }
     };
     if constexpr (V::MINMAX) {
@@ -407,26 +428,32 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const float Wrow = (rx.W[0][r] + rx.W[1][r]) + (rx.W[2][r] + rx.W[3][r]);
     const float WLrow =
         PROB ? (rx.WL[0][r] + rx.WL[1][r]) + (rx.WL[2][r] + rx.WL[3][r]) : Wrow;
-    // epilogue: this thread writes D/4 columns of its row
-    if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.o_full, 0, abort))) {
+    // epilogue: this thread stages D/4 columns of its row of O (and O_L) in
+    // the free K ring, laid out as the TMA store's 128-byte swizzle expects
+    // (16-byte chunk c of row r at chunk c ^ (r % 8)); one thread stores
+    const bool out_ok = !failed && __all_sync(0xffffffffu, mbar_wait(&bar.o_full, 0, abort));
+    float* sO = sK;                       // [D / 32][128 rows][32] per output
+    if (out_ok) {
       tc_fence_after();
       constexpr int kCols = D / kRowSplit;     // 16 or 32
       const uint32_t col = (uint32_t)(part * kCols);
       float o[kCols];
-      auto write_row = [&](uint32_t tcol, float* dst, float w) {
+      auto stage_row = [&](uint32_t tcol, float* dst, float w) {
         if constexpr (kCols == 16) tmem_ld16(tmem + lane_addr + tcol + col, o);
         else tmem_ld32(tmem + lane_addr + tcol + col, o);
-        tmem_ld_wait();
-        if (qrow < T) {
-          float4* o4 = reinterpret_cast<float4*>(dst + grow * D + col);
+        tmem_ld_wait_regs(o);
+        const float rw = __frcp_rn(w);
+        float* blk = dst + (col / 32) * (32 * KIA_TILE) + r * 32;
+        const int c0 = (col % 32) / 4;        // first 16-byte chunk in the 128-byte row
 #pragma unroll
-          for (int i = 0; i < kCols / 4; ++i)
-            o4[i] = make_float4(__fdiv_rn(o[4 * i], w), __fdiv_rn(o[4 * i + 1], w),
-                                __fdiv_rn(o[4 * i + 2], w), __fdiv_rn(o[4 * i + 3], w));
+        for (int i = 0; i < kCols / 4; ++i) {
+          const int ch = (c0 + i) ^ (r & 7);
+          *reinterpret_cast<float4*>(blk + ch * 4) =
+              make_float4(o[4 * i] * rw, o[4 * i + 1] * rw, o[4 * i + 2] * rw, o[4 * i + 3] * rw);
         }
       };
-      write_row(col_o, O, Wrow);
-      if constexpr (PROB) write_row(col_ol, st.OL, WLrow);
+      stage_row(col_o, sO, Wrow);
+      if constexpr (PROB) stage_row(col_ol, sO + D * KIA_TILE, WLrow);
       if (qrow < T && part == 0) {
         st.m[grow] = m;
         st.n[grow] = n;
@@ -441,6 +468,19 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     } else {
       failed = true;
     }
+    fence_proxy_async_smem();
+    mbar_arrive(&bar.out_ready);
+    if (threadIdx.x == 64) {
+      if (mbar_wait(&bar.out_ready, 0, abort) && !*abort) {
+        for (int b = 0; b < D / 32; ++b) {
+          tma_store_3d(&tmO, sO + b * 32 * KIA_TILE, b * 32, qt * KIA_TILE, bh);
+          if constexpr (PROB)
+            tma_store_3d(&tmOL, sO + D * KIA_TILE + b * 32 * KIA_TILE, b * 32, qt * KIA_TILE, bh);
+        }
+        tma_store_commit();
+        tma_store_wait_all();
+      }
+    }
   }
   if (failed || *abort) drain_in_flight();
   tc_fence_before();
@@ -448,35 +488,36 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D>
+template <int D, bool PROB>
 size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem) {
-  constexpr int NS = FwdCfg<D>::kStages;
+  using Cfg = FwdCfg<D, PROB>;
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
-  return 1024 + (size_t)(1 + 2 * NS) * FwdCfg<D>::kTileBytes + sizeof(FwdRowX) +
+  return 1024 + (size_t)(1 + Cfg::kKStages + Cfg::kVStages) * Cfg::kTileBytes + sizeof(FwdRowX) +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
 }
 
 template <int D, class V>
 int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, float* O,
                  const StatsView& st, int B, int H, int T, const OpParams& p, cudaStream_t s) {
+  CUtensorMap to, tol;
+  if (!make_tmap(&to, O, B * H, T, D) ||
+      !make_tmap(&tol, V::PROB ? st.OL : O, B * H, T, D))
+    return KIA_ERR_CUDA;
   bool tab_in_smem = true;
-  size_t smem = tc_fwd_smem<D>(p, true);
+  size_t smem = tc_fwd_smem<D, V::PROB>(p, true);
   if (smem > 232448) {
     tab_in_smem = false;
-    smem = tc_fwd_smem<D>(p, false);
+    smem = tc_fwd_smem<D, V::PROB>(p, false);
   }
   if (smem > 232448) return KIA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(tc_fwd_kernel<D, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return KIA_ERR_CUDA;
-  // TMEM: S buffers (128 columns each), P_L (128, Prob-STE), O and O_L (D each)
-  int nsb = 2;
-  if (256 + (V::PROB ? 128 + 2 * D : D) > 512) nsb = 1;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   dim3 grid(B * H, nt);
-  tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, O, st, p, B, H, T, nsb,
+  tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, to, tol, st, p, B, H, T,
                                                      tab_in_smem ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
 }

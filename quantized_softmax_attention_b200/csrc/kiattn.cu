@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -84,16 +86,22 @@ OpParams make_params(const kia_config* cfg) {
   return p;
 }
 
-int launch_status() {
-  const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
+// With KIATTN_DEBUG set in the environment, a failed CUDA call prints the
+// runtime's message to stderr; the return code is KIA_ERR_CUDA either way.
+int cuda_fail(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return KIA_OK;
+  if (getenv("KIATTN_DEBUG")) fprintf(stderr, "kiattn: %s: %s\n", where, cudaGetErrorString(e));
+  return KIA_ERR_CUDA;
 }
+
+int launch_status() { return cuda_fail(cudaGetLastError(), "kernel launch"); }
 
 template <typename Kern>
 int set_smem(Kern k, size_t bytes) {
   if (bytes > 48 * 1024) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
-        cudaSuccess)
+    if (cuda_fail(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bytes),
+                  "shared memory attribute"))
       return KIA_ERR_CUDA;
   }
   return KIA_OK;
