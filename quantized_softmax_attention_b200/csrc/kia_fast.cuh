@@ -209,7 +209,8 @@ __device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, flo
 }
 
 // Backward of one element in the key pass: the forward probability P (for
-// dV) and the detached dS (for dK), from one grid position.
+// dV) and the detached dS (for dK), from one grid position.  FWM's tail
+// (u > K) has zero weight and zero slope.
 template <class V, class G>
 __device__ __forceinline__ void kv_elem(const G& grid, float m, float rh, float dg, float rWf,
                                         float Kf, float Km1f, float s, float dw, float& P,
@@ -220,20 +221,20 @@ __device__ __forceinline__ void kv_elem(const G& grid, float m, float rh, float 
     dS = w * dw;
   } else {
     const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
-    float2 g = grid.pair(p.k);
-    float wf = V::NEAREST ? ((p.t >= 0.5f) ? g.y : g.x) : __fmaf_rn(p.t, __fsub_rn(g.y, g.x), g.x);
-    if constexpr (V::FWM) {
-      const bool tail = p.u > Kf;
-      g.x = tail ? 0.0f : g.x;
-      g.y = tail ? 0.0f : g.y;
-      wf = tail ? 0.0f : wf;
-    }
+    const float2 g = grid.pair(p.k);
+    const float a = __fsub_rn(g.y, g.x);
+    const float wf = V::NEAREST ? ((p.t >= 0.5f) ? g.y : g.x) : __fmaf_rn(p.t, a, g.x);
     P = wf * rWf;
-    const float da = dw * __fsub_rn(g.y, g.x);
+    const float da = dw * a;
     if constexpr (V::MINMAX) {
       dS = fmaf(dw, dg, -(da * rh));
     } else {
       dS = -(da * rh);
+    }
+    if constexpr (V::FWM) {
+      const bool tail = p.u > Kf;
+      P = tail ? 0.0f : P;
+      dS = tail ? 0.0f : dS;
     }
   }
 }

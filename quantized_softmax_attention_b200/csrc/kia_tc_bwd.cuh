@@ -35,7 +35,7 @@
 
 namespace kia {
 
-constexpr int kBwdSmemTabK = 32;  // key pass: per-query grids up to K = 32 in shared memory
+constexpr int kBwdSmemTabK = 16;  // key pass: per-query grids up to K = 16 in shared memory
 constexpr int kBwdRegions = 3;    // TMEM regions of 128 columns (S | dP) in rotation
 
 struct BwdQBars {
@@ -56,8 +56,8 @@ struct BwdKBars {
   uint64_t qd_full, qd_empty;     // Q_i, dO_i K-major (for S^T, dP^T)
   uint64_t mn_full, mn_empty;     // Q_i, dO_i MN-major (for dK, dV)
   uint64_t sp_full[3];            // S^T and dP^T of a half tile in TMEM region r
-  uint64_t qc_ready[2];           // per-query constants of group g's unit loaded
-  uint64_t qc_free[2];            // group g done with its unit's constants
+  uint64_t qc_ready[4];           // per-query constants of a unit loaded into slot s
+  uint64_t qc_free[4];            // the unit's group done with slot s
   uint64_t elem_done[3];          // P^T, dS^T written into region r
   uint64_t st_free[3];            // dV, dK MMAs of region r done
   uint64_t acc_full;              // all dV, dK MMAs done
@@ -295,6 +295,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_arrive(&bar.row_sync);
     if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
     const float Dc = sDc[r];
+    const float nDr = -Dc * rWb;            // dw = (dP - D) / W_bar as one fma
     float A = 0.0f, C = 0.0f;
     for (int u = grp; u < nunits && !failed; u += 2) {
       const int j = u >> 1, rg = u % R;
@@ -312,7 +313,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!edge) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float dw = (g[i] - Dc) * rWb;
+            const float dw = fmaf(g[i], rWb, nDr);
             v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
           }
         } else {
@@ -320,7 +321,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int i = 0; i < 16; ++i) {
             const int key = key0 + i;
             const bool ok = key < T && (!p.causal || key <= q);
-            const float dw = ok ? (g[i] - Dc) * rWb : 0.0f;
+            const float dw = ok ? fmaf(g[i], rWb, nDr) : 0.0f;
             v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
           }
         }
@@ -436,12 +437,22 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float* sG = reinterpret_cast<float*>(base + 3 * kTile);
   float* sQmn = reinterpret_cast<float*>(base + 4 * kTile);
   float* sGmn = reinterpret_cast<float*>(base + 5 * kTile);
-  float4* sC4 = reinterpret_cast<float4*>(base + 6 * kTile);  // (m, rh, D, rWb) per query
-  float4* sCA = sC4 + KIA_TILE;                               // (rWf, dg, g_m or c, g_n)
-  int2* sCI = reinterpret_cast<int2*>(sCA + KIA_TILE);         // argmax, argmin keys - tile start
-  float* sTab = reinterpret_cast<float*>(sCI + KIA_TILE);
+  // Per-query constants of a unit (64 queries) in four slots, filled ahead of
+  // the element groups by the constant warp: unit u uses slot
+  // 2 (u % 2) + (u / 2) % 2.
+  constexpr int kSlots = 4, kSlotQ = 64;
+  float4* sC4 = reinterpret_cast<float4*>(base + 6 * kTile);  // (m, rh, rWb, -D rWb)
+  float2* sC2 = reinterpret_cast<float2*>(sC4 + kSlots * kSlotQ);  // (rWf, dg or projection shift c)
+  // calibration terms, read only where a query's argmax (argmin) key is this
+  // thread's key: key - tile start, and the coefficient
+  int2* sCI = reinterpret_cast<int2*>(sC2 + kSlots * kSlotQ);  // (argmax, argmin) - kt * 128
+  float2* sCG = reinterpret_cast<float2*>(sCI + kSlots * kSlotQ);  // (g_m, g_n)
+  // which queries of a unit have their argmax (argmin) key in lanes
+  // 32 quad..32 quad + 31: [slot][argmax / argmin][quad][query half]
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sCG + kSlots * kSlotQ);
+  float* sTab = reinterpret_cast<float*>(sMask + kSlots * 2 * 4 * 2);   // [slot][64][K + 1]
   const int K1 = p.K + 1;
-  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? K1 * KIA_TILE : 0) : 4 * K1);
+  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? kSlots * kSlotQ * K1 : 0) : 4 * K1);
   BwdKBars& bar = *reinterpret_cast<BwdKBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -465,9 +476,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(&bar.elem_done[b], kGroupThreads);
       mbar_init(&bar.st_free[b], 1);
     }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&bar.qc_ready[g], kGroupThreads);
-      mbar_init(&bar.qc_free[g], kGroupThreads);
+    for (int sl = 0; sl < 4; ++sl) {
+      mbar_init(&bar.qc_ready[sl], 32);
+      mbar_init(&bar.qc_free[sl], kGroupThreads);
     }
     mbar_init(&bar.acc_full, 1);
     bar.abort = 0;
@@ -588,6 +599,95 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       if (!failed) tc_commit(&bar.acc_full);
     }
+  } else if (warp == kScoreWarp + 1) {
+    // -------------------------------------------- query-constant producer
+    // Loads the per-query constants of each unit into its slot while the
+    // element groups work on earlier units (lane l: queries l and l + 32).
+    const long long rowbase = (long long)bh * T;
+    // FWM: each group's copy of the shared grid's pairs, published with the
+    // first units' constants
+    if (!V::SOFTMAX && !V::MINMAX) {
+      for (int k = lane; k < p.K; k += 32) {
+        const float2 pr = make_float2(st.table[k], st.table[k + 1]);
+        reinterpret_cast<float2*>(sTab)[k] = pr;
+        reinterpret_cast<float2*>(sTab)[K1 + k] = pr;
+      }
+    }
+    // raw per-query values of one unit (lane l: queries l and l + 32), loaded
+    // one unit ahead so that their latency overlaps the wait for a free slot
+    struct Raw {
+      float m[2], rh[2], D[2], Wb[2], Wf[2], gm[2], gn[2];
+      int am[2], an[2];
+    };
+    auto load_raw = [&](int u, Raw& x) {
+      const int qi = q0 + (u >> 1);
+#pragma unroll
+      for (int hq = 0; hq < 2; ++hq) {
+        const int q = qi * KIA_TILE + 64 * (u & 1) + 32 * hq + lane;
+        const long long qr = rowbase + (q < T ? q : T - 1);
+        x.m[hq] = st.m[qr];
+        x.rh[hq] = st.rh[qr];
+        x.D[hq] = wk.D[qr];
+        x.Wb[hq] = st.Wb[qr];
+        x.Wf[hq] = st.Wf[qr];
+        x.gm[hq] = wk.gm[qr];
+        x.gn[hq] = V::MINMAX ? wk.gn[qr] : 0.0f;
+        x.am[hq] = PROJ ? 0 : wk.am[qr];
+        x.an[hq] = (V::MINMAX && !PROJ) ? wk.an[qr] : 0;
+      }
+    };
+    Raw cur;
+    if (nunits > 0) load_raw(0, cur);
+    for (int u = 0; u < nunits && !failed; ++u) {
+      const int sl = 2 * (u & 1) + ((u >> 1) & 1);
+      Raw nxt;
+      if (u + 1 < nunits) load_raw(u + 1, nxt);
+      if (u >= kSlots && !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[sl], ((u >> 2) - 1) & 1, abort))) {
+        failed = true;
+        break;
+      }
+      const int qi = q0 + (u >> 1);
+#pragma unroll
+      for (int hq = 0; hq < 2; ++hq) {
+        const int ql = 64 * (u & 1) + 32 * hq + lane;        // query in the tile
+        const int e = sl * kSlotQ + 32 * hq + lane;          // its slot entry
+        const int q = qi * KIA_TILE + ql;
+        const int Lq = p.causal ? q + 1 : T;
+        const float rWb = Lq == 1 ? 0.0f : __fdiv_rn(1.0f, cur.Wb[hq]);
+        sC4[e] = make_float4(cur.m[hq], cur.rh[hq], rWb, -cur.D[hq] * rWb);
+        // calibration terms of the query's row, added to dS^T before dK:
+        // g_m at the argmax key, g_n at the argmin key, or the projection
+        // shift c on every visible key
+        const bool live = q < T;
+        const float gm = live ? cur.gm[hq] : 0.0f, gn = live ? cur.gn[hq] : 0.0f;
+        sC2[e] = make_float2(__fdiv_rn(1.0f, cur.Wf[hq]),
+                             PROJ ? gm : ((V::MINMAX && cur.rh[hq] == 0.0f) ? 1.0f : 0.0f));
+        if constexpr (!PROJ && !V::SOFTMAX) {
+          const int ka = cur.am[hq] - kt * KIA_TILE;
+          const int kn = V::MINMAX ? cur.an[hq] - kt * KIA_TILE : -1;
+          sCI[e] = make_int2(ka, kn);
+          sCG[e] = make_float2(gm, gn);
+          const bool hit_m = gm != 0.0f && ka >= 0 && ka < KIA_TILE;
+          const bool hit_n = V::MINMAX && gn != 0.0f && kn >= 0 && kn < KIA_TILE;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            const uint32_t bm = __ballot_sync(0xffffffffu, hit_m && (ka >> 5) == qd);
+            const uint32_t bn = __ballot_sync(0xffffffffu, hit_n && (kn >> 5) == qd);
+            if (lane == 0) {
+              sMask[((sl * 2 + 0) * 4 + qd) * 2 + hq] = bm;
+              sMask[((sl * 2 + 1) * 4 + qd) * 2 + hq] = bn;
+            }
+          }
+        }
+        if (V::MINMAX && tab_in_smem) {
+          const long long qr = rowbase + (q < T ? q : T - 1);
+          for (int kk = 0; kk < K1; ++kk) sTab[e * K1 + kk] = st.table[qr * K1 + kk];
+        }
+      }
+      __syncwarp();
+      mbar_arrive(&bar.qc_ready[sl]);
+      cur = nxt;
+    }
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
@@ -595,47 +695,18 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int grp = part >> 1;               // half tiles u with u % 2 == grp
     const int sub = part & 1;                // query columns 32 sub .. 32 sub + 31 of a unit
     const int r = quad * 32 + lane;
-    const int eg = ((int)threadIdx.x - 64) & (kGroupThreads - 1);   // thread of the group
     const int kj = kt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const long long rowbase = (long long)bh * T;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     // FWM: each group keeps its own copy of the shared grid's pairs
     const float2* sPairG = reinterpret_cast<const float2*>(sTab) + grp * K1;
-    if (!V::SOFTMAX && !V::MINMAX && eg < p.K)
-      reinterpret_cast<float2*>(sTab)[grp * K1 + eg] = make_float2(st.table[eg], st.table[eg + 1]);
     for (int u = grp; u < nunits && !failed; u += 2) {
       const int s = u >> 1;
       const int qi = q0 + s;
       const int rg = u % R;
-      // per-query constants of this unit's 64 queries (the group's own half
-      // of the arrays), once every thread of the group is done with its
-      // previous unit
-      if (u >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[grp], (s - 1) & 1, abort))) {
-        failed = true;
-        break;
-      }
-      if (eg < 64) {
-        const int ql = 64 * grp + eg;
-        const int q = qi * KIA_TILE + ql;
-        const long long qr = rowbase + (q < T ? q : T - 1);
-        const float rhq = st.rh[qr];
-        const int Lq = p.causal ? q + 1 : T;
-        sC4[ql] = make_float4(st.m[qr], rhq, wk.D[qr], Lq == 1 ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]));
-        // calibration terms of the query's row, added to dS^T before dK:
-        // g_m at the argmax key, g_n at the argmin key, or the projection
-        // shift c on every visible key
-        const bool live = q < T;
-        sCA[ql] = make_float4(__fdiv_rn(1.0f, st.Wf[qr]), (V::MINMAX && rhq == 0.0f) ? 1.0f : 0.0f,
-                              live ? wk.gm[qr] : 0.0f, live ? wk.gn[qr] : 0.0f);
-        sCI[ql] = make_int2(PROJ ? -1 : wk.am[qr] - kt * KIA_TILE,
-                            PROJ ? -1 : wk.an[qr] - kt * KIA_TILE);
-        if (V::MINMAX && tab_in_smem)
-          for (int k = 0; k < K1; ++k) sTab[ql * K1 + k] = st.table[qr * K1 + k];
-      }
-      mbar_arrive(&bar.qc_ready[grp]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[grp], s & 1, abort))) { failed = true; break; }
+      const int sl = 2 * grp + ((u >> 1) & 1);           // this unit's constant slot
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[sl], (u >> 2) & 1, abort))) { failed = true; break; }
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (u / R) & 1, abort))) { failed = true; break; }
       tc_fence_after();
       const bool edge =
@@ -648,28 +719,26 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tmem_ld16(tmem + lane_addr + cs + 64u, g);
         tmem_ld_wait_regs(v, g);
         const int ql0 = 64 * grp + 32 * sub + 16 * c;   // first query (in the tile) of the chunk
+        const int e0 = sl * kSlotQ + 32 * sub + 16 * c;  // its slot entry
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int ql = ql0 + i;
-          const float4 c4 = sC4[ql];
-          const float4 ca = sCA[ql];
-          const float dw = (g[i] - c4.z) * c4.w;
+          const float4 c4 = sC4[e0 + i];
+          const float2 c2 = sC2[e0 + i];
+          const float dw = fmaf(g[i], c4.z, c4.w);
           float P, dS;
           if constexpr (V::MINMAX) {
-            const GridF grid{tab_in_smem ? sTab + ql * K1
+            const GridF grid{tab_in_smem ? sTab + (e0 + i) * K1
                                          : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
                              1};
-            kv_elem<V>(grid, c4.x, c4.y, ca.y, ca.x, Kf, Km1f, v[i], dw, P, dS);
+            // degenerate rows (rh = 0) take dS = dw; under the projection c2.y
+            // holds the shift, so the flag comes from rh itself
+            const float dg = PROJ ? (c4.y == 0.0f ? 1.0f : 0.0f) : c2.y;
+            kv_elem<V>(grid, c4.x, c4.y, dg, c2.x, Kf, Km1f, v[i], dw, P, dS);
           } else {
-            kv_elem<V>(GridP{sPairG}, c4.x, c4.y, ca.y, ca.x, Kf, Km1f, v[i], dw, P, dS);
+            kv_elem<V>(GridP{sPairG}, c4.x, c4.y, 0.0f, c2.x, Kf, Km1f, v[i], dw, P, dS);
           }
-          if constexpr (PROJ) {
-            dS += ca.z;
-          } else if constexpr (!V::SOFTMAX) {
-            const int2 ci = sCI[ql];
-            dS += (ci.x == r) ? ca.z : 0.0f;
-            if constexpr (V::MINMAX) dS += (ci.y == r) ? ca.w : 0.0f;
-          }
+          if constexpr (PROJ) dS += c2.y;
           if (edge) {
             const int q = qi * KIA_TILE + ql;
             if (!(kj < T && q < T && (!p.causal || kj <= q))) {
@@ -680,13 +749,32 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           v[i] = P;
           g[i] = dS;
         }
+        if constexpr (!PROJ && !V::SOFTMAX) {
+          // the chunk's queries whose argmax (argmin) key lies in this warp's
+          // 32 keys: a warp-uniform test, the per-element work only for them
+          const int sh = 16 * c;
+          const uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu;
+          const uint32_t bn =
+              V::MINMAX ? (sMask[((sl * 2 + 1) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu : 0u;
+          if ((bm | bn) != 0u) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if ((bm | bn) & (1u << i)) {
+                const int2 ci = sCI[e0 + i];
+                const float2 cg = sCG[e0 + i];
+                if ((bm >> i) & 1u) g[i] += (ci.x == r) ? cg.x : 0.0f;
+                if (V::MINMAX && ((bn >> i) & 1u)) g[i] += (ci.y == r) ? cg.y : 0.0f;
+              }
+            }
+          }
+        }
         tmem_st16(tmem + lane_addr + cs, v);
         tmem_st16(tmem + lane_addr + cs + 64u, g);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar.elem_done[rg]);
-      mbar_arrive(&bar.qc_free[grp]);
+      mbar_arrive(&bar.qc_free[sl]);
     }
     if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.acc_full, 0, abort))) {
       tc_fence_after();
@@ -727,8 +815,8 @@ template <int D>
 size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
-      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 4 * (p.K + 1));
-  return 1024 + 6 * (size_t)D * KIA_TILE * 4 + KIA_TILE * (16 + 16 + 8) +
+      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? 4 * 64 * (p.K + 1) : 0) : 4 * (p.K + 1));
+  return 1024 + 6 * (size_t)D * KIA_TILE * 4 + 4 * 64 * (16 + 8 + 8 + 8) + 4 * 2 * 4 * 2 * 4 +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdKBars);
 }
 
@@ -745,7 +833,7 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
       !make_tmap(&tv, Vv, BH, T, D))
     return KIA_ERR_CUDA;
   const size_t smq = tc_bwd_q_smem<D>(p);
-  const bool kv_tab_smem = p.K <= kBwdSmemTabK;
+  const bool kv_tab_smem = p.K <= kBwdSmemTabK && tc_bwd_kv_smem<D>(p, true) <= 232448;
   const size_t smk = tc_bwd_kv_smem<D>(p, kv_tab_smem);
   if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
   const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
