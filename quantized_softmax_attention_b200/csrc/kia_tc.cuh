@@ -41,16 +41,29 @@ inline EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [BH, T, d] fp32 tensor; box = 32 columns x 128 rows x 1, 128-byte swizzle
+// Number of SMs of the current device (cached per device; 0 on error).
+inline int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// [BH, T, d] fp32 tensor; box = 32 columns x box_rows rows x 1, 128-byte swizzle
 // (16-byte atoms for K-major use, 32-byte atoms for MN-major use),
 // out-of-range rows read as zero.
 inline bool make_tmap(CUtensorMap* m, const float* base, int BH, int T, int d,
-                      bool mn_major = false) {
+                      bool mn_major = false, int box_rows = KIA_TILE) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)T * d * 4};
-  cuuint32_t box[3] = {32, KIA_TILE, 1};
+  cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -85,6 +98,19 @@ __host__ __device__ constexpr uint64_t kstep_kmajor(int ks) {
 }
 // MN-major: K step ks = rows 8ks..8ks+7
 __host__ __device__ constexpr uint64_t kstep_mnmajor(int ks) { return desc_step((uint32_t)ks * 1024u); }
+
+// Half tiles (64 rows, loaded with a 64-row box): column blocks are 8 KB
+// apart instead of 16 KB.
+constexpr uint32_t kHalfBlockBytes = 64 * 128;
+__device__ __forceinline__ uint64_t desc_kmajor_half(uint32_t tile) {
+  return smem_desc(tile, 16u, 1024u, kLayoutSW128);
+}
+__host__ __device__ constexpr uint64_t kstep_kmajor_half(int ks) {
+  return desc_step((uint32_t)(ks >> 2) * kHalfBlockBytes + (uint32_t)(ks & 3) * 32u);
+}
+__device__ __forceinline__ uint64_t desc_mnmajor_half(uint32_t tile) {
+  return smem_desc(tile, kHalfBlockBytes, 512u, kLayoutSW128Atom32);
+}
 
 // ------------------------------------------------------ score tile kernel
 

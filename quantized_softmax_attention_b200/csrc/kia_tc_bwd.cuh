@@ -28,6 +28,7 @@
 // reaches TMEM lanes 32*(w%4)..+31; the two warps of a group that share
 // those lanes split a half tile's 64 columns.
 #pragma once
+#include <algorithm>
 #include <type_traits>
 
 #include "kia_fast.cuh"
@@ -37,15 +38,19 @@ namespace kia {
 
 constexpr int kBwdSmemTabK = 16;  // key pass: per-query grids up to K = 16 in shared memory
 constexpr int kBwdRegions = 3;    // TMEM regions of 128 columns (S | dP) in rotation
+constexpr int kBwdSlots = 3;      // query pass: slots of the half-tile key rings
+constexpr uint32_t kHalfTile = 64 * 64 * 4;       // one operand's half tile (64 rows, d = 64)
+constexpr uint32_t kHalfPair = 2 * kHalfTile;     // K half and V half
 
 struct BwdQBars {
-  uint64_t qd_full;               // Q_i, dO_i (K-major), once
-  uint64_t kv_full, kv_empty;     // K_j, V_j K-major (for S, dP)
-  uint64_t kmn_full, kmn_empty;   // K_j MN-major (for dQ)
+  uint64_t qd_full, qd_empty;     // Q_i, dO_i (K-major), per item
+  uint64_t kv_full[3], kv_empty[3];     // half tiles of K, V K-major (for S, dP)
+  uint64_t kmn_full[3], kmn_empty[3];   // half tiles of K MN-major (for dQ)
   uint64_t sp_full[3];            // S and dP of a half tile in TMEM region r
   uint64_t elem_done[3];          // dS written into region r
   uint64_t st_free[3];            // dQ MMA of region r done
-  uint64_t dq_full;               // all dQ MMAs done
+  uint64_t dq_full;               // all dQ MMAs of an item done
+  uint64_t dq_free;               // the item's dQ read out of TMEM
   uint64_t row_sync;              // element-thread rendezvous
   uint32_t tmem_base;
   int abort;
@@ -74,7 +79,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmV, const float* __restrict__ Kt,
                 const float* __restrict__ O, const float* __restrict__ dO, StatsView st,
                 WorkView wk, float* __restrict__ dQ, float* __restrict__ dS_dbg, OpParams p, int B,
-                int H, int T) {
+                int H, int T, int tab_in_smem) {
   static_assert(D == 64, "tensor-core backward tiles are laid out for d = 64");
   constexpr uint32_t kTile = D * KIA_TILE * 4;
   // the stats must come from a forward of this shape and configuration
@@ -82,46 +87,55 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (threadIdx.x == 0) {
     const bool ok = header_matches(st.header, B, H, T, D, p);
     s_hdr_ok = ok ? 1 : 0;
-    if (blockIdx.x == 0 && blockIdx.y == 0) *wk.status = ok ? 0 : 1;
+    if (blockIdx.x == 0) *wk.status = ok ? 0 : 1;
     if (!ok) atomicExch(&g_kia_device_error, KIA_ERR_STATS_MISMATCH);
   }
   __syncthreads();
   if (!s_hdr_ok) return;
   extern __shared__ uint8_t smraw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
+  // Q_i and dO_i stay for an item; the keys stream through two rings of half tiles
+  // (64 keys): K and V K-major (for S and dP) and K MN-major (for dQ), three
+  // slots each, so that a slot refills while the next two are in use.
   float* sQ = reinterpret_cast<float*>(base);
   float* sG = reinterpret_cast<float*>(base + kTile);
-  float* sK = reinterpret_cast<float*>(base + 2 * kTile);
-  float* sKmn = reinterpret_cast<float*>(base + 3 * kTile);
-  float* sV = reinterpret_cast<float*>(base + 4 * kTile);
-  float* sAC = reinterpret_cast<float*>(base + 5 * kTile);   // [kRowSplit][2][128]
+  uint8_t* sKV = base + 2 * kTile;                           // [3][K half | V half]
+  uint8_t* sKmn = sKV + kBwdSlots * kHalfPair;                // [3][K half, MN-major]
+  float* sAC = reinterpret_cast<float*>(sKmn + kBwdSlots * kHalfTile);   // [kRowSplit][2][128]
   float* sDc = sAC + 2 * kRowSplit * KIA_TILE;               // [128] centering D
   float* sTab = sDc + KIA_TILE;
-  const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (p.K + 1) * KIA_TILE : 2 * (p.K + 1));
+  const int tab_floats =
+      V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   BwdQBars& bar = *reinterpret_cast<BwdQBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
+  const int BH = B * H;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
-  const int qt = nt - 1 - blockIdx.y;
-  const int nkt = p.causal ? qt + 1 : nt;
-  const int nunits = 2 * nkt;          // half key tiles
+  const int nitems = BH * nt;
+  // item it -> (query tile, batch*head), heaviest causal tiles first; this
+  // CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+  auto item_qt = [&](int it) { return nt - 1 - it / BH; };
+  auto item_bh = [&](int it) { return it % BH; };
+  auto item_units = [&](int it) { return 2 * (p.causal ? item_qt(it) + 1 : nt); };
   constexpr int R = kBwdRegions;
   constexpr uint32_t kColDQ = 128u * R;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.qd_full, 1);
-    mbar_init(&bar.kv_full, 1);
-    mbar_init(&bar.kv_empty, 1);
-    mbar_init(&bar.kmn_full, 1);
-    mbar_init(&bar.kmn_empty, 1);
+    mbar_init(&bar.qd_empty, 1);
+    for (int sl = 0; sl < kBwdSlots; ++sl) {
+      mbar_init(&bar.kv_full[sl], 1);
+      mbar_init(&bar.kv_empty[sl], 1);
+      mbar_init(&bar.kmn_full[sl], 1);
+      mbar_init(&bar.kmn_empty[sl], 1);
+    }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&bar.sp_full[b], 1);
       mbar_init(&bar.elem_done[b], kGroupThreads);
       mbar_init(&bar.st_free[b], 1);
     }
     mbar_init(&bar.dq_full, 1);
+    mbar_init(&bar.dq_free, kElemThreads);
     mbar_init(&bar.row_sync, kElemThreads);
     bar.abort = 0;
     fence_barrier_init();
@@ -139,37 +153,61 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
+    // Q_i, dO_i of each item once its previous item's MMAs are done with
+    // them; the two key rings refill independently, each as soon as its
+    // slot is free (half tiles numbered across the CTA's items).
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmG);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmKmn);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar.qd_full, 2 * kTile);
-      for (int b = 0; b < D / 32; ++b) {
-        tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, qt * KIA_TILE, bh);
-        tma_load_3d(sG + b * 32 * KIA_TILE, &tmG, &bar.qd_full, b * 32, qt * KIA_TILE, bh);
-      }
-      // the two rings refill independently, each as soon as its slot is free
-      int jk = 0, jm = 0;                // next K / V tile, next K MN-major tile
+      int iq = blockIdx.x, nq = 0;                   // next item for Q / dO
+      int ik = blockIdx.x, uk = 0, gk = 0;            // K / V ring: item, unit, global unit
+      int im = blockIdx.x, um = 0, gm = 0;            // K MN-major ring
       PollGuard guard;
-      while ((jk < nkt || jm < nkt) && !failed) {
+      while ((iq < nitems || ik < nitems || im < nitems) && !failed) {
         bool moved = false;
-        if (jk < nkt && mbar_test(&bar.kv_empty, (jk & 1) ^ 1)) {
-          mbar_arrive_expect_tx(&bar.kv_full, 2 * kTile);
+        if (iq < nitems && mbar_test(&bar.qd_empty, (nq & 1) ^ 1)) {
+          mbar_arrive_expect_tx(&bar.qd_full, 2 * kTile);
           for (int b = 0; b < D / 32; ++b) {
-            tma_load_3d(sK + b * 32 * KIA_TILE, &tmK, &bar.kv_full, b * 32, jk * KIA_TILE, bh);
-            tma_load_3d(sV + b * 32 * KIA_TILE, &tmV, &bar.kv_full, b * 32, jk * KIA_TILE, bh);
+            tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, item_qt(iq) * KIA_TILE,
+                        item_bh(iq));
+            tma_load_3d(sG + b * 32 * KIA_TILE, &tmG, &bar.qd_full, b * 32, item_qt(iq) * KIA_TILE,
+                        item_bh(iq));
           }
-          ++jk;
+          iq += gridDim.x;
+          ++nq;
           moved = true;
         }
-        if (jm < nkt && mbar_test(&bar.kmn_empty, (jm & 1) ^ 1)) {
-          mbar_arrive_expect_tx(&bar.kmn_full, kTile);
-          for (int b = 0; b < D / 32; ++b)
-            tma_load_3d(sKmn + b * 32 * KIA_TILE, &tmKmn, &bar.kmn_full, b * 32, jm * KIA_TILE, bh);
-          ++jm;
-          moved = true;
+        if (ik < nitems) {
+          const int sl = gk % kBwdSlots;
+          if (mbar_test(&bar.kv_empty[sl], ((gk / kBwdSlots) & 1) ^ 1)) {
+            uint8_t* dst = sKV + sl * kHalfPair;
+            mbar_arrive_expect_tx(&bar.kv_full[sl], kHalfPair);
+            for (int b = 0; b < D / 32; ++b) {
+              tma_load_3d(dst + b * kHalfBlockBytes, &tmK, &bar.kv_full[sl], b * 32, 64 * uk,
+                          item_bh(ik));
+              tma_load_3d(dst + kHalfTile + b * kHalfBlockBytes, &tmV, &bar.kv_full[sl], b * 32,
+                          64 * uk, item_bh(ik));
+            }
+            ++gk;
+            if (++uk == item_units(ik)) { uk = 0; ik += gridDim.x; }
+            moved = true;
+          }
+        }
+        if (im < nitems) {
+          const int sl = gm % kBwdSlots;
+          if (mbar_test(&bar.kmn_empty[sl], ((gm / kBwdSlots) & 1) ^ 1)) {
+            uint8_t* dst = sKmn + sl * kHalfTile;
+            mbar_arrive_expect_tx(&bar.kmn_full[sl], kHalfTile);
+            for (int b = 0; b < D / 32; ++b)
+              tma_load_3d(dst + b * kHalfBlockBytes, &tmKmn, &bar.kmn_full[sl], b * 32, 64 * um,
+                          item_bh(im));
+            ++gm;
+            if (++um == item_units(im)) { um = 0; im += gridDim.x; }
+            moved = true;
+          }
         }
         if (moved) guard.progress();
         else if (!guard.idle(abort)) failed = true;
@@ -181,55 +219,69 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
       // descriptors built once; each MMA only adds a constant step
       const uint64_t dqa = desc_kmajor(smem_u32(sQ), 0), dga = desc_kmajor(smem_u32(sG), 0),
-                     dka = desc_kmajor(smem_u32(sK), 0), dva = desc_kmajor(smem_u32(sV), 0);
+                     dkv = desc_kmajor_half(smem_u32(sKV));
       uint32_t sf_par = 0;                // per-region phase bits of the st_free waits
-      failed = !mbar_wait(&bar.qd_full, 0, abort);
-      // S, dP of half tile u (keys 64 (u % 2).. of tile u / 2) into region
-      // u % R, once the dQ MMA of unit u - R has released the region
-      for (int u = 0; u < nunits && !failed; ++u) {
-        const int r = u % R, j = u >> 1, h = u & 1;
-        if (u >= R) {
-          if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
-          sf_par ^= 1u << r;
+      int g = 0, n = 0;                   // global half tile, item count
+      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+        if (!mbar_wait(&bar.qd_full, n & 1, abort)) { failed = true; break; }
+        // S, dP of half tile u (keys 64 u..) into region g % R, once the dQ
+        // MMA of half tile g - R has released the region
+        const int nunits = item_units(it);
+        for (int u = 0; u < nunits; ++u, ++g) {
+          const int r = g % R;
+          if (g >= R) {
+            if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+            sf_par ^= 1u << r;
+          }
+          const int sl = g % kBwdSlots;
+          if (!mbar_wait(&bar.kv_full[sl], (g / kBwdSlots) & 1, abort)) { failed = true; break; }
+          tc_fence_after();
+          const uint64_t dk = dkv + desc_step((uint32_t)sl * kHalfPair);   // K half, V half after it
+          const uint64_t dv = dk + desc_step(kHalfTile);
+          const uint32_t dst = tmem + 128u * r;
+#pragma unroll
+          for (int ks = 0; ks < D / 8; ++ks)
+            mma_tf32_ss(dst, dqa + kstep_kmajor(ks), dk + kstep_kmajor_half(ks), id_s, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < D / 8; ++ks)
+            mma_tf32_ss(dst + 64u, dga + kstep_kmajor(ks), dv + kstep_kmajor_half(ks), id_s, ks > 0);
+          tc_commit(&bar.sp_full[r]);
+          tc_commit(&bar.kv_empty[sl]);
         }
-        if (h == 0 && !mbar_wait(&bar.kv_full, j & 1, abort)) { failed = true; break; }
-        tc_fence_after();
-        const uint64_t koff = desc_step((uint32_t)h * 64u * 128u);   // rows 64h.. of the key tile
-        const uint32_t dst = tmem + 128u * r;
-#pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(dst, dqa + kstep_kmajor(ks), dka + koff + kstep_kmajor(ks), id_s, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(dst + 64u, dga + kstep_kmajor(ks), dva + koff + kstep_kmajor(ks), id_s,
-                      ks > 0);
-        tc_commit(&bar.sp_full[r]);
-        if (h == 1) tc_commit(&bar.kv_empty);
+        if (!failed) tc_commit(&bar.qd_empty);     // Q_i, dO_i free once these MMAs are done
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------- dQ-MMA issuer
     if (lane == 0) {
       const uint32_t id_dq = idesc_tf32(128, D, 0, 1);
-      const uint64_t dkm = desc_mnmajor(smem_u32(sKmn), 0);
+      const uint64_t dkm = desc_mnmajor_half(smem_u32(sKmn));
       uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
-      // dQ of half tile u: A = dS in region u % R, B = rows 64 (u % 2).. of K_j (MN-major)
-      for (int u = 0; u < nunits && !failed; ++u) {
-        const int r = u % R, j = u >> 1, h = u & 1;
-        if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
-        ed_par ^= 1u << r;
-        if (h == 0 && !mbar_wait(&bar.kmn_full, j & 1, abort)) { failed = true; break; }
-        tc_fence_after();
-        const uint64_t db = dkm + kstep_mnmajor(8 * h);
-        const uint32_t pa = tmem + 128u * r;
-        const uint32_t acc0 = u > 0 ? 1u : 0u;
+      int g = 0, n = 0;
+      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+        const int nunits = item_units(it);
+        // dQ of half tile u: A = dS in region g % R, B = K half (MN-major)
+        for (int u = 0; u < nunits; ++u, ++g) {
+          const int r = g % R, sl = g % kBwdSlots;
+          if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
+          ed_par ^= 1u << r;
+          if (!mbar_wait(&bar.kmn_full[sl], (g / kBwdSlots) & 1, abort)) { failed = true; break; }
+          // the accumulator restarts with this item: the previous item's
+          // epilogue must have read it
+          if (u == 0 && n > 0 && !mbar_wait(&bar.dq_free, (n - 1) & 1, abort)) { failed = true; break; }
+          tc_fence_after();
+          const uint64_t db = dkm + desc_step((uint32_t)sl * kHalfTile);
+          const uint32_t pa = tmem + 128u * r;
+          const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_tf32_ts(tmem + kColDQ, pa + 8u * kk, db + kstep_mnmajor(kk), id_dq, kk > 0 ? 1u : acc0);
-        tc_commit(&bar.st_free[r]);
-        if (h == 1) tc_commit(&bar.kmn_empty);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_tf32_ts(tmem + kColDQ, pa + 8u * kk, db + kstep_mnmajor(kk), id_dq,
+                        kk > 0 ? 1u : acc0);
+          tc_commit(&bar.st_free[r]);
+          tc_commit(&bar.kmn_empty[sl]);
+        }
+        if (!failed) tc_commit(&bar.dq_full);
       }
-      if (!failed) tc_commit(&bar.dq_full);
     }
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
@@ -238,112 +290,128 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int grp = part >> 1;              // half tiles u with u % 2 == grp
     const int sub = part & 1;               // columns 32 sub .. 32 sub + 31 of a unit
     const int r = quad * 32 + lane;
-    const int q = qt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const long long rowbase = (long long)bh * T;
-    const long long qr = rowbase + (q < T ? q : T - 1);
-    // this row's calibration and centering (written by the forward and prep)
-    const float m = st.m[qr];
-    const float n = st.n[qr];
-    const int am = st.am[qr], an = V::MINMAX ? st.an[qr] : am;
-    const float rh = st.rh[qr];
-    const float nrh = -rh;
-    const float dg = (V::MINMAX && rh == 0.0f) ? 1.0f : 0.0f;
-    const int L = p.causal ? q + 1 : T;
-    // a one-key row has P = 1 whatever its score: zero gradient
-    const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]);
-    // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE): four
-    // consecutive element threads read one row's D values (coalesced), add
-    // their partial sums by shuffles and leave the row's D in shared memory
-    {
-      const int e = (int)threadIdx.x - 64;
-      const int rr = e >> 2, cc = e & 3;     // row of the tile, quarter of the row
-      const int qq = qt * KIA_TILE + rr;
-      const long long qrr = rowbase + (qq < T ? qq : T - 1);
-      const float4* g4 = reinterpret_cast<const float4*>(dO + qrr * D) + cc * (D / 16);
-      const float4* o4 =
-          reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qrr * D) + cc * (D / 16);
-      float acc = 0.0f;
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        const float4 a = g4[c], b4 = o4[c];
-        acc = fmaf(a.x, b4.x, acc);
-        acc = fmaf(a.y, b4.y, acc);
-        acc = fmaf(a.z, b4.z, acc);
-        acc = fmaf(a.w, b4.w, acc);
-      }
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if (cc == 0) {
-        sDc[rr] = acc;
-        if (qq < T) wk.D[qrr] = acc;
-      }
-    }
-
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     float2* sPair = reinterpret_cast<float2*>(sTab);
-    if constexpr (V::MINMAX) {
-      for (int k = part; k <= p.K; k += kRowSplit) sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
-    } else if constexpr (!V::SOFTMAX) {
+    if constexpr (!V::MINMAX && !V::SOFTMAX) {
       const int k = (int)threadIdx.x - 64;
       if (k >= 0 && k < p.K) sPair[k] = make_float2(st.table[k], st.table[k + 1]);
     }
-    using Grid = std::conditional_t<V::MINMAX, GridF, GridP>;
-    Grid grid;
-    if constexpr (V::MINMAX) grid = GridF{sTab + r, KIA_TILE};
-    else grid = GridP{sPair};
-    mbar_arrive(&bar.row_sync);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
-    const float Dc = sDc[r];
-    const float nDr = -Dc * rWb;            // dw = (dP - D) / W_bar as one fma
-    float A = 0.0f, C = 0.0f;
-    for (int u = grp; u < nunits && !failed; u += 2) {
-      const int j = u >> 1, rg = u % R;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (u / R) & 1, abort))) { failed = true; break; }
-      tc_fence_after();
-      const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        float v[16], g[16];
-        const uint32_t cs = 128u * rg + 32u * sub + 16u * c;    // 16 columns of S
-        tmem_ld16(tmem + lane_addr + cs, v);
-        tmem_ld16(tmem + lane_addr + cs + 64u, g);
-        tmem_ld_wait_regs(v, g);
-        const int key0 = j * KIA_TILE + 64 * grp + 32 * sub + 16 * c;
-        if (!edge) {
+    int gbase = 0, n = 0;
+    for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      const int qt = item_qt(it), bh = item_bh(it), nunits = item_units(it);
+      const int q = qt * KIA_TILE + r;
+      const long long rowbase = (long long)bh * T;
+      const long long qr = rowbase + (q < T ? q : T - 1);
+      // this row's calibration and centering (written by the forward)
+      const float m = st.m[qr];
+      const int am = st.am[qr], an = V::MINMAX ? st.an[qr] : am;
+      const float rh = st.rh[qr];
+      const float nrh = -rh;
+      const float dg = (V::MINMAX && rh == 0.0f) ? 1.0f : 0.0f;
+      const int L = p.causal ? q + 1 : T;
+      // a one-key row has P = 1 whatever its score: zero gradient
+      const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]);
+      // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE): four
+      // consecutive element threads read one row's D values (coalesced), add
+      // their partial sums by shuffles and leave the row's D in shared memory
+      {
+        const int e = (int)threadIdx.x - 64;
+        const int rr = e >> 2, cc = e & 3;     // row of the tile, quarter of the row
+        const int qq = qt * KIA_TILE + rr;
+        const long long qrr = rowbase + (qq < T ? qq : T - 1);
+        const float4* g4 = reinterpret_cast<const float4*>(dO + qrr * D) + cc * (D / 16);
+        const float4* o4 =
+            reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qrr * D) + cc * (D / 16);
+        float acc = 0.0f;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float dw = fmaf(g[i], rWb, nDr);
-            v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int key = key0 + i;
-            const bool ok = key < T && (!p.causal || key <= q);
-            const float dw = ok ? fmaf(g[i], rWb, nDr) : 0.0f;
-            v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
-          }
+        for (int c = 0; c < D / 16; ++c) {
+          const float4 a = g4[c], b4 = o4[c];
+          acc = fmaf(a.x, b4.x, acc);
+          acc = fmaf(a.y, b4.y, acc);
+          acc = fmaf(a.z, b4.z, acc);
+          acc = fmaf(a.w, b4.w, acc);
         }
-        tmem_st16(tmem + lane_addr + cs, v);
-        if (dS_dbg && q < T) {
-          float* dst = dS_dbg + (rowbase + q) * T + key0;
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (key0 + i < T) dst[i] = v[i];
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (cc == 0) {
+          sDc[rr] = acc;
+          if (qq < T) wk.D[qrr] = acc;
         }
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bar.elem_done[rg]);
-    }
-    // row sums of the four column groups
-    sAC[(part * 2 + 0) * KIA_TILE + r] = A;
-    sAC[(part * 2 + 1) * KIA_TILE + r] = C;
-    mbar_arrive(&bar.row_sync);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 1, abort))) failed = true;
-    if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.dq_full, 0, abort))) {
+      if constexpr (V::MINMAX) {
+        if (tab_in_smem)
+          for (int k = part; k <= p.K; k += kRowSplit)
+            sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
+      }
+      using Grid = std::conditional_t<V::MINMAX, GridF, GridP>;
+      Grid grid;
+      if constexpr (V::MINMAX)
+        grid = tab_in_smem ? GridF{sTab + r, KIA_TILE} : GridF{st.table + qr * (p.K + 1), 1};
+      else grid = GridP{sPair};
+      mbar_arrive(&bar.row_sync);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (2 * n) & 1, abort))) { failed = true; break; }
+      const float Dc = sDc[r];
+      const float nDr = -Dc * rWb;            // dw = (dP - D) / W_bar as one fma
+      float A = 0.0f, C = 0.0f;
+      for (int u = grp; u < nunits && !failed; u += 2) {
+        const int j = u >> 1, gu = gbase + u, rg = gu % R;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (gu / R) & 1, abort))) { failed = true; break; }
+        tc_fence_after();
+        const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float v[16], g[16];
+          const uint32_t cs = 128u * rg + 32u * sub + 16u * c;    // 16 columns of S
+          tmem_ld16(tmem + lane_addr + cs, v);
+          tmem_ld16(tmem + lane_addr + cs + 64u, g);
+          tmem_ld_wait_regs(v, g);
+          const int key0 = j * KIA_TILE + 64 * grp + 32 * sub + 16 * c;
+          if (!edge) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float dw = fmaf(g[i], rWb, nDr);
+              v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int key = key0 + i;
+              const bool ok = key < T && (!p.causal || key <= q);
+              const float dw = ok ? fmaf(g[i], rWb, nDr) : 0.0f;
+              v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+            }
+          }
+          tmem_st16(tmem + lane_addr + cs, v);
+          if (dS_dbg && q < T) {
+            float* dst = dS_dbg + (rowbase + q) * T + key0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (key0 + i < T) dst[i] = v[i];
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar.elem_done[rg]);
+      }
+      if (failed) break;
+      gbase += nunits;
+      // row sums of the four column groups
+      sAC[(part * 2 + 0) * KIA_TILE + r] = A;
+      sAC[(part * 2 + 1) * KIA_TILE + r] = C;
+      mbar_arrive(&bar.row_sync);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (2 * n + 1) & 1, abort))) { failed = true; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.dq_full, n & 1, abort))) { failed = true; break; }
       tc_fence_after();
+      // this thread's 16 columns of dQ, then the accumulator is free for the
+      // next item
+      constexpr int kCols = D / kRowSplit;   // 16
+      const uint32_t col = (uint32_t)(part * kCols);
+      float o[kCols];
+      tmem_ld16(tmem + lane_addr + kColDQ + col, o);
+      tmem_ld_wait_regs(o);
+      tc_fence_before();
+      mbar_arrive(&bar.dq_free);
       // calibration terms of this row (section 3, Calibration gradients;
       // Appendix B): dS gains g_m at the argmax key and g_n at the argmin key
       const float Arow = (sAC[0 * KIA_TILE + r] + sAC[2 * KIA_TILE + r]) +
@@ -354,42 +422,33 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       calibration_coeffs(p, Arow, Crow, rh, L, gm, gn);
       const bool proj = p.grad == KIA_GRAD_PROJECT;
       const float gmq = proj ? 0.0f : gm;   // the projection shift is applied by the scan pass
-      const float* ka = Kt + (rowbase + am) * D;
-      const float* kn = Kt + (rowbase + an) * D;
-      {
-        constexpr int kCols = D / kRowSplit;   // 16
-        const uint32_t col = (uint32_t)(part * kCols);
-        float o[kCols];
-        tmem_ld16(tmem + lane_addr + kColDQ + col, o);
-        tmem_ld_wait();
-        if (q < T) {
-          if (gmq != 0.0f) {
-            const float4* k4 = reinterpret_cast<const float4*>(ka + col);
+      if (q < T) {
+        if (gmq != 0.0f) {
+          const float4* k4 = reinterpret_cast<const float4*>(Kt + (rowbase + am) * D + col);
 #pragma unroll
-            for (int i = 0; i < kCols / 4; ++i) {
-              const float4 kk = k4[i];
-              o[4 * i] = fmaf(gmq, kk.x, o[4 * i]);
-              o[4 * i + 1] = fmaf(gmq, kk.y, o[4 * i + 1]);
-              o[4 * i + 2] = fmaf(gmq, kk.z, o[4 * i + 2]);
-              o[4 * i + 3] = fmaf(gmq, kk.w, o[4 * i + 3]);
-            }
+          for (int i = 0; i < kCols / 4; ++i) {
+            const float4 kk = k4[i];
+            o[4 * i] = fmaf(gmq, kk.x, o[4 * i]);
+            o[4 * i + 1] = fmaf(gmq, kk.y, o[4 * i + 1]);
+            o[4 * i + 2] = fmaf(gmq, kk.z, o[4 * i + 2]);
+            o[4 * i + 3] = fmaf(gmq, kk.w, o[4 * i + 3]);
           }
-          if (V::MINMAX && gn != 0.0f) {
-            const float4* k4 = reinterpret_cast<const float4*>(kn + col);
-#pragma unroll
-            for (int i = 0; i < kCols / 4; ++i) {
-              const float4 kk = k4[i];
-              o[4 * i] = fmaf(gn, kk.x, o[4 * i]);
-              o[4 * i + 1] = fmaf(gn, kk.y, o[4 * i + 1]);
-              o[4 * i + 2] = fmaf(gn, kk.z, o[4 * i + 2]);
-              o[4 * i + 3] = fmaf(gn, kk.w, o[4 * i + 3]);
-            }
-          }
-          float4* o4 = reinterpret_cast<float4*>(dQ + (rowbase + q) * D + col);
-#pragma unroll
-          for (int i = 0; i < kCols / 4; ++i)
-            o4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
+        if (V::MINMAX && gn != 0.0f) {
+          const float4* k4 = reinterpret_cast<const float4*>(Kt + (rowbase + an) * D + col);
+#pragma unroll
+          for (int i = 0; i < kCols / 4; ++i) {
+            const float4 kk = k4[i];
+            o[4 * i] = fmaf(gn, kk.x, o[4 * i]);
+            o[4 * i + 1] = fmaf(gn, kk.y, o[4 * i + 1]);
+            o[4 * i + 2] = fmaf(gn, kk.z, o[4 * i + 2]);
+            o[4 * i + 3] = fmaf(gn, kk.w, o[4 * i + 3]);
+          }
+        }
+        float4* o4 = reinterpret_cast<float4*>(dQ + (rowbase + q) * D + col);
+#pragma unroll
+        for (int i = 0; i < kCols / 4; ++i)
+          o4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
       }
       if (q < T && part == 0) {
         wk.gm[rowbase + q] = gm;
@@ -406,8 +465,6 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-    } else {
-      failed = true;
     }
   }
   if (failed || *abort) drain_in_flight();
@@ -804,11 +861,12 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 template <int D>
-size_t tc_bwd_q_smem(const OpParams& p) {
+size_t tc_bwd_q_smem(const OpParams& p, bool tab_in_smem) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
-  const int tab = p.softmax ? 0 : (minmax_tab ? (p.K + 1) * KIA_TILE : 2 * (p.K + 1));
-  return 1024 + 5 * (size_t)D * KIA_TILE * 4 + (2 * kRowSplit + 1) * KIA_TILE * 4 +
-         (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdQBars);
+  const int tab =
+      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
+  return 1024 + 2 * (size_t)D * KIA_TILE * 4 + kBwdSlots * (size_t)(kHalfPair + kHalfTile) +
+         (2 * kRowSplit + 1) * KIA_TILE * 4 + (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdQBars);
 }
 
 template <int D>
@@ -826,13 +884,15 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
                   float* dV, float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
                   void (*mark)(int, cudaStream_t)) {
   const int BH = B * H;
-  CUtensorMap tq, tqm, tg, tgm, tk, tkm, tv;
+  CUtensorMap tq, tqm, tg, tgm, tk, tkm, tv, tkh, tkmh, tvh;
   if (!make_tmap(&tq, Q, BH, T, D) || !make_tmap(&tqm, Q, BH, T, D, true) ||
       !make_tmap(&tg, dO, BH, T, D) || !make_tmap(&tgm, dO, BH, T, D, true) ||
       !make_tmap(&tk, Kt, BH, T, D) || !make_tmap(&tkm, Kt, BH, T, D, true) ||
-      !make_tmap(&tv, Vv, BH, T, D))
+      !make_tmap(&tv, Vv, BH, T, D) || !make_tmap(&tkh, Kt, BH, T, D, false, 64) ||
+      !make_tmap(&tkmh, Kt, BH, T, D, true, 64) || !make_tmap(&tvh, Vv, BH, T, D, false, 64))
     return KIA_ERR_CUDA;
-  const size_t smq = tc_bwd_q_smem<D>(p);
+  const bool q_tab_smem = tc_bwd_q_smem<D>(p, true) <= 232448;
+  const size_t smq = tc_bwd_q_smem<D>(p, q_tab_smem);
   const bool kv_tab_smem = p.K <= kBwdSmemTabK && tc_bwd_kv_smem<D>(p, true) <= 232448;
   const size_t smk = tc_bwd_kv_smem<D>(p, kv_tab_smem);
   if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
@@ -840,18 +900,24 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
                                     p.grad == KIA_GRAD_MIN_ONLY);
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   dim3 grid(BH, nt);
+  // the query pass is persistent: one CTA per SM walks the items
+  const int sms = num_sms();
+  if (sms <= 0) return KIA_ERR_CUDA;
+  const dim3 qgrid(std::min(sms, BH * nt));
   if (need_c) {
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
-    tc_bwd_q_kernel<D, V, true><<<grid, kTcThreads, smq, s>>>(tq, tg, tk, tkm, tv, Kt, O, dO, st,
-                                                              wk, dQ, dS_dbg, p, B, H, T);
+    tc_bwd_q_kernel<D, V, true><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
+                                                              st, wk, dQ, dS_dbg, p, B, H, T,
+                                                              q_tab_smem ? 1 : 0);
   } else {
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
-    tc_bwd_q_kernel<D, V, false><<<grid, kTcThreads, smq, s>>>(tq, tg, tk, tkm, tv, Kt, O, dO,
-                                                               st, wk, dQ, dS_dbg, p, B, H, T);
+    tc_bwd_q_kernel<D, V, false><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
+                                                               st, wk, dQ, dS_dbg, p, B, H, T,
+                                                               q_tab_smem ? 1 : 0);
   }
   if (cudaGetLastError() != cudaSuccess) return KIA_ERR_CUDA;
   mark(4, s);
