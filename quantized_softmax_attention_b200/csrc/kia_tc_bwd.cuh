@@ -40,7 +40,8 @@ constexpr int kBwdSmemTabK = 16;  // key pass: per-query grids up to K = 16 in s
 constexpr int kBwdRegions = 3;    // TMEM regions of 128 columns (S | dP) in rotation
 constexpr int kBwdSlots = 3;      // query pass: slots of the half-tile key rings
 constexpr uint32_t kHalfTile = 64 * 64 * 4;       // one operand's half tile (64 rows, d = 64)
-constexpr uint32_t kHalfPair = 2 * kHalfTile;     // K half and V half
+constexpr uint32_t kHalfPair = 2 * kHalfTile;     // K half and V half (Q half and dO half)
+constexpr int kKvSlots = 2;       // key pass: slots of each half-tile query ring
 
 struct BwdQBars {
   uint64_t qd_full, qd_empty;     // Q_i, dO_i (K-major), per item
@@ -57,15 +58,16 @@ struct BwdQBars {
 };
 
 struct BwdKBars {
-  uint64_t kv_full;               // K_j, V_j K-major, once
-  uint64_t qd_full, qd_empty;     // Q_i, dO_i K-major (for S^T, dP^T)
-  uint64_t mn_full, mn_empty;     // Q_i, dO_i MN-major (for dK, dV)
+  uint64_t kv_full, kv_empty;     // K_j, V_j K-major, per item
+  uint64_t qd_full[2], qd_empty[2];     // half tiles of Q, dO K-major (for S^T, dP^T)
+  uint64_t mn_full[2], mn_empty[2];     // half tiles of Q, dO MN-major (for dK, dV)
   uint64_t sp_full[3];            // S^T and dP^T of a half tile in TMEM region r
   uint64_t qc_ready[4];           // per-query constants of a unit loaded into slot s
   uint64_t qc_free[4];            // the unit's group done with slot s
   uint64_t elem_done[3];          // P^T, dS^T written into region r
   uint64_t st_free[3];            // dV, dK MMAs of region r done
-  uint64_t acc_full;              // all dV, dK MMAs done
+  uint64_t acc_full;              // all dV, dK MMAs of an item done
+  uint64_t acc_free;              // the item's dV, dK read out of TMEM
   uint32_t tmem_base;
   int abort;
 };
@@ -481,24 +483,24 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmGmn,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  StatsView st, WorkView wk, float* __restrict__ dK, float* __restrict__ dV,
-                 OpParams p, int T, int tab_in_smem) {
+                 OpParams p, int BH, int T, int tab_in_smem) {
   static_assert(D == 64, "tensor-core backward tiles are laid out for d = 64");
   constexpr uint32_t kTile = D * KIA_TILE * 4;
   if (*wk.status != 0) return;
   extern __shared__ uint8_t smraw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
+  // K_j and V_j stay for an item; the queries stream through two rings of
+  // half tiles (64 queries): Q and dO K-major (for S^T, dP^T) and Q and dO
+  // MN-major (for dK, dV), two slots each.
   float* sK = reinterpret_cast<float*>(base);
   float* sV = reinterpret_cast<float*>(base + kTile);
-  float* sQ = reinterpret_cast<float*>(base + 2 * kTile);
-  float* sG = reinterpret_cast<float*>(base + 3 * kTile);
-  float* sQmn = reinterpret_cast<float*>(base + 4 * kTile);
-  float* sGmn = reinterpret_cast<float*>(base + 5 * kTile);
+  uint8_t* sQD = base + 2 * kTile;                            // [2][Q half | dO half]
+  uint8_t* sQDmn = sQD + kKvSlots * kHalfPair;                // [2][Q half | dO half], MN-major
   // Per-query constants of a unit (64 queries) in four slots, filled ahead of
-  // the element groups by the constant warp: unit u uses slot
-  // 2 (u % 2) + (u / 2) % 2.
+  // the element groups by the constant warp: half tile g (numbered across the
+  // CTA's items) uses slot 2 (g % 2) + (g / 2) % 2.
   constexpr int kSlots = 4, kSlotQ = 64;
-  float4* sC4 = reinterpret_cast<float4*>(base + 6 * kTile);  // (m, rh, rWb, -D rWb)
+  float4* sC4 = reinterpret_cast<float4*>(sQDmn + kKvSlots * kHalfPair);  // (m, rh, rWb, -D rWb)
   float2* sC2 = reinterpret_cast<float2*>(sC4 + kSlots * kSlotQ);  // (rWf, dg or projection shift c)
   // calibration terms, read only where a query's argmax (argmin) key is this
   // thread's key: key - tile start, and the coefficient
@@ -507,27 +509,34 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   // which queries of a unit have their argmax (argmin) key in lanes
   // 32 quad..32 quad + 31: [slot][argmax / argmin][quad][query half]
   uint32_t* sMask = reinterpret_cast<uint32_t*>(sCG + kSlots * kSlotQ);
-  float* sTab = reinterpret_cast<float*>(sMask + kSlots * 2 * 4 * 2);   // [slot][64][K + 1]
+  // epilogue: 1 KB per element warp to turn its rows into full-sector stores
+  float* sStage = reinterpret_cast<float*>(sMask + kSlots * 2 * 4 * 2);   // [16 warps][32][8]
+  float* sTab = sStage + kElemThreads / 32 * 256;   // [slot][64][K + 1]
   const int K1 = p.K + 1;
   const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? kSlots * kSlotQ * K1 : 0) : 4 * K1);
   BwdKBars& bar = *reinterpret_cast<BwdKBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
-  const int kt = blockIdx.y;
-  const int q0 = p.causal ? kt : 0;
-  const int ntiles = nt - q0;
-  const int nunits = 2 * ntiles;       // half query tiles
+  const int nitems = BH * nt;
+  // item it -> (key tile, batch*head), heaviest causal tiles (most queries)
+  // first; this CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+  auto item_kt = [&](int it) { return it / BH; };
+  auto item_bh = [&](int it) { return it % BH; };
+  auto item_q0 = [&](int it) { return p.causal ? item_kt(it) : 0; };
+  auto item_units = [&](int it) { return 2 * (nt - item_q0(it)); };
   constexpr int R = kBwdRegions;
   constexpr uint32_t kColDV = 128u * R, kColDK = kColDV + D;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.kv_full, 1);
-    mbar_init(&bar.qd_full, 1);
-    mbar_init(&bar.qd_empty, 1);
-    mbar_init(&bar.mn_full, 1);
-    mbar_init(&bar.mn_empty, 1);
+    mbar_init(&bar.kv_empty, 1);
+    for (int sl = 0; sl < kKvSlots; ++sl) {
+      mbar_init(&bar.qd_full[sl], 1);
+      mbar_init(&bar.qd_empty[sl], 1);
+      mbar_init(&bar.mn_full[sl], 1);
+      mbar_init(&bar.mn_empty[sl], 1);
+    }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&bar.sp_full[b], 1);
       mbar_init(&bar.elem_done[b], kGroupThreads);
@@ -538,6 +547,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(&bar.qc_free[sl], kGroupThreads);
     }
     mbar_init(&bar.acc_full, 1);
+    mbar_init(&bar.acc_free, kElemThreads);
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -554,6 +564,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
+    // K_j, V_j of each item once the previous item's MMAs are done with
+    // them; the two query rings refill independently, each as soon as its
+    // slot is free (half tiles numbered across the CTA's items).
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmQmn);
@@ -561,35 +574,56 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tma_prefetch_desc(&tmGmn);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar.kv_full, 2 * kTile);
-      for (int b = 0; b < D / 32; ++b) {
-        tma_load_3d(sK + b * 32 * KIA_TILE, &tmK, &bar.kv_full, b * 32, kt * KIA_TILE, bh);
-        tma_load_3d(sV + b * 32 * KIA_TILE, &tmV, &bar.kv_full, b * 32, kt * KIA_TILE, bh);
-      }
-      // the two rings refill independently, each as soon as its slot is free
-      int sk = 0, sm = 0;                // next K-major tile, next MN-major tile
+      int ikv = blockIdx.x, nkv = 0;                 // next item for K / V
+      int iq = blockIdx.x, uq = 0, gq = 0;            // K-major ring: item, unit, global unit
+      int im = blockIdx.x, um = 0, gm = 0;            // MN-major ring
       PollGuard guard;
-      while ((sk < ntiles || sm < ntiles) && !failed) {
+      while ((ikv < nitems || iq < nitems || im < nitems) && !failed) {
         bool moved = false;
-        if (sk < ntiles && mbar_test(&bar.qd_empty, (sk & 1) ^ 1)) {
-          const int qi = q0 + sk;
-          mbar_arrive_expect_tx(&bar.qd_full, 2 * kTile);
+        if (ikv < nitems && mbar_test(&bar.kv_empty, (nkv & 1) ^ 1)) {
+          mbar_arrive_expect_tx(&bar.kv_full, 2 * kTile);
           for (int b = 0; b < D / 32; ++b) {
-            tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, qi * KIA_TILE, bh);
-            tma_load_3d(sG + b * 32 * KIA_TILE, &tmG, &bar.qd_full, b * 32, qi * KIA_TILE, bh);
+            tma_load_3d(sK + b * 32 * KIA_TILE, &tmK, &bar.kv_full, b * 32, item_kt(ikv) * KIA_TILE,
+                        item_bh(ikv));
+            tma_load_3d(sV + b * 32 * KIA_TILE, &tmV, &bar.kv_full, b * 32, item_kt(ikv) * KIA_TILE,
+                        item_bh(ikv));
           }
-          ++sk;
+          ikv += gridDim.x;
+          ++nkv;
           moved = true;
         }
-        if (sm < ntiles && mbar_test(&bar.mn_empty, (sm & 1) ^ 1)) {
-          const int qi = q0 + sm;
-          mbar_arrive_expect_tx(&bar.mn_full, 2 * kTile);
-          for (int b = 0; b < D / 32; ++b) {
-            tma_load_3d(sQmn + b * 32 * KIA_TILE, &tmQmn, &bar.mn_full, b * 32, qi * KIA_TILE, bh);
-            tma_load_3d(sGmn + b * 32 * KIA_TILE, &tmGmn, &bar.mn_full, b * 32, qi * KIA_TILE, bh);
+        if (iq < nitems) {
+          const int sl = gq % kKvSlots;
+          if (mbar_test(&bar.qd_empty[sl], ((gq / kKvSlots) & 1) ^ 1)) {
+            uint8_t* dst = sQD + sl * kHalfPair;
+            const int row = 64 * (2 * item_q0(iq) + uq);
+            mbar_arrive_expect_tx(&bar.qd_full[sl], kHalfPair);
+            for (int b = 0; b < D / 32; ++b) {
+              tma_load_3d(dst + b * kHalfBlockBytes, &tmQ, &bar.qd_full[sl], b * 32, row, item_bh(iq));
+              tma_load_3d(dst + kHalfTile + b * kHalfBlockBytes, &tmG, &bar.qd_full[sl], b * 32,
+                          row, item_bh(iq));
+            }
+            ++gq;
+            if (++uq == item_units(iq)) { uq = 0; iq += gridDim.x; }
+            moved = true;
           }
-          ++sm;
-          moved = true;
+        }
+        if (im < nitems) {
+          const int sl = gm % kKvSlots;
+          if (mbar_test(&bar.mn_empty[sl], ((gm / kKvSlots) & 1) ^ 1)) {
+            uint8_t* dst = sQDmn + sl * kHalfPair;
+            const int row = 64 * (2 * item_q0(im) + um);
+            mbar_arrive_expect_tx(&bar.mn_full[sl], kHalfPair);
+            for (int b = 0; b < D / 32; ++b) {
+              tma_load_3d(dst + b * kHalfBlockBytes, &tmQmn, &bar.mn_full[sl], b * 32, row,
+                          item_bh(im));
+              tma_load_3d(dst + kHalfTile + b * kHalfBlockBytes, &tmGmn, &bar.mn_full[sl], b * 32,
+                          row, item_bh(im));
+            }
+            ++gm;
+            if (++um == item_units(im)) { um = 0; im += gridDim.x; }
+            moved = true;
+          }
         }
         if (moved) guard.progress();
         else if (!guard.idle(abort)) failed = true;
@@ -601,66 +635,78 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
       // descriptors built once; each MMA only adds a constant step
       const uint64_t dka = desc_kmajor(smem_u32(sK), 0), dva = desc_kmajor(smem_u32(sV), 0),
-                     dqa = desc_kmajor(smem_u32(sQ), 0), dga = desc_kmajor(smem_u32(sG), 0);
+                     dqd = desc_kmajor_half(smem_u32(sQD));
       uint32_t sf_par = 0;                // per-region phase bits of the st_free waits
-      failed = !mbar_wait(&bar.kv_full, 0, abort);
-      // S^T, dP^T of half tile u (queries 64 (u % 2).. of tile u / 2) into
-      // region u % R, once the dV / dK MMAs of unit u - R have released it
-      for (int u = 0; u < nunits && !failed; ++u) {
-        const int r = u % R, s = u >> 1, h = u & 1;
-        if (u >= R) {
-          if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
-          sf_par ^= 1u << r;
+      int g = 0, n = 0;
+      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+        if (!mbar_wait(&bar.kv_full, n & 1, abort)) { failed = true; break; }
+        // S^T, dP^T of half tile u (queries 64 (2 q0 + u)..) into region
+        // g % R, once the dV / dK MMAs of half tile g - R have released it
+        const int nunits = item_units(it);
+        for (int u = 0; u < nunits; ++u, ++g) {
+          const int r = g % R, sl = g % kKvSlots;
+          if (g >= R) {
+            if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+            sf_par ^= 1u << r;
+          }
+          if (!mbar_wait(&bar.qd_full[sl], (g / kKvSlots) & 1, abort)) { failed = true; break; }
+          tc_fence_after();
+          const uint64_t dq = dqd + desc_step((uint32_t)sl * kHalfPair);   // Q half, dO half after it
+          const uint64_t dg = dq + desc_step(kHalfTile);
+          const uint32_t dst = tmem + 128u * r;
+#pragma unroll
+          for (int ks = 0; ks < D / 8; ++ks)
+            mma_tf32_ss(dst, dka + kstep_kmajor(ks), dq + kstep_kmajor_half(ks), id_s, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < D / 8; ++ks)
+            mma_tf32_ss(dst + 64u, dva + kstep_kmajor(ks), dg + kstep_kmajor_half(ks), id_s, ks > 0);
+          tc_commit(&bar.sp_full[r]);
+          tc_commit(&bar.qd_empty[sl]);
         }
-        if (h == 0 && !mbar_wait(&bar.qd_full, s & 1, abort)) { failed = true; break; }
-        tc_fence_after();
-        const uint64_t qoff = desc_step((uint32_t)h * 64u * 128u);   // query rows 64h.. of the tile
-        const uint32_t dst = tmem + 128u * r;
-#pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(dst, dka + kstep_kmajor(ks), dqa + qoff + kstep_kmajor(ks), id_s, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(dst + 64u, dva + kstep_kmajor(ks), dga + qoff + kstep_kmajor(ks), id_s,
-                      ks > 0);
-        tc_commit(&bar.sp_full[r]);
-        if (h == 1) tc_commit(&bar.qd_empty);
+        if (!failed) tc_commit(&bar.kv_empty);     // K_j, V_j free once these MMAs are done
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------- dV / dK-MMA issuer
     if (lane == 0) {
       const uint32_t id_acc = idesc_tf32(128, D, 0, 1);
-      const uint64_t dqm = desc_mnmajor(smem_u32(sQmn), 0), dgm = desc_mnmajor(smem_u32(sGmn), 0);
+      const uint64_t dmn = desc_mnmajor_half(smem_u32(sQDmn));
       uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
-      // dV += P^T dO, dK += dS^T Q for half tile u (A operands in region u % R)
-      for (int u = 0; u < nunits && !failed; ++u) {
-        const int r = u % R, s = u >> 1, h = u & 1;
-        if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
-        ed_par ^= 1u << r;
-        if (h == 0 && !mbar_wait(&bar.mn_full, s & 1, abort)) { failed = true; break; }
-        tc_fence_after();
-        const uint64_t hoff = kstep_mnmajor(8 * h);
-        const uint32_t pa = tmem + 128u * r;
-        const uint32_t acc0 = u > 0 ? 1u : 0u;
+      int g = 0, n = 0;
+      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+        const int nunits = item_units(it);
+        // dV += P^T dO, dK += dS^T Q for half tile u (A operands in region g % R)
+        for (int u = 0; u < nunits; ++u, ++g) {
+          const int r = g % R, sl = g % kKvSlots;
+          if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
+          ed_par ^= 1u << r;
+          if (!mbar_wait(&bar.mn_full[sl], (g / kKvSlots) & 1, abort)) { failed = true; break; }
+          // the accumulators restart with this item: the previous item's
+          // epilogue must have read them
+          if (u == 0 && n > 0 && !mbar_wait(&bar.acc_free, (n - 1) & 1, abort)) { failed = true; break; }
+          tc_fence_after();
+          const uint64_t dqm = dmn + desc_step((uint32_t)sl * kHalfPair);   // Q half, dO half after it
+          const uint64_t dgm = dqm + desc_step(kHalfTile);
+          const uint32_t pa = tmem + 128u * r;
+          const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_tf32_ts(tmem + kColDV, pa + 8u * kk, dgm + hoff + kstep_mnmajor(kk), id_acc,
-                      kk > 0 ? 1u : acc0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_tf32_ts(tmem + kColDV, pa + 8u * kk, dgm + kstep_mnmajor(kk), id_acc,
+                        kk > 0 ? 1u : acc0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_tf32_ts(tmem + kColDK, pa + 64u + 8u * kk, dqm + hoff + kstep_mnmajor(kk), id_acc,
-                      kk > 0 ? 1u : acc0);
-        tc_commit(&bar.st_free[r]);
-        if (h == 1) tc_commit(&bar.mn_empty);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_tf32_ts(tmem + kColDK, pa + 64u + 8u * kk, dqm + kstep_mnmajor(kk), id_acc,
+                        kk > 0 ? 1u : acc0);
+          tc_commit(&bar.st_free[r]);
+          tc_commit(&bar.mn_empty[sl]);
+        }
+        if (!failed) tc_commit(&bar.acc_full);
       }
-      if (!failed) tc_commit(&bar.acc_full);
     }
   } else if (warp == kScoreWarp + 1) {
     // -------------------------------------------- query-constant producer
     // Loads the per-query constants of each unit into its slot while the
     // element groups work on earlier units (lane l: queries l and l + 32).
-    const long long rowbase = (long long)bh * T;
     // FWM: each group's copy of the shared grid's pairs, published with the
     // first units' constants
     if (!V::SOFTMAX && !V::MINMAX) {
@@ -676,11 +722,11 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       float m[2], rh[2], D[2], Wb[2], Wf[2], gm[2], gn[2];
       int am[2], an[2];
     };
-    auto load_raw = [&](int u, Raw& x) {
-      const int qi = q0 + (u >> 1);
+    auto load_raw = [&](int it, int u, Raw& x) {
+      const long long rowbase = (long long)item_bh(it) * T;
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
-        const int q = qi * KIA_TILE + 64 * (u & 1) + 32 * hq + lane;
+        const int q = 64 * (2 * item_q0(it) + u) + 32 * hq + lane;
         const long long qr = rowbase + (q < T ? q : T - 1);
         x.m[hq] = st.m[qr];
         x.rh[hq] = st.rh[qr];
@@ -694,21 +740,25 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
     };
     Raw cur;
-    if (nunits > 0) load_raw(0, cur);
-    for (int u = 0; u < nunits && !failed; ++u) {
-      const int sl = 2 * (u & 1) + ((u >> 1) & 1);
+    int it = blockIdx.x, u = 0;
+    if (it < nitems) load_raw(it, 0, cur);
+    for (int g = 0; it < nitems && !failed; ++g) {
+      const int sl = 2 * (g & 1) + ((g >> 1) & 1);
+      // the next half tile (possibly of the next item)
+      int it2 = it, u2 = u + 1;
+      if (u2 == item_units(it)) { u2 = 0; it2 += gridDim.x; }
       Raw nxt;
-      if (u + 1 < nunits) load_raw(u + 1, nxt);
-      if (u >= kSlots && !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[sl], ((u >> 2) - 1) & 1, abort))) {
+      if (it2 < nitems) load_raw(it2, u2, nxt);
+      if (g >= kSlots && !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[sl], ((g >> 2) - 1) & 1, abort))) {
         failed = true;
         break;
       }
-      const int qi = q0 + (u >> 1);
+      const int kt = item_kt(it);
+      const long long rowbase = (long long)item_bh(it) * T;
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
-        const int ql = 64 * (u & 1) + 32 * hq + lane;        // query in the tile
+        const int q = 64 * (2 * item_q0(it) + u) + 32 * hq + lane;
         const int e = sl * kSlotQ + 32 * hq + lane;          // its slot entry
-        const int q = qi * KIA_TILE + ql;
         const int Lq = p.causal ? q + 1 : T;
         const float rWb = Lq == 1 ? 0.0f : __fdiv_rn(1.0f, cur.Wb[hq]);
         sC4[e] = make_float4(cur.m[hq], cur.rh[hq], rWb, -cur.D[hq] * rWb);
@@ -744,6 +794,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       __syncwarp();
       mbar_arrive(&bar.qc_ready[sl]);
       cur = nxt;
+      it = it2;
+      u = u2;
     }
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
@@ -752,88 +804,93 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int grp = part >> 1;               // half tiles u with u % 2 == grp
     const int sub = part & 1;                // query columns 32 sub .. 32 sub + 31 of a unit
     const int r = quad * 32 + lane;
-    const int kj = kt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const long long rowbase = (long long)bh * T;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     // FWM: each group keeps its own copy of the shared grid's pairs
     const float2* sPairG = reinterpret_cast<const float2*>(sTab) + grp * K1;
-    for (int u = grp; u < nunits && !failed; u += 2) {
-      const int s = u >> 1;
-      const int qi = q0 + s;
-      const int rg = u % R;
-      const int sl = 2 * grp + ((u >> 1) & 1);           // this unit's constant slot
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[sl], (u >> 2) & 1, abort))) { failed = true; break; }
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (u / R) & 1, abort))) { failed = true; break; }
-      tc_fence_after();
-      const bool edge =
-          (p.causal && qi == kt) || (qi + 1) * KIA_TILE > T || (kt + 1) * KIA_TILE > T;
+    int gbase = 0, n = 0;
+    for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      const int kt = item_kt(it), q0 = item_q0(it), nunits = item_units(it);
+      const int kj = kt * KIA_TILE + r;
+      const long long rowbase = (long long)item_bh(it) * T;
+      for (int u = grp; u < nunits && !failed; u += 2) {
+        const int gu = gbase + u;
+        const int qi = q0 + (u >> 1);
+        const int rg = gu % R;
+        const int sl = 2 * grp + ((gu >> 1) & 1);           // this unit's constant slot
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[sl], (gu >> 2) & 1, abort))) { failed = true; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (gu / R) & 1, abort))) { failed = true; break; }
+        tc_fence_after();
+        const bool edge =
+            (p.causal && qi == kt) || (qi + 1) * KIA_TILE > T || (kt + 1) * KIA_TILE > T;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        float v[16], g[16];
-        const uint32_t cs = 128u * rg + 32u * sub + 16u * c;
-        tmem_ld16(tmem + lane_addr + cs, v);
-        tmem_ld16(tmem + lane_addr + cs + 64u, g);
-        tmem_ld_wait_regs(v, g);
-        const int ql0 = 64 * grp + 32 * sub + 16 * c;   // first query (in the tile) of the chunk
-        const int e0 = sl * kSlotQ + 32 * sub + 16 * c;  // its slot entry
+        for (int c = 0; c < 2; ++c) {
+          float v[16], g[16];
+          const uint32_t cs = 128u * rg + 32u * sub + 16u * c;
+          tmem_ld16(tmem + lane_addr + cs, v);
+          tmem_ld16(tmem + lane_addr + cs + 64u, g);
+          tmem_ld_wait_regs(v, g);
+          const int ql0 = 64 * (u & 1) + 32 * sub + 16 * c;   // first query (in the tile) of the chunk
+          const int e0 = sl * kSlotQ + 32 * sub + 16 * c;     // its slot entry
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int ql = ql0 + i;
-          const float4 c4 = sC4[e0 + i];
-          const float2 c2 = sC2[e0 + i];
-          const float dw = fmaf(g[i], c4.z, c4.w);
-          float P, dS;
-          if constexpr (V::MINMAX) {
-            const GridF grid{tab_in_smem ? sTab + (e0 + i) * K1
-                                         : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
-                             1};
-            // degenerate rows (rh = 0) take dS = dw; under the projection c2.y
-            // holds the shift, so the flag comes from rh itself
-            const float dg = PROJ ? (c4.y == 0.0f ? 1.0f : 0.0f) : c2.y;
-            kv_elem<V>(grid, c4.x, c4.y, dg, c2.x, Kf, Km1f, v[i], dw, P, dS);
-          } else {
-            kv_elem<V>(GridP{sPairG}, c4.x, c4.y, 0.0f, c2.x, Kf, Km1f, v[i], dw, P, dS);
-          }
-          if constexpr (PROJ) dS += c2.y;
-          if (edge) {
-            const int q = qi * KIA_TILE + ql;
-            if (!(kj < T && q < T && (!p.causal || kj <= q))) {
-              P = 0.0f;
-              dS = 0.0f;
+          for (int i = 0; i < 16; ++i) {
+            const int ql = ql0 + i;
+            const float4 c4 = sC4[e0 + i];
+            const float2 c2 = sC2[e0 + i];
+            const float dw = fmaf(g[i], c4.z, c4.w);
+            float P, dS;
+            if constexpr (V::MINMAX) {
+              const GridF grid{tab_in_smem ? sTab + (e0 + i) * K1
+                                           : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
+                               1};
+              // degenerate rows (rh = 0) take dS = dw; under the projection c2.y
+              // holds the shift, so the flag comes from rh itself
+              const float dg = PROJ ? (c4.y == 0.0f ? 1.0f : 0.0f) : c2.y;
+              kv_elem<V>(grid, c4.x, c4.y, dg, c2.x, Kf, Km1f, v[i], dw, P, dS);
+            } else {
+              kv_elem<V>(GridP{sPairG}, c4.x, c4.y, 0.0f, c2.x, Kf, Km1f, v[i], dw, P, dS);
             }
+            if constexpr (PROJ) dS += c2.y;
+            if (edge) {
+              const int q = qi * KIA_TILE + ql;
+              if (!(kj < T && q < T && (!p.causal || kj <= q))) {
+                P = 0.0f;
+                dS = 0.0f;
+              }
+            }
+            v[i] = P;
+            g[i] = dS;
           }
-          v[i] = P;
-          g[i] = dS;
-        }
-        if constexpr (!PROJ && !V::SOFTMAX) {
-          // the chunk's queries whose argmax (argmin) key lies in this warp's
-          // 32 keys: a warp-uniform test, the per-element work only for them
-          const int sh = 16 * c;
-          const uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu;
-          const uint32_t bn =
-              V::MINMAX ? (sMask[((sl * 2 + 1) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu : 0u;
-          if ((bm | bn) != 0u) {
+          if constexpr (!PROJ && !V::SOFTMAX) {
+            // the chunk's queries whose argmax (argmin) key lies in this warp's
+            // 32 keys: a warp-uniform test, the per-element work only for them
+            const int sh = 16 * c;
+            const uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu;
+            const uint32_t bn =
+                V::MINMAX ? (sMask[((sl * 2 + 1) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu : 0u;
+            if ((bm | bn) != 0u) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              if ((bm | bn) & (1u << i)) {
-                const int2 ci = sCI[e0 + i];
-                const float2 cg = sCG[e0 + i];
-                if ((bm >> i) & 1u) g[i] += (ci.x == r) ? cg.x : 0.0f;
-                if (V::MINMAX && ((bn >> i) & 1u)) g[i] += (ci.y == r) ? cg.y : 0.0f;
+              for (int i = 0; i < 16; ++i) {
+                if ((bm | bn) & (1u << i)) {
+                  const int2 ci = sCI[e0 + i];
+                  const float2 cg = sCG[e0 + i];
+                  if ((bm >> i) & 1u) g[i] += (ci.x == r) ? cg.x : 0.0f;
+                  if (V::MINMAX && ((bn >> i) & 1u)) g[i] += (ci.y == r) ? cg.y : 0.0f;
+                }
               }
             }
           }
+          tmem_st16(tmem + lane_addr + cs, v);
+          tmem_st16(tmem + lane_addr + cs + 64u, g);
         }
-        tmem_st16(tmem + lane_addr + cs, v);
-        tmem_st16(tmem + lane_addr + cs + 64u, g);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar.elem_done[rg]);
+        mbar_arrive(&bar.qc_free[sl]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bar.elem_done[rg]);
-      mbar_arrive(&bar.qc_free[sl]);
-    }
-    if (!failed && __all_sync(0xffffffffu, mbar_wait(&bar.acc_full, 0, abort))) {
+      if (failed) break;
+      gbase += nunits;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.acc_full, n & 1, abort))) { failed = true; break; }
       tc_fence_after();
       constexpr int kCols = D / kRowSplit;   // 16
       const uint32_t col = (uint32_t)(part * kCols);
@@ -841,17 +898,30 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_ld16(tmem + lane_addr + kColDV + col, v);
       tmem_ld16(tmem + lane_addr + kColDK + col, g);
       tmem_ld_wait_regs(v, g);
-      if (kj < T) {
-        float4* dv4 = reinterpret_cast<float4*>(dV + (rowbase + kj) * D + col);
-        float4* dk4 = reinterpret_cast<float4*>(dK + (rowbase + kj) * D + col);
+      tc_fence_before();
+      mbar_arrive(&bar.acc_free);            // the accumulators are free for the next item
+      // this warp's 32 rows x 16 columns of dV and dK, 8 columns at a time
+      // through its staging block: each store instruction then writes 16
+      // rows x 32 contiguous bytes (whole sectors) instead of 32 rows x 16
+      float* stg = sStage + (warp - 2) * 256;
+      const int row0 = kt * KIA_TILE + quad * 32;
 #pragma unroll
-        for (int i = 0; i < kCols / 4; ++i) {
-          dv4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          dk4[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+      for (int pass = 0; pass < 4; ++pass) {
+        const float* src = (pass < 2 ? v : g) + 8 * (pass & 1);
+        float* out = pass < 2 ? dV : dK;
+        *reinterpret_cast<float4*>(stg + lane * 8) = make_float4(src[0], src[1], src[2], src[3]);
+        *reinterpret_cast<float4*>(stg + lane * 8 + 4) = make_float4(src[4], src[5], src[6], src[7]);
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int rl = 16 * h + (lane >> 1);
+          const float4 val = *reinterpret_cast<const float4*>(stg + rl * 8 + (lane & 1) * 4);
+          if (row0 + rl < T)
+            *reinterpret_cast<float4*>(out + (rowbase + row0 + rl) * D + col + 8 * (pass & 1) +
+                                       (lane & 1) * 4) = val;
         }
+        __syncwarp();
       }
-    } else {
-      failed = true;
     }
   }
   if (failed || *abort) drain_in_flight();
@@ -874,7 +944,8 @@ size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? 4 * 64 * (p.K + 1) : 0) : 4 * (p.K + 1));
-  return 1024 + 6 * (size_t)D * KIA_TILE * 4 + 4 * 64 * (16 + 8 + 8 + 8) + 4 * 2 * 4 * 2 * 4 +
+  return 1024 + 2 * (size_t)D * KIA_TILE * 4 + 2 * kKvSlots * (size_t)kHalfPair +
+         4 * 64 * (16 + 8 + 8 + 8) + 4 * 2 * 4 * 2 * 4 + kElemThreads / 32 * 1024 +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdKBars);
 }
 
@@ -884,12 +955,13 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
                   float* dV, float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
                   void (*mark)(int, cudaStream_t)) {
   const int BH = B * H;
-  CUtensorMap tq, tqm, tg, tgm, tk, tkm, tv, tkh, tkmh, tvh;
-  if (!make_tmap(&tq, Q, BH, T, D) || !make_tmap(&tqm, Q, BH, T, D, true) ||
-      !make_tmap(&tg, dO, BH, T, D) || !make_tmap(&tgm, dO, BH, T, D, true) ||
-      !make_tmap(&tk, Kt, BH, T, D) || !make_tmap(&tkm, Kt, BH, T, D, true) ||
-      !make_tmap(&tv, Vv, BH, T, D) || !make_tmap(&tkh, Kt, BH, T, D, false, 64) ||
-      !make_tmap(&tkmh, Kt, BH, T, D, true, 64) || !make_tmap(&tvh, Vv, BH, T, D, false, 64))
+  CUtensorMap tq, tg, tk, tv, tqh, tqmh, tgh, tgmh, tkh, tkmh, tvh;
+  if (!make_tmap(&tq, Q, BH, T, D) || !make_tmap(&tg, dO, BH, T, D) ||
+      !make_tmap(&tk, Kt, BH, T, D) || !make_tmap(&tv, Vv, BH, T, D) ||
+      !make_tmap(&tqh, Q, BH, T, D, false, 64) || !make_tmap(&tqmh, Q, BH, T, D, true, 64) ||
+      !make_tmap(&tgh, dO, BH, T, D, false, 64) || !make_tmap(&tgmh, dO, BH, T, D, true, 64) ||
+      !make_tmap(&tkh, Kt, BH, T, D, false, 64) || !make_tmap(&tkmh, Kt, BH, T, D, true, 64) ||
+      !make_tmap(&tvh, Vv, BH, T, D, false, 64))
     return KIA_ERR_CUDA;
   const bool q_tab_smem = tc_bwd_q_smem<D>(p, true) <= 232448;
   const size_t smq = tc_bwd_q_smem<D>(p, q_tab_smem);
@@ -899,8 +971,7 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
   const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
                                     p.grad == KIA_GRAD_MIN_ONLY);
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
-  dim3 grid(BH, nt);
-  // the query pass is persistent: one CTA per SM walks the items
+  // both passes are persistent: one CTA per SM walks the items
   const int sms = num_sms();
   if (sms <= 0) return KIA_ERR_CUDA;
   const dim3 qgrid(std::min(sms, BH * nt));
@@ -925,8 +996,8 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk) !=
         cudaSuccess)
       return KIA_ERR_CUDA;
-    kern<<<grid, kTcThreads, smk, s>>>(tq, tqm, tg, tgm, tk, tv, st, wk, dK, dV, p, T,
-                                       kv_tab_smem ? 1 : 0);
+    kern<<<qgrid, kTcThreads, smk, s>>>(tqh, tqmh, tgh, tgmh, tk, tv, st, wk, dK, dV, p, BH, T,
+                                        kv_tab_smem ? 1 : 0);
     return KIA_OK;
   };
   const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;
