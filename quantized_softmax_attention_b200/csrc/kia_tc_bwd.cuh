@@ -38,7 +38,8 @@ namespace kia {
 
 constexpr int kBwdSmemTabK = 16;  // key pass: per-query grids up to K = 16 in shared memory
 constexpr int kBwdRegions = 3;    // TMEM regions of 128 columns (S | dP) in rotation
-constexpr int kBwdSlots = 3;      // query pass: slots of the half-tile key rings
+constexpr int kBwdSlots = 3;      // query pass: slots of the K / V half-tile ring
+constexpr int kKmnSlots = 2;      // query pass: slots of the K MN-major half-tile ring
 constexpr uint32_t kHalfTile = 64 * 64 * 4;       // one operand's half tile (64 rows, d = 64)
 constexpr uint32_t kHalfPair = 2 * kHalfTile;     // K half and V half (Q half and dO half)
 constexpr int kKvSlots = 2;       // key pass: slots of each half-tile query ring
@@ -102,8 +103,10 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   float* sQ = reinterpret_cast<float*>(base);
   float* sG = reinterpret_cast<float*>(base + kTile);
   uint8_t* sKV = base + 2 * kTile;                           // [3][K half | V half]
-  uint8_t* sKmn = sKV + kBwdSlots * kHalfPair;                // [3][K half, MN-major]
-  float* sAC = reinterpret_cast<float*>(sKmn + kBwdSlots * kHalfTile);   // [kRowSplit][2][128]
+  uint8_t* sKmn = sKV + kBwdSlots * kHalfPair;                // [2][K half, MN-major]
+  // epilogue: 1 KB per element warp to turn its rows into full-sector stores
+  float* sStage = reinterpret_cast<float*>(sKmn + kKmnSlots * kHalfTile);   // [16 warps][32][8]
+  float* sAC = sStage + kElemThreads / 32 * 256;              // [kRowSplit][2][128]
   float* sDc = sAC + 2 * kRowSplit * KIA_TILE;               // [128] centering D
   float* sTab = sDc + KIA_TILE;
   const int tab_floats =
@@ -199,8 +202,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
         if (im < nitems) {
-          const int sl = gm % kBwdSlots;
-          if (mbar_test(&bar.kmn_empty[sl], ((gm / kBwdSlots) & 1) ^ 1)) {
+          const int sl = gm % kKmnSlots;
+          if (mbar_test(&bar.kmn_empty[sl], ((gm / kKmnSlots) & 1) ^ 1)) {
             uint8_t* dst = sKmn + sl * kHalfTile;
             mbar_arrive_expect_tx(&bar.kmn_full[sl], kHalfTile);
             for (int b = 0; b < D / 32; ++b)
@@ -264,10 +267,10 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int nunits = item_units(it);
         // dQ of half tile u: A = dS in region g % R, B = K half (MN-major)
         for (int u = 0; u < nunits; ++u, ++g) {
-          const int r = g % R, sl = g % kBwdSlots;
+          const int r = g % R, sl = g % kKmnSlots;
           if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
           ed_par ^= 1u << r;
-          if (!mbar_wait(&bar.kmn_full[sl], (g / kBwdSlots) & 1, abort)) { failed = true; break; }
+          if (!mbar_wait(&bar.kmn_full[sl], (g / kKmnSlots) & 1, abort)) { failed = true; break; }
           // the accumulator restarts with this item: the previous item's
           // epilogue must have read it
           if (u == 0 && n > 0 && !mbar_wait(&bar.dq_free, (n - 1) & 1, abort)) { failed = true; break; }
@@ -447,10 +450,29 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             o[4 * i + 3] = fmaf(gn, kk.w, o[4 * i + 3]);
           }
         }
-        float4* o4 = reinterpret_cast<float4*>(dQ + (rowbase + q) * D + col);
+      }
+      // this warp's 32 rows x 16 columns of dQ, 8 columns at a time through
+      // its staging block, so that each store writes 16 rows x 32 bytes
+      {
+        float* stg = sStage + (warp - 2) * 256;
+        const int row0 = qt * KIA_TILE + quad * 32;
 #pragma unroll
-        for (int i = 0; i < kCols / 4; ++i)
-          o4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        for (int pass = 0; pass < 2; ++pass) {
+          const float* src = o + 8 * pass;
+          *reinterpret_cast<float4*>(stg + lane * 8) = make_float4(src[0], src[1], src[2], src[3]);
+          *reinterpret_cast<float4*>(stg + lane * 8 + 4) =
+              make_float4(src[4], src[5], src[6], src[7]);
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int rl = 16 * h + (lane >> 1);
+            const float4 val = *reinterpret_cast<const float4*>(stg + rl * 8 + (lane & 1) * 4);
+            if (row0 + rl < T)
+              *reinterpret_cast<float4*>(dQ + (rowbase + row0 + rl) * D + col + 8 * pass +
+                                         (lane & 1) * 4) = val;
+          }
+          __syncwarp();
+        }
       }
       if (q < T && part == 0) {
         wk.gm[rowbase + q] = gm;
@@ -935,7 +957,8 @@ size_t tc_bwd_q_smem(const OpParams& p, bool tab_in_smem) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
-  return 1024 + 2 * (size_t)D * KIA_TILE * 4 + kBwdSlots * (size_t)(kHalfPair + kHalfTile) +
+  return 1024 + 2 * (size_t)D * KIA_TILE * 4 + kBwdSlots * (size_t)kHalfPair +
+         kKmnSlots * (size_t)kHalfTile + kElemThreads / 32 * 1024 +
          (2 * kRowSplit + 1) * KIA_TILE * 4 + (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdQBars);
 }
 
