@@ -31,6 +31,8 @@
 // through shared memory.  O and O_L leave through shared memory and TMA
 // stores.
 #pragma once
+#include <algorithm>
+
 #include "kia_fast.cuh"
 #include "kia_tc.cuh"
 
@@ -57,16 +59,16 @@ struct FwdCfg {
 };
 
 struct FwdBars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;       // Q of an item / free once its S MMAs are done
   uint64_t k_full[3], k_empty[3];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[3];    // S of a unit ready in region r (tcgen05.commit)
   uint64_t s_free[3];    // sweep 1: the unit's group done reading region r
   uint64_t p_ready[3];   // sweep 2: P (and P_L) written into region r
   uint64_t pv_done[3];   // sweep 2: P V of region r finished (tcgen05.commit)
-  uint64_t o_full;       // all P V done
-  uint64_t out_ready;    // O (and O_L) staged in shared memory
-  uint64_t row_sync;     // element-thread rendezvous, used 3 times
+  uint64_t o_full;       // all P V of an item done
+  uint64_t o_free;       // the item's O (and O_L) read out of TMEM
+  uint64_t row_sync;     // element-thread rendezvous, three times per item
   uint32_t tmem_base;
   int abort;
 };
@@ -84,9 +86,8 @@ struct FwdRowX {
 template <int D, class V>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-              const __grid_constant__ CUtensorMap tmOL, StatsView st, OpParams p, int B, int H,
-              int T, int tab_in_smem) {
+              const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, StatsView st,
+              OpParams p, int B, int H, int T, int tab_in_smem) {
   constexpr bool PROB = V::PROB;
   using Cfg = FwdCfg<D, PROB>;
   constexpr int NSK = Cfg::kKStages, NSV = Cfg::kVStages, R = Cfg::kRegions;
@@ -97,23 +98,29 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   float* sK = sQ + kTileF;
   float* sV = sK + NSK * kTileF;
   FwdRowX& rx = *reinterpret_cast<FwdRowX*>(sV + NSV * kTileF);
-  float* sTab = reinterpret_cast<float*>(&rx + 1);
+  // epilogue: 1 KB per element warp to turn its rows into full-sector stores
+  float* sStage = reinterpret_cast<float*>(&rx + 1);      // [16 warps][32][8]
+  float* sTab = sStage + kElemThreads / 32 * 256;
   const int tab_floats =
       V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   FwdBars& bar = *reinterpret_cast<FwdBars*>(sTab + ((tab_floats + 31) & ~31));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
+  const int BH = B * H;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
-  const int qt = nt - 1 - blockIdx.y;
-  const int nkt = p.causal ? qt + 1 : nt;
-  const int nunits = 2 * nkt;          // half key tiles per sweep
+  const int nitems = BH * nt;
+  // item it -> (query tile, batch*head), heaviest causal tiles first; this
+  // CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+  auto item_qt = [&](int it) { return nt - 1 - it / BH; };
+  auto item_bh = [&](int it) { return it % BH; };
+  auto item_nkt = [&](int it) { return p.causal ? item_qt(it) + 1 : nt; };
   // TMEM columns: region r = [128 r, 128 r + 128); then O and O_L (D each)
   constexpr uint32_t col_o = 128u * R;
   constexpr uint32_t col_ol = col_o + D;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
+    mbar_init(&bar.q_empty, 1);
     for (int s = 0; s < 3; ++s) {
       mbar_init(&bar.k_full[s], 1);
       mbar_init(&bar.k_empty[s], 1);
@@ -127,7 +134,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(&bar.v_empty[s], 1);
     }
     mbar_init(&bar.o_full, 1);
-    mbar_init(&bar.out_ready, kElemThreads);
+    mbar_init(&bar.o_free, kElemThreads);
     mbar_init(&bar.row_sync, kElemThreads);
     bar.abort = 0;
     fence_barrier_init();
@@ -149,29 +156,34 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar.q_full, Cfg::kTileBytes);
-      for (int b = 0; b < D / 32; ++b)
-        tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.q_full, b * 32, qt * KIA_TILE, bh);
-      int kc = 0, vc = 0;
-      for (int sweep = 0; sweep < 2 && !failed; ++sweep) {
-        for (int j = 0; j < nkt; ++j) {
-          {
-            const int s = kc % NSK, n = kc / NSK;
-            if (!mbar_wait(&bar.k_empty[s], (n & 1) ^ 1, abort)) { failed = true; break; }
-            mbar_arrive_expect_tx(&bar.k_full[s], Cfg::kTileBytes);
-            float* dst = sK + s * kTileF;
-            for (int b = 0; b < D / 32; ++b)
-              tma_load_3d(dst + b * 32 * KIA_TILE, &tmK, &bar.k_full[s], b * 32, j * KIA_TILE, bh);
-            ++kc;
-          }
-          if (sweep == 1) {
-            const int s = vc % NSV, n = vc / NSV;
-            if (!mbar_wait(&bar.v_empty[s], (n & 1) ^ 1, abort)) { failed = true; break; }
-            mbar_arrive_expect_tx(&bar.v_full[s], Cfg::kTileBytes);
-            float* dst = sV + s * kTileF;
-            for (int b = 0; b < D / 32; ++b)
-              tma_load_3d(dst + b * 32 * KIA_TILE, &tmV, &bar.v_full[s], b * 32, j * KIA_TILE, bh);
-            ++vc;
+      int kc = 0, vc = 0, n = 0;
+      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+        const int qt = item_qt(it), bh = item_bh(it), nkt = item_nkt(it);
+        // Q of this item once the previous item's S MMAs are done with it
+        if (!mbar_wait(&bar.q_empty, (n & 1) ^ 1, abort)) { failed = true; break; }
+        mbar_arrive_expect_tx(&bar.q_full, Cfg::kTileBytes);
+        for (int b = 0; b < D / 32; ++b)
+          tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.q_full, b * 32, qt * KIA_TILE, bh);
+        for (int sweep = 0; sweep < 2 && !failed; ++sweep) {
+          for (int j = 0; j < nkt; ++j) {
+            {
+              const int s = kc % NSK, nn = kc / NSK;
+              if (!mbar_wait(&bar.k_empty[s], (nn & 1) ^ 1, abort)) { failed = true; break; }
+              mbar_arrive_expect_tx(&bar.k_full[s], Cfg::kTileBytes);
+              float* dst = sK + s * kTileF;
+              for (int b = 0; b < D / 32; ++b)
+                tma_load_3d(dst + b * 32 * KIA_TILE, &tmK, &bar.k_full[s], b * 32, j * KIA_TILE, bh);
+              ++kc;
+            }
+            if (sweep == 1) {
+              const int s = vc % NSV, nn = vc / NSV;
+              if (!mbar_wait(&bar.v_empty[s], (nn & 1) ^ 1, abort)) { failed = true; break; }
+              mbar_arrive_expect_tx(&bar.v_full[s], Cfg::kTileBytes);
+              float* dst = sV + s * kTileF;
+              for (int b = 0; b < D / 32; ++b)
+                tma_load_3d(dst + b * 32 * KIA_TILE, &tmV, &bar.v_full[s], b * 32, j * KIA_TILE, bh);
+              ++vc;
+            }
           }
         }
       }
@@ -179,40 +191,56 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------- score-MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_tf32(128, 64, 0, 0);
+      const uint32_t idesc_s = idesc_tf32(128, 64, 0, 0);    // sweep 2: half tiles
+      const uint32_t idesc_t = idesc_tf32(128, 128, 0, 0);   // sweep 1: whole tiles
       // descriptors built once; each MMA only adds a constant step
       const uint64_t dq0 = desc_kmajor(smem_u32(sQ), 0);
       const uint64_t dk0 = desc_kmajor(smem_u32(sK), 0);
-      int kc = 0;
-      uint32_t pv_par = 0;                // per-region phase bits of the pv_done waits
-      failed = !mbar_wait(&bar.q_full, 0, abort);
-      // S of unit U (sweep U / nunits, keys 64 (U % nunits) ..) into region
-      // U % R, once the unit R before it has released the region
-      const int total = 2 * nunits;
-      for (int U = 0; U < total && !failed; ++U) {
-        const int r = U % R, prev = U - R;
-        if (prev >= 0) {
-          if (prev < nunits) {
-            if (!mbar_wait(&bar.s_free[r], (prev / R) & 1, abort)) { failed = true; break; }
+      int kc = 0, n = 0, G = 0;           // K tiles, items, units (numbered across items)
+      // per region: phase bits of the s_free / pv_done waits, and whether its
+      // last unit was a sweep-2 unit (released by pv_done) or not (s_free)
+      uint32_t sf_par = 0, pv_par = 0, last_pv = 0;
+      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+        if (!mbar_wait(&bar.q_full, n & 1, abort)) { failed = true; break; }
+        const int nkt = item_nkt(it), nunits = 2 * nkt;
+        // units of an item: sweep 1 key tiles j (N = 128), then sweep 2 half
+        // tiles u (N = 64); unit G goes into region G % R once the unit R
+        // before it has released the region
+        for (int v = 0; v < nkt + nunits; ++v, ++G) {
+          const bool sweep2 = v >= nkt;
+          const int r = G % R;
+          if (G >= R) {
+            if ((last_pv >> r) & 1u) {
+              if (!mbar_wait(&bar.pv_done[r], (pv_par >> r) & 1u, abort)) { failed = true; break; }
+              pv_par ^= 1u << r;
+            } else {
+              if (!mbar_wait(&bar.s_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+              sf_par ^= 1u << r;
+            }
+          }
+          last_pv = sweep2 ? (last_pv | (1u << r)) : (last_pv & ~(1u << r));
+          const int h = sweep2 ? ((v - nkt) & 1) : 0;   // half of the key tile (sweep 2)
+          const int s = kc % NSK, nn = kc / NSK;
+          if (h == 0 && !mbar_wait(&bar.k_full[s], nn & 1, abort)) { failed = true; break; }
+          tc_fence_after();
+          const uint64_t dk = dk0 + desc_step((uint32_t)s * Cfg::kTileBytes + (uint32_t)h * 64u * 128u);
+          const uint32_t dst = tmem + 128u * r;
+          if (!sweep2) {
+#pragma unroll
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_t, ks > 0 ? 1u : 0u);
           } else {
-            if (!mbar_wait(&bar.pv_done[r], (pv_par >> r) & 1u, abort)) { failed = true; break; }
-            pv_par ^= 1u << r;
+#pragma unroll
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_s, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(&bar.s_full[r]);
+          if (!sweep2 || h == 1) {
+            tc_commit(&bar.k_empty[s]);
+            ++kc;
           }
         }
-        const int h = U & 1;              // half of the key tile
-        const int s = kc % NSK, n = kc / NSK;
-        if (h == 0 && !mbar_wait(&bar.k_full[s], n & 1, abort)) { failed = true; break; }
-        tc_fence_after();
-        const uint64_t dk = dk0 + desc_step((uint32_t)s * Cfg::kTileBytes + (uint32_t)h * 64u * 128u);
-        const uint32_t dst = tmem + 128u * r;
-#pragma unroll
-        for (int ks = 0; ks < D / 8; ++ks)
-          mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_s, ks > 0 ? 1u : 0u);
-        tc_commit(&bar.s_full[r]);
-        if (h == 1) {
-          tc_commit(&bar.k_empty[s]);
-          ++kc;
-        }
+        if (!failed) tc_commit(&bar.q_empty);    // Q free once these MMAs are done
       }
     }
   } else if (warp == 1) {
@@ -220,35 +248,42 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (lane == 0) {
       const uint32_t idesc_o = idesc_tf32(128, D, 0, 1);
       const uint64_t dv0 = desc_mnmajor(smem_u32(sV), 0);
-      int vc = 0;
+      int vc = 0, n = 0, G = 0;
       uint32_t pr_par = 0;                // per-region phase bits of the p_ready waits
-      for (int u = 0; u < nunits && !failed; ++u) {
-        const int U = nunits + u, r = U % R, h = u & 1;
-        if (!mbar_wait(&bar.p_ready[r], (pr_par >> r) & 1u, abort)) { failed = true; break; }
-        pr_par ^= 1u << r;
-        const int s = vc % NSV, n = vc / NSV;
-        if (h == 0 && !mbar_wait(&bar.v_full[s], n & 1, abort)) { failed = true; break; }
-        tc_fence_after();
-        const uint64_t dv = dv0 + desc_step((uint32_t)s * Cfg::kTileBytes) + kstep_mnmajor(8 * h);
-        const uint32_t pa = tmem + 128u * r;
-        const uint32_t acc0 = u > 0 ? 1u : 0u;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_tf32_ts(tmem + col_o, pa + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
-                      kk > 0 ? 1u : acc0);
-        if constexpr (PROB) {
+      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+        const int nunits = 2 * item_nkt(it);
+        G += item_nkt(it);                // this item's sweep-1 units (whole tiles)
+        for (int u = 0; u < nunits; ++u, ++G) {
+          const int r = G % R, h = u & 1;
+          if (!mbar_wait(&bar.p_ready[r], (pr_par >> r) & 1u, abort)) { failed = true; break; }
+          pr_par ^= 1u << r;
+          const int s = vc % NSV, nn = vc / NSV;
+          if (h == 0 && !mbar_wait(&bar.v_full[s], nn & 1, abort)) { failed = true; break; }
+          // the accumulators restart with this item: the previous item's
+          // epilogue must have read them
+          if (u == 0 && n > 0 && !mbar_wait(&bar.o_free, (n - 1) & 1, abort)) { failed = true; break; }
+          tc_fence_after();
+          const uint64_t dv = dv0 + desc_step((uint32_t)s * Cfg::kTileBytes) + kstep_mnmajor(8 * h);
+          const uint32_t pa = tmem + 128u * r;
+          const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + col_ol, pa + 64u + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
+            mma_tf32_ts(tmem + col_o, pa + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
                         kk > 0 ? 1u : acc0);
+          if constexpr (PROB) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_tf32_ts(tmem + col_ol, pa + 64u + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
+                          kk > 0 ? 1u : acc0);
+          }
+          tc_commit(&bar.pv_done[r]);
+          if (h == 1) {
+            tc_commit(&bar.v_empty[s]);
+            ++vc;
+          }
         }
-        tc_commit(&bar.pv_done[r]);
-        if (h == 1) {
-          tc_commit(&bar.v_empty[s]);
-          ++vc;
-        }
+        if (!failed) tc_commit(&bar.o_full);
       }
-      if (!failed) tc_commit(&bar.o_full);
     }
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
@@ -257,206 +292,239 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int grp = part >> 1;                 // units U with U % 2 == grp
     const int sub = part & 1;                  // columns 32 sub .. 32 sub + 31 of a unit
     const int r = quad * 32 + lane;            // query row in the tile
-    const int qrow = qt * KIA_TILE + r;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const long long grow = (long long)bh * T + (qrow < T ? qrow : T - 1);
-    // a unit holds masked keys when it reaches past the first row of the
-    // tile (causal) or past the sequence end
-    const int edge_from = p.causal ? (qt * KIA_TILE) / 64 : nunits;
-    auto is_edge = [&](int u) { return u >= edge_from || (u + 1) * 64 > T; };
-    // row extrema and the keys of their first occurrences
-    float m = -INFINITY, n = INFINITY;
-    int am = 0, an = 0;
-    // sweep 1: statistics of this thread's 32 columns of each of its units
-    for (int U = grp; U < nunits; U += 2) {
-      const int rg = U % R;
-      float v[32];
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[rg], (U / R) & 1, abort))) { failed = true; break; }
-      tc_fence_after();
-      tmem_ld32(tmem + lane_addr + 128u * rg + 32u * sub, v);
-      tmem_ld_wait_regs(v);
-      tc_fence_before();
-      mbar_arrive(&bar.s_free[rg]);
-      const int key0 = 64 * U + 32 * sub;
-      if (!is_edge(U)) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          // strict comparisons keep the lowest index on ties
-          if (v[i] > m) am = key0 + i;
-          m = fmaxf(m, v[i]);
-          if constexpr (V::MINMAX) {
-            if (v[i] < n) an = key0 + i;
-            n = fminf(n, v[i]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = key0 + i;
-          const bool ok = key < T && (!p.causal || key <= qrow);
-          const float vx = ok ? v[i] : -INFINITY;
-          if (vx > m) am = key;
-          m = fmaxf(m, vx);
-          if constexpr (V::MINMAX) {
-            const float vn = ok ? v[i] : INFINITY;
-            if (vn < n) an = key;
-            n = fminf(n, vn);
-          }
-        }
-      }
-    }
-    // merge the four threads of the row (lowest index on ties)
-    rx.m[part][r] = m;
-    rx.n[part][r] = n;
-    rx.am[part][r] = am;
-    rx.an[part][r] = an;
-    mbar_arrive(&bar.row_sync);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
-    m = rx.m[0][r];
-    am = rx.am[0][r];
-    n = rx.n[0][r];
-    an = rx.an[0][r];
-#pragma unroll
-    for (int h = 1; h < kRowSplit; ++h) {
-      const float mh = rx.m[h][r], nh = rx.n[h][r];
-      const int ah = rx.am[h][r], bh2 = rx.an[h][r];
-      am = (mh > m) ? ah : (mh == m ? min(am, ah) : am);
-      m = fmaxf(m, mh);
-      an = (nh < n) ? bh2 : (nh == n ? min(an, bh2) : an);
-      n = fminf(n, nh);
-    }
-    if constexpr (!V::MINMAX) {
-      n = m;   // FWM and softmax do not use the row minimum
-      an = am;
-    }
-    // calibration (section 3) and the grid
-    const RowCal rc = row_calibration(p, m, n);
-    const bool degen = V::MINMAX && rc.h == 0.0f;
-    float2* sPair = reinterpret_cast<float2*>(sTab);
-    if constexpr (V::MINMAX) {
-      if (tab_in_smem) {
-        for (int k = part; k <= p.K; k += kRowSplit) {
-          const float G = degen ? 1.0f : grid_value(k, rc.h);
-          sTab[k * KIA_TILE + r] = G;
-          if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
-        }
-      } else {
-        for (int k = part; k <= p.K; k += kRowSplit) {
-          const float G = degen ? 1.0f : grid_value(k, rc.h);
-          if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
-        }
-        __threadfence_block();
-      }
-    } else if constexpr (!V::SOFTMAX) {
-      // one grid for every row: pairs (G_k, G_{k+1}), k = 0..K-1
-      const int k = (int)threadIdx.x - 64;
-      if (k >= 0 && k < p.K) {
-        const float G0 = grid_value(k, p.fwm_h), G1 = grid_value(k + 1, p.fwm_h);
-        sPair[k] = make_float2(G0, G1);
-        if (bh == 0 && qt == nt - 1) {
-          st.table[k] = G0;
-          if (k == p.K - 1) st.table[k + 1] = G1;
-        }
-      }
-    }
-    mbar_arrive(&bar.row_sync);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 1, abort))) failed = true;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
-    // sweep 2: weights -> P (and P_L) in TMEM, normalisers
-    float W = 0.0f, WL = 0.0f;
-    auto sweep2 = [&](auto grid) {
-      for (int u = grp; u < nunits && !failed; u += 2) {
-        const int U = nunits + u, rg = U % R;
+    int gbase = 0, n = 0;
+    for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      const int qt = item_qt(it), bh = item_bh(it), nunits = 2 * item_nkt(it);
+      const int qrow = qt * KIA_TILE + r;
+      const long long grow = (long long)bh * T + (qrow < T ? qrow : T - 1);
+      // a unit holds masked keys when it reaches past the first row of the
+      // tile (causal) or past the sequence end
+      const int edge_from = p.causal ? (qt * KIA_TILE) / 64 : nunits;
+      auto is_edge = [&](int u) { return u >= edge_from || (u + 1) * 64 > T; };
+      // row extrema and the keys of their first occurrences
+      float m = -INFINITY, n_ = INFINITY;
+      int am = 0, an = 0;
+      // sweep 1: statistics of this thread's 64 columns of each of its key
+      // tiles (group g takes the tiles j with j % 2 == g)
+      const int nkt = nunits / 2;
+      for (int j = grp; j < nkt; j += 2) {
+        const int U = gbase + j, rg = U % R;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[rg], (U / R) & 1, abort))) { failed = true; break; }
         tc_fence_after();
-        const bool edge = is_edge(u);
-        const uint32_t col_s = 128u * rg + 32u * sub;   // this thread's S / P columns
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
-          float w16[16], vl[16];
-          tmem_ld16(tmem + lane_addr + col_s + 16u * c, w16);
-          tmem_ld_wait_regs(w16);
-          const int key0 = 64 * u + 32 * sub + 16 * c;
-          if (!edge) {
+          float v[32];
+          tmem_ld32(tmem + lane_addr + 128u * rg + 64u * sub + 32u * c, v);
+          tmem_ld_wait_regs(v);
+          if (c == 1) {
+            tc_fence_before();
+            mbar_arrive(&bar.s_free[rg]);
+          }
+          const int key0 = KIA_TILE * j + 64 * sub + 32 * c;
+          if (!is_edge(2 * j + sub)) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float wf, wl;
-              fwd_weights<V, false>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
-              W += wf;
-              w16[i] = wf;
-              if constexpr (PROB) {
-                WL += wl;
-                vl[i] = wl;
+            for (int i = 0; i < 32; ++i) {
+              // strict comparisons keep the lowest index on ties
+              if (v[i] > m) am = key0 + i;
+              m = fmaxf(m, v[i]);
+              if constexpr (V::MINMAX) {
+                if (v[i] < n_) an = key0 + i;
+                n_ = fminf(n_, v[i]);
               }
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float wf, wl;
-              fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
+            for (int i = 0; i < 32; ++i) {
               const int key = key0 + i;
               const bool ok = key < T && (!p.causal || key <= qrow);
-              wf = ok ? wf : 0.0f;
-              wl = ok ? wl : 0.0f;
-              W += wf;
-              w16[i] = wf;
-              if constexpr (PROB) {
-                WL += wl;
-                vl[i] = wl;
+              const float vx = ok ? v[i] : -INFINITY;
+              if (vx > m) am = key;
+              m = fmaxf(m, vx);
+              if constexpr (V::MINMAX) {
+                const float vn = ok ? v[i] : INFINITY;
+                if (vn < n_) an = key;
+                n_ = fminf(n_, vn);
               }
             }
           }
-          tmem_st16(tmem + lane_addr + col_s + 16u * c, w16);
-          if constexpr (PROB) tmem_st16(tmem + lane_addr + col_s + 64u + 16u * c, vl);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bar.p_ready[rg]);
       }
-    };
-    if constexpr (V::MINMAX) {
-      if (tab_in_smem) sweep2(GridF{sTab + r, KIA_TILE});
-      else sweep2(GridF{st.table + grow * (p.K + 1), 1});
-    } else {
-      sweep2(GridP{sPair});
-    }
-    // normalisers of the whole row
-    rx.W[part][r] = W;
-    rx.WL[part][r] = WL;
-    mbar_arrive(&bar.row_sync);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, 0, abort))) failed = true;
-    const float Wrow = (rx.W[0][r] + rx.W[1][r]) + (rx.W[2][r] + rx.W[3][r]);
-    const float WLrow =
-        PROB ? (rx.WL[0][r] + rx.WL[1][r]) + (rx.WL[2][r] + rx.WL[3][r]) : Wrow;
-    // epilogue: this thread stages D/4 columns of its row of O (and O_L) in
-    // the free K ring, laid out as the TMA store's 128-byte swizzle expects
-    // (16-byte chunk c of row r at chunk c ^ (r % 8)); one thread stores
-    const bool out_ok = !failed && __all_sync(0xffffffffu, mbar_wait(&bar.o_full, 0, abort));
-    float* sO = sK;                       // [D / 32][128 rows][32] per output
-    if (out_ok) {
+      if (failed) break;
+      // merge the four threads of the row (lowest index on ties)
+      rx.m[part][r] = m;
+      rx.n[part][r] = n_;
+      rx.am[part][r] = am;
+      rx.an[part][r] = an;
+      mbar_arrive(&bar.row_sync);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n) & 1, abort))) { failed = true; break; }
+      m = rx.m[0][r];
+      am = rx.am[0][r];
+      n_ = rx.n[0][r];
+      an = rx.an[0][r];
+#pragma unroll
+      for (int h = 1; h < kRowSplit; ++h) {
+        const float mh = rx.m[h][r], nh = rx.n[h][r];
+        const int ah = rx.am[h][r], bh2 = rx.an[h][r];
+        am = (mh > m) ? ah : (mh == m ? min(am, ah) : am);
+        m = fmaxf(m, mh);
+        an = (nh < n_) ? bh2 : (nh == n_ ? min(an, bh2) : an);
+        n_ = fminf(n_, nh);
+      }
+      if constexpr (!V::MINMAX) {
+        n_ = m;   // FWM and softmax do not use the row minimum
+        an = am;
+      }
+      // calibration (section 3) and the grid
+      const RowCal rc = row_calibration(p, m, n_);
+      const bool degen = V::MINMAX && rc.h == 0.0f;
+      float2* sPair = reinterpret_cast<float2*>(sTab);
+      if constexpr (V::MINMAX) {
+        if (tab_in_smem) {
+          for (int k = part; k <= p.K; k += kRowSplit) {
+            const float G = degen ? 1.0f : grid_value(k, rc.h);
+            sTab[k * KIA_TILE + r] = G;
+            if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
+          }
+        } else {
+          for (int k = part; k <= p.K; k += kRowSplit) {
+            const float G = degen ? 1.0f : grid_value(k, rc.h);
+            if (qrow < T) st.table[grow * (p.K + 1) + k] = G;
+          }
+          __threadfence_block();
+        }
+      } else if constexpr (!V::SOFTMAX) {
+        // one grid for every row: pairs (G_k, G_{k+1}), k = 0..K-1
+        const int k = (int)threadIdx.x - 64;
+        if (k >= 0 && k < p.K) {
+          const float G0 = grid_value(k, p.fwm_h), G1 = grid_value(k + 1, p.fwm_h);
+          sPair[k] = make_float2(G0, G1);
+          if (bh == 0 && qt == nt - 1) {
+            st.table[k] = G0;
+            if (k == p.K - 1) st.table[k + 1] = G1;
+          }
+        }
+      }
+      mbar_arrive(&bar.row_sync);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n + 1) & 1, abort))) { failed = true; break; }
+      // sweep 2: weights -> P (and P_L) in TMEM, normalisers
+      float W = 0.0f, WL = 0.0f;
+      auto sweep2 = [&](auto grid) {
+        for (int u = grp; u < nunits && !failed; u += 2) {
+          const int U = gbase + nkt + u, rg = U % R;
+          if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[rg], (U / R) & 1, abort))) { failed = true; break; }
+          tc_fence_after();
+          const bool edge = is_edge(u);
+          const uint32_t col_s = 128u * rg + 32u * sub;   // this thread's S / P columns
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            float w16[16], vl[16];
+            tmem_ld16(tmem + lane_addr + col_s + 16u * c, w16);
+            tmem_ld_wait_regs(w16);
+            const int key0 = 64 * u + 32 * sub + 16 * c;
+            if (!edge) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float wf, wl;
+                fwd_weights<V, false>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
+                W += wf;
+                w16[i] = wf;
+                if constexpr (PROB) {
+                  WL += wl;
+                  vl[i] = wl;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float wf, wl;
+                fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
+                const int key = key0 + i;
+                const bool ok = key < T && (!p.causal || key <= qrow);
+                wf = ok ? wf : 0.0f;
+                wl = ok ? wl : 0.0f;
+                W += wf;
+                w16[i] = wf;
+                if constexpr (PROB) {
+                  WL += wl;
+                  vl[i] = wl;
+                }
+              }
+            }
+            tmem_st16(tmem + lane_addr + col_s + 16u * c, w16);
+            if constexpr (PROB) tmem_st16(tmem + lane_addr + col_s + 64u + 16u * c, vl);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&bar.p_ready[rg]);
+        }
+      };
+      if constexpr (V::MINMAX) {
+        if (tab_in_smem) sweep2(GridF{sTab + r, KIA_TILE});
+        else sweep2(GridF{st.table + grow * (p.K + 1), 1});
+      } else {
+        sweep2(GridP{sPair});
+      }
+      if (failed) break;
+      gbase += nkt + nunits;
+      // normalisers of the whole row
+      rx.W[part][r] = W;
+      rx.WL[part][r] = WL;
+      mbar_arrive(&bar.row_sync);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n + 2) & 1, abort))) { failed = true; break; }
+      const float Wrow = (rx.W[0][r] + rx.W[1][r]) + (rx.W[2][r] + rx.W[3][r]);
+      const float WLrow =
+          PROB ? (rx.WL[0][r] + rx.WL[1][r]) + (rx.WL[2][r] + rx.WL[3][r]) : Wrow;
+      // epilogue: this thread's D/4 columns of O (and O_L) out of TMEM, the
+      // accumulators released, then stores staged per warp into whole sectors
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.o_full, n & 1, abort))) { failed = true; break; }
       tc_fence_after();
       constexpr int kCols = D / kRowSplit;     // 16 or 32
       const uint32_t col = (uint32_t)(part * kCols);
-      float o[kCols];
-      auto stage_row = [&](uint32_t tcol, float* dst, float w) {
-        if constexpr (kCols == 16) tmem_ld16(tmem + lane_addr + tcol + col, o);
-        else tmem_ld32(tmem + lane_addr + tcol + col, o);
-        tmem_ld_wait_regs(o);
-        const float rw = __frcp_rn(w);
-        float* blk = dst + (col / 32) * (32 * KIA_TILE) + r * 32;
-        const int c0 = (col % 32) / 4;        // first 16-byte chunk in the 128-byte row
+      float o[kCols], ol[PROB ? kCols : 1];
+      if constexpr (kCols == 16) tmem_ld16(tmem + lane_addr + col_o + col, o);
+      else tmem_ld32(tmem + lane_addr + col_o + col, o);
+      tmem_ld_wait_regs(o);
+      if constexpr (PROB) {
+        if constexpr (kCols == 16) tmem_ld16(tmem + lane_addr + col_ol + col, ol);
+        else tmem_ld32(tmem + lane_addr + col_ol + col, ol);
+        tmem_ld_wait_regs(ol);
+      }
+      tc_fence_before();
+      mbar_arrive(&bar.o_free);
+      {
+        float* stg = sStage + (warp - 2) * 256;
+        const int row0 = qt * KIA_TILE + quad * 32;
+        const long long rb = (long long)bh * T;
+        const float rw = __frcp_rn(Wrow), rwl = __frcp_rn(WLrow);
 #pragma unroll
-        for (int i = 0; i < kCols / 4; ++i) {
-          const int ch = (c0 + i) ^ (r & 7);
-          *reinterpret_cast<float4*>(blk + ch * 4) =
-              make_float4(o[4 * i] * rw, o[4 * i + 1] * rw, o[4 * i + 2] * rw, o[4 * i + 3] * rw);
+        for (int pass = 0; pass < (PROB ? 2 : 1) * kCols / 8; ++pass) {
+          constexpr int kPer = kCols / 8;             // passes per output
+          const bool second = PROB && pass >= kPer;
+          const int cp = second ? pass - kPer : pass;
+          const float* src = ((PROB && second) ? ol : o) + 8 * cp;
+          const float sc = second ? rwl : rw;
+          float* out = second ? st.OL : O;
+          *reinterpret_cast<float4*>(stg + lane * 8) =
+              make_float4(src[0] * sc, src[1] * sc, src[2] * sc, src[3] * sc);
+          *reinterpret_cast<float4*>(stg + lane * 8 + 4) =
+              make_float4(src[4] * sc, src[5] * sc, src[6] * sc, src[7] * sc);
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int rl = 16 * h + (lane >> 1);
+            const float4 val = *reinterpret_cast<const float4*>(stg + rl * 8 + (lane & 1) * 4);
+            if (row0 + rl < T)
+              *reinterpret_cast<float4*>(out + (rb + row0 + rl) * D + col + 8 * cp +
+                                         (lane & 1) * 4) = val;
+          }
+          __syncwarp();
         }
-      };
-      stage_row(col_o, sO, Wrow);
-      if constexpr (PROB) stage_row(col_ol, sO + D * KIA_TILE, WLrow);
+      }
       if (qrow < T && part == 0) {
         st.m[grow] = m;
-        st.n[grow] = n;
+        st.n[grow] = n_;
         st.am[grow] = am;
         st.an[grow] = an;
         st.rh[grow] = degen ? 0.0f : rc.rh;
@@ -465,21 +533,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         st.Wb[grow] = (!V::SOFTMAX && lerp_normpoint(p)) ? WLrow : Wrow;
       }
       if (bh == 0 && qt == nt - 1 && threadIdx.x == 64) write_header(st.header, B, H, T, D, p);
-    } else {
-      failed = true;
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&bar.out_ready);
-    if (threadIdx.x == 64) {
-      if (mbar_wait(&bar.out_ready, 0, abort) && !*abort) {
-        for (int b = 0; b < D / 32; ++b) {
-          tma_store_3d(&tmO, sO + b * 32 * KIA_TILE, b * 32, qt * KIA_TILE, bh);
-          if constexpr (PROB)
-            tma_store_3d(&tmOL, sO + D * KIA_TILE + b * 32 * KIA_TILE, b * 32, qt * KIA_TILE, bh);
-        }
-        tma_store_commit();
-        tma_store_wait_all();
-      }
     }
   }
   if (failed || *abort) drain_in_flight();
@@ -495,16 +548,12 @@ size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem) {
   const int tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   return 1024 + (size_t)(1 + Cfg::kKStages + Cfg::kVStages) * Cfg::kTileBytes + sizeof(FwdRowX) +
-         (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
+         kElemThreads / 32 * 1024 + (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
 }
 
 template <int D, class V>
 int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, float* O,
                  const StatsView& st, int B, int H, int T, const OpParams& p, cudaStream_t s) {
-  CUtensorMap to, tol;
-  if (!make_tmap(&to, O, B * H, T, D) ||
-      !make_tmap(&tol, V::PROB ? st.OL : O, B * H, T, D))
-    return KIA_ERR_CUDA;
   bool tab_in_smem = true;
   size_t smem = tc_fwd_smem<D, V::PROB>(p, true);
   if (smem > 232448) {
@@ -515,9 +564,12 @@ int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   if (cudaFuncSetAttribute(tc_fwd_kernel<D, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return KIA_ERR_CUDA;
+  // persistent: one CTA per SM walks the (query tile, batch*head) items
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
-  dim3 grid(B * H, nt);
-  tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, to, tol, st, p, B, H, T,
+  const int sms = num_sms();
+  if (sms <= 0) return KIA_ERR_CUDA;
+  const dim3 grid(std::min(sms, B * H * nt));
+  tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, O, st, p, B, H, T,
                                                      tab_in_smem ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
 }
