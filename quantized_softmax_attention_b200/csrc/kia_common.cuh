@@ -284,6 +284,25 @@ struct PollGuard {
   }
 };
 
+// A persistent CTA's work items: round r of gridDim.x items gives CTA c the
+// item r * G + c in even rounds and r * G + (G - 1 - c) in odd ones.  Items
+// are numbered heaviest first, so the serpentine order evens out the sums.
+struct ItemSeq {
+  int r, n;
+  __device__ __forceinline__ explicit ItemSeq(int nitems) : r(-1), n(nitems) {}
+  // the next item of this CTA, or -1 when there is none
+  __device__ __forceinline__ int next() {
+    const int G = (int)gridDim.x;
+    for (;;) {
+      ++r;
+      if ((long long)r * G >= n) return -1;
+      const int c = (r & 1) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x;
+      const int it = r * G + c;
+      if (it < n) return it;
+    }
+  }
+};
+
 // After an abort: let copies and MMAs already in flight land before the CTA
 // releases its shared and tensor memory (bounded: ~200 us).
 __device__ __forceinline__ void drain_in_flight() {

@@ -118,7 +118,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   const int nitems = BH * nt;
   // item it -> (query tile, batch*head), heaviest causal tiles first; this
-  // CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+  // CTA takes its items in the serpentine order of ItemSeq
   auto item_qt = [&](int it) { return nt - 1 - it / BH; };
   auto item_bh = [&](int it) { return it % BH; };
   auto item_units = [&](int it) { return 2 * (p.causal ? item_qt(it) + 1 : nt); };
@@ -167,13 +167,14 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmKmn);
       tma_prefetch_desc(&tmV);
-      int iq = blockIdx.x, nq = 0;                   // next item for Q / dO
-      int ik = blockIdx.x, uk = 0, gk = 0;            // K / V ring: item, unit, global unit
-      int im = blockIdx.x, um = 0, gm = 0;            // K MN-major ring
+      ItemSeq sq(nitems), sk(nitems), sm(nitems);
+      int iq = sq.next(), nq = 0;                    // next item for Q / dO
+      int ik = sk.next(), uk = 0, gk = 0;             // K / V ring: item, unit, global unit
+      int im = sm.next(), um = 0, gm = 0;             // K MN-major ring
       PollGuard guard;
-      while ((iq < nitems || ik < nitems || im < nitems) && !failed) {
+      while ((iq >= 0 || ik >= 0 || im >= 0) && !failed) {
         bool moved = false;
-        if (iq < nitems && mbar_test(&bar.qd_empty, (nq & 1) ^ 1)) {
+        if (iq >= 0 && mbar_test(&bar.qd_empty, (nq & 1) ^ 1)) {
           mbar_arrive_expect_tx(&bar.qd_full, 2 * kTile);
           for (int b = 0; b < D / 32; ++b) {
             tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, item_qt(iq) * KIA_TILE,
@@ -181,11 +182,11 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tma_load_3d(sG + b * 32 * KIA_TILE, &tmG, &bar.qd_full, b * 32, item_qt(iq) * KIA_TILE,
                         item_bh(iq));
           }
-          iq += gridDim.x;
+          iq = sq.next();
           ++nq;
           moved = true;
         }
-        if (ik < nitems) {
+        if (ik >= 0) {
           const int sl = gk % kBwdSlots;
           if (mbar_test(&bar.kv_empty[sl], ((gk / kBwdSlots) & 1) ^ 1)) {
             uint8_t* dst = sKV + sl * kHalfPair;
@@ -197,11 +198,11 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                           64 * uk, item_bh(ik));
             }
             ++gk;
-            if (++uk == item_units(ik)) { uk = 0; ik += gridDim.x; }
+            if (++uk == item_units(ik)) { uk = 0; ik = sk.next(); }
             moved = true;
           }
         }
-        if (im < nitems) {
+        if (im >= 0) {
           const int sl = gm % kKmnSlots;
           if (mbar_test(&bar.kmn_empty[sl], ((gm / kKmnSlots) & 1) ^ 1)) {
             uint8_t* dst = sKmn + sl * kHalfTile;
@@ -210,7 +211,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               tma_load_3d(dst + b * kHalfBlockBytes, &tmKmn, &bar.kmn_full[sl], b * 32, 64 * um,
                           item_bh(im));
             ++gm;
-            if (++um == item_units(im)) { um = 0; im += gridDim.x; }
+            if (++um == item_units(im)) { um = 0; im = sm.next(); }
             moved = true;
           }
         }
@@ -227,7 +228,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                      dkv = desc_kmajor_half(smem_u32(sKV));
       uint32_t sf_par = 0;                // per-region phase bits of the st_free waits
       int g = 0, n = 0;                   // global half tile, item count
-      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      ItemSeq seq(nitems);
+      for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         if (!mbar_wait(&bar.qd_full, n & 1, abort)) { failed = true; break; }
         // S, dP of half tile u (keys 64 u..) into region g % R, once the dQ
         // MMA of half tile g - R has released the region
@@ -263,7 +265,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint64_t dkm = desc_mnmajor_half(smem_u32(sKmn));
       uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
       int g = 0, n = 0;
-      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      ItemSeq seq(nitems);
+      for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         const int nunits = item_units(it);
         // dQ of half tile u: A = dS in region g % R, B = K half (MN-major)
         for (int u = 0; u < nunits; ++u, ++g) {
@@ -303,7 +306,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (k >= 0 && k < p.K) sPair[k] = make_float2(st.table[k], st.table[k + 1]);
     }
     int gbase = 0, n = 0;
-    for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+    ItemSeq seq(nitems);
+    for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       const int qt = item_qt(it), bh = item_bh(it), nunits = item_units(it);
       const int q = qt * KIA_TILE + r;
       const long long rowbase = (long long)bh * T;
@@ -542,7 +546,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   const int nitems = BH * nt;
   // item it -> (key tile, batch*head), heaviest causal tiles (most queries)
-  // first; this CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+  // first; this CTA takes its items in the serpentine order of ItemSeq
   auto item_kt = [&](int it) { return it / BH; };
   auto item_bh = [&](int it) { return it % BH; };
   auto item_q0 = [&](int it) { return p.causal ? item_kt(it) : 0; };
@@ -596,13 +600,14 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tma_prefetch_desc(&tmGmn);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int ikv = blockIdx.x, nkv = 0;                 // next item for K / V
-      int iq = blockIdx.x, uq = 0, gq = 0;            // K-major ring: item, unit, global unit
-      int im = blockIdx.x, um = 0, gm = 0;            // MN-major ring
+      ItemSeq skv(nitems), sq(nitems), sm(nitems);
+      int ikv = skv.next(), nkv = 0;                 // next item for K / V
+      int iq = sq.next(), uq = 0, gq = 0;             // K-major ring: item, unit, global unit
+      int im = sm.next(), um = 0, gm = 0;             // MN-major ring
       PollGuard guard;
-      while ((ikv < nitems || iq < nitems || im < nitems) && !failed) {
+      while ((ikv >= 0 || iq >= 0 || im >= 0) && !failed) {
         bool moved = false;
-        if (ikv < nitems && mbar_test(&bar.kv_empty, (nkv & 1) ^ 1)) {
+        if (ikv >= 0 && mbar_test(&bar.kv_empty, (nkv & 1) ^ 1)) {
           mbar_arrive_expect_tx(&bar.kv_full, 2 * kTile);
           for (int b = 0; b < D / 32; ++b) {
             tma_load_3d(sK + b * 32 * KIA_TILE, &tmK, &bar.kv_full, b * 32, item_kt(ikv) * KIA_TILE,
@@ -610,11 +615,11 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tma_load_3d(sV + b * 32 * KIA_TILE, &tmV, &bar.kv_full, b * 32, item_kt(ikv) * KIA_TILE,
                         item_bh(ikv));
           }
-          ikv += gridDim.x;
+          ikv = skv.next();
           ++nkv;
           moved = true;
         }
-        if (iq < nitems) {
+        if (iq >= 0) {
           const int sl = gq % kKvSlots;
           if (mbar_test(&bar.qd_empty[sl], ((gq / kKvSlots) & 1) ^ 1)) {
             uint8_t* dst = sQD + sl * kHalfPair;
@@ -626,11 +631,11 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                           row, item_bh(iq));
             }
             ++gq;
-            if (++uq == item_units(iq)) { uq = 0; iq += gridDim.x; }
+            if (++uq == item_units(iq)) { uq = 0; iq = sq.next(); }
             moved = true;
           }
         }
-        if (im < nitems) {
+        if (im >= 0) {
           const int sl = gm % kKvSlots;
           if (mbar_test(&bar.mn_empty[sl], ((gm / kKvSlots) & 1) ^ 1)) {
             uint8_t* dst = sQDmn + sl * kHalfPair;
@@ -643,7 +648,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                           row, item_bh(im));
             }
             ++gm;
-            if (++um == item_units(im)) { um = 0; im += gridDim.x; }
+            if (++um == item_units(im)) { um = 0; im = sm.next(); }
             moved = true;
           }
         }
@@ -660,7 +665,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                      dqd = desc_kmajor_half(smem_u32(sQD));
       uint32_t sf_par = 0;                // per-region phase bits of the st_free waits
       int g = 0, n = 0;
-      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      ItemSeq seq(nitems);
+      for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         if (!mbar_wait(&bar.kv_full, n & 1, abort)) { failed = true; break; }
         // S^T, dP^T of half tile u (queries 64 (2 q0 + u)..) into region
         // g % R, once the dV / dK MMAs of half tile g - R have released it
@@ -695,7 +701,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const uint64_t dmn = desc_mnmajor_half(smem_u32(sQDmn));
       uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
       int g = 0, n = 0;
-      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      ItemSeq seq(nitems);
+      for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         const int nunits = item_units(it);
         // dV += P^T dO, dK += dS^T Q for half tile u (A operands in region g % R)
         for (int u = 0; u < nunits; ++u, ++g) {
@@ -762,15 +769,16 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
     };
     Raw cur;
-    int it = blockIdx.x, u = 0;
-    if (it < nitems) load_raw(it, 0, cur);
-    for (int g = 0; it < nitems && !failed; ++g) {
+    ItemSeq cseq(nitems);
+    int it = cseq.next(), u = 0;
+    if (it >= 0) load_raw(it, 0, cur);
+    for (int g = 0; it >= 0 && !failed; ++g) {
       const int sl = 2 * (g & 1) + ((g >> 1) & 1);
       // the next half tile (possibly of the next item)
       int it2 = it, u2 = u + 1;
-      if (u2 == item_units(it)) { u2 = 0; it2 += gridDim.x; }
+      if (u2 == item_units(it)) { u2 = 0; it2 = cseq.next(); }
       Raw nxt;
-      if (it2 < nitems) load_raw(it2, u2, nxt);
+      if (it2 >= 0) load_raw(it2, u2, nxt);
       if (g >= kSlots && !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[sl], ((g >> 2) - 1) & 1, abort))) {
         failed = true;
         break;
@@ -831,7 +839,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // FWM: each group keeps its own copy of the shared grid's pairs
     const float2* sPairG = reinterpret_cast<const float2*>(sTab) + grp * K1;
     int gbase = 0, n = 0;
-    for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+    ItemSeq seq(nitems);
+    for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       const int kt = item_kt(it), q0 = item_q0(it), nunits = item_units(it);
       const int kj = kt * KIA_TILE + r;
       const long long rowbase = (long long)item_bh(it) * T;

@@ -110,7 +110,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   const int nitems = BH * nt;
   // item it -> (query tile, batch*head), heaviest causal tiles first; this
-  // CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+  // CTA takes its items in the serpentine order of ItemSeq
   auto item_qt = [&](int it) { return nt - 1 - it / BH; };
   auto item_bh = [&](int it) { return it % BH; };
   auto item_nkt = [&](int it) { return p.causal ? item_qt(it) + 1 : nt; };
@@ -157,7 +157,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       int kc = 0, vc = 0, n = 0;
-      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      ItemSeq seq(nitems);
+      for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         const int qt = item_qt(it), bh = item_bh(it), nkt = item_nkt(it);
         // Q of this item once the previous item's S MMAs are done with it
         if (!mbar_wait(&bar.q_empty, (n & 1) ^ 1, abort)) { failed = true; break; }
@@ -200,7 +201,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // per region: phase bits of the s_free / pv_done waits, and whether its
       // last unit was a sweep-2 unit (released by pv_done) or not (s_free)
       uint32_t sf_par = 0, pv_par = 0, last_pv = 0;
-      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      ItemSeq seq(nitems);
+      for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         if (!mbar_wait(&bar.q_full, n & 1, abort)) { failed = true; break; }
         const int nkt = item_nkt(it), nunits = 2 * nkt;
         // units of an item: sweep 1 key tiles j (N = 128), then sweep 2 half
@@ -250,7 +252,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const uint64_t dv0 = desc_mnmajor(smem_u32(sV), 0);
       int vc = 0, n = 0, G = 0;
       uint32_t pr_par = 0;                // per-region phase bits of the p_ready waits
-      for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+      ItemSeq seq(nitems);
+      for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         const int nunits = 2 * item_nkt(it);
         G += item_nkt(it);                // this item's sweep-1 units (whole tiles)
         for (int u = 0; u < nunits; ++u, ++G) {
@@ -295,7 +298,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     int gbase = 0, n = 0;
-    for (int it = blockIdx.x; it < nitems && !failed; it += gridDim.x, ++n) {
+    ItemSeq seq(nitems);
+    for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       const int qt = item_qt(it), bh = item_bh(it), nunits = 2 * item_nkt(it);
       const int qrow = qt * KIA_TILE + r;
       const long long grow = (long long)bh * T + (qrow < T ? qrow : T - 1);
