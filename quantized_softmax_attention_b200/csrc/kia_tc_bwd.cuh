@@ -863,35 +863,41 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           tmem_ld_wait_regs(v, g);
           const int ql0 = 64 * (u & 1) + 32 * sub + 16 * c;   // first query (in the tile) of the chunk
           const int e0 = sl * kSlotQ + 32 * sub + 16 * c;     // its slot entry
+          // the element loop, without the mask test on units with no masked pair
+          auto body = [&](auto edge_c) {
+            constexpr bool EDGE = decltype(edge_c)::value;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int ql = ql0 + i;
-            const float4 c4 = sC4[e0 + i];
-            const float2 c2 = sC2[e0 + i];
-            const float dw = fmaf(g[i], c4.z, c4.w);
-            float P, dS;
-            if constexpr (V::MINMAX) {
-              const GridF grid{tab_in_smem ? sTab + (e0 + i) * K1
-                                           : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
-                               1};
-              // degenerate rows (rh = 0) take dS = dw; under the projection c2.y
-              // holds the shift, so the flag comes from rh itself
-              const float dg = PROJ ? (c4.y == 0.0f ? 1.0f : 0.0f) : c2.y;
-              kv_elem<V>(grid, c4.x, c4.y, dg, c2.x, Kf, Km1f, v[i], dw, P, dS);
-            } else {
-              kv_elem<V>(GridP{sPairG}, c4.x, c4.y, 0.0f, c2.x, Kf, Km1f, v[i], dw, P, dS);
-            }
-            if constexpr (PROJ) dS += c2.y;
-            if (edge) {
-              const int q = qi * KIA_TILE + ql;
-              if (!(kj < T && q < T && (!p.causal || kj <= q))) {
-                P = 0.0f;
-                dS = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+              const int ql = ql0 + i;
+              const float4 c4 = sC4[e0 + i];
+              const float2 c2 = sC2[e0 + i];
+              const float dw = fmaf(g[i], c4.z, c4.w);
+              float P, dS;
+              if constexpr (V::MINMAX) {
+                const GridF grid{tab_in_smem ? sTab + (e0 + i) * K1
+                                             : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
+                                 1};
+                // degenerate rows (rh = 0) take dS = dw; under the projection c2.y
+                // holds the shift, so the flag comes from rh itself
+                const float dg = PROJ ? (c4.y == 0.0f ? 1.0f : 0.0f) : c2.y;
+                kv_elem<V>(grid, c4.x, c4.y, dg, c2.x, Kf, Km1f, v[i], dw, P, dS);
+              } else {
+                kv_elem<V>(GridP{sPairG}, c4.x, c4.y, 0.0f, c2.x, Kf, Km1f, v[i], dw, P, dS);
               }
+              if constexpr (PROJ) dS += c2.y;
+              if constexpr (EDGE) {
+                const int q = qi * KIA_TILE + ql;
+                if (!(kj < T && q < T && (!p.causal || kj <= q))) {
+                  P = 0.0f;
+                  dS = 0.0f;
+                }
+              }
+              v[i] = P;
+              g[i] = dS;
             }
-            v[i] = P;
-            g[i] = dS;
-          }
+          };
+          if (edge) body(std::true_type{});
+          else body(std::false_type{});
           if constexpr (!PROJ && !V::SOFTMAX) {
             // the chunk's queries whose argmax (argmin) key lies in this warp's
             // 32 keys: a warp-uniform test, the per-element work only for them
