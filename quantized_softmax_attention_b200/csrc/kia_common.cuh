@@ -327,6 +327,11 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
+// Bring the 128-byte line holding addr into L2 (no register result).
+__device__ __forceinline__ void prefetch_l2(const void* addr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(addr));
+}
+
 // 3-D tiled store: the box at (x, y, z) of the tensor map from shared
 // memory (rows outside the tensor are not written), as one bulk group.
 __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int x, int y, int z) {

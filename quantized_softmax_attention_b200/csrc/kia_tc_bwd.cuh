@@ -321,6 +321,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int L = p.causal ? q + 1 : T;
       // a one-key row has P = 1 whatever its score: zero gradient
       const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]);
+      // the key rows this row's epilogue gathers (argmax, argmin) into L2 now
+      prefetch_l2(Kt + (rowbase + am) * D + part * (D / kRowSplit));
+      if constexpr (V::MINMAX) prefetch_l2(Kt + (rowbase + an) * D + part * (D / kRowSplit));
       // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE): four
       // consecutive element threads read one row's D values (coalesced), add
       // their partial sums by shuffles and leave the row's D in shared memory
@@ -405,6 +408,31 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (failed) break;
       gbase += nunits;
+      {
+        // the next item's rows (statistics, dO and O_bar for its centering)
+        // into L2 while this item's epilogue runs
+        ItemSeq peek = seq;
+        const int nx = peek.next();
+        if (nx >= 0) {
+          const int e = (int)threadIdx.x - 64;
+          const int qn = item_qt(nx) * KIA_TILE + (e >> 2);
+          const long long rn = (long long)item_bh(nx) * T + (qn < T ? qn : T - 1);
+          prefetch_l2(dO + rn * D + (e & 3) * (D / 4));
+          prefetch_l2((V::PROB ? st.OL : O) + rn * D + (e & 3) * (D / 4));
+          if (e < 5 * 4) {
+            // 128 rows of one per-row array = four 128-byte lines
+            const long long r0 = (long long)item_bh(nx) * T + item_qt(nx) * KIA_TILE +
+                                 32 * (e & 3);
+            const int a = e >> 2;
+            const void* ptr = a == 0 ? (const void*)(st.m + r0)
+                            : a == 1 ? (const void*)(st.am + r0)
+                            : a == 2 ? (const void*)(st.an + r0)
+                            : a == 3 ? (const void*)(st.rh + r0)
+                                     : (const void*)(st.Wb + r0);
+            if (item_qt(nx) * KIA_TILE + 32 * (e & 3) < T) prefetch_l2(ptr);
+          }
+        }
+      }
       // row sums of the four column groups
       sAC[(part * 2 + 0) * KIA_TILE + r] = A;
       sAC[(part * 2 + 1) * KIA_TILE + r] = C;
