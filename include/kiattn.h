@@ -166,6 +166,26 @@ int kiattn_weights_from_S(const float* S, int rows, int cols, const int* row_len
 int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T, int d,
                   const kia_config* cfg, void* stream);
 
+/* Fixed-upstream decomposition of the score gradient (Appendix F, "The
+ * detached-gradient record and its replication"; Table S24): for each row i,
+ * out[3 i + 0] = ||dS_i||^2 (the backward's dS of the mode it ran with),
+ * out[3 i + 1] = the squared norm of that mode's maximum-side calibration
+ * term (g_m^2 for full and max-only; under the zero-sum projection the
+ * common-mode shift c_i on every visible key, c_i^2 |J_i|; 0 otherwise),
+ * out[3 i + 2] = that of the minimum-side term (g_n^2 for full and min-only,
+ * 0 otherwise), i.e. the norms of (mode - detach) split by extremum.  The
+ * maximum- and minimum-dependent norm ratios of the appendix are
+ * sqrt(sum out[.,1] / sum out[.,0]) and sqrt(sum out[.,2] / sum out[.,0])
+ * over the rows of interest.
+ * dS: the dS_dbg [B,H,T,T] written by kiattn_bwd; workspace: the workspace of
+ * that same kiattn_bwd call (it holds g_m, g_n per row); cfg as in that call;
+ * out: device fp64 [B*H*T*3], caller-owned.  Sums run in fp64.  Nothing is
+ * written when the kiattn_bwd call rejected its stats (workspace status set).
+ * Errors: INVALID_ARG (null pointer, B, H or T < 1), UNSUPPORTED (shape
+ * beyond the operator's limits), CUDA (launch failure). */
+int kiattn_grad_decomposition(const float* dS, const void* workspace, int B, int H, int T,
+                              const kia_config* cfg, double* out, void* stream);
+
 /* Error word raised by device code since the last reset: KIA_ERR_TIMEOUT
  * when a bounded wait inside a kernel gave up, KIA_ERR_STATS_MISMATCH when
  * kiattn_bwd was handed stats written for another shape or config (the

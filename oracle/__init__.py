@@ -195,6 +195,37 @@ def attention(Q, K, V, dO, cfg: RefConfig, bh_range=None, want_bwd=True, dump=Fa
     return out
 
 
+def grad_decomposition(Q, K, V, dO, cfg: RefConfig, bh_range=None):
+    """Fixed-upstream decomposition of the score gradient (Appendix F, "The
+    detached-gradient record and its replication"; Table S24), fp64, by
+    definition: the calibration terms of a mode are what it adds to the
+    detached gradient at the same upstream, dS_mode - dS_detach; the
+    maximum-dependent term is that difference at the row's argmax key (under
+    the zero-sum projection the whole common-mode shift), the
+    minimum-dependent term the difference at the argmin key.  Returns
+    [BH, T, 3]: ||dS_mode,i||^2, ||max term||^2, ||min term||^2 per row."""
+    mode = attention(Q, K, V, dO, cfg, bh_range=bh_range, dump=True)
+    det = attention(Q, K, V, dO, cfg.replace(grad=GRAD_DETACH), bh_range=bh_range,
+                    dump=True)
+    dS, diff = mode["dS"], mode["dS"] - det["dS"]
+    T = dS.shape[-1]
+    dS = dS.reshape(-1, T, T)
+    diff = diff.reshape(-1, T, T)
+    st = mode["stats"].reshape(-1, T, ST_COUNT)
+    out = np.zeros((dS.shape[0], T, 3))
+    out[..., 0] = np.sum(dS * dS, axis=-1)
+    am = st[..., ST_AM].astype(np.int64)
+    an = st[..., ST_AN].astype(np.int64)
+    at_m = np.take_along_axis(diff, am[..., None], axis=-1)[..., 0]
+    at_n = np.take_along_axis(diff, an[..., None], axis=-1)[..., 0]
+    if cfg.grad == GRAD_PROJECT:
+        out[..., 1] = np.sum(diff * diff, axis=-1)
+    else:
+        out[..., 1] = at_m * at_m
+        out[..., 2] = np.where(an != am, at_n * at_n, 0.0)
+    return out
+
+
 def weights_fp32(S, row_len, cfg: RefConfig):
     """The fp32 weight stage as a fixed sequence of fp32 operations (the
     bit-exact contract of the CUDA weight stage).  Returns w, bin, t, m, n."""

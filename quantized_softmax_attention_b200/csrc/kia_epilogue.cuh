@@ -205,4 +205,34 @@ bwd_project_scan_kernel(const float* __restrict__ Q, const float* __restrict__ K
   }
 }
 
+// Fixed-upstream decomposition of the score gradient (Appendix F; Table
+// S24): per row, ||dS_i||^2 over the visible keys and the squared norms of
+// the maximum- and minimum-side calibration terms the backward applied.  One
+// warp per row, fp64 sums.
+__global__ void __launch_bounds__(32 * kRowWarps)
+grad_decomp_kernel(const float* __restrict__ dS, WorkView wk, long long rows, int T, int causal,
+                   int grad, double* __restrict__ out) {
+  if (*wk.status != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kRowWarps + warp;
+  if (row >= rows) return;
+  const int i = (int)(row % T);
+  const int L = causal ? i + 1 : T;
+  const float* ds = dS + row * (long long)T;
+  double s2 = 0.0;
+  for (int j = lane; j < L; j += 32) {
+    const double v = (double)ds[j];
+    s2 += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  if (lane == 0) {
+    const double gm = (double)wk.gm[row], gn = (double)wk.gn[row];
+    const bool proj = grad == KIA_GRAD_PROJECT;
+    out[3 * row + 0] = s2;
+    out[3 * row + 1] = proj ? gm * gm * (double)L : gm * gm;
+    out[3 * row + 2] = proj ? 0.0 : gn * gn;
+  }
+}
+
 }  // namespace kia

@@ -335,6 +335,21 @@ int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T
   return d == 64 ? tc_scores<64>(Q, Kt, S, B, H, T, p, s) : tc_scores<128>(Q, Kt, S, B, H, T, p, s);
 }
 
+int kiattn_grad_decomposition(const float* dS, const void* workspace, int B, int H, int T,
+                              const kia_config* cfg, double* out, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_shape(B, H, T, 64))) return rc;
+  if (!dS || !workspace || !out) return KIA_ERR_INVALID_ARG;
+  const long long rows = (long long)B * H * T;
+  WorkView wk = work_view(const_cast<void*>(workspace), rows);
+  const long long blocks = (rows + kRowWarps - 1) / kRowWarps;
+  if (blocks > 0x7fffffffll) return KIA_ERR_UNSUPPORTED;
+  grad_decomp_kernel<<<(unsigned)blocks, 32 * kRowWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+      dS, wk, rows, T, cfg->causal, cfg->grad, out);
+  return launch_status();
+}
+
 const char* kiattn_strerror(int code) {
   switch (code) {
     case KIA_OK: return "ok";

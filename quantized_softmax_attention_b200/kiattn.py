@@ -30,7 +30,7 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error", 
 SYMBOLS = ("kiattn_stats_bytes", "kiattn_workspace_bytes", "kiattn_fwd", "kiattn_bwd",
            "kiattn_weights_from_S", "kiattn_scores", "kiattn_strerror", "kiattn_version",
            "kiattn_device_error", "kiattn_profile_enable", "kiattn_profile_read",
-           "kiattn_bwd_noalloc")
+           "kiattn_bwd_noalloc", "kiattn_grad_decomposition")
 NOALLOC_MAX_ROWS = 1 << 20
 PHASES = ("fwd", "bwd_prep", "bwd_query_pass", "bwd_key_pass", "bwd_calibration")
 
@@ -91,6 +91,8 @@ def _load():
     lib.kiattn_bwd_noalloc.restype = i
     lib.kiattn_weights_from_S.argtypes = [vp, i, i, vp, cp, vp, vp, vp, vp, vp, vp]
     lib.kiattn_scores.argtypes = [vp, vp, vp, i, i, i, i, cp, vp]
+    lib.kiattn_grad_decomposition.argtypes = [vp, vp, i, i, i, cp, vp, vp]
+    lib.kiattn_grad_decomposition.restype = i
     lib.kiattn_strerror.argtypes = [i]
     lib.kiattn_strerror.restype = ctypes.c_char_p
     lib.kiattn_version.restype = i
@@ -172,6 +174,16 @@ def kiattn_weights_from_S(S, row_len, cfg: Config, w, bin=None, t=None, row_m=No
     _check("kiattn_weights_from_S",
            _lib.kiattn_weights_from_S(_p(S), rows, cols, _p(row_len), ctypes.byref(cfg.c()), _p(w),
                                       _p(bin), _p(t), _p(row_m), _p(row_n), _stream(stream)))
+
+
+def kiattn_grad_decomposition(dS, workspace, out, cfg: Config, stream=None):
+    """Per-row ||dS_i||^2 and the squared norms of the maximum- and
+    minimum-side calibration terms (out: device fp64 [B, H, T, 3]) from the
+    dS_dbg and workspace of one kiattn_bwd call with the same cfg."""
+    B, H, T, _ = dS.shape
+    _check("kiattn_grad_decomposition",
+           _lib.kiattn_grad_decomposition(_p(dS), _p(workspace), B, H, T, ctypes.byref(cfg.c()),
+                                          _p(out), _stream(stream)))
 
 
 def kiattn_scores(Q, K, S, cfg: Config, stream=None):

@@ -221,3 +221,62 @@ def test_tc_d128_forward_and_backward():
         # the d = 128 backward runs the exact-fp32 kernels on the TF32 forward
         for name in ("dQ", "dK", "dV"):
             assert errs[name] < 2e-3, (cal, rec, ste, errs)
+
+
+# ---------------------------------------- fixed-upstream decomposition
+
+@pytest.mark.parametrize("gemm,rule,tol", [(K.GEMM_TF32, TF32_RULE, 5e-3),
+                                           (K.GEMM_FP32, ref.ROUND_NONE, 5e-5)])
+@pytest.mark.parametrize("cal", [K.CAL_MINMAX, K.CAL_FWM])
+def test_grad_decomposition_matches_oracle(gemm, rule, tol, cal):
+    """Per-row ||dS||^2 and squared maximum- / minimum-side calibration terms
+    from kiattn_grad_decomposition (after a kiattn_bwd that dumped dS) against
+    the oracle's mode-minus-detach decomposition, every gradient mode.  The
+    quantities are squares, so the bound is about twice the operator's."""
+    from parity_util import ref_cfg
+    B, H, T, d = 1, 2, 200, 64
+    Q, Kt, V, dO = _inputs(B, H, T, d, 61 + cal, qscale=0.5)
+    for rec, ste in RECSTE:
+        for grad in MODES:
+            cfg = K.Config(K=4, cal=cal, rec=rec, ste=ste, grad=grad, gemm=gemm)
+            flags = flag_rows(Q, Kt, cfg, rule, 1e-4)
+            dO2 = dO.copy()
+            dO2[flags] = 0.0
+            q, k, v, g = (torch.from_numpy(np.ascontiguousarray(x)).cuda() for x in (Q, Kt, V, dO2))
+            bufs = K.Buffers(B, H, T, d, cfg)
+            dS = torch.empty((B, H, T, T), dtype=torch.float32, device="cuda")
+            out = torch.full((B, H, T, 3), float("nan"), dtype=torch.float64, device="cuda")
+            K.kiattn_fwd(q, k, v, bufs.O, bufs.stats, cfg)
+            K.kiattn_bwd(q, k, v, bufs.O, g, bufs.stats, bufs.dQ, bufs.dK, bufs.dV, bufs.work, cfg,
+                         dS_dbg=dS)
+            K.kiattn_grad_decomposition(dS, bufs.work, out, cfg)
+            torch.cuda.synchronize()
+            assert K.kiattn_device_error(True) == 0
+            got = out.cpu().numpy().reshape(B * H, T, 3)
+            want = ref.grad_decomposition(Q, Kt, V, dO2, ref_cfg(cfg, rule))
+            assert np.isfinite(got).all()
+            for c in range(3):
+                err = rel_l2(got[..., c], want[..., c])
+                assert err < tol, (rec, ste, grad, c, err)
+            if grad in (K.GRAD_DETACH,):
+                assert np.all(got[..., 1:] == 0.0)
+            if grad == K.GRAD_MAX_ONLY or grad == K.GRAD_PROJECT or cal == K.CAL_FWM:
+                assert np.all(got[..., 2] == 0.0)
+            if grad == K.GRAD_MIN_ONLY:
+                assert np.all(got[..., 1] == 0.0)
+            # the appendix's norm ratios
+            for c in (1, 2):
+                rg = np.sqrt(got[..., c].sum() / got[..., 0].sum())
+                rw = np.sqrt(want[..., c].sum() / want[..., 0].sum())
+                assert abs(rg - rw) <= tol * max(rw, 1e-3), (grad, c, rg, rw)
+
+
+def test_grad_decomposition_rejects_bad_arguments():
+    cfg = K.Config()
+    dS = torch.zeros((1, 1, 128, 128), device="cuda")
+    out = torch.zeros((1, 1, 128, 3), dtype=torch.float64, device="cuda")
+    bufs = K.Buffers(1, 1, 128, 64, cfg)
+    with pytest.raises(RuntimeError):
+        K.kiattn_grad_decomposition(dS, None, out, cfg)
+    with pytest.raises(RuntimeError):
+        K.kiattn_grad_decomposition(dS[:, :, :0], bufs.work, out, cfg)

@@ -44,7 +44,8 @@ def _near_kink(S, L, cfg, tol):
     for i in range(S.shape[0]):
         s = S[i, :L[i]]
         h = st[i, ref.ST_H]
-        u = (st[i, ref.ST_M] - s) / h
+        with np.errstate(invalid="ignore", divide="ignore"):
+            u = (st[i, ref.ST_M] - s) / h
         frac = np.abs(u - np.round(u))
         if cfg.cal == ref.CAL_FWM:
             frac = np.where(u > cfg.K + 0.5, 1.0, frac)
@@ -569,3 +570,101 @@ def test_fp32_weight_stage_tracks_fp64(cal, rec):
         assert err.max() <= 2e-6 * max(1.0, K / 4), (K, err.max())
         if rec == ref.REC_NEAREST:
             assert np.all(f["w"][mask] == w64[mask].astype(np.float32)) or err.max() < 1e-7
+
+
+# --------------------------------------- fixed-upstream decomposition
+
+def _decomp_inputs(seed, B=1, H=2, T=20, d=8):
+    rng = np.random.default_rng(seed)
+    Q = (rng.standard_normal((B, H, T, d)) * 1.5).astype(np.float32)
+    K = rng.standard_normal((B, H, T, d)).astype(np.float32)
+    V = rng.standard_normal((B, H, T, d)).astype(np.float32)
+    dO = rng.standard_normal((B, H, T, d)).astype(np.float32)
+    return Q, K, V, dO
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_decomposition_max_and_min_terms_are_extremum_derivatives(causal):
+    """Appendix F, fixed-upstream decomposition (Table S24): at a fixed
+    upstream dP = dO V^T the maximum-dependent term is the derivative of the
+    row loss sum_j P_ij dP_ij with respect to the row maximum m_i (minimum
+    frozen), the minimum-dependent term the derivative with respect to n_i;
+    both checked by central differences of the LERP forward with the other
+    extremum frozen."""
+    Q, K, V, dO = _decomp_inputs(21)
+    T = Q.shape[2]
+    for cal in CALS:
+        cfg = ref.RefConfig(K=4, cal=cal, rec=ref.REC_LERP, causal=causal)
+        dec = ref.grad_decomposition(Q, K, V, dO, cfg)
+        for hh in range(Q.shape[1]):
+            q, k, v, g = (x[0, hh].astype(np.float64) for x in (Q, K, V, dO))
+            S, dP = q @ k.T, g @ v.T
+            Ls = np.arange(1, T + 1) if causal else np.full(T, T)
+            Sm = np.where(np.arange(T)[None, :] < Ls[:, None], S, -np.inf)
+            Sn = np.where(np.arange(T)[None, :] < Ls[:, None], S, np.inf)
+            m0, n0 = Sm.max(1), Sn.min(1)
+            ok = ~_near_kink(S, Ls, cfg, 1e-3) & (Ls >= 3)
+            assert ok.sum() >= T // 2
+            eps = 1e-6
+            d_m = (_loss(S, Ls, cfg, dP, m0 + eps, n0) - _loss(S, Ls, cfg, dP, m0 - eps, n0)) / (2 * eps)
+            d_n = (_loss(S, Ls, cfg, dP, m0, n0 + eps) - _loss(S, Ls, cfg, dP, m0, n0 - eps)) / (2 * eps)
+            np.testing.assert_allclose(dec[hh, :, 1][ok], (d_m ** 2)[ok], rtol=1e-6, atol=1e-12)
+            np.testing.assert_allclose(dec[hh, :, 2][ok], (d_n ** 2)[ok], rtol=1e-6, atol=1e-12)
+            if cal == ref.CAL_FWM:
+                assert np.all(dec[hh, :, 2] == 0.0)
+
+
+@pytest.mark.parametrize("rec,ste", RECSTE)
+def test_decomposition_modes_split_the_full_terms(rec, ste):
+    """The terms a partial mode keeps are the full mode's own (Appendix B:
+    max-only keeps the maximum-dependent term, min-only the minimum one,
+    detach neither), ||dS||^2 is the squared norm of the mode's dump, and
+    under the zero-sum projection the maximum slot holds |J_i| c_i^2 with
+    c_i minus the mean of the detached row (the dump's rows then sum to zero)."""
+    Q, K, V, dO = _decomp_inputs(22)
+    for cal in CALS:
+        base = ref.RefConfig(K=4, cal=cal, rec=rec, ste=ste)
+        dec = {m: ref.grad_decomposition(Q, K, V, dO, base.replace(grad=m)) for m in MODES}
+        full = dec[ref.GRAD_FULL]
+        np.testing.assert_array_equal(dec[ref.GRAD_MAX_ONLY][..., 1], full[..., 1])
+        np.testing.assert_array_equal(dec[ref.GRAD_MAX_ONLY][..., 2], 0.0)
+        np.testing.assert_array_equal(dec[ref.GRAD_MIN_ONLY][..., 2], full[..., 2])
+        np.testing.assert_array_equal(dec[ref.GRAD_MIN_ONLY][..., 1], 0.0)
+        np.testing.assert_array_equal(dec[ref.GRAD_DETACH][..., 1:], 0.0)
+        T = Q.shape[2]
+        for m in MODES:
+            dS = ref.attention(Q, K, V, dO, base.replace(grad=m), dump=True)["dS"][0]
+            np.testing.assert_allclose(dec[m][..., 0], np.einsum("htj,htj->ht", dS, dS),
+                                       rtol=1e-12)
+        det = ref.attention(Q, K, V, dO, base.replace(grad=ref.GRAD_DETACH), dump=True)["dS"][0]
+        Ls = np.arange(1, T + 1)
+        c = -det.sum(-1) / Ls
+        np.testing.assert_allclose(dec[ref.GRAD_PROJECT][..., 1], c * c * Ls, rtol=1e-10,
+                                   atol=1e-30)
+        np.testing.assert_array_equal(dec[ref.GRAD_PROJECT][..., 2], 0.0)
+        # a full-mode row's calibration norm splits into its two extremum terms
+        dfull = ref.attention(Q, K, V, dO, base, dump=True)["dS"][0]
+        diff = dfull - det
+        np.testing.assert_allclose(full[..., 1] + full[..., 2], np.sum(diff * diff, -1),
+                                   rtol=1e-10, atol=1e-30)
+
+
+def test_decomposition_closed_forms_from_row_statistics():
+    """Appendix B closed forms: MinMax g_m = A/h + C/K, g_n = -C/K; FWM
+    g_m = A/h, g_n = 0, with A, C the row sums the backward records."""
+    Q, K, V, dO = _decomp_inputs(23)
+    for cal in CALS:
+        for rec, ste in RECSTE:
+            cfg = ref.RefConfig(K=4, cal=cal, rec=rec, ste=ste)
+            dec = ref.grad_decomposition(Q, K, V, dO, cfg)
+            st = ref.attention(Q, K, V, dO, cfg)["stats"][0]
+            live = st[..., ref.ST_DEGEN] == 0
+            A, C, h = st[..., ref.ST_A], st[..., ref.ST_C], st[..., ref.ST_H]
+            hs = np.where(live, h, 1.0)
+            if cal == ref.CAL_MINMAX:
+                gm, gn = A / hs + C / cfg.K, -C / cfg.K
+            else:
+                gm, gn = A / hs, np.zeros_like(A)
+            np.testing.assert_allclose(dec[..., 1][live], (gm * gm)[live], rtol=1e-9, atol=1e-28)
+            np.testing.assert_allclose(dec[..., 2][live], (gn * gn)[live], rtol=1e-9, atol=1e-28)
+            np.testing.assert_array_equal(dec[..., 1:][~live], 0.0)
