@@ -27,6 +27,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -44,16 +46,19 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gpt2_fwm",
-                    choices=["gpt2_fwm", "gpt2_heavy", "tiny"])
+                    choices=["gpt2_fwm", "gpt2_heavy", "gpt2_fixed", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--diag", default=None, choices=["geometry", "decomposition"],
+                    help="time one of the diagnostic row kernels instead of the step")
     return ap.parse_args()
 
 
 def workload(name):
     from quantized_softmax_attention_b200 import workloads as W
-    return {"gpt2_fwm": W.gpt2_fwm, "gpt2_heavy": W.gpt2_heavy, "tiny": W.tiny}[name]()
+    return {"gpt2_fwm": W.gpt2_fwm, "gpt2_heavy": W.gpt2_heavy, "gpt2_fixed": W.gpt2_fixed,
+            "tiny": W.tiny}[name]()
 
 
 def gemm_units(w):
@@ -68,9 +73,9 @@ def algorithmic_flops(w):
 
 
 def config_dict(w, n):
-    names = {0: "MinMax", 1: "FWM"}
+    names = {0: "MinMax", 1: "FWM", 2: "fixed step (untruncated)"}
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "K": w.K,
-            "calibration": names[w.cal], "tau": w.tau if w.cal == 1 else None,
+            "calibration": names[w.cal], "tau": w.tau if w.cal != 0 else None,
             "reconstruction": "LERP" if w.rec == 0 else "Nearest",
             "surrogate": None if w.rec == 0 else ("Prob-STE" if w.ste else "Weight-STE"),
             "grad": "full", "causal": w.causal, "parallelism": f"dp{n}",
@@ -252,10 +257,141 @@ def weak_scaling_value(flops_per_rank_step: float, world: int, ms_per_step: floa
 
 # ------------------------------------------------------------------ GPU side
 
+# ------------------------------------------------------ diagnostic kernels
+
+def diag_main(args):
+    """One JSON line for a diagnostic row kernel on the benchmark's workload:
+    the geometry probe over the scores S = Q K^T, or the fixed-upstream
+    decomposition over the backward's dS dump.  Both read each row's visible
+    scores once: algorithmic bytes = 4 sum_i L_i + per-row side inputs and
+    outputs; HBM-bound by design."""
+    import torch
+    from quantized_softmax_attention_b200 import kiattn as K
+    from quantized_softmax_attention_b200 import workloads as W
+    torch.cuda.set_device(0)
+    w = workload(args.workload)
+    cfg = K.Config(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
+                   causal=w.causal, gemm=K.GEMM_TF32)
+    host = W.make_inputs(w)
+    q, k, v, g = (x.cuda() for x in host)
+    B, H, T, d = w.B, w.H, w.T, w.d
+    rows = B * H * T
+    vis = B * H * (T * (T + 1) // 2 if w.causal else T * T)
+    S = torch.empty((B, H, T, T), dtype=torch.float32, device="cuda")
+    if args.diag == "geometry":
+        K.kiattn_scores(q, k, S, cfg)
+        out = torch.empty((B, H, T, K.GEO_FIELD_COUNT), dtype=torch.float32, device="cuda")
+        nbytes = 4 * vis + rows * (4 * d + 4 * K.GEO_FIELD_COUNT)
+
+        def run(src, dst, stream=None):
+            K.kiattn_geometry(src, dst, cfg, Q=q, stream=stream)
+        kname, metric = "geometry_kernel", "geometry probe GB/s (per-row span, width, norm, " \
+            "entropies, TV, top-bucket mass) over the scores of B8·H12·T1024"
+    else:
+        bufs = K.Buffers(B, H, T, d, cfg)
+        K.kiattn_fwd(q, k, v, bufs.O, bufs.stats, cfg)
+        K.kiattn_bwd(q, k, v, bufs.O, g, bufs.stats, bufs.dQ, bufs.dK, bufs.dV, bufs.work, cfg,
+                     dS_dbg=S)
+        out = torch.empty((B, H, T, 3), dtype=torch.float64, device="cuda")
+        nbytes = 4 * vis + rows * (8 + 24)
+
+        def run(src, dst, stream=None):
+            K.kiattn_grad_decomposition(src, bufs.work, dst, cfg, stream=stream)
+        kname, metric = "grad_decomp_kernel", "fixed-upstream gradient decomposition GB/s " \
+            "over the dS of B8·H12·T1024"
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        run(S, out)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0, enabled=not args.no_clocks)
+    time.sleep(0.3 if sampler.proc else 0.0)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        run(S, out)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    err = K.kiattn_device_error(True)
+    if err != 0:
+        raise RuntimeError(f"device error word {err}")
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    _, hbm, src = peaks()
+
+    # end to end: the step's scores (or dS) copied in from pinned host memory,
+    # the kernel, the per-row record copied out
+    e2e = None
+    if not args.no_e2e:
+        hS = S.cpu().pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        nrep = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(nrep):
+            S.copy_(hS, non_blocking=True)
+            run(S, out)
+            hout.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = e0.elapsed_time(e1) / nrep
+        e2e = {"value": nbytes / (te * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": hS.numel() * 4,
+               "d2h_bytes_per_step": hout.numel() * hout.element_size(), "ms_per_step": te}
+    line = {"metric": metric, "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {**config_dict(w, 1), "diagnostic": args.diag,
+                       "l2": "flushed between timed launches (256 MiB write)"},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm,
+                         "unit": "GB/s", "frac": gbs / hbm, "traffic": None,
+                         "bytes_per_launch": nbytes, "peak_source": f"{src} HBM copy"},
+            "gpu_launches": args.steps}
+    if e2e:
+        line["e2e"] = e2e
+    if clocks:
+        line["clocks"] = clocks
+    if not args.no_cpu_baseline:
+        import oracle as ref
+        rcfg = ref.RefConfig(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
+                             causal=w.causal)
+        Sh = S.cpu().numpy()
+        Qh = host[0].numpy()
+        ln = np.arange(1, T + 1) if w.causal else np.full(T, T)
+        t0, n = time.perf_counter(), 0
+        while time.perf_counter() - t0 < 10.0 and n < B * H:
+            b, h = divmod(n, H)
+            if args.diag == "geometry":
+                ref.geometry(Sh[b, h], ln, rcfg, Q=Qh[b, h])
+            else:
+                ref.grad_decomposition(host[0][b:b + 1, h:h + 1].numpy(),
+                                       host[1][b:b + 1, h:h + 1].numpy(),
+                                       host[2][b:b + 1, h:h + 1].numpy(),
+                                       host[3][b:b + 1, h:h + 1].numpy(), rcfg)
+            n += 1
+        secs = time.perf_counter() - t0
+        per_head = nbytes / (B * H)
+        line["cpu_baseline"] = {"value": n * per_head / secs / 1e9, "unit": "GB/s",
+                                "cores": int(os.environ.get("OMP_NUM_THREADS",
+                                                            os.cpu_count() or 1)),
+                                "kind": "oracle",
+                                "sample": f"{n} of {B * H} (b, h) pairs ({secs:.1f} s, fp64)"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         reference_arm(args)
+        return
+    if args.diag:
+        diag_main(args)
         return
     import torch
     import torch.distributed as dist

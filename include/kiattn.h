@@ -51,6 +51,12 @@ extern "C" {
 /* calibration (section 3, Calibration) */
 #define KIA_CAL_MINMAX 0 /* h = row span / K */
 #define KIA_CAL_FWM 1    /* window [m - tau, m], h = tau / K, zero tail */
+/* untruncated fixed step (Appendix D.4): h = tau / K anchored at the row
+ * maximum like FWM, with the grid continued past node K over the whole row
+ * span (nodes until e^{-k h} underflows in fp32, k h >= 104.5); calibration
+ * gradient as FWM's (the maximum only).  Needs ceil(104.5 K / tau) <= 400,
+ * else KIA_ERR_UNSUPPORTED (e.g. tau = 6 allows K <= 22). */
+#define KIA_CAL_FIXED 2
 /* reconstruction (section 3, Reconstruction) */
 #define KIA_REC_LERP 0
 #define KIA_REC_NEAREST 1
@@ -82,7 +88,7 @@ extern "C" {
 typedef struct {
   int n_intervals; /* K >= 1 */
   int cal;         /* KIA_CAL_* */
-  float tau;       /* FWM window width in nats (6 in the paper) */
+  float tau;       /* FWM window width in nats (6 in the paper); fixed-step K h */
   int rec;         /* KIA_REC_* */
   int ste;         /* KIA_STE_* (ignored for LERP) */
   int grad;        /* KIA_GRAD_* (backward only) */
@@ -179,12 +185,47 @@ int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T
  * over the rows of interest.
  * dS: the dS_dbg [B,H,T,T] written by kiattn_bwd; workspace: the workspace of
  * that same kiattn_bwd call (it holds g_m, g_n per row); cfg as in that call;
- * out: device fp64 [B*H*T*3], caller-owned.  Sums run in fp64.  Nothing is
+ * out: device fp64 [B*H*T*3], caller-owned.  Sums run in fp64 (groups of
+ * four squares in fp32 first).  Nothing is
  * written when the kiattn_bwd call rejected its stats (workspace status set).
  * Errors: INVALID_ARG (null pointer, B, H or T < 1), UNSUPPORTED (shape
  * beyond the operator's limits), CUDA (launch failure). */
 int kiattn_grad_decomposition(const float* dS, const void* workspace, int B, int H, int T,
                               const kia_config* cfg, double* out, void* stream);
+
+/* Geometry probe (section 4, geometry probe; section 5.4; Appendix D.6,
+ * Figure S4): per query row, on given scores, the quantities the paper
+ * records to describe learned score geometry.  Fields of out[row * 8 + f]:
+ *   KIA_GEO_SPAN         m - n over the row's visible keys
+ *   KIA_GEO_H            native interval width h (MinMax span / K, 0 for a
+ *                        degenerate row; FWM tau / K)
+ *   KIA_GEO_QNORM        ||q_i||_2 (0 when Q is NULL)
+ *   KIA_GEO_ENT_SOFTMAX  entropy (nats) of softmax(s_i)
+ *   KIA_GEO_ENT_OP       entropy of the operator's forward probabilities
+ *   KIA_GEO_TV           total variation 1/2 sum_j |P_op - P_softmax|
+ *   KIA_GEO_TOP_SOFTMAX  softmax mass on the keys whose nearest grid node is
+ *                        node 0 (the top rounding bucket)
+ *   KIA_GEO_TOP_OP       the operator's mass on the same keys
+ * The operator weights and the grid decisions are the forward's fp32 weight
+ * stage (bit-identical to kiattn_weights_from_S); sums run in fp32.
+ * S: device fp32 [B,H,T,T] row-major scores (e.g. from kiattn_scores); row i
+ * sees keys j <= i when cfg->causal, else all T.  Q: device fp32 [B,H,T,d]
+ * or NULL.  cfg: the grid to measure against (cal, K, tau, rec, causal;
+ * op must be KIA_OP_KINTERVAL; grad and ste are ignored).  out: device fp32
+ * [B*H*T*8], caller-owned.  Runs on `stream`, allocates nothing.
+ * Errors: INVALID_ARG (null S or out, B, H or T < 1, d < 1 with Q given, op
+ * not K-interval), UNSUPPORTED (shape beyond the operator's limits), CUDA. */
+#define KIA_GEO_SPAN 0
+#define KIA_GEO_H 1
+#define KIA_GEO_QNORM 2
+#define KIA_GEO_ENT_SOFTMAX 3
+#define KIA_GEO_ENT_OP 4
+#define KIA_GEO_TV 5
+#define KIA_GEO_TOP_SOFTMAX 6
+#define KIA_GEO_TOP_OP 7
+#define KIA_GEO_FIELDS 8
+int kiattn_geometry(const float* S, const float* Q, int B, int H, int T, int d,
+                    const kia_config* cfg, float* out, void* stream);
 
 /* Error word raised by device code since the last reset: KIA_ERR_TIMEOUT
  * when a bounded wait inside a kernel gave up, KIA_ERR_STATS_MISMATCH when

@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kiattn_ref.c")
 _LIB = os.path.join(_HERE, "libkiattn_ref.so")
 
-CAL_MINMAX, CAL_FWM = 0, 1
+CAL_MINMAX, CAL_FWM, CAL_FIXED = 0, 1, 2
 REC_LERP, REC_NEAREST = 0, 1
 STE_WEIGHT, STE_PROB = 0, 1
 GRAD_FULL, GRAD_DETACH, GRAD_MAX_ONLY, GRAD_MIN_ONLY, GRAD_PROJECT = 0, 1, 2, 3, 4
@@ -246,6 +246,58 @@ def weights_fp32(S, row_len, cfg: RefConfig):
     if rc != 0:
         raise ValueError("kiattn_ref_weights_fp32: bad arguments")
     return {"w": w, "bin": b, "t": t, "m": m, "n": n}
+
+
+GEO_SPAN, GEO_H, GEO_QNORM, GEO_ENT_SOFTMAX, GEO_ENT_OP, GEO_TV, GEO_TOP_SOFTMAX, GEO_TOP_OP = range(8)
+GEO_FIELDS = 8
+
+
+def geometry(S, row_len, cfg: RefConfig, Q=None):
+    """Geometry probe per row ("Pretraining Transformers with Quantized Softmax
+    in Attention", section 4 geometry probe, section 5.4, Appendix D.6 and
+    Figure S4): span m - n, native width h, ||q_i||, entropy of softmax(s_i)
+    and of the operator's forward probabilities, their total variation, and
+    the softmax and operator mass on the keys whose nearest grid node is
+    node 0 (the top rounding bucket).  The grid decisions (node, tail) and
+    the operator weights are those of the fp32 weight stage, so that both
+    sides take them in the same precision; everything else is fp64.
+    S: [rows, cols] scores (rounded to fp32), row_len: visible keys per row;
+    Q: [rows, d] or None.  Returns [rows, GEO_FIELDS]."""
+    S32 = np.ascontiguousarray(S, dtype=np.float32)
+    rws, cols = S32.shape
+    row_len = np.asarray(row_len, dtype=np.int64)
+    ws = weights_fp32(S32, row_len, cfg)
+    vis = np.arange(cols)[None, :] < row_len[:, None]
+    m = ws["m"].astype(np.float64)
+    n = ws["n"].astype(np.float64)
+    out = np.zeros((rws, GEO_FIELDS))
+    out[:, GEO_SPAN] = m - n
+    if cfg.cal == CAL_MINMAX:
+        out[:, GEO_H] = np.where(m - n < 1e-12, 0.0, (m - n) / cfg.K)
+    else:
+        out[:, GEO_H] = float(np.float32(cfg.tau)) / cfg.K
+    if Q is not None:
+        out[:, GEO_QNORM] = np.linalg.norm(np.asarray(Q, np.float64).reshape(rws, -1), axis=1)
+    x = np.where(vis, S32.astype(np.float64) - m[:, None], -np.inf)
+    e = np.exp(x)
+    Psm = e / e.sum(axis=1, keepdims=True)
+    w = np.where(vis, ws["w"].astype(np.float64), 0.0)
+    Pop = w / w.sum(axis=1, keepdims=True)
+
+    def entropy(P):
+        with np.errstate(divide="ignore", invalid="ignore"):
+            return -np.sum(np.where(P > 0, P * np.log(P), 0.0), axis=1)
+
+    out[:, GEO_ENT_SOFTMAX] = entropy(Psm)
+    out[:, GEO_ENT_OP] = entropy(Pop)
+    out[:, GEO_TV] = 0.5 * np.abs(Pop - Psm).sum(axis=1)
+    node = ws["bin"].astype(np.int64)
+    if cfg.rec == REC_LERP:   # the stage records k and t; the nearest node is k + [t >= 1/2]
+        node = np.where(node >= 0, node + (ws["t"] >= np.float32(0.5)), node)
+    top = vis & (node == 0)
+    out[:, GEO_TOP_SOFTMAX] = np.where(top, Psm, 0.0).sum(axis=1)
+    out[:, GEO_TOP_OP] = np.where(top, Pop, 0.0).sum(axis=1)
+    return out
 
 
 def own_exp(x: float) -> float:

@@ -47,6 +47,7 @@
 
 #define REF_CAL_MINMAX 0
 #define REF_CAL_FWM 1
+#define REF_CAL_FIXED 2 /* untruncated fixed step (Appendix D.4): h = tau / K, no window */
 #define REF_REC_LERP 0
 #define REF_REC_NEAREST 1
 #define REF_STE_WEIGHT 0
@@ -158,7 +159,8 @@ static void row_forward(const double* s, int L, const ref_cfg* c, const double* 
         wL[j] = 0.0; wN[j] = 0.0; kk[j] = -1; tt[j] = 0.0;
       } else {
         int k = (int)floor(u);
-        if (k > K - 1) k = K - 1;
+        /* the fixed-step grid continues past node K down to the row minimum */
+        if (c->cal != REF_CAL_FIXED && k > K - 1) k = K - 1;
         if (k < 0) k = 0;
         double t = u - k;
         double Gk = exp(-(double)k * h);
@@ -550,8 +552,9 @@ int kiattn_ref_weights_fp32(const float* S, int rows, int cols, const int* row_l
       h = tau / Kf;
       rh = Kf / tau;
     }
+    const int fixed = c->cal == REF_CAL_FIXED;
     float G[1024 + 1];
-    if (!degen) {
+    if (!degen && !fixed) {
       for (int k = 0; k <= K; ++k) G[k] = (float)own_exp(-(double)k * (double)h);
     }
     for (int j = 0; j < cols; ++j) {
@@ -566,20 +569,23 @@ int kiattn_ref_weights_fp32(const float* S, int rows, int cols, const int* row_l
           int tail = 0;
           if (c->cal == REF_CAL_MINMAX) {
             if (uu > Kf) uu = Kf;
-          } else {
+          } else if (c->cal == REF_CAL_FWM) {
             tail = uu > Kf;
           }
           if (!tail) {
             int k = (int)floorf(uu);
-            if (k > K - 1) k = K - 1;
+            if (!fixed && k > K - 1) k = K - 1;
             float t = uu - (float)k;
+            /* fixed step: grid values on demand, G_k = RN32(E(-k h)) for any k */
+            const float Gk = fixed ? (float)own_exp(-(double)k * (double)h) : G[k];
+            const float Gk1 = fixed ? (float)own_exp(-(double)(k + 1) * (double)h) : G[k + 1];
             if (c->rec == REF_REC_LERP) {
-              float a = G[k + 1] - G[k];
-              wj = fmaf(t, a, G[k]);
+              float a = Gk1 - Gk;
+              wj = fmaf(t, a, Gk);
               bj = k;
             } else {
               int r = k + (t >= 0.5f ? 1 : 0);
-              wj = G[r];
+              wj = r == k ? Gk : Gk1;
               bj = r;
             }
             tj = t;

@@ -13,6 +13,8 @@
 #include "../../include/kiattn.h"
 
 #define KIA_MAX_K 64
+// fixed-step grids: at most this many intervals before G_k underflows
+#define KIA_MAX_KCAP 400
 #define KIA_TILE 128
 
 namespace kia {
@@ -32,6 +34,8 @@ struct OpParams {
   float fwm_h;    // tau / K  (fp32 division)
   float fwm_rh;   // K / tau  (fp32 division)
   int tf32_ops;   // CUDA-core kernels: truncate product operands to TF32 like tcgen05
+  int fixed_step; // untruncated fixed step (Appendix D.4), run as FWM with K = the grid's
+                  // extent, the first node count at which G_k underflows to zero in fp32
 };
 
 // The tcgen05 kind::tf32 MMA reads fp32 operands and ignores their low 13

@@ -220,9 +220,29 @@ grad_decomp_kernel(const float* __restrict__ dS, WorkView wk, long long rows, in
   const int L = causal ? i + 1 : T;
   const float* ds = dS + row * (long long)T;
   double s2 = 0.0;
-  for (int j = lane; j < L; j += 32) {
-    const double v = (double)ds[j];
-    s2 += v * v;
+  if ((T & 3) == 0 && (reinterpret_cast<uintptr_t>(dS) & 15) == 0) {
+    // four 128-key chunks in flight per lane; each float4's four squares are
+    // summed in fp32 (exact to 2^-22 relative), the rest in fp64
+    for (int j0 = 4 * lane; j0 < L; j0 += 512) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + 128 * u;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j + 3 < L) {
+          v[u] = __ldg(reinterpret_cast<const float4*>(ds + j));
+        } else if (j < L) {
+          v[u].x = ds[j];
+          if (j + 1 < L) v[u].y = ds[j + 1];
+          if (j + 2 < L) v[u].z = ds[j + 2];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        s2 += (double)fmaf(v[u].x, v[u].x, fmaf(v[u].y, v[u].y, fmaf(v[u].z, v[u].z, v[u].w * v[u].w)));
+    }
+  } else {
+    for (int j = lane; j < L; j += 32) s2 = fma((double)ds[j], (double)ds[j], s2);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);

@@ -89,10 +89,11 @@ simt_fwd_kernel(const float* __restrict__ Q, const float* __restrict__ Kt,
         for (int k = 0; k <= p.K; ++k) st.table[(size_t)(bh * T + i) * (p.K + 1) + k] = 1.0f;
       }
     } else {
-      if (r <= p.K) {
-        const float G = grid_value(r, p.fwm_h);
-        sTab[r] = G;
-        if (blockIdx.x == 0 && blockIdx.y == 0) st.table[r] = G;
+      // one grid for every row (the fixed-step grid may outnumber the threads)
+      for (int k = r; k <= p.K; k += kSimtRows) {
+        const float G = grid_value(k, p.fwm_h);
+        sTab[k] = G;
+        if (blockIdx.x == 0 && blockIdx.y == 0) st.table[k] = G;
       }
     }
   }
@@ -183,8 +184,8 @@ simt_bwd_q_kernel(const float* __restrict__ Q, const float* __restrict__ Kt,
   if (!p.softmax) {
     if (p.cal == KIA_CAL_MINMAX) {
       for (int k = 0; k <= p.K; ++k) sTab[k * kSimtRows + r] = st.table[row * (p.K + 1) + k];
-    } else if (r <= p.K) {
-      sTab[r] = st.table[r];
+    } else {
+      for (int k = r; k <= p.K; k += kSimtRows) sTab[k] = st.table[k];
     }
   }
   float acc[D];
@@ -274,8 +275,8 @@ simt_bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ Kt,
           const size_t qr = (size_t)bh * T + (qi < T ? qi : 0);
           sTab[e] = st.table[qr * K1 + e % K1];
         }
-      } else if (threadIdx.x < K1) {
-        sTab[threadIdx.x] = st.table[threadIdx.x];
+      } else {
+        for (int e = threadIdx.x; e < K1; e += blockDim.x) sTab[e] = st.table[e];
       }
     }
     __syncthreads();

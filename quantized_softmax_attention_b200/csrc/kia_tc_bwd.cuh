@@ -302,8 +302,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     float2* sPair = reinterpret_cast<float2*>(sTab);
     if constexpr (!V::MINMAX && !V::SOFTMAX) {
-      const int k = (int)threadIdx.x - 64;
-      if (k >= 0 && k < p.K) sPair[k] = make_float2(st.table[k], st.table[k + 1]);
+      for (int k = (int)threadIdx.x - 64; k < p.K; k += kElemThreads)
+        sPair[k] = make_float2(st.table[k], st.table[k + 1]);
     }
     int gbase = 0, n = 0;
     ItemSeq seq(nitems);

@@ -401,15 +401,16 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       } else if constexpr (!V::SOFTMAX) {
         // one grid for every row and item: pairs (G_k, G_{k+1}), k = 0..K-1,
         // computed with the CTA's first item and kept
-        const int k = (int)threadIdx.x - 64;
-        if (n == 0 && k >= 0 && k < p.K) {
-          const float G0 = grid_value(k, p.fwm_h), G1 = grid_value(k + 1, p.fwm_h);
-          sPair[k] = make_float2(G0, G1);
-        }
-        if (bh == 0 && qt == nt - 1 && k >= 0 && k < p.K) {
-          const float2 G = sPair[k];
-          st.table[k] = G.x;
-          if (k == p.K - 1) st.table[k + 1] = G.y;
+        for (int k = (int)threadIdx.x - 64; k < p.K; k += kElemThreads) {
+          if (n == 0) {
+            const float G0 = grid_value(k, p.fwm_h), G1 = grid_value(k + 1, p.fwm_h);
+            sPair[k] = make_float2(G0, G1);
+          }
+          if (bh == 0 && qt == nt - 1) {
+            const float2 G = sPair[k];
+            st.table[k] = G.x;
+            if (k == p.K - 1) st.table[k + 1] = G.y;
+          }
         }
       }
       mbar_arrive(&bar.row_sync);

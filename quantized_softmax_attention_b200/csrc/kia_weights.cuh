@@ -15,7 +15,7 @@ weights_from_S_kernel(const float* __restrict__ S, int rows, int cols,
                       const int* __restrict__ row_len, OpParams p, float* __restrict__ w,
                       int* __restrict__ bin, float* __restrict__ tout, float* __restrict__ row_m,
                       float* __restrict__ row_n) {
-  __shared__ float sG[kWeightsWarps][KIA_MAX_K + 1];
+  __shared__ float sG[kWeightsWarps][KIA_MAX_KCAP + 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWeightsWarps + warp;
   if (row >= rows) return;

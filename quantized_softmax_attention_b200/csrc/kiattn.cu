@@ -14,6 +14,7 @@
 #include "kia_common.cuh"
 #include "kia_elem.cuh"
 #include "kia_epilogue.cuh"
+#include "kia_geometry.cuh"
 #include "kia_simt.cuh"
 #include "kia_stats.cuh"
 #include "kia_tc.cuh"
@@ -37,17 +38,32 @@ void prof_mark(int i, cudaStream_t s) {
   if (g_prof_on) cudaEventRecord(g_prof_ev[i], s);
 }
 
+// Extent of the untruncated fixed-step grid (Appendix D.4): the node count
+// Kc at which G_Kc = RN32(e^{-Kc h}) is zero (every Kc h >= 104.5 nats, since
+// e^{-103.98} is already below half the least fp32 subnormal), so that keys
+// past node Kc carry exactly zero weight and may be treated as a tail.
+int fixed_step_extent(const kia_config* cfg) {
+  const float h = cfg->tau / (float)cfg->n_intervals;
+  const double kc = ceil(104.5 / (double)h);
+  return kc < 1.0 ? 1 : (kc > 1e9 ? 1000000000 : (int)kc);
+}
+
 int check_config(const kia_config* cfg) {
   if (!cfg) return KIA_ERR_INVALID_ARG;
   if (cfg->n_intervals < 1 || cfg->n_intervals > KIA_MAX_K) return KIA_ERR_UNSUPPORTED;
-  if (cfg->cal != KIA_CAL_MINMAX && cfg->cal != KIA_CAL_FWM) return KIA_ERR_INVALID_ARG;
+  if (cfg->cal != KIA_CAL_MINMAX && cfg->cal != KIA_CAL_FWM && cfg->cal != KIA_CAL_FIXED)
+    return KIA_ERR_INVALID_ARG;
   if (cfg->rec != KIA_REC_LERP && cfg->rec != KIA_REC_NEAREST) return KIA_ERR_INVALID_ARG;
   if (cfg->ste != KIA_STE_WEIGHT && cfg->ste != KIA_STE_PROB) return KIA_ERR_INVALID_ARG;
   if (cfg->grad < KIA_GRAD_FULL || cfg->grad > KIA_GRAD_PROJECT) return KIA_ERR_INVALID_ARG;
   if (cfg->gemm != KIA_GEMM_TF32 && cfg->gemm != KIA_GEMM_FP32) return KIA_ERR_INVALID_ARG;
   if (cfg->op != KIA_OP_KINTERVAL && cfg->op != KIA_OP_SOFTMAX) return KIA_ERR_INVALID_ARG;
   if (cfg->causal != 0 && cfg->causal != 1) return KIA_ERR_INVALID_ARG;
-  if (cfg->cal == KIA_CAL_FWM && !(cfg->tau > 0.0f && cfg->tau < 1e30f)) return KIA_ERR_INVALID_ARG;
+  if (cfg->cal != KIA_CAL_MINMAX && !(cfg->tau > 0.0f && cfg->tau < 1e30f))
+    return KIA_ERR_INVALID_ARG;
+  if (cfg->cal == KIA_CAL_FIXED && cfg->op == KIA_OP_KINTERVAL &&
+      fixed_step_extent(cfg) > KIA_MAX_KCAP)
+    return KIA_ERR_UNSUPPORTED;
   return KIA_OK;
 }
 
@@ -71,9 +87,18 @@ OpParams make_params(const kia_config* cfg) {
   p.causal = cfg->causal;
   p.softmax = cfg->op == KIA_OP_SOFTMAX;
   p.tau = cfg->tau;
-  p.fwm_h = (cfg->cal == KIA_CAL_FWM) ? cfg->tau / p.Kf : 0.0f;
-  p.fwm_rh = (cfg->cal == KIA_CAL_FWM) ? p.Kf / cfg->tau : 0.0f;
+  p.fwm_h = (cfg->cal != KIA_CAL_MINMAX) ? cfg->tau / p.Kf : 0.0f;
+  p.fwm_rh = (cfg->cal != KIA_CAL_MINMAX) ? p.Kf / cfg->tau : 0.0f;
   p.tf32_ops = 0;
+  p.fixed_step = 0;
+  if (cfg->cal == KIA_CAL_FIXED) {
+    // the fixed-step operator is FWM's grid (h = tau / K, anchored at the row
+    // maximum) with its window widened to the grid's full extent
+    p.cal = KIA_CAL_FWM;
+    p.fixed_step = 1;
+    p.K = fixed_step_extent(cfg);
+    p.Kf = (float)p.K;
+  }
   if (p.softmax) {  // the softmax row has no grid: normalise the unused axes
     p.cal = KIA_CAL_MINMAX;
     p.rec = KIA_REC_LERP;
@@ -82,6 +107,7 @@ OpParams make_params(const kia_config* cfg) {
     p.Kf = 1.0f;
     p.tau = 0.0f;
     p.fwm_h = p.fwm_rh = 0.0f;
+    p.fixed_step = 0;
   }
   return p;
 }
@@ -347,6 +373,36 @@ int kiattn_grad_decomposition(const float* dS, const void* workspace, int B, int
   if (blocks > 0x7fffffffll) return KIA_ERR_UNSUPPORTED;
   grad_decomp_kernel<<<(unsigned)blocks, 32 * kRowWarps, 0, static_cast<cudaStream_t>(stream)>>>(
       dS, wk, rows, T, cfg->causal, cfg->grad, out);
+  return launch_status();
+}
+
+int kiattn_geometry(const float* S, const float* Q, int B, int H, int T, int d,
+                    const kia_config* cfg, float* out, void* stream) {
+  static_assert(kGeoFields == KIA_GEO_FIELDS, "geometry field count");
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_shape(B, H, T, 64))) return rc;
+  if (!S || !out || cfg->op != KIA_OP_KINTERVAL || (Q && (d < 1 || d > 4096)))
+    return KIA_ERR_INVALID_ARG;
+  const long long rows = (long long)B * H * T;
+  const long long blocks = (rows + kGeoWarps - 1) / kGeoWarps;
+  if (blocks > 0x7fffffffll) return KIA_ERR_UNSUPPORTED;
+  const OpParams p = make_params(cfg);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dq = Q ? d : 0;
+  auto launch = [&](auto var) {
+    using V = decltype(var);
+    geometry_kernel<V><<<(unsigned)blocks, 32 * kGeoWarps, 0, s>>>(S, Q, rows, T, dq,
+                                                                  cfg->causal, p, out);
+  };
+  const bool lerp = p.rec == KIA_REC_LERP;
+  if (p.cal == KIA_CAL_MINMAX) {
+    if (lerp) launch(Var<KIA_CAL_MINMAX, KIA_REC_LERP, false, false>{});
+    else launch(Var<KIA_CAL_MINMAX, KIA_REC_NEAREST, false, false>{});
+  } else {
+    if (lerp) launch(Var<KIA_CAL_FWM, KIA_REC_LERP, false, false>{});
+    else launch(Var<KIA_CAL_FWM, KIA_REC_NEAREST, false, false>{});
+  }
   return launch_status();
 }
 

@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkiattn.so")
 
-CAL_MINMAX, CAL_FWM = 0, 1
+CAL_MINMAX, CAL_FWM, CAL_FIXED = 0, 1, 2
 REC_LERP, REC_NEAREST = 0, 1
 STE_WEIGHT, STE_PROB = 0, 1
 GRAD_FULL, GRAD_DETACH, GRAD_MAX_ONLY, GRAD_MIN_ONLY, GRAD_PROJECT = 0, 1, 2, 3, 4
@@ -30,7 +30,7 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error", 
 SYMBOLS = ("kiattn_stats_bytes", "kiattn_workspace_bytes", "kiattn_fwd", "kiattn_bwd",
            "kiattn_weights_from_S", "kiattn_scores", "kiattn_strerror", "kiattn_version",
            "kiattn_device_error", "kiattn_profile_enable", "kiattn_profile_read",
-           "kiattn_bwd_noalloc", "kiattn_grad_decomposition")
+           "kiattn_bwd_noalloc", "kiattn_grad_decomposition", "kiattn_geometry")
 NOALLOC_MAX_ROWS = 1 << 20
 PHASES = ("fwd", "bwd_prep", "bwd_query_pass", "bwd_key_pass", "bwd_calibration")
 
@@ -93,6 +93,8 @@ def _load():
     lib.kiattn_scores.argtypes = [vp, vp, vp, i, i, i, i, cp, vp]
     lib.kiattn_grad_decomposition.argtypes = [vp, vp, i, i, i, cp, vp, vp]
     lib.kiattn_grad_decomposition.restype = i
+    lib.kiattn_geometry.argtypes = [vp, vp, i, i, i, i, cp, vp, vp]
+    lib.kiattn_geometry.restype = i
     lib.kiattn_strerror.argtypes = [i]
     lib.kiattn_strerror.restype = ctypes.c_char_p
     lib.kiattn_version.restype = i
@@ -184,6 +186,21 @@ def kiattn_grad_decomposition(dS, workspace, out, cfg: Config, stream=None):
     _check("kiattn_grad_decomposition",
            _lib.kiattn_grad_decomposition(_p(dS), _p(workspace), B, H, T, ctypes.byref(cfg.c()),
                                           _p(out), _stream(stream)))
+
+
+GEO_FIELDS = ("span", "h", "q_norm", "entropy_softmax", "entropy_op", "tv", "top_softmax",
+              "top_op")
+GEO_FIELD_COUNT = len(GEO_FIELDS)
+
+
+def kiattn_geometry(S, out, cfg: Config, Q=None, stream=None):
+    """Per-row geometry probe of scores S [B, H, T, T] against cfg's grid;
+    out: device fp32 [B, H, T, 8] in the order of GEO_FIELDS."""
+    B, H, T, _ = S.shape
+    d = Q.shape[-1] if Q is not None else 0
+    _check("kiattn_geometry", _lib.kiattn_geometry(_p(S), _p(Q), B, H, T, d,
+                                                   ctypes.byref(cfg.c()), _p(out),
+                                                   _stream(stream)))
 
 
 def kiattn_scores(Q, K, S, cfg: Config, stream=None):

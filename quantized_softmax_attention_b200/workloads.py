@@ -17,7 +17,7 @@ from dataclasses import dataclass, field
 
 import torch
 
-CAL_MINMAX, CAL_FWM = 0, 1
+CAL_MINMAX, CAL_FWM, CAL_FIXED = 0, 1, 2
 REC_LERP, REC_NEAREST = 0, 1
 STE_WEIGHT, STE_PROB = 0, 1
 GRAD_FULL, GRAD_DETACH, GRAD_MAX_ONLY, GRAD_MIN_ONLY, GRAD_PROJECT = 0, 1, 2, 3, 4
@@ -58,6 +58,13 @@ def gpt2_fwm() -> Workload:
     from 8 to 40 nats; seed 1."""
     return Workload("gpt2_124M_B8H12T1024d64_fwm_nearest_probste_K4", 8, 12, 1024, 64, 4,
                     CAL_FWM, REC_NEAREST, STE_PROB, seed=1, scores="span_ladder")
+
+
+def gpt2_fixed() -> Workload:
+    """The gpt2_fwm workload under the untruncated fixed-step operator
+    (Appendix D.4): h = tau / K = 1.5 without the tail cut; seed 1."""
+    return Workload("gpt2_124M_B8H12T1024d64_fixedstep_nearest_probste_K4", 8, 12, 1024, 64, 4,
+                    CAL_FIXED, REC_NEAREST, STE_PROB, seed=1, scores="span_ladder")
 
 
 def gpt2_heavy() -> Workload:

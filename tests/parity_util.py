@@ -69,7 +69,7 @@ def flag_rows(Q, Kt, cfg: K.Config, rule: int, delta: float) -> np.ndarray:
         u = (m - s) / hs
         bad = np.zeros((B, H), bool)
         if cfg.rec == K.REC_NEAREST:
-            inw = u <= cfg.K + delta
+            inw = (u <= cfg.K + delta) if cfg.cal == K.CAL_FWM else np.ones_like(u, bool)
             frac = np.abs(u - np.floor(u) - 0.5)
             bad |= np.any(inw & (frac < delta), -1)
         if cfg.cal == K.CAL_FWM:

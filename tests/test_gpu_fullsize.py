@@ -82,6 +82,14 @@ def test_gpt2_124M_fwm_nearest_probste_full_size():
     assert flags.mean() < 0.25
 
 
+def test_gpt2_124M_fixed_step_full_size():
+    """The same workload under the untruncated fixed-step operator (Appendix
+    D.4): heads whose spans reach past the FWM window, all five modes."""
+    w = W.gpt2_fixed()
+    q, k, v, g = (x.numpy() for x in W.make_inputs(w))
+    _check_heads(q, k, v, g, _cfg(w), [(2, 11), (6, 4)], tuple(MODES))
+
+
 def test_gpt2_124M_minmax_heavy_tail_full_size():
     """MinMax + Nearest + Weight-STE with heavy-tailed head scales; head 0
     reaches a span about seven times the softmax span (grid values at or

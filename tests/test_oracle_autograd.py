@@ -28,7 +28,9 @@ def autograd_row(s_np, dP_np, K, cal, tau, rec, ste, mode):
         n = n.detach()
     h = (m - n) / K if cal == ref.CAL_MINMAX else torch.tensor(tau / K, dtype=torch.float64)
     u = (m - s) / h
-    k = torch.clamp(torch.floor(u.detach()), 0, K - 1)
+    # the untruncated fixed step (Appendix D.4) keeps counting nodes past K
+    k_hi = float("inf") if cal == ref.CAL_FIXED else K - 1
+    k = torch.clamp(torch.floor(u.detach()), min=0, max=k_hi)
     t = u - k
     g_lo = torch.exp(-k * h)
     g_hi = torch.exp(-(k + 1) * h)
@@ -54,7 +56,7 @@ def autograd_row(s_np, dP_np, K, cal, tau, rec, ste, mode):
     return P.detach().numpy(), g
 
 
-@pytest.mark.parametrize("cal", [ref.CAL_MINMAX, ref.CAL_FWM])
+@pytest.mark.parametrize("cal", [ref.CAL_MINMAX, ref.CAL_FWM, ref.CAL_FIXED])
 @pytest.mark.parametrize("rec,ste", [(ref.REC_LERP, ref.STE_WEIGHT),
                                      (ref.REC_NEAREST, ref.STE_WEIGHT),
                                      (ref.REC_NEAREST, ref.STE_PROB)])

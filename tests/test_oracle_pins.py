@@ -15,7 +15,7 @@ import oracle as ref
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 
-CALS = [ref.CAL_MINMAX, ref.CAL_FWM]
+CALS = [ref.CAL_MINMAX, ref.CAL_FWM, ref.CAL_FIXED]
 MODES = [ref.GRAD_FULL, ref.GRAD_DETACH, ref.GRAD_MAX_ONLY, ref.GRAD_MIN_ONLY, ref.GRAD_PROJECT]
 RECSTE = [(ref.REC_LERP, ref.STE_WEIGHT), (ref.REC_NEAREST, ref.STE_WEIGHT),
           (ref.REC_NEAREST, ref.STE_PROB)]
@@ -344,13 +344,15 @@ def _linear_scan_forward(s, K, cal, tau, rec):
     m - k h from the top, no floor()."""
     m, n = s.max(), s.min()
     h = (m - n) / K if cal == ref.CAL_MINMAX else tau / K
-    nodes = m - h * np.arange(K + 1)
+    # the untruncated fixed step (Appendix D.4) continues the grid down to n
+    Kn = max(K, math.ceil((m - n) / h)) if cal == ref.CAL_FIXED else K
+    nodes = m - h * np.arange(Kn + 1)
     w = np.zeros_like(s)
     for j, x in enumerate(s):
         if cal == ref.CAL_FWM and x < nodes[K] - 1e-15 * max(1, abs(x)):
             continue
         k = 0
-        while k < K - 1 and x < nodes[k + 1]:
+        while k < Kn - 1 and x < nodes[k + 1]:
             k += 1
         lo, hi = nodes[k], nodes[k + 1]
         t = (lo - x) / (lo - hi)
@@ -668,3 +670,37 @@ def test_decomposition_closed_forms_from_row_statistics():
             np.testing.assert_allclose(dec[..., 1][live], (gm * gm)[live], rtol=1e-9, atol=1e-28)
             np.testing.assert_allclose(dec[..., 2][live], (gn * gn)[live], rtol=1e-9, atol=1e-28)
             np.testing.assert_array_equal(dec[..., 1:][~live], 0.0)
+
+
+# ------------------------------------------ untruncated fixed step
+
+@pytest.mark.parametrize("rec,ste", RECSTE)
+@pytest.mark.parametrize("mode", MODES)
+def test_fixed_step_is_fwm_with_a_window_covering_the_span(rec, ste, mode):
+    """Appendix D.4: the untruncated fixed-step operator keeps FWM's step
+    h = tau / K but drops the tail cut, so it equals FWM with K' = 64 K
+    intervals over a window tau' = 64 tau (the same h) wide enough to hold
+    every row's span; on rows whose span is within tau it equals FWM itself."""
+    rng = np.random.default_rng(31 + 5 * mode + rec + ste)
+    S = _rows(rng, 40, 24, 1.0, 60.0)
+    Ls = rng.integers(1, 25, 40)
+    dP = rng.standard_normal(S.shape)
+    fixed = ref.rows(S, Ls, ref.RefConfig(K=4, cal=ref.CAL_FIXED, tau=6.0, rec=rec, ste=ste,
+                                          grad=mode), dP=dP)
+    wide = ref.rows(S, Ls, ref.RefConfig(K=256, cal=ref.CAL_FWM, tau=384.0, rec=rec, ste=ste,
+                                         grad=mode), dP=dP)
+    np.testing.assert_allclose(fixed["P"], wide["P"], rtol=1e-13, atol=1e-300)
+    np.testing.assert_allclose(fixed["dS"], wide["dS"], rtol=1e-12, atol=1e-14)
+    fwm = ref.rows(S, Ls, ref.RefConfig(K=4, cal=ref.CAL_FWM, tau=6.0, rec=rec, ste=ste,
+                                        grad=mode), dP=dP)
+    span = fixed["stats"][:, ref.ST_M] - fixed["stats"][:, ref.ST_N]
+    inside = span < 6.0 - 1e-9
+    assert inside.any() and (~inside).any()
+    np.testing.assert_array_equal(fixed["P"][inside], fwm["P"][inside])
+    np.testing.assert_array_equal(fixed["dS"][inside], fwm["dS"][inside])
+    # past the window FWM puts no mass, the fixed step keeps e^{-k h}-scale weight
+    out = ~inside
+    assert np.all(fixed["P"][out].sum(1) == pytest.approx(1.0))
+    tail = (S[out] < (fixed["stats"][out, ref.ST_M] - 6.0 - 1e-9)[:, None]) & \
+        (np.arange(24)[None] < Ls[out][:, None])
+    assert np.all(fixed["P"][out][tail] > 0) and np.all(fwm["P"][out][tail] == 0)
