@@ -46,7 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gpt2_fwm",
-                    choices=["gpt2_fwm", "gpt2_heavy", "gpt2_fixed", "tiny"])
+                    choices=["gpt2_fwm", "gpt2_heavy", "gpt2_fixed", "gpt2_bf16exp",
+                             "gpt2_fp8exp", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -58,7 +59,21 @@ def parse():
 def workload(name):
     from quantized_softmax_attention_b200 import workloads as W
     return {"gpt2_fwm": W.gpt2_fwm, "gpt2_heavy": W.gpt2_heavy, "gpt2_fixed": W.gpt2_fixed,
-            "tiny": W.tiny}[name]()
+            "gpt2_bf16exp": lambda: W.gpt2_rounded_exp(False),
+            "gpt2_fp8exp": lambda: W.gpt2_rounded_exp(True), "tiny": W.tiny}[name]()
+
+
+def lib_config(w, K):
+    """The library's operator configuration of workload w (TF32 products)."""
+    return K.Config(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
+                    causal=w.causal, gemm=K.GEMM_TF32, op=w.operator)
+
+
+def oracle_config(w, ref):
+    """The oracle's configuration of workload w."""
+    return ref.RefConfig(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
+                         causal=w.causal, softmax=w.operator != 0,
+                         exp_round={2: ref.EXP_BF16, 3: ref.EXP_FP8}.get(w.operator, ref.EXP_EXACT))
 
 
 def gemm_units(w):
@@ -68,12 +83,17 @@ def gemm_units(w):
 def algorithmic_flops(w):
     """Forward 3U (+1U with Prob-STE) and backward 5U, U = B H T^2 d
     (2 flops per multiply-add over the causal half counts T^2 d per GEMM)."""
-    prob = w.rec == 1 and w.ste == 1
+    prob = w.operator == 0 and w.rec == 1 and w.ste == 1
     return (8 + (1 if prob else 0)) * gemm_units(w)
 
 
 def config_dict(w, n):
     names = {0: "MinMax", 1: "FWM", 2: "fixed step (untruncated)"}
+    if w.operator != 0:
+        ops = {1: "softmax", 2: "softmax, bf16-rounded exp", 3: "softmax, FP8-rounded exp"}
+        return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d,
+                "operator": ops[w.operator], "causal": w.causal, "parallelism": f"dp{n}",
+                "l2": "flushed between timed steps (256 MiB write)"}
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "K": w.K,
             "calibration": names[w.cal], "tau": w.tau if w.cal != 0 else None,
             "reconstruction": "LERP" if w.rec == 0 else "Nearest",
@@ -153,8 +173,7 @@ def cpu_oracle_rate(w, target_s=10.0, max_reps=20):
     import oracle as ref
     from quantized_softmax_attention_b200 import workloads as W
     q, k, v, g = (x.numpy() for x in W.make_inputs(w))
-    cfg = ref.RefConfig(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
-                        causal=w.causal)
+    cfg = oracle_config(w, ref)
     t0 = time.perf_counter()
     reps = 0
     while True:
@@ -178,8 +197,7 @@ def reference_arm(args):
     w = workload(args.workload)
     heads = min(w.H, 4)
     q, k, v, g = (x.numpy() for x in W.make_inputs(w, B=1, H=heads))
-    cfg = ref.RefConfig(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
-                        causal=w.causal)
+    cfg = oracle_config(w, ref)
     flops = algorithmic_flops(w) * heads / (w.B * w.H)
     for _ in range(args.warmup):
         ref.attention(q, k, v, g, cfg)
@@ -270,8 +288,7 @@ def diag_main(args):
     from quantized_softmax_attention_b200 import workloads as W
     torch.cuda.set_device(0)
     w = workload(args.workload)
-    cfg = K.Config(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
-                   causal=w.causal, gemm=K.GEMM_TF32)
+    cfg = lib_config(w, K)
     host = W.make_inputs(w)
     q, k, v, g = (x.cuda() for x in host)
     B, H, T, d = w.B, w.H, w.T, w.d
@@ -359,8 +376,7 @@ def diag_main(args):
         line["clocks"] = clocks
     if not args.no_cpu_baseline:
         import oracle as ref
-        rcfg = ref.RefConfig(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
-                             causal=w.causal)
+        rcfg = oracle_config(w, ref)
         Sh = S.cpu().numpy()
         Qh = host[0].numpy()
         ln = np.arange(1, T + 1) if w.causal else np.full(T, T)
@@ -407,8 +423,7 @@ def main():
     from quantized_softmax_attention_b200 import workloads as W
 
     w = workload(args.workload)
-    cfg = K.Config(K=w.K, cal=w.cal, tau=w.tau, rec=w.rec, ste=w.ste, grad=w.grad,
-                   causal=w.causal, gemm=K.GEMM_TF32)
+    cfg = lib_config(w, K)
     w_rank = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
     host = [x.pin_memory() for x in W.make_inputs(w_rank)]
     dev = [x.cuda() for x in host]

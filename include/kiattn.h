@@ -75,6 +75,15 @@ extern "C" {
 /* operator */
 #define KIA_OP_KINTERVAL 0
 #define KIA_OP_SOFTMAX 1 /* exact softmax attention (Appendix G reference row) */
+/* reduced-precision exponential baselines (Appendix D.5): softmax whose
+ * numerator e^{s-m} (fp32) is rounded to nearest-even bfloat16, or to
+ * nearest-even FP8 E4M3; P = R(e) / sum R(e).  The backward passes straight
+ * through the rounding (dS_j = e_j (dP_j - D) / W, e unrounded, D the row's
+ * dO . O, W the rounded normaliser) with the row maximum held fixed, as
+ * softmax's stabilising shift.  The calibration and gradient-mode fields do
+ * not apply. */
+#define KIA_OP_SOFTMAX_BF16EXP 2
+#define KIA_OP_SOFTMAX_FP8EXP 3
 
 /* error codes */
 #define KIA_OK 0

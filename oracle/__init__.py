@@ -24,6 +24,7 @@ _SRC = os.path.join(_HERE, "kiattn_ref.c")
 _LIB = os.path.join(_HERE, "libkiattn_ref.so")
 
 CAL_MINMAX, CAL_FWM, CAL_FIXED = 0, 1, 2
+EXP_EXACT, EXP_BF16, EXP_FP8 = 0, 1, 2
 REC_LERP, REC_NEAREST = 0, 1
 STE_WEIGHT, STE_PROB = 0, 1
 GRAD_FULL, GRAD_DETACH, GRAD_MAX_ONLY, GRAD_MIN_ONLY, GRAD_PROJECT = 0, 1, 2, 3, 4
@@ -45,6 +46,7 @@ class _Cfg(ctypes.Structure):
         ("causal", ctypes.c_int),
         ("softmax", ctypes.c_int),
         ("rounding", ctypes.c_int),
+        ("exp_round", ctypes.c_int),
     ]
 
 
@@ -61,11 +63,12 @@ class RefConfig:
     causal: bool = True
     softmax: bool = False
     rounding: int = ROUND_NONE
+    exp_round: int = EXP_EXACT   # softmax numerator: exact, bfloat16 or FP8 E4M3 (App. D.5)
 
     def c(self) -> _Cfg:
         return _Cfg(int(self.K), int(self.cal), float(self.tau), int(self.rec), int(self.ste),
                     int(self.grad), int(bool(self.causal)), int(bool(self.softmax)),
-                    int(self.rounding))
+                    int(self.rounding), int(self.exp_round))
 
     def replace(self, **kw) -> "RefConfig":
         d = dict(self.__dict__)
@@ -104,6 +107,8 @@ def lib():
                                               dp, dp, dp, dp, dp, dp, dp, dp]
         _lib.kiattn_ref_weights_fp32.argtypes = [fp, ctypes.c_int, ctypes.c_int, ip, cp, fp, ip,
                                                  fp, fp, fp]
+        _lib.kiattn_ref_round_exp_format.argtypes = [ctypes.c_float, ctypes.c_int]
+        _lib.kiattn_ref_round_exp_format.restype = ctypes.c_float
         _lib.kiattn_ref_own_exp.argtypes = [ctypes.c_double]
         _lib.kiattn_ref_own_exp.restype = ctypes.c_double
     return _lib
@@ -298,6 +303,12 @@ def geometry(S, row_len, cfg: RefConfig, Q=None):
     out[:, GEO_TOP_SOFTMAX] = np.where(top, Psm, 0.0).sum(axis=1)
     out[:, GEO_TOP_OP] = np.where(top, Pop, 0.0).sum(axis=1)
     return out
+
+
+def round_exp_format(x: float, mode: int) -> float:
+    """The oracle's rounding of an fp32 value to bfloat16 (mode 1) or FP8
+    E4M3 (mode 2), nearest-even (Appendix D.5 baselines)."""
+    return lib().kiattn_ref_round_exp_format(float(x), int(mode))
 
 
 def own_exp(x: float) -> float:

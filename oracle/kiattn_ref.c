@@ -73,6 +73,7 @@ typedef struct {
   int causal;   /* 1: key j is visible to query i iff j <= i */
   int softmax;  /* 1: exact softmax attention instead of K-interval */
   int rounding; /* REF_ROUND_* */
+  int exp_round; /* softmax only (Appendix D.5): 0 exact, 1 bfloat16, 2 FP8 E4M3 numerator */
 } ref_cfg;
 
 /* per-row statistics exported by the oracle, in this order */
@@ -251,9 +252,53 @@ static void row_backward(const double* s, int L, const ref_cfg* c, const rowstat
   *Aout = A; *Cout = C;
 }
 
-/* Exact softmax row (reference row of the sweep; Appendix G: softmax runs use
- * softmax's own backward). */
-static void softmax_row(const double* s, int L, double* P, rowstat* st) {
+/* Rounding of an fp32 value to bfloat16 (8 significand bits, fp32's
+ * exponent range), to nearest, ties to even: keep the top 16 bits. */
+static float round_bf16(float x) {
+  uint32_t b;
+  memcpy(&b, &x, 4);
+  if ((b & 0x7f800000u) == 0x7f800000u) return x;
+  b += 0x7fffu + ((b >> 16) & 1u);
+  b &= 0xffff0000u;
+  float y;
+  memcpy(&y, &b, 4);
+  return y;
+}
+
+/* Rounding to FP8 E4M3 (4 exponent bits with bias 7, 3 fraction bits;
+ * normal numbers from 2^-6, subnormals in steps of 2^-9, largest finite 448),
+ * to nearest, ties to even, saturating at 448. */
+static float round_e4m3(float x) {
+  const double a = fabs((double)x);
+  if (a != a) return x;
+  if (a >= 448.0) return x < 0 ? -448.0f : 448.0f;
+  int e;
+  frexp(a, &e);            /* a in [2^(e-1), 2^e) */
+  int E = e - 1;
+  if (E < -6) E = -6;      /* subnormal range: fixed step 2^-9 */
+  const double q = ldexp(1.0, E - 3);
+  const double r = nearbyint(a / q) * q;   /* a / q is exact; nearbyint: ties to even */
+  return (float)(x < 0 ? -r : r);
+}
+
+/* The numerator of the reduced-precision exponential baselines (Appendix
+ * D.5): e^{s-m} as fp32, then rounded to the format. */
+static double rounded_exp(double x, int mode) {
+  const float e32 = (float)exp(x);
+  if (mode == 1) return (double)round_bf16(e32);
+  if (mode == 2) return (double)round_e4m3(e32);
+  return exp(x);
+}
+
+float kiattn_ref_round_exp_format(float x, int mode) {
+  return mode == 1 ? round_bf16(x) : (mode == 2 ? round_e4m3(x) : x);
+}
+
+/* Softmax row (reference row of the sweep; Appendix G: softmax runs use
+ * softmax's own backward), or a reduced-precision exponential baseline:
+ * P = R(e^{s-m}) / sum R(e^{s-m}).  E receives the unrounded e^{s-m} (the
+ * straight-through slope of the baselines' backward). */
+static void softmax_row_r(const double* s, int L, int mode, double* P, double* E, rowstat* st) {
   double m = s[0];
   int am = 0;
   double n = s[0];
@@ -263,11 +308,16 @@ static void softmax_row(const double* s, int L, double* P, rowstat* st) {
     if (s[j] < n) { n = s[j]; an = j; }
   }
   double W = 0.0;
-  for (int j = 0; j < L; ++j) { P[j] = exp(s[j] - m); W += P[j]; }
+  for (int j = 0; j < L; ++j) {
+    E[j] = exp(s[j] - m);
+    P[j] = mode ? rounded_exp(s[j] - m, mode) : E[j];
+    W += P[j];
+  }
   for (int j = 0; j < L; ++j) P[j] /= W;
   st->m = m; st->n = n; st->am = am; st->an = an; st->h = 0.0;
   st->WL = W; st->WN = W; st->degen = 0;
 }
+
 
 /* ------------------------------------------------------------- row API */
 
@@ -301,7 +351,7 @@ int kiattn_ref_rows(const double* S, const int* row_len, int rows, int cols,
       rowstat st;
       double A = 0.0, C = 0.0;
       if (c->softmax) {
-        softmax_row(s, L, Pb, &st);
+        softmax_row_r(s, L, c->exp_round, Pb, ds, &st);
         if (pf) { for (int j = 0; j < cols; ++j) pf[j] = j < L ? Pb[j] : 0.0; }
         if (P_L) { for (int j = 0; j < cols; ++j) P_L[(size_t)i * cols + j] = j < L ? Pb[j] : 0.0; }
         if (P_N) { for (int j = 0; j < cols; ++j) P_N[(size_t)i * cols + j] = j < L ? Pb[j] : 0.0; }
@@ -309,7 +359,10 @@ int kiattn_ref_rows(const double* S, const int* row_len, int rows, int cols,
           const double* dp = dP + (size_t)i * cols;
           double D = 0.0;
           for (int j = 0; j < L; ++j) D += Pb[j] * dp[j];
-          for (int j = 0; j < cols; ++j) dS[(size_t)i * cols + j] = j < L ? Pb[j] * (dp[j] - D) : 0.0;
+          /* e^{s-m} (dP - D) / W: the softmax Jacobian, taken straight through
+           * the rounding of the reduced-precision baselines */
+          for (int j = 0; j < cols; ++j)
+            dS[(size_t)i * cols + j] = j < L ? ds[j] / st.WL * (dp[j] - D) : 0.0;
         }
       } else {
         row_forward(s, L, c, frozen_m ? frozen_m + i : NULL, frozen_n ? frozen_n + i : NULL,
@@ -409,8 +462,8 @@ int kiattn_ref_attention(const float* Q, const float* Kt, const float* V, const 
         double Wfwd, Wbar;
         const double *wf, *wb;
         if (c->softmax) {
-          softmax_row(s, L, P, &st);
-          /* unnormalised weights e^{s-m} so that O = sum(w v)/W like the rest */
+          softmax_row_r(s, L, c->exp_round, P, wN, &st);   /* wN: unrounded e^{s-m} */
+          /* unnormalised weights so that O = sum(w v)/W like the rest */
           for (int j = 0; j < L; ++j) wL[j] = P[j] * st.WL;
           wf = wL; wb = wL; Wfwd = st.WL; Wbar = st.WL;
         } else {
@@ -447,7 +500,8 @@ int kiattn_ref_attention(const float* Q, const float* Kt, const float* V, const 
           double D = 0.0;
           for (int x = 0; x < d; ++x) D += (double)dO[base + (size_t)i * d + x] * ob[x];
           if (c->softmax) {
-            for (int j = 0; j < L; ++j) ds[j] = P[j] * (dp[j] - D);
+            /* straight through the baselines' rounding: slope e^{s-m} / W */
+            for (int j = 0; j < L; ++j) ds[j] = wN[j] / st.WL * (dp[j] - D);
           } else {
             row_backward(s, L, c, &st, wL, wN, kk, tt, win, dp, D, ds, &A, &C);
           }

@@ -7,6 +7,9 @@
 // Attention", section 3 (Calibration, Reconstruction) and Appendix A.
 #pragma once
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,7 +39,26 @@ struct OpParams {
   int tf32_ops;   // CUDA-core kernels: truncate product operands to TF32 like tcgen05
   int fixed_step; // untruncated fixed step (Appendix D.4), run as FWM with K = the grid's
                   // extent, the first node count at which G_k underflows to zero in fp32
+  int exp_round;  // softmax only: 0 exact e^{s-m}; 1 rounded to bf16; 2 rounded to FP8 E4M3
 };
+
+// Reduced-precision exponential baselines (Appendix D.5): the softmax
+// numerator e^{s-m} (fp32) rounded to bfloat16 (R = 1) or to FP8 E4M3 (R =
+// 2), both to nearest, ties to even; R = 0 leaves it exact.
+template <int R>
+__device__ __forceinline__ float round_exp(float e) {
+  if constexpr (R == 1) {
+    return __bfloat162float(__float2bfloat16_rn(e));
+  } else if constexpr (R == 2) {
+    const __nv_fp8_storage_t q = __nv_cvt_float_to_fp8(e, __NV_SATFINITE, __NV_E4M3);
+    return __half2float(__half(__nv_cvt_fp8_to_halfraw(q, __NV_E4M3)));
+  } else {
+    return e;
+  }
+}
+__device__ __forceinline__ float round_exp_rt(float e, int mode) {
+  return mode == 1 ? round_exp<1>(e) : (mode == 2 ? round_exp<2>(e) : e);
+}
 
 // The tcgen05 kind::tf32 MMA reads fp32 operands and ignores their low 13
 // mantissa bits; CUDA-core kernels standing in for it apply the same mask.

@@ -32,7 +32,7 @@ __device__ __forceinline__ ElemFwd elem_forward(const OpParams& p, const RowStat
                                                 const float* tab, int ts, float s) {
   ElemFwd e;
   if (p.softmax) {
-    e.wf = expf(s - r.cal.m);
+    e.wf = round_exp_rt(expf(s - r.cal.m), p.exp_round);
     e.wl = e.wf;
     return e;
   }
@@ -63,7 +63,9 @@ __device__ __forceinline__ ElemFwd elem_forward(const OpParams& p, const RowStat
 __device__ __forceinline__ float elem_backward(const OpParams& p, const RowState& r,
                                                const float* tab, int ts, float s, float wf,
                                                float dw, float& A, float& C) {
-  if (p.softmax) return wf * dw;   // P (dP - D) with P = w / W, dw = (dP - D) / W
+  // softmax: e^{s-m} (dP - D) / W; the reduced-precision baselines pass
+  // straight through their rounding, so the slope is the unrounded e^{s-m}
+  if (p.softmax) return (p.exp_round ? expf(s - r.cal.m) : wf) * dw;
   if (r.degen) return dw;          // uniform P: (dP - mean dP) / |J|
   const GridPos g = grid_position(p, r.cal, s);
   if (g.tail) return 0.0f;         // FWM tail: zero gradient through mask and clamp

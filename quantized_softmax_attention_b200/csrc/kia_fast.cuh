@@ -16,8 +16,9 @@
 
 namespace kia {
 
-template <int CAL_, int REC_, bool PROB_, bool SOFTMAX_>
+template <int CAL_, int REC_, bool PROB_, bool SOFTMAX_, int EXPR_ = 0>
 struct Var {
+  static constexpr int EXPR = EXPR_;         // softmax numerator rounding (round_exp)
   static constexpr int CAL = CAL_;
   static constexpr int REC = REC_;
   static constexpr bool PROB = PROB_;        // Nearest + Prob-STE: forward also keeps P_L
@@ -115,7 +116,7 @@ __device__ __forceinline__ void fwd_weights2(const G& grid, float m, float rh, f
                                              float Km1f, float s0, float s1, float2& wf2,
                                              float2& wl2) {
   if constexpr (V::SOFTMAX) {
-    wf2 = make_float2(__expf(s0 - m), __expf(s1 - m));
+    wf2 = make_float2(round_exp<V::EXPR>(__expf(s0 - m)), round_exp<V::EXPR>(__expf(s1 - m)));
     wl2 = wf2;
   } else {
     float2 u = mul2(sub2(make_float2(m, m), make_float2(s0, s1)), make_float2(rh, rh));
@@ -152,7 +153,7 @@ template <class V, bool CLAMP0, class G>
 __device__ __forceinline__ void fwd_weights(const G& grid, float m, float rh, float Kf,
                                             float Km1f, float s, float& wf, float& wl) {
   if constexpr (V::SOFTMAX) {
-    wf = __expf(s - m);
+    wf = round_exp<V::EXPR>(__expf(s - m));
     wl = wf;
   } else {
     const Pos p = grid_pos<V, CLAMP0>(m, rh, Kf, Km1f, s);
@@ -182,6 +183,8 @@ __device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, flo
                                            float Kf, float Km1f, float s, float dw, float& A,
                                            float& C) {
   if constexpr (V::SOFTMAX) {
+    // straight through the rounding of the reduced-precision baselines:
+    // the slope is the unrounded e^{s-m}
     return __expf(s - m) * dw;
   } else {
     const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
@@ -217,8 +220,8 @@ __device__ __forceinline__ void kv_elem(const G& grid, float m, float rh, float 
                                         float& dS) {
   if constexpr (V::SOFTMAX) {
     const float w = __expf(s - m);
-    P = w * rWf;
-    dS = w * dw;
+    P = round_exp<V::EXPR>(w) * rWf;   // the forward's (rounded) probability
+    dS = w * dw;                       // straight through the rounding
   } else {
     const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
     const float2 g = grid.pair(p.k);

@@ -115,7 +115,7 @@ enum HeaderWord {
 __device__ inline void write_header(uint32_t* hdr, int B, int H, int T, int d, const OpParams& p) {
   hdr[HW_B] = B; hdr[HW_H] = H; hdr[HW_T] = T; hdr[HW_D] = d; hdr[HW_K] = p.K;
   hdr[HW_CAL] = p.fixed_step ? KIA_CAL_FIXED : p.cal; hdr[HW_REC] = p.rec; hdr[HW_STE] = p.ste; hdr[HW_CAUSAL] = p.causal;
-  hdr[HW_OP] = p.softmax; hdr[HW_TAU_BITS] = __float_as_uint(p.tau);
+  hdr[HW_OP] = p.softmax ? 1 + p.exp_round : 0; hdr[HW_TAU_BITS] = __float_as_uint(p.tau);
   __threadfence();
   hdr[HW_MAGIC] = kStatsMagic;
 }
@@ -127,7 +127,7 @@ __device__ inline bool header_matches(const uint32_t* hdr, int B, int H, int T, 
          hdr[HW_CAL] == (uint32_t)(p.fixed_step ? KIA_CAL_FIXED : p.cal) &&
          hdr[HW_REC] == (uint32_t)p.rec &&
          (p.rec == KIA_REC_LERP || hdr[HW_STE] == (uint32_t)p.ste) &&
-         hdr[HW_CAUSAL] == (uint32_t)p.causal && hdr[HW_OP] == (uint32_t)p.softmax &&
+         hdr[HW_CAUSAL] == (uint32_t)p.causal && hdr[HW_OP] == (uint32_t)(p.softmax ? 1 + p.exp_round : 0) &&
          hdr[HW_TAU_BITS] == __float_as_uint(p.tau);
 }
 

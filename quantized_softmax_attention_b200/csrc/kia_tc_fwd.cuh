@@ -584,7 +584,13 @@ int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
 // Calls f.template operator()<V>() with the compile-time variant of p.
 template <class F>
 int dispatch_variant(const OpParams& p, F&& f) {
-  if (p.softmax) return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_LERP, false, true>>();
+  if (p.softmax) {
+    if (p.exp_round == 1)
+      return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_LERP, false, true, 1>>();
+    if (p.exp_round == 2)
+      return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_LERP, false, true, 2>>();
+    return f.template operator()<Var<KIA_CAL_MINMAX, KIA_REC_LERP, false, true>>();
+  }
   const bool prob = p.rec == KIA_REC_NEAREST && p.ste == KIA_STE_PROB;
   if (p.cal == KIA_CAL_MINMAX) {
     if (p.rec == KIA_REC_LERP)

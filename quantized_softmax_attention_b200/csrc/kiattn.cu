@@ -57,7 +57,7 @@ int check_config(const kia_config* cfg) {
   if (cfg->ste != KIA_STE_WEIGHT && cfg->ste != KIA_STE_PROB) return KIA_ERR_INVALID_ARG;
   if (cfg->grad < KIA_GRAD_FULL || cfg->grad > KIA_GRAD_PROJECT) return KIA_ERR_INVALID_ARG;
   if (cfg->gemm != KIA_GEMM_TF32 && cfg->gemm != KIA_GEMM_FP32) return KIA_ERR_INVALID_ARG;
-  if (cfg->op != KIA_OP_KINTERVAL && cfg->op != KIA_OP_SOFTMAX) return KIA_ERR_INVALID_ARG;
+  if (cfg->op < KIA_OP_KINTERVAL || cfg->op > KIA_OP_SOFTMAX_FP8EXP) return KIA_ERR_INVALID_ARG;
   if (cfg->causal != 0 && cfg->causal != 1) return KIA_ERR_INVALID_ARG;
   if (cfg->cal != KIA_CAL_MINMAX && !(cfg->tau > 0.0f && cfg->tau < 1e30f))
     return KIA_ERR_INVALID_ARG;
@@ -85,7 +85,8 @@ OpParams make_params(const kia_config* cfg) {
   p.ste = (cfg->rec == KIA_REC_LERP) ? KIA_STE_WEIGHT : cfg->ste;
   p.grad = cfg->grad;
   p.causal = cfg->causal;
-  p.softmax = cfg->op == KIA_OP_SOFTMAX;
+  p.softmax = cfg->op != KIA_OP_KINTERVAL;
+  p.exp_round = cfg->op == KIA_OP_SOFTMAX_BF16EXP ? 1 : (cfg->op == KIA_OP_SOFTMAX_FP8EXP ? 2 : 0);
   p.tau = cfg->tau;
   p.fwm_h = (cfg->cal != KIA_CAL_MINMAX) ? cfg->tau / p.Kf : 0.0f;
   p.fwm_rh = (cfg->cal != KIA_CAL_MINMAX) ? p.Kf / cfg->tau : 0.0f;

@@ -22,7 +22,7 @@ REC_LERP, REC_NEAREST = 0, 1
 STE_WEIGHT, STE_PROB = 0, 1
 GRAD_FULL, GRAD_DETACH, GRAD_MAX_ONLY, GRAD_MIN_ONLY, GRAD_PROJECT = 0, 1, 2, 3, 4
 GEMM_TF32, GEMM_FP32 = 0, 1
-OP_KINTERVAL, OP_SOFTMAX = 0, 1
+OP_KINTERVAL, OP_SOFTMAX, OP_SOFTMAX_BF16EXP, OP_SOFTMAX_FP8EXP = 0, 1, 2, 3
 
 ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error", -4: "timeout",
           -5: "stats mismatch", -6: "capacity exceeded"}

@@ -39,6 +39,7 @@ class Workload:
     causal: bool = True
     seed: int = 0
     scores: str = "iid"          # iid | span_ladder | heavy
+    operator: int = 0            # 0 K-interval, 1 softmax, 2 / 3 bf16- / FP8-rounded exp softmax
     extra: dict = field(default_factory=dict, compare=False)
 
     def op(self) -> dict:
@@ -65,6 +66,15 @@ def gpt2_fixed() -> Workload:
     (Appendix D.4): h = tau / K = 1.5 without the tail cut; seed 1."""
     return Workload("gpt2_124M_B8H12T1024d64_fixedstep_nearest_probste_K4", 8, 12, 1024, 64, 4,
                     CAL_FIXED, REC_NEAREST, STE_PROB, seed=1, scores="span_ladder")
+
+
+def gpt2_rounded_exp(fp8: bool) -> Workload:
+    """The gpt2_fwm inputs under a reduced-precision exponential baseline
+    (Appendix D.5): softmax with its numerator rounded to bfloat16 or FP8."""
+    tag = "fp8exp" if fp8 else "bf16exp"
+    return Workload(f"gpt2_124M_B8H12T1024d64_softmax_{tag}", 8, 12, 1024, 64, 4, CAL_MINMAX,
+                    REC_LERP, STE_WEIGHT, seed=1, scores="span_ladder",
+                    operator=3 if fp8 else 2)
 
 
 def gpt2_heavy() -> Workload:

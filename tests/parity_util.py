@@ -42,13 +42,41 @@ def tf32_round(x: np.ndarray, rule: int) -> np.ndarray:
 def ref_cfg(cfg: K.Config, rounding: int) -> ref.RefConfig:
     return ref.RefConfig(K=cfg.K, cal=cfg.cal, tau=float(np.float32(cfg.tau)), rec=cfg.rec,
                          ste=cfg.ste, grad=cfg.grad, causal=bool(cfg.causal),
-                         softmax=cfg.op == K.OP_SOFTMAX, rounding=rounding)
+                         softmax=cfg.op != K.OP_KINTERVAL, rounding=rounding,
+                         exp_round={K.OP_SOFTMAX_BF16EXP: ref.EXP_BF16,
+                                    K.OP_SOFTMAX_FP8EXP: ref.EXP_FP8}.get(cfg.op, ref.EXP_EXACT))
 
 
 def oracle_scores(Q, Kt, rule):
     q = tf32_round(Q, rule)
     k = tf32_round(Kt, rule)
     return np.einsum("bhid,bhjd->bhij", q, k)
+
+
+def _round_format(x: np.ndarray, op: int) -> np.ndarray:
+    """Nearest-even rounding of fp32 values to bfloat16 or FP8 E4M3 by torch's
+    own dtype conversions (test-side)."""
+    t = torch.from_numpy(np.ascontiguousarray(x, np.float32))
+    dt = torch.bfloat16 if op == K.OP_SOFTMAX_BF16EXP else torch.float8_e4m3fn
+    return t.to(dt).to(torch.float32).numpy()
+
+
+def _rounding_flags(S, cfg: K.Config) -> np.ndarray:
+    """Rows with a numerator e^{s-m} >= 1e-6 whose rounding to the baseline's
+    format would change under a relative perturbation of the exponential's
+    error size (the kernels' fast exponential and the oracle's fp64 one may
+    land on either side of a rounding boundary there)."""
+    B, H, T, _ = S.shape
+    flags = np.zeros((B, H, T), bool)
+    for i in range(T):
+        L = i + 1 if cfg.causal else T
+        x = S[:, :, i, :L] - S[:, :, i, :L].max(-1, keepdims=True)
+        e = np.exp(x)
+        rel = 2.0 ** -21 + np.abs(x) * 2.0 ** -22
+        lo = _round_format((e * (1 - rel)).astype(np.float32), cfg.op)
+        hi = _round_format((e * (1 + rel)).astype(np.float32), cfg.op)
+        flags[:, :, i] = np.any((lo != hi) & (e >= 1e-6), -1)
+    return flags
 
 
 def flag_rows(Q, Kt, cfg: K.Config, rule: int, delta: float) -> np.ndarray:
@@ -58,6 +86,8 @@ def flag_rows(Q, Kt, cfg: K.Config, rule: int, delta: float) -> np.ndarray:
     flags = np.zeros((B, H, T), bool)
     if cfg.op == K.OP_SOFTMAX:
         return flags
+    if cfg.op in (K.OP_SOFTMAX_BF16EXP, K.OP_SOFTMAX_FP8EXP):
+        return _rounding_flags(S, cfg)
     tau = float(np.float32(cfg.tau))
     for i in range(T):
         L = i + 1 if cfg.causal else T

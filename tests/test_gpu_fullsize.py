@@ -140,6 +140,14 @@ def test_exact_softmax_reference_row_full_size():
     _check_heads(q, k, v, g, _cfg(w, op=K.OP_SOFTMAX), [(0, 0), (9, 4)], (None,))
 
 
+@pytest.mark.parametrize("op", [K.OP_SOFTMAX_BF16EXP, K.OP_SOFTMAX_FP8EXP])
+def test_reduced_precision_exp_baselines_full_size(op):
+    """Appendix D.5 baselines at the bench shape B8 H12 T1024 d64."""
+    w = W.gpt2_fwm()
+    q, k, v, g = (x.numpy() for x in W.make_inputs(w))
+    _check_heads(q, k, v, g, _cfg(w, op=op), [(1, 2), (6, 10)], (None,))
+
+
 # ----------------------------------------------------------------- edges
 
 @pytest.mark.parametrize("T", [1, 2, 5, 127, 129])

@@ -213,6 +213,36 @@ def test_tc_path_softmax_and_noncausal():
             assert errs[name] < 2e-3, (causal, op, errs)
 
 
+REDUCED_EXP = [K.OP_SOFTMAX_BF16EXP, K.OP_SOFTMAX_FP8EXP]
+
+
+@pytest.mark.parametrize("op", REDUCED_EXP)
+@pytest.mark.parametrize("shape", [(1, 2, 200, 64), (2, 1, 384, 64)])
+def test_tc_reduced_precision_exp_baselines(op, shape):
+    """Appendix D.5 baselines on the tcgen05 path: softmax with a bfloat16-
+    or FP8-rounded numerator, straight-through backward; TF32 tolerance."""
+    B, H, T, d = shape
+    Q, Kt, V, dO = _inputs(B, H, T, d, 71 + op + T, qscale=0.5)
+    for causal in (True, False):
+        cfg = K.Config(op=op, causal=causal)
+        errs, _, _ = compare(Q, Kt, V, dO, cfg, TF32_RULE, 2e-3, 1e-4)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 2e-3, (op, causal, errs)
+        assert errs["flagged"] < errs["rows"] // 4
+
+
+@pytest.mark.parametrize("op", REDUCED_EXP)
+@pytest.mark.parametrize("shape", [(1, 2, 200, 64), (1, 1, 160, 128)])
+def test_fp32_reduced_precision_exp_baselines(op, shape):
+    B, H, T, d = shape
+    Q, Kt, V, dO = _inputs(B, H, T, d, 81 + op + T, qscale=0.5)
+    for causal in (True, False):
+        cfg = K.Config(op=op, causal=causal, gemm=K.GEMM_FP32)
+        errs, _, _ = compare(Q, Kt, V, dO, cfg, ref.ROUND_NONE, 1e-5, 1e-4)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 1e-5, (op, causal, errs)
+
+
 def test_tc_forward_bitwise_identical_across_modes_and_surrogates():
     Q, Kt, V, dO = _inputs(2, 2, 256, 64, 42, qscale=0.7)
     from parity_util import run_gpu
