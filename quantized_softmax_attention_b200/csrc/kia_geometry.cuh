@@ -9,8 +9,10 @@
 // One warp per row, specialised at compile time on calibration and
 // reconstruction.  Rows of at most kGeoRegKeys keys (T a multiple of 4) are
 // read from HBM once into registers, four keys per lane per 128-key chunk,
-// and only the chunks the row reaches are touched; other rows take three
-// sweeps over global memory, the later two served by L1/L2.  The operator
+// and only the chunks the row reaches are touched; the third sweep
+// recomputes e and w from the held scores rather than keeping them, for
+// occupancy.  Other rows take three sweeps over global memory, the later two
+// served by L1/L2.  The operator
 // weights are the fused kernels' paired fp32 weight stage (kia_fast.cuh), so
 // the grid decisions are the forward's; a key is in the top bucket iff its
 // grid coordinate u = (m - s) / h is below 1/2 (nearest node 0).
@@ -85,7 +87,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <class V>
-__global__ void __launch_bounds__(32 * kGeoWarps)
+__global__ void __launch_bounds__(32 * kGeoWarps, 4)
 geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long long rows, int T,
                 int d, int causal, OpParams p, float* __restrict__ out) {
   // (G_k, G_{k+1}) pairs: one per warp under MinMax (the grid follows the
@@ -105,6 +107,13 @@ geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long l
   const bool in_regs = (T & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&
                        L <= kGeoRegKeys;
   const int nch = (L + 127) >> 7;   // chunks the row reaches (warp-uniform)
+  // the query's squared norm, loaded up front so that its latency overlaps
+  // the score loads
+  float qn = 0.0f;
+  if (Q) {
+    const float* q = Q + row * (long long)d;
+    for (int k = lane; k < d; k += 32) qn = fmaf(q[k], q[k], qn);
+  }
 
   // sweep 1: row extrema (section 3, calibration statistics)
   float4 v[kGeoChunks];
@@ -155,20 +164,22 @@ geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long l
     r.g.q = sPair[0];
   }
 
-  // sweep 2: normalisers, entropy sums and top-bucket masses
+  // sweep 2: normalisers, entropy sums and top-bucket masses (the scores
+  // stay in registers; sweep 3 recomputes e and w from them, which keeps the
+  // register count low enough for more resident warps)
   GeoSums a = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  float4 w4[kGeoChunks];
   if (in_regs) {
 #pragma unroll
     for (int cc = 0; cc < kGeoChunks; ++cc) {
       if (cc < nch) {
         const int j = 4 * lane + 128 * cc;
+        float x0 = v[cc].x, x1 = v[cc].y, x2 = v[cc].z, x3 = v[cc].w, w0, w1, w2, w3;
         if (128 * cc + 128 <= L) {
-          geo_pair<V, false>(r, v[cc].x, v[cc].y, w4[cc].x, w4[cc].y, true, true, a);
-          geo_pair<V, false>(r, v[cc].z, v[cc].w, w4[cc].z, w4[cc].w, true, true, a);
+          geo_pair<V, false>(r, x0, x1, w0, w1, true, true, a);
+          geo_pair<V, false>(r, x2, x3, w2, w3, true, true, a);
         } else {
-          geo_pair<V, true>(r, v[cc].x, v[cc].y, w4[cc].x, w4[cc].y, j < L, j + 1 < L, a);
-          geo_pair<V, true>(r, v[cc].z, v[cc].w, w4[cc].z, w4[cc].w, j + 2 < L, j + 3 < L, a);
+          geo_pair<V, true>(r, x0, x1, w0, w1, j < L, j + 1 < L, a);
+          geo_pair<V, true>(r, x2, x3, w2, w3, j + 2 < L, j + 3 < L, a);
         }
       }
     }
@@ -185,11 +196,16 @@ geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long l
   // sweep 3: total variation 1/2 sum_j |P_op,j - P_softmax,j|
   float tv = 0.0f;
   if (in_regs) {
+    GeoSums dummy = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int cc = 0; cc < kGeoChunks; ++cc) {
       if (cc < nch) {
-        tv += fabsf(fmaf(w4[cc].x, rW, -v[cc].x * rZ)) + fabsf(fmaf(w4[cc].y, rW, -v[cc].y * rZ)) +
-              fabsf(fmaf(w4[cc].z, rW, -v[cc].z * rZ)) + fabsf(fmaf(w4[cc].w, rW, -v[cc].w * rZ));
+        const int j = 4 * lane + 128 * cc;
+        float x0 = v[cc].x, x1 = v[cc].y, x2 = v[cc].z, x3 = v[cc].w, w0, w1, w2, w3;
+        geo_pair<V, true>(r, x0, x1, w0, w1, j < L, j + 1 < L, dummy);
+        geo_pair<V, true>(r, x2, x3, w2, w3, j + 2 < L, j + 3 < L, dummy);
+        tv += fabsf(fmaf(w0, rW, -x0 * rZ)) + fabsf(fmaf(w1, rW, -x1 * rZ)) +
+              fabsf(fmaf(w2, rW, -x2 * rZ)) + fabsf(fmaf(w3, rW, -x3 * rZ));
       }
     }
   } else {
@@ -202,12 +218,7 @@ geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long l
   }
   tv = 0.5f * warp_sum(tv);
 
-  float qn = 0.0f;
-  if (Q) {
-    const float* q = Q + row * (long long)d;
-    for (int k = lane; k < d; k += 32) qn = fmaf(q[k], q[k], qn);
-    qn = sqrtf(warp_sum(qn));
-  }
+  if (Q) qn = sqrtf(warp_sum(qn));
   if (lane < kGeoFields) {
     float val;
     switch (lane) {
