@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--diag", default=None, choices=["geometry", "decomposition"],
                     help="time one of the diagnostic row kernels instead of the step")
+    ap.add_argument("--matrix", default=None, choices=["variants", "sweep"],
+                    help="one JSON line per operator variant (every calibration x "
+                         "reconstruction x surrogate x gradient mode at the 124M shape) or per "
+                         "point of the B16 H12 T 1024-4096 throughput sweep")
     return ap.parse_args()
 
 
@@ -83,6 +87,8 @@ def gemm_units(w):
 def algorithmic_flops(w):
     """Forward 3U (+1U with Prob-STE) and backward 5U, U = B H T^2 d
     (2 flops per multiply-add over the causal half counts T^2 d per GEMM)."""
+    if w.operator == 1:
+        return 7 * gemm_units(w)   # exact softmax: one S in the forward (online rescaling)
     prob = w.operator == 0 and w.rec == 1 and w.ste == 1
     return (8 + (1 if prob else 0)) * gemm_units(w)
 
@@ -401,6 +407,81 @@ def diag_main(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------ variant matrices
+
+def matrix_main(args):
+    """Fwd+bwd throughput over a matrix of operator variants: `variants` runs
+    the 124M span-ladder inputs under every calibration x reconstruction x
+    surrogate x gradient mode; `sweep` runs the B16 H12 d64 throughput sweep
+    (T in 1024..4096, K in 2..64, both calibrations, three reconstructions,
+    plus exact softmax per T).  Same timing rules as the step: warm-up, L2
+    flushed between timed steps, CUDA events on the launching stream."""
+    import torch
+    from quantized_softmax_attention_b200 import kiattn as K
+    from quantized_softmax_attention_b200 import workloads as W
+    torch.cuda.set_device(0)
+    bf16, _, src = peaks()
+    peak = bf16 * TF32_OVER_BF16
+    recs = [(W.REC_LERP, W.STE_WEIGHT), (W.REC_NEAREST, W.STE_WEIGHT),
+            (W.REC_NEAREST, W.STE_PROB)]
+    runs = []
+    if args.matrix == "variants":
+        base = W.gpt2_fwm()
+        for cal in (W.CAL_MINMAX, W.CAL_FWM, W.CAL_FIXED):
+            for rec, ste in recs:
+                for grad in range(5):
+                    runs.append(W.Workload(**{**base.__dict__, "cal": cal, "rec": rec, "ste": ste,
+                                              "grad": grad, "name": base.name}))
+    else:
+        for T in (1024, 2048, 4096):
+            for Kint in (2, 4, 16, 32, 64):
+                for cal in (W.CAL_MINMAX, W.CAL_FWM):
+                    for rec, ste in recs:
+                        runs.append(W.sweep(T, Kint, cal, rec, ste))
+            runs.append(W.Workload(**{**W.sweep(T, 4, W.CAL_MINMAX, W.REC_LERP,
+                                                W.STE_WEIGHT).__dict__, "operator": 1}))
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    inputs = {}
+    for w in runs:
+        key = (w.B, w.H, w.T, w.d, w.seed, w.scores)
+        if key not in inputs:
+            inputs.clear()
+            inputs[key] = [x.cuda() for x in W.make_inputs(w)]
+        q, k, v, g = inputs[key]
+        cfg = lib_config(w, K)
+        bufs = K.Buffers(w.B, w.H, w.T, w.d, cfg)
+
+        def step():
+            K.kiattn_fwd(q, k, v, bufs.O, bufs.stats, cfg)
+            K.kiattn_bwd(q, k, v, bufs.O, g, bufs.stats, bufs.dQ, bufs.dK, bufs.dV, bufs.work, cfg)
+
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        err = K.kiattn_device_error(True)
+        if err != 0:
+            raise RuntimeError(f"device error word {err}")
+        ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+        tf = algorithmic_flops(w) / (ms * 1e-3) / 1e12
+        cd = config_dict(w, 1)
+        cd["grad"] = ("full", "detach", "max-only", "min-only", "projection")[w.grad]
+        print(json.dumps({"matrix": args.matrix, "config": cd, "value": tf, "unit": "TFLOP/s",
+                          "ms_per_step": ms, "frac_of_tf32_roofline": tf / peak,
+                          "peak_source": f"{src} bf16 dense x {TF32_OVER_BF16:.4f}",
+                          "steps": args.steps, "warmup": args.warmup}), flush=True)
+        del bufs
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -408,6 +489,9 @@ def main():
         return
     if args.diag:
         diag_main(args)
+        return
+    if args.matrix:
+        matrix_main(args)
         return
     import torch
     import torch.distributed as dist
@@ -571,6 +655,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32",
             "data": "synthetic", "config": config_dict(w, world), "roofline": roof,
             "frac_of_tf32_roofline": value / world / peak,
+            "softmax_equivalent": {"value": value * 7.0 / (flops / gemm_units(w)),
+                                   "unit": "TFLOP/s", "flops_per_step": "7U (exact softmax)"},
             "gpu_launches": launches_per_step * args.steps}
     if e2e:
         line["e2e"] = e2e

@@ -150,9 +150,10 @@ bwd_scatter_kernel(const float* __restrict__ Q, WorkView wk, float* __restrict__
 }
 
 // Zero-sum projection, common-mode part.  Block = (bh, 32-column chunk);
-// 8 groups of 32 threads split the T rows into contiguous ranges; fp64
+// 32 groups of 32 threads split the T rows into contiguous ranges (enough
+// resident warps to keep the row loads in flight); fp64
 // running sums.
-constexpr int kScanGroups = 8;
+constexpr int kScanGroups = 32;
 
 template <int D>
 __global__ void __launch_bounds__(32 * kScanGroups)

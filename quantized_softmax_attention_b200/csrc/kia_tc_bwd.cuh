@@ -356,16 +356,15 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int k = part; k <= p.K; k += kRowSplit)
             sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
       }
-      using Grid = std::conditional_t<V::MINMAX, GridF, GridP>;
-      Grid grid;
-      if constexpr (V::MINMAX)
-        grid = tab_in_smem ? GridF{sTab + r, KIA_TILE} : GridF{st.table + qr * (p.K + 1), 1};
-      else grid = GridP{sPair};
       mbar_arrive(&bar.row_sync);
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (2 * n) & 1, abort))) { failed = true; break; }
       const float Dc = sDc[r];
       const float nDr = -Dc * rWb;            // dw = (dP - D) / W_bar as one fma
       float A = 0.0f, C = 0.0f;
+      // the unit loop, instantiated per grid placement so that the grid
+      // loads of the element loop are shared-memory loads when the grid is
+      // in shared memory (a runtime choice of pointer makes them generic)
+      auto unit_loop = [&](const auto& grid) {
       for (int u = grp; u < nunits && !failed; u += 2) {
         const int j = u >> 1, gu = gbase + u, rg = gu % R;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (gu / R) & 1, abort))) { failed = true; break; }
@@ -405,6 +404,13 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bar.elem_done[rg]);
+      }
+      };
+      if constexpr (V::MINMAX) {
+        if (tab_in_smem) unit_loop(GridF{sTab + r, KIA_TILE});
+        else unit_loop(GridF{st.table + qr * (p.K + 1), 1});
+      } else {
+        unit_loop(GridP{sPair});
       }
       if (failed) break;
       gbase += nunits;
@@ -844,9 +850,30 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
           }
         }
-        if (V::MINMAX && tab_in_smem) {
-          const long long qr = rowbase + (q < T ? q : T - 1);
-          for (int kk = 0; kk < K1; ++kk) sTab[e * K1 + kk] = st.table[qr * K1 + kk];
+      }
+      if (V::MINMAX && tab_in_smem) {
+        // the unit's 64 per-query grids are consecutive rows of the stats
+        // table: one coalesced copy, its loads issued together in four batches
+        // (rows past T are filled with ones; their queries are masked)
+        const int qf = 64 * (2 * item_q0(it) + u);
+        const int nvalid = max(0, min(kSlotQ, T - qf)) * K1, ntot = kSlotQ * K1;
+        const float* src = st.table + (rowbase + qf) * K1;
+        float* dst = sTab + (size_t)sl * kSlotQ * K1;
+        constexpr int kBatches = 4;
+        constexpr int kBatch = (kSlotQ * (kBwdSmemTabK + 1) + 32 * kBatches - 1) / (32 * kBatches);
+#pragma unroll
+        for (int b = 0; b < kBatches; ++b) {
+          float buf[kBatch];
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) {
+            const int x = lane + 32 * (b * kBatch + i);
+            buf[i] = x < nvalid ? src[x] : 1.0f;
+          }
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) {
+            const int x = lane + 32 * (b * kBatch + i);
+            if (x < ntot) dst[x] = buf[i];
+          }
         }
       }
       __syncwarp();
@@ -892,8 +919,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           const int ql0 = 64 * (u & 1) + 32 * sub + 16 * c;   // first query (in the tile) of the chunk
           const int e0 = sl * kSlotQ + 32 * sub + 16 * c;     // its slot entry
           // the element loop, without the mask test on units with no masked pair
-          auto body = [&](auto edge_c) {
+          auto body = [&](auto edge_c, auto tabs_c) {
             constexpr bool EDGE = decltype(edge_c)::value;
+            constexpr bool TABS = decltype(tabs_c)::value;   // per-query grids in shared memory
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int ql = ql0 + i;
@@ -902,9 +930,10 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
               const float dw = fmaf(g[i], c4.z, c4.w);
               float P, dS;
               if constexpr (V::MINMAX) {
-                const GridF grid{tab_in_smem ? sTab + (e0 + i) * K1
-                                             : st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1,
-                                 1};
+                const float* gp;
+                if constexpr (TABS) gp = sTab + (e0 + i) * K1;
+                else gp = st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1;
+                const GridF grid{gp, 1};
                 // degenerate rows (rh = 0) take dS = dw; under the projection c2.y
                 // holds the shift, so the flag comes from rh itself
                 const float dg = PROJ ? (c4.y == 0.0f ? 1.0f : 0.0f) : c2.y;
@@ -924,8 +953,16 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
               g[i] = dS;
             }
           };
-          if (edge) body(std::true_type{});
-          else body(std::false_type{});
+          auto run = [&](auto tabs_c) {
+            if (edge) body(std::true_type{}, tabs_c);
+            else body(std::false_type{}, tabs_c);
+          };
+          if constexpr (V::MINMAX) {
+            if (tab_in_smem) run(std::true_type{});
+            else run(std::false_type{});
+          } else {
+            run(std::true_type{});
+          }
           if constexpr (!PROJ && !V::SOFTMAX) {
             // the chunk's queries whose argmax (argmin) key lies in this warp's
             // 32 keys: a warp-uniform test, the per-element work only for them
