@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--workload", default="gpt2_fwm",
                     choices=["gpt2_fwm", "gpt2_heavy", "gpt2_fixed", "gpt2_bf16exp",
                              "gpt2_fp8exp", "tiny"])
+    ap.add_argument("--grad", default=None,
+                    choices=["full", "detach", "max-only", "min-only", "projection"],
+                    help="override the workload's gradient mode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -60,8 +63,14 @@ def parse():
     return ap.parse_args()
 
 
-def workload(name):
+GRAD_NAMES = ("full", "detach", "max-only", "min-only", "projection")
+
+
+def workload(name, grad=None):
     from quantized_softmax_attention_b200 import workloads as W
+    if grad is not None:
+        w = workload(name)
+        return W.Workload(**{**w.__dict__, "grad": GRAD_NAMES.index(grad)})
     return {"gpt2_fwm": W.gpt2_fwm, "gpt2_heavy": W.gpt2_heavy, "gpt2_fixed": W.gpt2_fixed,
             "gpt2_bf16exp": lambda: W.gpt2_rounded_exp(False),
             "gpt2_fp8exp": lambda: W.gpt2_rounded_exp(True), "tiny": W.tiny}[name]()
@@ -104,7 +113,7 @@ def config_dict(w, n):
             "calibration": names[w.cal], "tau": w.tau if w.cal != 0 else None,
             "reconstruction": "LERP" if w.rec == 0 else "Nearest",
             "surrogate": None if w.rec == 0 else ("Prob-STE" if w.ste else "Weight-STE"),
-            "grad": "full", "causal": w.causal, "parallelism": f"dp{n}",
+            "grad": GRAD_NAMES[w.grad], "causal": w.causal, "parallelism": f"dp{n}",
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
@@ -200,7 +209,7 @@ def reference_arm(args):
         return
     import oracle as ref
     from quantized_softmax_attention_b200 import workloads as W
-    w = workload(args.workload)
+    w = workload(args.workload, args.grad)
     heads = min(w.H, 4)
     q, k, v, g = (x.numpy() for x in W.make_inputs(w, B=1, H=heads))
     cfg = oracle_config(w, ref)
@@ -293,7 +302,7 @@ def diag_main(args):
     from quantized_softmax_attention_b200 import kiattn as K
     from quantized_softmax_attention_b200 import workloads as W
     torch.cuda.set_device(0)
-    w = workload(args.workload)
+    w = workload(args.workload, args.grad)
     cfg = lib_config(w, K)
     host = W.make_inputs(w)
     q, k, v, g = (x.cuda() for x in host)
@@ -474,7 +483,6 @@ def matrix_main(args):
         ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
         tf = algorithmic_flops(w) / (ms * 1e-3) / 1e12
         cd = config_dict(w, 1)
-        cd["grad"] = ("full", "detach", "max-only", "min-only", "projection")[w.grad]
         print(json.dumps({"matrix": args.matrix, "config": cd, "value": tf, "unit": "TFLOP/s",
                           "ms_per_step": ms, "frac_of_tf32_roofline": tf / peak,
                           "peak_source": f"{src} bf16 dense x {TF32_OVER_BF16:.4f}",
@@ -506,7 +514,7 @@ def main():
     from quantized_softmax_attention_b200 import kiattn as K
     from quantized_softmax_attention_b200 import workloads as W
 
-    w = workload(args.workload)
+    w = workload(args.workload, args.grad)
     cfg = lib_config(w, K)
     w_rank = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
     host = [x.pin_memory() for x in W.make_inputs(w_rank)]

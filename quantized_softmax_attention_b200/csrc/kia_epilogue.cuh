@@ -149,57 +149,80 @@ bwd_scatter_kernel(const float* __restrict__ Q, WorkView wk, float* __restrict__
     dK[(rowbase + base) * D + e] += acc[e];
 }
 
-// Zero-sum projection, common-mode part.  Block = (bh, 32-column chunk);
-// 32 groups of 32 threads split the T rows into contiguous ranges (enough
-// resident warps to keep the row loads in flight); fp64
-// running sums.
-constexpr int kScanGroups = 32;
+// Zero-sum projection, common-mode part: dQ_i += c_i sum_{j in J_i} k_j and
+// (with_dk) dK_j += sum_{i : j in J_i} c_i q_i.  Block = (bh, 32-column chunk,
+// 128-row chunk); each of its 8 warps owns 16 consecutive rows.  The sums
+// over the rows before (for dQ) and after (for dK) the chunk are re-read by
+// the block (from L2 after the first blocks of a head), the in-chunk prefix
+// is exclusive across warps; fp64 running sums.
+constexpr int kScanRows = 128, kScanWarps = 8;
 
 template <int D>
-__global__ void __launch_bounds__(32 * kScanGroups)
+__global__ void __launch_bounds__(32 * kScanWarps)
 bwd_project_scan_kernel(const float* __restrict__ Q, const float* __restrict__ Kt, WorkView wk,
                         float* __restrict__ dQ, float* __restrict__ dK, OpParams p, int T,
                         int with_dk) {
   if (*wk.status != 0) return;
-  __shared__ double sK[kScanGroups][32];
-  __shared__ double sQ[kScanGroups][32];
+  __shared__ double sK[kScanWarps][32];   // per-warp partial sums of k (rows before / own)
+  __shared__ double sQ[kScanWarps][32];   // per-warp partial sums of c q (rows after / own)
   const int bh = blockIdx.x;
-  const int col = blockIdx.y * 32 + (threadIdx.x & 31);
-  const int grp = threadIdx.x >> 5;
-  const int per = (T + kScanGroups - 1) / kScanGroups;
-  const int r0 = grp * per, r1 = min(T, r0 + per);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int col = blockIdx.y * 32 + lane;
+  const int c0 = blockIdx.z * kScanRows, c1 = min(T, c0 + kScanRows);
   const size_t base = (size_t)bh * T * D;
   const float* cc = wk.gm + (size_t)bh * T;
-  double sk = 0.0, sq = 0.0;
-  for (int r = r0; r < r1; ++r) {
-    sk += (double)Kt[base + (size_t)r * D + col];
-    sq += (double)cc[r] * (double)Q[base + (size_t)r * D + col];
+  const bool causal = p.causal;
+  // rows outside the chunk that every row of the chunk sees
+  const int kb = causal ? c0 : 0, ke = causal ? c0 : T;    // dQ: keys [0, c0) (or all)
+  double ok = 0.0, oq = 0.0;
+  if (causal) {
+    for (int r = warp; r < kb; r += kScanWarps) ok += (double)Kt[base + (size_t)r * D + col];
+    if (with_dk)
+      for (int r = c1 + warp; r < T; r += kScanWarps)
+        oq += (double)cc[r] * (double)Q[base + (size_t)r * D + col];
+  } else {
+    for (int r = warp; r < ke; r += kScanWarps) {
+      ok += (double)Kt[base + (size_t)r * D + col];
+      if (with_dk) oq += (double)cc[r] * (double)Q[base + (size_t)r * D + col];
+    }
   }
-  sK[grp][threadIdx.x & 31] = sk;
-  sQ[grp][threadIdx.x & 31] = sq;
+  sK[warp][lane] = ok;
+  sQ[warp][lane] = oq;
   __syncthreads();
-  double allK = 0.0, allQ = 0.0, preK = 0.0, sufQ = 0.0;
-  for (int g = 0; g < kScanGroups; ++g) {
-    allK += sK[g][threadIdx.x & 31];
-    allQ += sQ[g][threadIdx.x & 31];
-    if (g < grp) preK += sK[g][threadIdx.x & 31];
-    if (g > grp) sufQ += sQ[g][threadIdx.x & 31];
-  }
-  if (!p.causal) {
-    for (int r = r0; r < r1; ++r) {
-      dQ[base + (size_t)r * D + col] += (float)((double)cc[r] * allK);
-      if (with_dk) dK[base + (size_t)r * D + col] += (float)allQ;
+  double outK = 0.0, outQ = 0.0;
+#pragma unroll
+  for (int w = 0; w < kScanWarps; ++w) { outK += sK[w][lane]; outQ += sQ[w][lane]; }
+  __syncthreads();
+  if (!causal) {
+    for (int r = c0 + warp; r < c1; r += kScanWarps) {
+      dQ[base + (size_t)r * D + col] += (float)((double)cc[r] * outK);
+      if (with_dk) dK[base + (size_t)r * D + col] += (float)outQ;
     }
     return;
   }
-  // prefix over keys for dQ (j <= i), suffix over queries for dK (i >= j)
-  double runK = preK;
+  // causal: this warp's 16 rows, with the exclusive in-chunk prefix (keys)
+  // and suffix (queries) of the other warps' rows
+  const int per = kScanRows / kScanWarps;
+  const int r0 = c0 + warp * per, r1 = min(c1, r0 + per);
+  double mk = 0.0, mq = 0.0;
+  for (int r = r0; r < r1; ++r) {
+    mk += (double)Kt[base + (size_t)r * D + col];
+    if (with_dk) mq += (double)cc[r] * (double)Q[base + (size_t)r * D + col];
+  }
+  sK[warp][lane] = mk;
+  sQ[warp][lane] = mq;
+  __syncthreads();
+  double runK = outK, runQ = outQ;
+#pragma unroll
+  for (int w = 0; w < kScanWarps; ++w) {
+    if (w < warp) runK += sK[w][lane];
+    if (w > warp) runQ += sQ[w][lane];
+  }
   for (int r = r0; r < r1; ++r) {
     runK += (double)Kt[base + (size_t)r * D + col];
     dQ[base + (size_t)r * D + col] += (float)((double)cc[r] * runK);
   }
   if (!with_dk) return;
-  double runQ = sufQ;
   for (int r = r1 - 1; r >= r0; --r) {
     runQ += (double)cc[r] * (double)Q[base + (size_t)r * D + col];
     dK[base + (size_t)r * D + col] += (float)runQ;

@@ -184,8 +184,8 @@ int backward_rows(const float* Q, const float* Kt, const float* O, const float* 
   bwd_calib_kernel<D><<<nb, 32 * kRowWarps, 0, s>>>(Q, Kt, st, wk, dQ, dK, dS_dbg, p, B, H, T);
   if (launch_status()) return KIA_ERR_CUDA;
   if (!p.softmax && p.grad == KIA_GRAD_PROJECT) {
-    dim3 g(B * H, D / 32);
-    bwd_project_scan_kernel<D><<<g, 32 * kScanGroups, 0, s>>>(Q, Kt, wk, dQ, dK, p, T, 1);
+    dim3 g(B * H, D / 32, (T + kScanRows - 1) / kScanRows);
+    bwd_project_scan_kernel<D><<<g, 32 * kScanWarps, 0, s>>>(Q, Kt, wk, dQ, dK, p, T, 1);
     if (launch_status()) return KIA_ERR_CUDA;
   }
   return KIA_OK;
@@ -213,8 +213,8 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
     if (rc) return rc;
     if (!p.softmax && p.grad == KIA_GRAD_PROJECT) {
       // the key pass already folded the projection shift into dK
-      dim3 g(B * H, D / 32);
-      bwd_project_scan_kernel<D><<<g, 32 * kScanGroups, 0, s>>>(Q, Kt, wk, dQ, dK, p, T, 0);
+      dim3 g(B * H, D / 32, (T + kScanRows - 1) / kScanRows);
+      bwd_project_scan_kernel<D><<<g, 32 * kScanWarps, 0, s>>>(Q, Kt, wk, dQ, dK, p, T, 0);
       if (launch_status()) return KIA_ERR_CUDA;
     }
     prof_mark(6, s);
