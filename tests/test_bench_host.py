@@ -62,3 +62,24 @@ def test_weak_scaling_aggregation_two_ranks_gloo():
     for rank, t, v in res:
         assert t == pytest.approx(15.0)
         assert v == pytest.approx(2 * 1e12 / 15e-3 / 1e12)
+
+
+def test_workload_overrides_and_flop_counts():
+    """The gradient-mode override, the operator workloads and the algorithmic
+    flop count: 8U, 9U with Prob-STE, 7U for exact softmax (one S in the
+    forward), 8U for the rounded-exponential baselines (they need the final
+    row maximum, so two passes over S)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from quantized_softmax_attention_b200 import workloads as W
+    w = bench.workload("gpt2_fwm", "projection")
+    assert w.grad == W.GRAD_PROJECT and w.cal == W.CAL_FWM
+    assert bench.config_dict(w, 1)["grad"] == "projection"
+    U = bench.gemm_units(w)
+    assert bench.algorithmic_flops(w) == 9 * U
+    assert bench.algorithmic_flops(bench.workload("gpt2_heavy")) == 8 * U
+    assert bench.algorithmic_flops(bench.workload("gpt2_bf16exp")) == 8 * U
+    sm = W.Workload(**{**w.__dict__, "operator": 1})
+    assert bench.algorithmic_flops(sm) == 7 * U
+    assert bench.config_dict(bench.workload("gpt2_fp8exp"), 1)["operator"].endswith("FP8-rounded exp")
+    assert bench.workload("gpt2_fixed").cal == W.CAL_FIXED
