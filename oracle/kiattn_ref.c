@@ -24,16 +24,22 @@
  *     Prob-STE share the hard forward and the LERP scalar derivatives but use
  *     different normalisation points.
  *
- * Readings of points the pages leave open (each is also listed in the design doc):
+ * Readings of points the pages leave open:
  *   grid nodes m - k h, k = 0..K (G_k = e^{-k h}); Nearest picks the nearer
  *   node, ties (t = 1/2) to the larger u; interval index k = min(floor u,
  *   K-1); FWM window u <= K for LERP and Nearest alike; degenerate MinMax rows
  *   (span < 1e-12) get uniform P and dS = (dP - mean dP)/|J|; arg-extrema take
  *   the lowest index; max-only keeps the live row max (n frozen), min-only
  *   keeps the live row min (m frozen); the projection subtracts the mean over
- *   all keys of the row; the caller pre-scales Q (no 1/sqrt(d) inside).
+ *   all keys of the row; the caller pre-scales Q (no 1/sqrt(d) inside); the
+ *   untruncated fixed step (Appendix D.4) is FWM's grid with no window, the
+ *   node index unbounded; the reduced-precision exponential baselines
+ *   (Appendix D.5) round e^{s-m} (as fp32) to bfloat16 or FP8 E4M3,
+ *   nearest-even, and pass straight through the rounding with the row
+ *   maximum held fixed.
  *
- * Parity pins (tests/test_oracle_pins.py, tests/test_oracle_autograd.py):
+ * Parity pins (tests/test_oracle_pins.py, tests/test_oracle_autograd.py,
+ * tests/test_oracle_reduced_exp.py, tests/test_oracle_geometry.py):
  * central finite differences, frozen-statistic finite differences, zero row
  * sums, bitwise-equal forwards across gradient modes, STE coincidence on grid
  * nodes, the softmax limit and the chord bound, the K = 1 closed form, brute
