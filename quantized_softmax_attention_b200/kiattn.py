@@ -126,6 +126,37 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(fn, name, t, numel=None, nbytes=None, dtype=None):
+    """Size and type checks of one argument, before any pointer is passed:
+    the library cannot see buffer sizes, so a short buffer is caught here."""
+    if t is None:
+        return
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{fn}: {name} must be {dtype}, got {t.dtype}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{fn}: {name} has {t.numel()} elements, needs {numel}")
+    if nbytes is not None and t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{fn}: {name} holds {t.numel() * t.element_size()} bytes, needs {nbytes}")
+
+
+def _need_qkv(fn, Q, rest, cfg, stats=None, workspace=None, dS=None):
+    f32 = torch.float32
+    if Q.dim() != 4:
+        raise ValueError(f"{fn}: Q must be [B, H, T, d], got {tuple(Q.shape)}")
+    B, H, T, d = Q.shape
+    _need(fn, "Q", Q, dtype=f32)
+    for name, t in rest.items():
+        _need(fn, name, t, numel=Q.numel(), dtype=f32)
+    if stats is not None:
+        sb = kiattn_stats_bytes(B, H, T, d, cfg)
+        _need(fn, "stats", stats, nbytes=sb if sb else None)
+    if workspace is not None:
+        wb = kiattn_workspace_bytes(B, H, T, d, cfg)
+        _need(fn, "workspace", workspace, nbytes=wb if wb else None)
+    _need(fn, "dS_dbg", dS, numel=B * H * T * T, dtype=f32)
+    return B, H, T, d
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -146,14 +177,16 @@ def kiattn_workspace_bytes(B, H, T, d, cfg: Config) -> int:
 
 
 def kiattn_fwd(Q, K, V, O, stats, cfg: Config, stream=None):
-    B, H, T, d = Q.shape
+    B, H, T, d = _need_qkv("kiattn_fwd", Q, {"K": K, "V": V, "O": O}, cfg, stats=stats)
     _check("kiattn_fwd", _lib.kiattn_fwd(_p(Q), _p(K), _p(V), _p(O), _p(stats), B, H, T, d,
                                          ctypes.byref(cfg.c()), _stream(stream)))
 
 
 def kiattn_bwd(Q, K, V, O, dO, stats, dQ, dK, dV, workspace, cfg: Config, dS_dbg=None,
                stream=None):
-    B, H, T, d = Q.shape
+    B, H, T, d = _need_qkv("kiattn_bwd", Q, {"K": K, "V": V, "O": O, "dO": dO, "dQ": dQ,
+                                             "dK": dK, "dV": dV}, cfg, stats=stats,
+                           workspace=workspace, dS=dS_dbg)
     _check("kiattn_bwd", _lib.kiattn_bwd(_p(Q), _p(K), _p(V), _p(O), _p(dO), _p(stats), _p(dQ),
                                          _p(dK), _p(dV), _p(dS_dbg), B, H, T, d,
                                          ctypes.byref(cfg.c()), _p(workspace), _stream(stream)))
@@ -164,6 +197,9 @@ def kiattn_bwd_noalloc(Q, K, V, O, dO, stats, dQ, dK, dV, cfg: Config, dS_dbg=No
     """Backward with the library's own fixed scratch (no workspace argument),
     for callers that cannot allocate device memory; B*H*T <= NOALLOC_MAX_ROWS."""
     B, H, T, d = Q.shape
+    if B * H * T <= NOALLOC_MAX_ROWS:   # beyond it the library refuses before any access
+        _need_qkv("kiattn_bwd_noalloc", Q, {"K": K, "V": V, "O": O, "dO": dO, "dQ": dQ, "dK": dK,
+                                            "dV": dV}, cfg, stats=stats, dS=dS_dbg)
     _check("kiattn_bwd_noalloc",
            _lib.kiattn_bwd_noalloc(_p(Q), _p(K), _p(V), _p(O), _p(dO), _p(stats), _p(dQ), _p(dK),
                                    _p(dV), _p(dS_dbg), B, H, T, d, ctypes.byref(cfg.c()),
@@ -172,7 +208,16 @@ def kiattn_bwd_noalloc(Q, K, V, O, dO, stats, dQ, dK, dV, cfg: Config, dS_dbg=No
 
 def kiattn_weights_from_S(S, row_len, cfg: Config, w, bin=None, t=None, row_m=None, row_n=None,
                           stream=None):
+    fn, f32, i32 = "kiattn_weights_from_S", torch.float32, torch.int32
+    if S.dim() != 2:
+        raise ValueError(f"{fn}: S must be [rows, cols], got {tuple(S.shape)}")
     rows, cols = S.shape
+    _need(fn, "S", S, dtype=f32)
+    _need(fn, "row_len", row_len, numel=rows, dtype=i32)
+    for name, x, dt in (("w", w, f32), ("bin", bin, i32), ("t", t, f32)):
+        _need(fn, name, x, numel=rows * cols, dtype=dt)
+    _need(fn, "row_m", row_m, numel=rows, dtype=f32)
+    _need(fn, "row_n", row_n, numel=rows, dtype=f32)
     _check("kiattn_weights_from_S",
            _lib.kiattn_weights_from_S(_p(S), rows, cols, _p(row_len), ctypes.byref(cfg.c()), _p(w),
                                       _p(bin), _p(t), _p(row_m), _p(row_n), _stream(stream)))
@@ -182,7 +227,14 @@ def kiattn_grad_decomposition(dS, workspace, out, cfg: Config, stream=None):
     """Per-row ||dS_i||^2 and the squared norms of the maximum- and
     minimum-side calibration terms (out: device fp64 [B, H, T, 3]) from the
     dS_dbg and workspace of one kiattn_bwd call with the same cfg."""
+    fn = "kiattn_grad_decomposition"
+    if dS.dim() != 4 or dS.shape[2] != dS.shape[3]:
+        raise ValueError(f"{fn}: dS must be [B, H, T, T], got {tuple(dS.shape)}")
     B, H, T, _ = dS.shape
+    _need(fn, "dS", dS, dtype=torch.float32)
+    wb = kiattn_workspace_bytes(B, H, T, 64, cfg)
+    _need(fn, "workspace", workspace, nbytes=wb if wb else None)
+    _need(fn, "out", out, numel=B * H * T * 3, dtype=torch.float64)
     _check("kiattn_grad_decomposition",
            _lib.kiattn_grad_decomposition(_p(dS), _p(workspace), B, H, T, ctypes.byref(cfg.c()),
                                           _p(out), _stream(stream)))
@@ -196,15 +248,22 @@ GEO_FIELD_COUNT = len(GEO_FIELDS)
 def kiattn_geometry(S, out, cfg: Config, Q=None, stream=None):
     """Per-row geometry probe of scores S [B, H, T, T] against cfg's grid;
     out: device fp32 [B, H, T, 8] in the order of GEO_FIELDS."""
+    fn = "kiattn_geometry"
+    if S.dim() != 4 or S.shape[2] != S.shape[3]:
+        raise ValueError(f"{fn}: S must be [B, H, T, T], got {tuple(S.shape)}")
     B, H, T, _ = S.shape
     d = Q.shape[-1] if Q is not None else 0
+    _need(fn, "S", S, dtype=torch.float32)
+    _need(fn, "out", out, numel=B * H * T * GEO_FIELD_COUNT, dtype=torch.float32)
+    _need(fn, "Q", Q, numel=B * H * T * d, dtype=torch.float32)
     _check("kiattn_geometry", _lib.kiattn_geometry(_p(S), _p(Q), B, H, T, d,
                                                    ctypes.byref(cfg.c()), _p(out),
                                                    _stream(stream)))
 
 
 def kiattn_scores(Q, K, S, cfg: Config, stream=None):
-    B, H, T, d = Q.shape
+    B, H, T, d = _need_qkv("kiattn_scores", Q, {"K": K}, cfg)
+    _need("kiattn_scores", "S", S, numel=B * H * T * T, dtype=torch.float32)
     _check("kiattn_scores", _lib.kiattn_scores(_p(Q), _p(K), _p(S), B, H, T, d,
                                                ctypes.byref(cfg.c()), _stream(stream)))
 

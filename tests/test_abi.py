@@ -97,3 +97,44 @@ def test_product_path_does_not_import_the_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "kiattn_ref" not in txt, f
+
+
+def test_binding_checks_buffer_sizes_before_passing_pointers():
+    """The library cannot see buffer sizes, so the binding checks them (and
+    the dtypes) before any pointer is formed; correctly sized host tensors
+    pass the checks and are then refused as not being CUDA tensors."""
+    import torch
+    K = pytest.importorskip("quantized_softmax_attention_b200.kiattn")
+    cfg = K.Config()
+    B, H, T, d = 1, 2, 128, 64
+    x = torch.zeros((B, H, T, d))
+    sb = K.kiattn_stats_bytes(B, H, T, d, cfg)
+    wb = K.kiattn_workspace_bytes(B, H, T, d, cfg)
+    st, wk = torch.zeros(sb, dtype=torch.uint8), torch.zeros(wb, dtype=torch.uint8)
+
+    def refused(fn, *a, **kw):
+        with pytest.raises(ValueError) as e:
+            fn(*a, **kw)
+        return str(e.value)
+
+    assert "CUDA" in refused(K.kiattn_fwd, x, x, x, x, st, cfg)
+    assert "needs" in refused(K.kiattn_fwd, x, x[:, :1], x, x, st, cfg)
+    assert "bytes" in refused(K.kiattn_fwd, x, x, x, x, st[:-1], cfg)
+    assert "float32" in refused(K.kiattn_fwd, x, x.double(), x, x, st, cfg)
+    assert "CUDA" in refused(K.kiattn_bwd, x, x, x, x, x, st, x, x, x, wk, cfg)
+    assert "bytes" in refused(K.kiattn_bwd, x, x, x, x, x, st, x, x, x, wk[:8], cfg)
+    assert "needs" in refused(K.kiattn_bwd, x, x, x, x, x, st, x, x, x, wk, cfg,
+                              dS_dbg=torch.zeros((B, H, T, T - 1)))
+    S = torch.zeros((B, H, T, T))
+    assert "CUDA" in refused(K.kiattn_scores, x, x, S, cfg)
+    assert "needs" in refused(K.kiattn_scores, x, x, S[..., :-1], cfg)
+    assert "CUDA" in refused(K.kiattn_geometry, S, torch.zeros((B, H, T, 8)), cfg, Q=x)
+    assert "needs" in refused(K.kiattn_geometry, S, torch.zeros((B, H, T, 7)), cfg)
+    assert "CUDA" in refused(K.kiattn_grad_decomposition, S, wk,
+                             torch.zeros((B, H, T, 3), dtype=torch.float64), cfg)
+    assert "float64" in refused(K.kiattn_grad_decomposition, S, wk, torch.zeros((B, H, T, 3)), cfg)
+    rows, cols = 4, 9
+    Sw = torch.zeros((rows, cols))
+    L = torch.full((rows,), cols, dtype=torch.int32)
+    assert "CUDA" in refused(K.kiattn_weights_from_S, Sw, L, cfg, torch.zeros((rows, cols)))
+    assert "int32" in refused(K.kiattn_weights_from_S, Sw, L.long(), cfg, torch.zeros((rows, cols)))

@@ -91,8 +91,10 @@ def test_geometry_rejects_bad_arguments():
     out = torch.zeros((1, 1, 8, 8), device="cuda")
     with pytest.raises(RuntimeError):
         K.kiattn_geometry(S, out, K.Config(op=K.OP_SOFTMAX))
-    with pytest.raises(RuntimeError):
+    with pytest.raises((RuntimeError, ValueError)):
         K.kiattn_geometry(S[:, :, :0], out, K.Config())
+    with pytest.raises(ValueError):   # the binding checks the output's size
+        K.kiattn_geometry(S, out[..., :4].contiguous(), K.Config())
 
 
 def test_geometry_full_size_sampled_rows():

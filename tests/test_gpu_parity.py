@@ -321,5 +321,7 @@ def test_grad_decomposition_rejects_bad_arguments():
     bufs = K.Buffers(1, 1, 128, 64, cfg)
     with pytest.raises(RuntimeError):
         K.kiattn_grad_decomposition(dS, None, out, cfg)
-    with pytest.raises(RuntimeError):
+    with pytest.raises((RuntimeError, ValueError)):
         K.kiattn_grad_decomposition(dS[:, :, :0], bufs.work, out, cfg)
+    with pytest.raises(ValueError):   # the binding checks the output's type
+        K.kiattn_grad_decomposition(dS, bufs.work, out.float(), cfg)
