@@ -138,3 +138,30 @@ def test_binding_checks_buffer_sizes_before_passing_pointers():
     L = torch.full((rows,), cols, dtype=torch.int32)
     assert "CUDA" in refused(K.kiattn_weights_from_S, Sw, L, cfg, torch.zeros((rows, cols)))
     assert "int32" in refused(K.kiattn_weights_from_S, Sw, L.long(), cfg, torch.zeros((rows, cols)))
+
+
+def test_fixed_step_and_rounded_exp_configs(K):
+    """The untruncated fixed step is accepted while its grid's extent,
+    ceil(104.5 K / tau) nodes, fits the library's 400-node limit (tau = 6:
+    K <= 22), and keeps its FWM-sized stats; the rounded-exponential softmax
+    operators are accepted and sized like softmax; unknown calibration or
+    operator codes are invalid arguments."""
+    B, H, T, d = 1, 2, 256, 64
+    fixed = K.Config(K=4, cal=K.CAL_FIXED, tau=6.0)
+    fwm = K.Config(K=4, cal=K.CAL_FWM, tau=6.0)
+    assert K.kiattn_stats_bytes(B, H, T, d, fixed) > 0
+    assert K.kiattn_stats_bytes(B, H, T, d, fixed.replace(K=22)) > 0
+    assert K.kiattn_stats_bytes(B, H, T, d, fixed.replace(K=23)) == 0
+    assert K.kiattn_stats_bytes(B, H, T, d, fixed.replace(K=64, tau=60.0)) > 0
+    # FWM keeps one grid; the fixed step's grid has ~70 nodes instead of 5
+    assert 0 < K.kiattn_stats_bytes(B, H, T, d, fixed) - K.kiattn_stats_bytes(B, H, T, d, fwm) < 4096
+    sm = K.kiattn_stats_bytes(B, H, T, d, K.Config(op=K.OP_SOFTMAX))
+    for op in (K.OP_SOFTMAX_BF16EXP, K.OP_SOFTMAX_FP8EXP):
+        assert K.kiattn_stats_bytes(B, H, T, d, K.Config(op=op)) == sm
+    assert K.kiattn_stats_bytes(B, H, T, d, K.Config(op=4)) == 0
+    assert K.kiattn_stats_bytes(B, H, T, d, K.Config(cal=3)) == 0
+    assert K.kiattn_stats_bytes(B, H, T, d, fixed.replace(tau=0.0)) == 0
+    lib = K.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    c = fixed.replace(K=23).c()
+    assert lib.kiattn_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, ctypes.byref(c), None) == -2
