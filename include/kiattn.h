@@ -195,8 +195,8 @@ int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T
  * dS: the dS_dbg [B,H,T,T] written by kiattn_bwd; workspace: the workspace of
  * that same kiattn_bwd call (it holds g_m, g_n per row); cfg as in that call;
  * out: device fp64 [B*H*T*3], caller-owned.  Sums run in fp64 (groups of
- * four squares in fp32 first).  Nothing is
- * written when the kiattn_bwd call rejected its stats (workspace status set).
+ * four squares in fp32 first).  Nothing is written when the kiattn_bwd call
+ * rejected its stats (workspace status set).
  * Errors: INVALID_ARG (null pointer, B, H or T < 1), UNSUPPORTED (shape
  * beyond the operator's limits), CUDA (launch failure). */
 int kiattn_grad_decomposition(const float* dS, const void* workspace, int B, int H, int T,
@@ -207,7 +207,7 @@ int kiattn_grad_decomposition(const float* dS, const void* workspace, int B, int
  * records to describe learned score geometry.  Fields of out[row * 8 + f]:
  *   KIA_GEO_SPAN         m - n over the row's visible keys
  *   KIA_GEO_H            native interval width h (MinMax span / K, 0 for a
- *                        degenerate row; FWM tau / K)
+ *                        degenerate row; FWM and fixed step tau / K)
  *   KIA_GEO_QNORM        ||q_i||_2 (0 when Q is NULL)
  *   KIA_GEO_ENT_SOFTMAX  entropy (nats) of softmax(s_i)
  *   KIA_GEO_ENT_OP       entropy of the operator's forward probabilities
