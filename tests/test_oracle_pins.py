@@ -339,6 +339,22 @@ def test_hand_worked_fwm_row():
     np.testing.assert_allclose(o["P"][0], wn / wn.sum(), rtol=1e-15)
 
 
+def test_hand_worked_fixed_step_row():
+    """The same row under the untruncated fixed step (Appendix D.4): the key
+    FWM drops (s = -10, u = 6 2/3) keeps the LERP weight between nodes 6 and
+    7, (1/3) e^-9 + (2/3) e^-10.5, and Nearest rounds it to node 7; the
+    in-window keys keep FWM's weights."""
+    S = np.array([[0.0, -1.5, -3.0, -0.75, -10.0]])
+    e1, e2 = math.exp(-1.5), math.exp(-3.0)
+    tail_l = math.exp(-9.0) / 3 + 2 * math.exp(-10.5) / 3
+    wl = np.array([1.0, e1, e2, (1 + e1) / 2, tail_l])
+    wn = np.array([1.0, e1, e2, e1, math.exp(-10.5)])
+    o = ref.rows(S, [5], ref.RefConfig(K=4, cal=ref.CAL_FIXED, tau=6.0, rec=ref.REC_LERP))
+    np.testing.assert_allclose(o["P"][0], wl / wl.sum(), rtol=1e-14)
+    o = ref.rows(S, [5], ref.RefConfig(K=4, cal=ref.CAL_FIXED, tau=6.0, rec=ref.REC_NEAREST))
+    np.testing.assert_allclose(o["P"][0], wn / wn.sum(), rtol=1e-14)
+
+
 def _linear_scan_forward(s, K, cal, tau, rec):
     """Second forward: find the bracketing nodes by scanning node scores
     m - k h from the top, no floor()."""
