@@ -147,14 +147,21 @@ int kiattn_bwd(const float* Q, const float* Kt, const float* V, const float* O, 
  *   - Capacity: B*H*T <= KIA_NOALLOC_MAX_ROWS rows; larger calls return
  *     KIA_ERR_CAPACITY and launch nothing.  Every GPU that loads the
  *     library holds the scratch (about 28 MiB) until the process exits.
- *   - The first call on a device, with that device current, looks up the
- *     scratch's device address; make that first call before any stream
- *     capture.
+ *   - The first call in a CUDA context (normally the device's primary
+ *     context, made current by cudaSetDevice) looks up the scratch's device
+ *     address in that context; make that first call before any stream
+ *     capture.  The address is kept per context, so after cudaDeviceReset,
+ *     or under another context of the same device, the next call looks it up
+ *     again (again outside capture).
  *   - It calls no cudaMalloc / cudaFree.  Each call clears the scratch
  *     fields that must start at zero; the scratch keeps the last call's
  *     contents otherwise.
  *   - All calls share one scratch per device: calls that overlap on the GPU
- *     (several streams, several host threads) race; serialise them. */
+ *     (several streams, several host threads) race; serialise them.
+ *   - The scratch is the library's own, so the caller has no handle to the
+ *     per-row calibration coefficients the backward leaves in it:
+ *     kiattn_grad_decomposition needs a kiattn_bwd call with a workspace of
+ *     the caller's. */
 #define KIA_NOALLOC_MAX_ROWS (1 << 20)
 int kiattn_bwd_noalloc(const float* Q, const float* Kt, const float* V, const float* O,
                        const float* dO, const void* stats, float* dQ, float* dK, float* dV,
@@ -242,6 +249,21 @@ int kiattn_geometry(const float* S, const float* Q, int B, int H, int T, int d,
  * backward kernels then skip their work), 0 otherwise.  Synchronous: it
  * copies the word from the device (and clears it when reset != 0). */
 int kiattn_device_error(int reset);
+
+/* Test hook for the bounded device-side waits (failure handling without a
+ * GPU fault; no counterpart in the paper).  Every wait inside the tensor-core
+ * kernels gives up after a time limit, raises KIA_ERR_TIMEOUT in the error
+ * word read by kiattn_device_error(), lets the copies and MMAs already in
+ * flight land, frees its tensor memory and returns, so the context stays
+ * usable.  what = 1 makes every following kiattn_fwd on the tensor-core
+ * path withhold one operand copy -- the first CTA never issues its first Q
+ * tile, so nothing is in flight for it and the waits on it run out; the
+ * outputs of that call are then undefined.  wait_limit_ns > 0 sets the limit
+ * of every wait (default 2 s) so that a test does not sit out the default.
+ * kiattn_debug_bounded_wait(0, 0) restores the defaults.  Synchronous (it
+ * writes the limit to the device); not thread-safe; meant for tests.
+ * Errors: INVALID_ARG (what not 0 or 1), CUDA. */
+int kiattn_debug_bounded_wait(int what, unsigned long long wait_limit_ns);
 
 /* Phase timing for profiling.  kiattn_profile_enable(1) makes kiattn_fwd
  * and kiattn_bwd record CUDA events on their stream around each internal

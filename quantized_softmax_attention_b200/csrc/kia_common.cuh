@@ -40,6 +40,8 @@ struct OpParams {
   int fixed_step; // untruncated fixed step (Appendix D.4), run as FWM with K = the grid's
                   // extent, the first node count at which G_k underflows to zero in fp32
   int exp_round;  // softmax only: 0 exact e^{s-m}; 1 rounded to bf16; 2 rounded to FP8 E4M3
+  int withhold;   // failure-handling test hook (forward only): 1 = the first CTA never
+                  // issues the first Q tile, so the waits on it run out; 0 normally
 };
 
 // Reduced-precision exponential baselines (Appendix D.5): the softmax
@@ -247,13 +249,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait.  Gives up after ~kWaitLimitNs or as soon as another thread
-// of the CTA has raised *abort; on giving up it raises *abort and the
+// Bounded wait.  Gives up after ~g_kia_wait_limit_ns or as soon as another
+// thread of the CTA has raised *abort; on giving up it raises *abort and the
 // library-wide error word, and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Library-wide device error word (the library is a single translation unit).
 __device__ int g_kia_device_error;
+// Limit of every bounded wait; the failure-handling test hook shortens it.
+__device__ unsigned long long g_kia_wait_limit_ns = kWaitLimitNs;
 
 // try_wait with a suspend-time hint: the thread sleeps in hardware until the
 // phase completes (or about hint_ns pass) instead of polling shared memory,
@@ -278,7 +282,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > g_kia_wait_limit_ns) {
       *abort = 1;
       atomicExch(&g_kia_device_error, KIA_ERR_TIMEOUT);
       return false;
@@ -288,8 +292,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Watchdog of a polling loop that serves several barriers: call idle() on
 // every pass that made no progress and progress() on every pass that did.
-// Gives up like mbar_wait: after ~kWaitLimitNs without progress, or at once
-// when *abort is raised.
+// Gives up like mbar_wait: after ~g_kia_wait_limit_ns without progress, or at
+// once when *abort is raised.
 struct PollGuard {
   uint64_t t0;
   uint32_t idle_passes;
@@ -300,7 +304,7 @@ struct PollGuard {
     __nanosleep(100);   // back off instead of hammering shared memory
     if ((++idle_passes & 15u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > g_kia_wait_limit_ns) {
         *abort = 1;
         atomicExch(&g_kia_device_error, KIA_ERR_TIMEOUT);
         return false;

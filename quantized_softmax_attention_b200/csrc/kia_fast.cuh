@@ -116,7 +116,7 @@ __device__ __forceinline__ void fwd_weights2(const G& grid, float m, float rh, f
                                              float Km1f, float s0, float s1, float2& wf2,
                                              float2& wl2) {
   if constexpr (V::SOFTMAX) {
-    wf2 = make_float2(round_exp<V::EXPR>(__expf(s0 - m)), round_exp<V::EXPR>(__expf(s1 - m)));
+    wf2 = make_float2(round_exp<V::EXPR>(expf(s0 - m)), round_exp<V::EXPR>(expf(s1 - m)));
     wl2 = wf2;
   } else {
     float2 u = mul2(sub2(make_float2(m, m), make_float2(s0, s1)), make_float2(rh, rh));
@@ -147,14 +147,18 @@ __device__ __forceinline__ void fwd_weights2(const G& grid, float m, float rh, f
 }
 
 // Forward weights: wf (forward probabilities' numerator) and wl (LERP
-// weight, used by Prob-STE's normalisation point).  CLAMP0 for tiles that
-// hold masked scores (which may lie above the row max).
+// weight, used by Prob-STE's normalisation point).  Returns the grid
+// position the weights came from (zero for softmax), so that the weight-stage
+// test entry point reports the bins and t of this very code.  CLAMP0 for
+// scores that may lie above the row max (recomputed by another contraction
+// order, or masked).
 template <class V, bool CLAMP0, class G>
-__device__ __forceinline__ void fwd_weights(const G& grid, float m, float rh, float Kf,
-                                            float Km1f, float s, float& wf, float& wl) {
+__device__ __forceinline__ Pos fwd_weights(const G& grid, float m, float rh, float Kf,
+                                           float Km1f, float s, float& wf, float& wl) {
   if constexpr (V::SOFTMAX) {
-    wf = round_exp<V::EXPR>(__expf(s - m));
+    wf = round_exp<V::EXPR>(expf(s - m));
     wl = wf;
+    return Pos{0.0f, 0.0f, 0.0f, 0};
   } else {
     const Pos p = grid_pos<V, CLAMP0>(m, rh, Kf, Km1f, s);
     const float2 g = grid.pair(p.k);
@@ -171,6 +175,7 @@ __device__ __forceinline__ void fwd_weights(const G& grid, float m, float rh, fl
       wf = tail ? 0.0f : wf;
       wl = tail ? 0.0f : wl;
     }
+    return p;
   }
 }
 
@@ -185,7 +190,7 @@ __device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, flo
   if constexpr (V::SOFTMAX) {
     // straight through the rounding of the reduced-precision baselines:
     // the slope is the unrounded e^{s-m}
-    return __expf(s - m) * dw;
+    return expf(s - m) * dw;
   } else {
     const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
     float2 g = grid.pair(p.k);
@@ -219,7 +224,7 @@ __device__ __forceinline__ void kv_elem(const G& grid, float m, float rh, float 
                                         float Kf, float Km1f, float s, float dw, float& P,
                                         float& dS) {
   if constexpr (V::SOFTMAX) {
-    const float w = __expf(s - m);
+    const float w = expf(s - m);
     P = round_exp<V::EXPR>(w) * rWf;   // the forward's (rounded) probability
     dS = w * dw;                       // straight through the rounding
   } else {

@@ -162,9 +162,15 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int qt = item_qt(it), bh = item_bh(it), nkt = item_nkt(it);
         // Q of this item once the previous item's S MMAs are done with it
         if (!mbar_wait(&bar.q_empty, (n & 1) ^ 1, abort)) { failed = true; break; }
-        mbar_arrive_expect_tx(&bar.q_full, Cfg::kTileBytes);
-        for (int b = 0; b < D / 32; ++b)
-          tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.q_full, b * 32, qt * KIA_TILE, bh);
+        // failure-handling test hook: the first CTA withholds its first Q tile
+        // (neither the expected-bytes arrival nor the copy is issued, so
+        // nothing is in flight for it) and the waits on it run out
+        const bool withhold = p.withhold == 1 && blockIdx.x == 0 && n == 0;
+        if (!withhold) {
+          mbar_arrive_expect_tx(&bar.q_full, Cfg::kTileBytes);
+          for (int b = 0; b < D / 32; ++b)
+            tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.q_full, b * 32, qt * KIA_TILE, bh);
+        }
         for (int sweep = 0; sweep < 2 && !failed; ++sweep) {
           for (int j = 0; j < nkt; ++j) {
             {
@@ -433,8 +439,11 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (!edge) {
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
+                // clamped like the edge tiles: these scores come from other
+                // MMAs than the ones the row max was taken from, and nothing
+                // makes the two bit-identical
                 float wf, wl;
-                fwd_weights<V, false>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
+                fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
                 W += wf;
                 w16[i] = wf;
                 if constexpr (PROB) {

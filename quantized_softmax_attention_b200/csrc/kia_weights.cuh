@@ -1,28 +1,44 @@
 // The fp32 weight stage on given scores (kiattn_weights_from_S): one warp
-// per row.  It runs exactly the per-row calibration and per-element grid
-// arithmetic of the fused kernels (kia_common.cuh), so a bit-exact match
-// against the oracle's fp32 definition here pins the fused kernels' weight
-// arithmetic too.
+// per row.  It runs the tensor-core forward's own weight code on the dumped
+// scores: the per-row calibration (row_calibration), the grid tables in the
+// forward's form (one pair table (G_k, G_{k+1}) per CTA for FWM and the fixed
+// step, one table per row for MinMax, both from grid_value), and the element
+// function fwd_weights<V, true> that the forward's sweep 2 calls on every
+// unit, compiled for the same operator variant V; keys past the row's last
+// visible one go through it too and are zeroed afterwards, as the forward's
+// masked keys are.  The bins and t written out are the grid position
+// fwd_weights returns, so a bit-exact match against the oracle's fp32
+// definition pins the forward's weights, bins and t themselves.
 #pragma once
-#include "kia_common.cuh"
+#include "kia_fast.cuh"
 
 namespace kia {
 
 constexpr int kWeightsWarps = 4;
 
+template <class V>
 __global__ void __launch_bounds__(32 * kWeightsWarps)
 weights_from_S_kernel(const float* __restrict__ S, int rows, int cols,
                       const int* __restrict__ row_len, OpParams p, float* __restrict__ w,
                       int* __restrict__ bin, float* __restrict__ tout, float* __restrict__ row_m,
                       float* __restrict__ row_n) {
-  __shared__ float sG[kWeightsWarps][KIA_MAX_KCAP + 1];
+  // FWM and the fixed step: the forward's per-CTA pairs (G_k, G_{k+1})
+  __shared__ float2 sPair[V::FWM ? KIA_MAX_KCAP : 1];
+  // MinMax: one grid per row, as the forward's per-row table
+  __shared__ float sTab[kWeightsWarps][V::MINMAX ? KIA_MAX_K + 1 : 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if constexpr (V::FWM) {
+    for (int k = (int)threadIdx.x; k < p.K; k += (int)blockDim.x)
+      sPair[k] = make_float2(grid_value(k, p.fwm_h), grid_value(k + 1, p.fwm_h));
+    __syncthreads();
+  }
   const int row = blockIdx.x * kWeightsWarps + warp;
   if (row >= rows) return;
   const float* s = S + (size_t)row * cols;
   int L = row_len[row];
   L = L < 1 ? 1 : (L > cols ? cols : L);
-  // row extrema (section 3: calibration statistics)
+  // row extrema (section 3: calibration statistics); max and min are exact
+  // in any order
   float m = -INFINITY, n = INFINITY;
   for (int j = lane; j < L; j += 32) {
     const float x = s[j];
@@ -38,37 +54,33 @@ weights_from_S_kernel(const float* __restrict__ S, int rows, int cols,
     if (row_m) row_m[row] = m;
     if (row_n) row_n[row] = n;
   }
-  const RowCal c = row_calibration(p, m, n);
-  const bool degen = (p.cal == KIA_CAL_MINMAX) && c.h == 0.0f;
-  if (!degen) {
-    for (int k = lane; k <= p.K; k += 32) sG[warp][k] = grid_value(k, c.h);
+  if constexpr (!V::MINMAX) n = m;   // as the forward: FWM does not use the row minimum
+  const RowCal rc = row_calibration(p, m, n);
+  if constexpr (V::MINMAX) {
+    // the forward's per-row grid: all ones on a degenerate row (rh = 0 then
+    // puts every key on node 0, weight 1)
+    const bool degen = rc.h == 0.0f;
+    for (int k = lane; k <= p.K; k += 32) sTab[warp][k] = degen ? 1.0f : grid_value(k, rc.h);
+    __syncwarp();
   }
-  __syncwarp();
-  for (int j = lane; j < cols; j += 32) {
-    float wj = 0.0f, tj = 0.0f;
-    int bj = -1;
-    if (j < L) {
-      if (degen) {
-        wj = 1.0f;
-        bj = 0;
-      } else {
-        const GridPos g = grid_position(p, c, s[j]);
-        if (!g.tail) {
-          if (p.rec == KIA_REC_LERP) {
-            wj = lerp_weight(g.t, sG[warp][g.k], sG[warp][g.k + 1]);
-            bj = g.k;
-          } else {
-            bj = nearest_node(g);
-            wj = sG[warp][bj];
-          }
-          tj = g.t;
-        }
-      }
+  const float Kf = p.Kf, Km1f = (float)(p.K - 1);
+  auto run = [&](const auto& grid) {
+    for (int j = lane; j < cols; j += 32) {
+      const float x = s[j];
+      const bool vis = j < L;
+      float wf, wl;
+      const Pos pos = fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, x, wf, wl);
+      const bool tail = V::FWM && pos.u > Kf;
+      const bool live = vis && !tail;
+      int b = pos.k;
+      if constexpr (V::NEAREST) b += pos.t >= 0.5f ? 1 : 0;
+      w[(size_t)row * cols + j] = vis ? wf : 0.0f;
+      if (bin) bin[(size_t)row * cols + j] = live ? b : -1;
+      if (tout) tout[(size_t)row * cols + j] = live ? pos.t : 0.0f;
     }
-    w[(size_t)row * cols + j] = wj;
-    if (bin) bin[(size_t)row * cols + j] = bj;
-    if (tout) tout[(size_t)row * cols + j] = tj;
-  }
+  };
+  if constexpr (V::MINMAX) run(GridF{sTab[warp], 1});
+  else run(GridP{sPair});
 }
 
 }  // namespace kia

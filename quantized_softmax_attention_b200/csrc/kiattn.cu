@@ -38,6 +38,9 @@ void prof_mark(int i, cudaStream_t s) {
   if (g_prof_on) cudaEventRecord(g_prof_ev[i], s);
 }
 
+// failure-handling test hook (kiattn_debug_bounded_wait)
+int g_withhold = 0;
+
 // Extent of the untruncated fixed-step grid (Appendix D.4): the node count
 // Kc at which G_Kc = RN32(e^{-Kc h}) is zero (every Kc h >= 104.5 nats, since
 // e^{-103.98} is already below half the least fp32 subnormal), so that keys
@@ -92,6 +95,7 @@ OpParams make_params(const kia_config* cfg) {
   p.fwm_rh = (cfg->cal != KIA_CAL_MINMAX) ? p.Kf / cfg->tau : 0.0f;
   p.tf32_ops = 0;
   p.fixed_step = 0;
+  p.withhold = g_withhold;
   if (cfg->cal == KIA_CAL_FIXED) {
     // the fixed-step operator is FWM's grid (h = tau / K, anchored at the row
     // maximum) with its window widened to the grid's full extent
@@ -238,13 +242,72 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
 
 // Scratch of kiattn_bwd_noalloc: the backward's workspace for up to
 // KIA_NOALLOC_MAX_ROWS rows, declared by the library so that the caller
-// allocates nothing.  Host code only ever uses its device address, looked up
-// once per device.
+// allocates nothing.  Host code only ever uses its device address.  That
+// address belongs to the CUDA context the module was loaded into, so it is
+// looked up once per context (keyed by the driver's context id, which is
+// never reused within a process): a device reset or a caller's own context
+// on the same device gets its own lookup instead of a stale address.
 constexpr size_t kNoallocScratchBytes = work_bytes_c(KIA_NOALLOC_MAX_ROWS);
 static __device__ __align__(256) unsigned char g_kia_noalloc_scratch[kNoallocScratchBytes];
-constexpr int kMaxDevices = 64;
-void* g_noalloc_addr[kMaxDevices] = {};
+constexpr int kMaxContexts = 64;
+struct NoallocSlot {
+  unsigned long long ctx_id;
+  void* addr;
+};
+NoallocSlot g_noalloc[kMaxContexts] = {};
+int g_noalloc_used = 0;
+int g_noalloc_next = 0;
 std::mutex g_noalloc_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context (the runtime's primary context
+// of the current device unless the caller made another one current); 0 on
+// error.  The runtime makes the primary context current on its first call
+// that needs one, so a thread with none yet gets it from cudaGetSymbolAddress.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_cur || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess)
+      return 0;
+    get_cur = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
+  }
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS) return 0;
+  if (!ctx) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kia_noalloc_scratch) != cudaSuccess) return 0;
+    if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  }
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+// Device address of the scratch in the calling thread's current context.
+void* noalloc_scratch() {
+  const unsigned long long id = current_context_id();
+  if (id == 0) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  for (int i = 0; i < g_noalloc_used; ++i)
+    if (g_noalloc[i].ctx_id == id) return g_noalloc[i].addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_kia_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+  // a process that cycles through more contexts than slots overwrites the
+  // oldest slot (its context is the likeliest to be gone)
+  g_noalloc[g_noalloc_next] = NoallocSlot{id, p};
+  g_noalloc_next = (g_noalloc_next + 1) % kMaxContexts;
+  if (g_noalloc_used < kMaxContexts) ++g_noalloc_used;
+  return p;
+}
 
 }  // namespace
 
@@ -313,20 +376,8 @@ int kiattn_bwd_noalloc(const float* Q, const float* Kt, const float* V, const fl
   const long long rows = (long long)B * H * T;
   if (rows > KIA_NOALLOC_MAX_ROWS || work_bytes(rows) > kNoallocScratchBytes)
     return KIA_ERR_CAPACITY;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KIA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return KIA_ERR_UNSUPPORTED;
-  void* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_kia_noalloc_scratch) != cudaSuccess || !p)
-        return KIA_ERR_CUDA;
-      g_noalloc_addr[dev] = p;
-    }
-    scratch = g_noalloc_addr[dev];
-  }
+  void* scratch = noalloc_scratch();
+  if (!scratch) return KIA_ERR_CUDA;
   return kiattn_bwd(Q, Kt, V, O, dO, stats, dQ, dK, dV, dS_dbg, B, H, T, d, cfg, scratch,
                     stream);
 }
@@ -341,9 +392,12 @@ int kiattn_weights_from_S(const float* S, int rows, int cols, const int* row_len
   if (cfg->op != KIA_OP_KINTERVAL) return KIA_ERR_INVALID_ARG;
   const OpParams p = make_params(cfg);
   const unsigned nb = (unsigned)((rows + kWeightsWarps - 1) / kWeightsWarps);
-  weights_from_S_kernel<<<nb, 32 * kWeightsWarps, 0, static_cast<cudaStream_t>(stream)>>>(
-      S, rows, cols, row_len, p, w, bin, t, row_m, row_n);
-  return launch_status();
+  // the forward's compile-time variant of this configuration
+  return dispatch_variant(p, [&]<class V>() {
+    weights_from_S_kernel<V><<<nb, 32 * kWeightsWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+        S, rows, cols, row_len, p, w, bin, t, row_m, row_n);
+    return launch_status();
+  });
 }
 
 int kiattn_scores(const float* Q, const float* Kt, float* S, int B, int H, int T, int d,
@@ -447,6 +501,15 @@ int kiattn_profile_read(float* ms, int n) {
     ms[w] = t;
   }
   return w;
+}
+
+int kiattn_debug_bounded_wait(int what, unsigned long long wait_limit_ns) {
+  if (what < 0 || what > 1) return KIA_ERR_INVALID_ARG;
+  const unsigned long long lim = wait_limit_ns ? wait_limit_ns : (unsigned long long)kWaitLimitNs;
+  if (cudaMemcpyToSymbol(g_kia_wait_limit_ns, &lim, sizeof(lim)) != cudaSuccess)
+    return KIA_ERR_CUDA;
+  g_withhold = what;
+  return KIA_OK;
 }
 
 int kiattn_device_error(int reset) {

@@ -30,7 +30,8 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error", 
 SYMBOLS = ("kiattn_stats_bytes", "kiattn_workspace_bytes", "kiattn_fwd", "kiattn_bwd",
            "kiattn_weights_from_S", "kiattn_scores", "kiattn_strerror", "kiattn_version",
            "kiattn_device_error", "kiattn_profile_enable", "kiattn_profile_read",
-           "kiattn_bwd_noalloc", "kiattn_grad_decomposition", "kiattn_geometry")
+           "kiattn_bwd_noalloc", "kiattn_grad_decomposition", "kiattn_geometry",
+           "kiattn_debug_bounded_wait")
 NOALLOC_MAX_ROWS = 1 << 20
 PHASES = ("fwd", "bwd_prep", "bwd_query_pass", "bwd_key_pass", "bwd_calibration")
 
@@ -95,6 +96,8 @@ def _load():
     lib.kiattn_grad_decomposition.restype = i
     lib.kiattn_geometry.argtypes = [vp, vp, i, i, i, i, cp, vp, vp]
     lib.kiattn_geometry.restype = i
+    lib.kiattn_debug_bounded_wait.argtypes = [i, ctypes.c_ulonglong]
+    lib.kiattn_debug_bounded_wait.restype = i
     lib.kiattn_strerror.argtypes = [i]
     lib.kiattn_strerror.restype = ctypes.c_char_p
     lib.kiattn_version.restype = i
@@ -278,6 +281,15 @@ def kiattn_version() -> int:
 
 def kiattn_device_error(reset: bool = True) -> int:
     return int(_lib.kiattn_device_error(1 if reset else 0))
+
+
+def kiattn_debug_bounded_wait(what: int, wait_limit_ns: int = 0):
+    """Test hook of the bounded device-side waits: what = 1 makes the
+    following tensor-core forwards withhold one operand copy so that their
+    waits run out (KIA_ERR_TIMEOUT in kiattn_device_error); wait_limit_ns > 0
+    shortens every wait's limit.  kiattn_debug_bounded_wait(0, 0) restores
+    the defaults."""
+    _check("kiattn_debug_bounded_wait", _lib.kiattn_debug_bounded_wait(int(what), int(wait_limit_ns)))
 
 
 def kiattn_profile_enable(on: bool = True):

