@@ -110,25 +110,44 @@ def flag_rows(Q, Kt, cfg: K.Config, rule: int, delta: float) -> np.ndarray:
             if cfg.cal == K.CAL_MINMAX:
                 bad |= (srt[..., 1] - srt[..., 0]) < delta * hs[..., 0]
                 span = (m - n)[..., 0]
-                bad |= np.abs(span - 1e-12) < 1e-13
+                near = np.abs(span - 1e-12) < 1e-13
+                # a row clearly in the degenerate branch has uniform P and no
+                # calibration term: neither its bins nor its arg-extrema matter
+                bad = np.where(span < 0.5e-12, near, bad | near)
         flags[:, :, i] = bad
     return flags
 
 
 def flag_budget(Q, Kt, cfg: K.Config, rule: int, delta: float) -> float:
     """Expected fraction of flagged rows for scores spread continuously: per
-    row, a union bound over the discontinuities flag_rows looks for -- each
+    row, a union bound over the discontinuities flag_rows looks for (for the
+    reduced-precision exponential baselines, the rounding boundaries its
+    numerators may straddle) -- each
     in-window key lies within delta of a Nearest rounding boundary with
     probability 2 delta (its position inside the interval is spread evenly),
     within delta of the FWM edge with probability 2 delta times the keys per
     unit of u around the edge, and the top (bottom) two scores come within
     delta h of each other with probability delta times the keys per unit of u
     next to the maximum (minimum)."""
-    if cfg.op != K.OP_KINTERVAL:
+    if cfg.op == K.OP_SOFTMAX:
         return 0.0
     S = oracle_scores(Q, Kt, rule)
     B, H, T, _ = Q.shape
     p = np.zeros((B, H, T))
+    if cfg.op in (K.OP_SOFTMAX_BF16EXP, K.OP_SOFTMAX_FP8EXP):
+        # _rounding_flags: a numerator e moved by a relative rel straddles a
+        # rounding boundary of the format with probability 2 rel e / ulp(e)
+        mbits, emin = (7, -126) if cfg.op == K.OP_SOFTMAX_BF16EXP else (3, -6)
+        for i in range(T):
+            L = i + 1 if cfg.causal else T
+            x = S[:, :, i, :L] - S[:, :, i, :L].max(-1, keepdims=True)
+            e = np.exp(x)
+            rel = 2.0 ** -21 + np.abs(x) * 2.0 ** -22
+            ex = np.maximum(np.floor(np.log2(np.maximum(e, 1e-300))), emin)
+            ulp = 2.0 ** (ex - mbits)
+            q = np.where(e >= 1e-6, 2 * rel * e / ulp, 0.0).sum(-1)
+            p[:, :, i] = np.minimum(q, 1.0)
+        return float(p.mean())
     tau = float(np.float32(cfg.tau))
     for i in range(T):
         L = i + 1 if cfg.causal else T
@@ -147,6 +166,8 @@ def flag_budget(Q, Kt, cfg: K.Config, rule: int, delta: float) -> float:
             q += delta * (u < 1).sum(-1)
             if cfg.cal == K.CAL_MINMAX:
                 q += delta * (u > cfg.K - 1).sum(-1)
+        if cfg.cal == K.CAL_MINMAX:
+            q = np.where((m - n)[..., 0] < 0.5e-12, 0.0, q)
         p[:, :, i] = np.minimum(q, 1.0)
     return float(p.mean())
 
