@@ -290,6 +290,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait by a whole warp (an MMA-issuing warp runs its loop converged
+// and elects one lane only to issue): every lane waits on the same phase and
+// the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
 // Watchdog of a polling loop that serves several barriers: call idle() on
 // every pass that made no progress and progress() on every pass that did.
 // Gives up like mbar_wait: after ~g_kia_wait_limit_ns without progress, or at

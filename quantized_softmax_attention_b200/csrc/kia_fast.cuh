@@ -44,6 +44,19 @@ struct GridP {
   const float2* q;
   __device__ __forceinline__ float2 pair(int k) const { return q[k]; }
 };
+// FWM / fixed-step grid in shared memory: pairs (G_k, G_{k+1}) for k = 0..K-1
+// followed by a zero pair at index K.  A tail key (u > K) fetches the zero
+// pair, which gives it weight 0 and slope 0 with no selects afterwards.
+struct GridZ {
+  const float2* q;   // pair 0 (shared memory)
+  int K;             // index of the zero pair
+  __device__ __forceinline__ float2 at(int k, bool tail) const { return q[tail ? K : k]; }
+};
+__device__ __forceinline__ GridZ make_gridz(const float2* pairs, int K) { return GridZ{pairs, K}; }
+template <class G>
+inline constexpr bool kZeroTail = false;
+template <>
+inline constexpr bool kZeroTail<GridZ> = true;
 
 struct Pos {
   float u;   // grid coordinate (MinMax: clamped to K)
@@ -161,7 +174,9 @@ __device__ __forceinline__ Pos fwd_weights(const G& grid, float m, float rh, flo
     return Pos{0.0f, 0.0f, 0.0f, 0};
   } else {
     const Pos p = grid_pos<V, CLAMP0>(m, rh, Kf, Km1f, s);
-    const float2 g = grid.pair(p.k);
+    float2 g;
+    if constexpr (kZeroTail<G>) g = grid.at(p.k, V::FWM && p.u > Kf);
+    else g = grid.pair(p.k);
     const float lerp = __fmaf_rn(p.t, __fsub_rn(g.y, g.x), g.x);
     if constexpr (V::NEAREST) {
       wf = (p.t >= 0.5f) ? g.y : g.x;
@@ -170,7 +185,7 @@ __device__ __forceinline__ Pos fwd_weights(const G& grid, float m, float rh, flo
       wf = lerp;
       wl = lerp;
     }
-    if constexpr (V::FWM) {
+    if constexpr (V::FWM && !kZeroTail<G>) {
       const bool tail = p.u > Kf;
       wf = tail ? 0.0f : wf;
       wl = tail ? 0.0f : wl;
@@ -193,11 +208,16 @@ __device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, flo
     return expf(s - m) * dw;
   } else {
     const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
-    float2 g = grid.pair(p.k);
-    if constexpr (V::FWM) {
-      const bool tail = p.u > Kf;
-      g.x = tail ? 0.0f : g.x;
-      g.y = tail ? 0.0f : g.y;
+    float2 g;
+    if constexpr (kZeroTail<G>) {
+      g = grid.at(p.k, V::FWM && p.u > Kf);
+    } else {
+      g = grid.pair(p.k);
+      if constexpr (V::FWM) {
+        const bool tail = p.u > Kf;
+        g.x = tail ? 0.0f : g.x;
+        g.y = tail ? 0.0f : g.y;
+      }
     }
     const float da = dw * __fsub_rn(g.y, g.x);
     A += da;
@@ -213,37 +233,6 @@ __device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, flo
       delta = da * nrh;
     }
     return delta;
-  }
-}
-
-// Backward of one element in the key pass: the forward probability P (for
-// dV) and the detached dS (for dK), from one grid position.  FWM's tail
-// (u > K) has zero weight and zero slope.
-template <class V, class G>
-__device__ __forceinline__ void kv_elem(const G& grid, float m, float rh, float dg, float rWf,
-                                        float Kf, float Km1f, float s, float dw, float& P,
-                                        float& dS) {
-  if constexpr (V::SOFTMAX) {
-    const float w = expf(s - m);
-    P = round_exp<V::EXPR>(w) * rWf;   // the forward's (rounded) probability
-    dS = w * dw;                       // straight through the rounding
-  } else {
-    const Pos p = grid_pos<V, true>(m, rh, Kf, Km1f, s);
-    const float2 g = grid.pair(p.k);
-    const float a = __fsub_rn(g.y, g.x);
-    const float wf = V::NEAREST ? ((p.t >= 0.5f) ? g.y : g.x) : __fmaf_rn(p.t, a, g.x);
-    P = wf * rWf;
-    const float da = dw * a;
-    if constexpr (V::MINMAX) {
-      dS = fmaf(dw, dg, -(da * rh));
-    } else {
-      dS = -(da * rh);
-    }
-    if constexpr (V::FWM) {
-      const bool tail = p.u > Kf;
-      P = tail ? 0.0f : P;
-      dS = tail ? 0.0f : dS;
-    }
   }
 }
 

@@ -221,7 +221,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------- score-MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptor
+    // arithmetic); one elected lane issues each unit's MMAs and commits.
+    {
       const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
       // descriptors built once; each MMA only adds a constant step
       const uint64_t dqa = desc_kmajor(smem_u32(sQ), 0), dga = desc_kmajor(smem_u32(sG), 0),
@@ -230,37 +232,44 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       int g = 0, n = 0;                   // global half tile, item count
       ItemSeq seq(nitems);
       for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
-        if (!mbar_wait(&bar.qd_full, n & 1, abort)) { failed = true; break; }
+        if (!warp_wait(&bar.qd_full, n & 1, abort)) { failed = true; break; }
         // S, dP of half tile u (keys 64 u..) into region g % R, once the dQ
         // MMA of half tile g - R has released the region
         const int nunits = item_units(it);
         for (int u = 0; u < nunits; ++u, ++g) {
           const int r = g % R;
           if (g >= R) {
-            if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+            if (!warp_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
             sf_par ^= 1u << r;
           }
           const int sl = g % kBwdSlots;
-          if (!mbar_wait(&bar.kv_full[sl], (g / kBwdSlots) & 1, abort)) { failed = true; break; }
-          tc_fence_after();
+          if (!warp_wait(&bar.kv_full[sl], (g / kBwdSlots) & 1, abort)) { failed = true; break; }
           const uint64_t dk = dkv + desc_step((uint32_t)sl * kHalfPair);   // K half, V half after it
           const uint64_t dv = dk + desc_step(kHalfTile);
           const uint32_t dst = tmem + 128u * r;
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ss(dst, dqa + kstep_kmajor(ks), dk + kstep_kmajor_half(ks), id_s, ks > 0);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ss(dst, dqa + kstep_kmajor(ks), dk + kstep_kmajor_half(ks), id_s, ks > 0);
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ss(dst + 64u, dga + kstep_kmajor(ks), dv + kstep_kmajor_half(ks), id_s, ks > 0);
-          tc_commit(&bar.sp_full[r]);
-          tc_commit(&bar.kv_empty[sl]);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ss(dst + 64u, dga + kstep_kmajor(ks), dv + kstep_kmajor_half(ks), id_s, ks > 0);
+            tc_commit(&bar.sp_full[r]);
+            tc_commit(&bar.kv_empty[sl]);
+          }
+          __syncwarp();
         }
-        if (!failed) tc_commit(&bar.qd_empty);     // Q_i, dO_i free once these MMAs are done
+        if (!failed) {
+          if (elect_one()) tc_commit(&bar.qd_empty);   // Q_i, dO_i free once these MMAs are done
+          __syncwarp();
+        }
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------- dQ-MMA issuer
-    if (lane == 0) {
+    // (whole warp, one elected lane issuing)
+    {
       const uint32_t id_dq = idesc_tf32(128, D, 0, 1);
       const uint64_t dkm = desc_mnmajor_half(smem_u32(sKmn));
       uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
@@ -271,24 +280,30 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // dQ of half tile u: A = dS in region g % R, B = K half (MN-major)
         for (int u = 0; u < nunits; ++u, ++g) {
           const int r = g % R, sl = g % kKmnSlots;
-          if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
+          if (!warp_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
           ed_par ^= 1u << r;
-          if (!mbar_wait(&bar.kmn_full[sl], (g / kKmnSlots) & 1, abort)) { failed = true; break; }
+          if (!warp_wait(&bar.kmn_full[sl], (g / kKmnSlots) & 1, abort)) { failed = true; break; }
           // the accumulator restarts with this item: the previous item's
           // epilogue must have read it
-          if (u == 0 && n > 0 && !mbar_wait(&bar.dq_free, (n - 1) & 1, abort)) { failed = true; break; }
-          tc_fence_after();
+          if (u == 0 && n > 0 && !warp_wait(&bar.dq_free, (n - 1) & 1, abort)) { failed = true; break; }
           const uint64_t db = dkm + desc_step((uint32_t)sl * kHalfTile);
           const uint32_t pa = tmem + 128u * r;
           const uint32_t acc0 = u > 0 ? 1u : 0u;
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + kColDQ, pa + 8u * kk, db + kstep_mnmajor(kk), id_dq,
-                        kk > 0 ? 1u : acc0);
-          tc_commit(&bar.st_free[r]);
-          tc_commit(&bar.kmn_empty[sl]);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_tf32_ts(tmem + kColDQ, pa + 8u * kk, db + kstep_mnmajor(kk), id_dq,
+                          kk > 0 ? 1u : acc0);
+            tc_commit(&bar.st_free[r]);
+            tc_commit(&bar.kmn_empty[sl]);
+          }
+          __syncwarp();
         }
-        if (!failed) tc_commit(&bar.dq_full);
+        if (!failed) {
+          if (elect_one()) tc_commit(&bar.dq_full);
+          __syncwarp();
+        }
       }
     }
   } else if (warp < kScoreWarp) {
@@ -302,8 +317,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
     float2* sPair = reinterpret_cast<float2*>(sTab);
     if constexpr (!V::MINMAX && !V::SOFTMAX) {
-      for (int k = (int)threadIdx.x - 64; k < p.K; k += kElemThreads)
-        sPair[k] = make_float2(st.table[k], st.table[k + 1]);
+      // pairs k = 0..K-1 and the tail's zero pair at K
+      for (int k = (int)threadIdx.x - 64; k <= p.K; k += kElemThreads)
+        sPair[k] = k < p.K ? make_float2(st.table[k], st.table[k + 1]) : make_float2(0.0f, 0.0f);
     }
     int gbase = 0, n = 0;
     ItemSeq seq(nitems);
@@ -409,8 +425,10 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if constexpr (V::MINMAX) {
         if (tab_in_smem) unit_loop(GridF{sTab + r, KIA_TILE});
         else unit_loop(GridF{st.table + qr * (p.K + 1), 1});
-      } else {
+      } else if constexpr (V::SOFTMAX) {
         unit_loop(GridP{sPair});
+      } else {
+        unit_loop(make_gridz(sPair, p.K));
       }
       if (failed) break;
       gbase += nunits;
@@ -559,12 +577,15 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   // Per-query constants of a unit (64 queries) in four slots, filled ahead of
   // the element groups by the constant warp: half tile g (numbered across the
   // CTA's items) uses slot 2 (g % 2) + (g / 2) % 2.
+  // sC4 = (m, k1, k0, 1/W_fwd): the score-gradient factor -dw/h = dP k1 + k0
+  // (softmax: dw itself); sX4 (MinMax or projection) = (1/h, the degenerate
+  // row's dw = dP x.y + x.z, 0 elsewhere, the projection shift c)
   constexpr int kSlots = 4, kSlotQ = 64;
-  float4* sC4 = reinterpret_cast<float4*>(sQDmn + kKvSlots * kHalfPair);  // (m, rh, rWb, -D rWb)
-  float2* sC2 = reinterpret_cast<float2*>(sC4 + kSlots * kSlotQ);  // (rWf, dg or projection shift c)
+  float4* sC4 = reinterpret_cast<float4*>(sQDmn + kKvSlots * kHalfPair);
+  float4* sX4 = sC4 + kSlots * kSlotQ;
   // calibration terms, read only where a query's argmax (argmin) key is this
   // thread's key: key - tile start, and the coefficient
-  int2* sCI = reinterpret_cast<int2*>(sC2 + kSlots * kSlotQ);  // (argmax, argmin) - kt * 128
+  int2* sCI = reinterpret_cast<int2*>(sX4 + kSlots * kSlotQ);  // (argmax, argmin) - kt * 128
   float2* sCG = reinterpret_cast<float2*>(sCI + kSlots * kSlotQ);  // (g_m, g_n)
   // which queries of a unit have their argmax (argmin) key in lanes
   // 32 quad..32 quad + 31: [slot][argmax / argmin][quad][query half]
@@ -692,7 +713,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------- score-MMA issuer
-    if (lane == 0) {
+    // (whole warp, one elected lane issuing)
+    {
       const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
       // descriptors built once; each MMA only adds a constant step
       const uint64_t dka = desc_kmajor(smem_u32(sK), 0), dva = desc_kmajor(smem_u32(sV), 0),
@@ -701,36 +723,43 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       int g = 0, n = 0;
       ItemSeq seq(nitems);
       for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
-        if (!mbar_wait(&bar.kv_full, n & 1, abort)) { failed = true; break; }
+        if (!warp_wait(&bar.kv_full, n & 1, abort)) { failed = true; break; }
         // S^T, dP^T of half tile u (queries 64 (2 q0 + u)..) into region
         // g % R, once the dV / dK MMAs of half tile g - R have released it
         const int nunits = item_units(it);
         for (int u = 0; u < nunits; ++u, ++g) {
           const int r = g % R, sl = g % kKvSlots;
           if (g >= R) {
-            if (!mbar_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+            if (!warp_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
             sf_par ^= 1u << r;
           }
-          if (!mbar_wait(&bar.qd_full[sl], (g / kKvSlots) & 1, abort)) { failed = true; break; }
-          tc_fence_after();
+          if (!warp_wait(&bar.qd_full[sl], (g / kKvSlots) & 1, abort)) { failed = true; break; }
           const uint64_t dq = dqd + desc_step((uint32_t)sl * kHalfPair);   // Q half, dO half after it
           const uint64_t dg = dq + desc_step(kHalfTile);
           const uint32_t dst = tmem + 128u * r;
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ss(dst, dka + kstep_kmajor(ks), dq + kstep_kmajor_half(ks), id_s, ks > 0);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ss(dst, dka + kstep_kmajor(ks), dq + kstep_kmajor_half(ks), id_s, ks > 0);
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ss(dst + 64u, dva + kstep_kmajor(ks), dg + kstep_kmajor_half(ks), id_s, ks > 0);
-          tc_commit(&bar.sp_full[r]);
-          tc_commit(&bar.qd_empty[sl]);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ss(dst + 64u, dva + kstep_kmajor(ks), dg + kstep_kmajor_half(ks), id_s, ks > 0);
+            tc_commit(&bar.sp_full[r]);
+            tc_commit(&bar.qd_empty[sl]);
+          }
+          __syncwarp();
         }
-        if (!failed) tc_commit(&bar.kv_empty);     // K_j, V_j free once these MMAs are done
+        if (!failed) {
+          if (elect_one()) tc_commit(&bar.kv_empty);   // K_j, V_j free once these MMAs are done
+          __syncwarp();
+        }
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------- dV / dK-MMA issuer
-    if (lane == 0) {
+    // (whole warp, one elected lane issuing)
+    {
       const uint32_t id_acc = idesc_tf32(128, D, 0, 1);
       const uint64_t dmn = desc_mnmajor_half(smem_u32(sQDmn));
       uint32_t ed_par = 0;                // per-region phase bits of the elem_done waits
@@ -741,29 +770,35 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // dV += P^T dO, dK += dS^T Q for half tile u (A operands in region g % R)
         for (int u = 0; u < nunits; ++u, ++g) {
           const int r = g % R, sl = g % kKvSlots;
-          if (!mbar_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
+          if (!warp_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
           ed_par ^= 1u << r;
-          if (!mbar_wait(&bar.mn_full[sl], (g / kKvSlots) & 1, abort)) { failed = true; break; }
+          if (!warp_wait(&bar.mn_full[sl], (g / kKvSlots) & 1, abort)) { failed = true; break; }
           // the accumulators restart with this item: the previous item's
           // epilogue must have read them
-          if (u == 0 && n > 0 && !mbar_wait(&bar.acc_free, (n - 1) & 1, abort)) { failed = true; break; }
-          tc_fence_after();
+          if (u == 0 && n > 0 && !warp_wait(&bar.acc_free, (n - 1) & 1, abort)) { failed = true; break; }
           const uint64_t dqm = dmn + desc_step((uint32_t)sl * kHalfPair);   // Q half, dO half after it
           const uint64_t dgm = dqm + desc_step(kHalfTile);
           const uint32_t pa = tmem + 128u * r;
           const uint32_t acc0 = u > 0 ? 1u : 0u;
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + kColDV, pa + 8u * kk, dgm + kstep_mnmajor(kk), id_acc,
-                        kk > 0 ? 1u : acc0);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_tf32_ts(tmem + kColDV, pa + 8u * kk, dgm + kstep_mnmajor(kk), id_acc,
+                          kk > 0 ? 1u : acc0);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + kColDK, pa + 64u + 8u * kk, dqm + kstep_mnmajor(kk), id_acc,
-                        kk > 0 ? 1u : acc0);
-          tc_commit(&bar.st_free[r]);
-          tc_commit(&bar.mn_empty[sl]);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_tf32_ts(tmem + kColDK, pa + 64u + 8u * kk, dqm + kstep_mnmajor(kk), id_acc,
+                          kk > 0 ? 1u : acc0);
+            tc_commit(&bar.st_free[r]);
+            tc_commit(&bar.mn_empty[sl]);
+          }
+          __syncwarp();
         }
-        if (!failed) tc_commit(&bar.acc_full);
+        if (!failed) {
+          if (elect_one()) tc_commit(&bar.acc_full);
+          __syncwarp();
+        }
       }
     }
   } else if (warp == kScoreWarp + 1) {
@@ -773,8 +808,9 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // FWM: each group's copy of the shared grid's pairs, published with the
     // first units' constants
     if (!V::SOFTMAX && !V::MINMAX) {
-      for (int k = lane; k < p.K; k += 32) {
-        const float2 pr = make_float2(st.table[k], st.table[k + 1]);
+      // pairs k = 0..K-1, then a zero pair at K: the target of tail keys
+      for (int k = lane; k <= p.K; k += 32) {
+        const float2 pr = k < p.K ? make_float2(st.table[k], st.table[k + 1]) : make_float2(0.0f, 0.0f);
         reinterpret_cast<float2*>(sTab)[k] = pr;
         reinterpret_cast<float2*>(sTab)[K1 + k] = pr;
       }
@@ -825,14 +861,19 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int e = sl * kSlotQ + 32 * hq + lane;          // its slot entry
         const int Lq = p.causal ? q + 1 : T;
         const float rWb = Lq == 1 ? 0.0f : __fdiv_rn(1.0f, cur.Wb[hq]);
-        sC4[e] = make_float4(cur.m[hq], cur.rh[hq], rWb, -cur.D[hq] * rWb);
+        const float nD = -cur.D[hq] * rWb;       // dw = dP rWb + nD
+        const float nrh = V::SOFTMAX ? 1.0f : -cur.rh[hq];
+        sC4[e] = make_float4(cur.m[hq], rWb * nrh, nD * nrh, __fdiv_rn(1.0f, cur.Wf[hq]));
         // calibration terms of the query's row, added to dS^T before dK:
         // g_m at the argmax key, g_n at the argmin key, or the projection
         // shift c on every visible key
         const bool live = q < T;
         const float gm = live ? cur.gm[hq] : 0.0f, gn = live ? cur.gn[hq] : 0.0f;
-        sC2[e] = make_float2(__fdiv_rn(1.0f, cur.Wf[hq]),
-                             PROJ ? gm : ((V::MINMAX && cur.rh[hq] == 0.0f) ? 1.0f : 0.0f));
+        if constexpr (V::MINMAX || PROJ) {
+          // a degenerate MinMax row (1/h = 0) has dS = dw: uniform P
+          const float dg = (V::MINMAX && cur.rh[hq] == 0.0f) ? 1.0f : 0.0f;
+          sX4[e] = make_float4(cur.rh[hq], dg * rWb, dg * nD, PROJ ? gm : 0.0f);
+        }
         if constexpr (!PROJ && !V::SOFTMAX) {
           const int ka = cur.am[hq] - kt * KIA_TILE;
           const int kn = V::MINMAX ? cur.an[hq] - kt * KIA_TILE : -1;
@@ -891,8 +932,12 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
-    // FWM: each group keeps its own copy of the shared grid's pairs
+    // FWM: each group keeps its own copy of the shared grid's pairs, with a
+    // zero pair at index K that tail keys are pointed at; a pair is fetched
+    // by its address computed from the floor trick's bits directly
     const float2* sPairG = reinterpret_cast<const float2*>(sTab) + grp * K1;
+    const GridZ gridz = make_gridz(sPairG, p.K);
+    const float rh_c = p.fwm_rh;
     int gbase = 0, n = 0;
     ItemSeq seq(nitems);
     for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
@@ -925,23 +970,40 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int ql = ql0 + i;
-              const float4 c4 = sC4[e0 + i];
-              const float2 c2 = sC2[e0 + i];
-              const float dw = fmaf(g[i], c4.z, c4.w);
+              const float4 cq = sC4[e0 + i];
+              float4 xq = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              if constexpr (V::MINMAX || PROJ) xq = sX4[e0 + i];
+              const float s = v[i], dP = g[i];
+              const float dSn = fmaf(dP, cq.y, cq.z);        // -dw / h  (softmax: dw)
               float P, dS;
-              if constexpr (V::MINMAX) {
-                const float* gp;
-                if constexpr (TABS) gp = sTab + (e0 + i) * K1;
-                else gp = st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1;
-                const GridF grid{gp, 1};
-                // degenerate rows (rh = 0) take dS = dw; under the projection c2.y
-                // holds the shift, so the flag comes from rh itself
-                const float dg = PROJ ? (c4.y == 0.0f ? 1.0f : 0.0f) : c2.y;
-                kv_elem<V>(grid, c4.x, c4.y, dg, c2.x, Kf, Km1f, v[i], dw, P, dS);
+              if constexpr (V::SOFTMAX) {
+                const float w = expf(s - cq.x);
+                P = round_exp<V::EXPR>(w) * cq.w;   // the forward's (rounded) probability
+                dS = w * dSn;                       // straight through the rounding
               } else {
-                kv_elem<V>(GridP{sPairG}, c4.x, c4.y, 0.0f, c2.x, Kf, Km1f, v[i], dw, P, dS);
+                const float rh = V::MINMAX ? xq.x : rh_c;
+                float u = __fmul_rn(__fsub_rn(cq.x, s), rh);
+                if constexpr (V::MINMAX) u = fminf(u, Kf);
+                const float uc = fmaxf(fminf(u, Km1f), 0.0f);
+                const float tmp = __fadd_rd(uc, kMagic);
+                const float t = __fsub_rn(u, __fsub_rn(tmp, kMagic));
+                float2 gp;
+                if constexpr (V::MINMAX) {
+                  const float* gq;
+                  if constexpr (TABS) gq = sTab + (e0 + i) * K1;
+                  else gq = st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * K1;
+                  gp = GridF{gq, 1}.pair(__float_as_int(tmp) - kMagicBits);
+                } else {
+                  // FWM tail (u > K): the zero pair, so P = 0 and dS = 0
+                  gp = gridz.at(__float_as_int(tmp) - kMagicBits, u > Kf);
+                }
+                const float a = __fsub_rn(gp.y, gp.x);
+                const float wf = V::NEAREST ? (t >= 0.5f ? gp.y : gp.x) : __fmaf_rn(t, a, gp.x);
+                P = wf * cq.w;
+                dS = a * dSn;
+                if constexpr (V::MINMAX) dS = fmaf(dP, xq.y, dS + xq.z);   // degenerate rows: dw
               }
-              if constexpr (PROJ) dS += c2.y;
+              if constexpr (PROJ) dS += xq.w;
               if constexpr (EDGE) {
                 const int q = qi * KIA_TILE + ql;
                 if (!(kj < T && q < T && (!p.causal || kj <= q))) {
@@ -1048,7 +1110,7 @@ size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem) {
   const int tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? 4 * 64 * (p.K + 1) : 0) : 4 * (p.K + 1));
   return 1024 + 2 * (size_t)D * KIA_TILE * 4 + 2 * kKvSlots * (size_t)kHalfPair +
-         4 * 64 * (16 + 8 + 8 + 8) + 4 * 2 * 4 * 2 * 4 + kElemThreads / 32 * 1024 +
+         4 * 64 * (16 + 16 + 8 + 8) + 4 * 2 * 4 * 2 * 4 + kElemThreads / 32 * 1024 +
          (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdKBars);
 }
 

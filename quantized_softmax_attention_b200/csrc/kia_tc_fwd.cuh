@@ -197,7 +197,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------- score-MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop, so that its waits and descriptor
+    // arithmetic stay warp-uniform; one elected lane issues each unit's MMAs
+    // and their commits (issuing from a lone lane halved the MMA rate).
+    {
       const uint32_t idesc_s = idesc_tf32(128, 64, 0, 0);    // sweep 2: half tiles
       const uint32_t idesc_t = idesc_tf32(128, 128, 0, 0);   // sweep 1: whole tiles
       // descriptors built once; each MMA only adds a constant step
@@ -209,7 +212,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       uint32_t sf_par = 0, pv_par = 0, last_pv = 0;
       ItemSeq seq(nitems);
       for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
-        if (!mbar_wait(&bar.q_full, n & 1, abort)) { failed = true; break; }
+        if (!warp_wait(&bar.q_full, n & 1, abort)) { failed = true; break; }
         const int nkt = item_nkt(it), nunits = 2 * nkt;
         // units of an item: sweep 1 key tiles j (N = 128), then sweep 2 half
         // tiles u (N = 64); unit G goes into region G % R once the unit R
@@ -219,41 +222,47 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           const int r = G % R;
           if (G >= R) {
             if ((last_pv >> r) & 1u) {
-              if (!mbar_wait(&bar.pv_done[r], (pv_par >> r) & 1u, abort)) { failed = true; break; }
+              if (!warp_wait(&bar.pv_done[r], (pv_par >> r) & 1u, abort)) { failed = true; break; }
               pv_par ^= 1u << r;
             } else {
-              if (!mbar_wait(&bar.s_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
+              if (!warp_wait(&bar.s_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
               sf_par ^= 1u << r;
             }
           }
           last_pv = sweep2 ? (last_pv | (1u << r)) : (last_pv & ~(1u << r));
           const int h = sweep2 ? ((v - nkt) & 1) : 0;   // half of the key tile (sweep 2)
           const int s = kc % NSK, nn = kc / NSK;
-          if (h == 0 && !mbar_wait(&bar.k_full[s], nn & 1, abort)) { failed = true; break; }
-          tc_fence_after();
+          if (h == 0 && !warp_wait(&bar.k_full[s], nn & 1, abort)) { failed = true; break; }
           const uint64_t dk = dk0 + desc_step((uint32_t)s * Cfg::kTileBytes + (uint32_t)h * 64u * 128u);
           const uint32_t dst = tmem + 128u * r;
-          if (!sweep2) {
+          const bool last_half = !sweep2 || h == 1;
+          if (elect_one()) {
+            tc_fence_after();
+            if (!sweep2) {
 #pragma unroll
-            for (int ks = 0; ks < D / 8; ++ks)
-              mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_t, ks > 0 ? 1u : 0u);
-          } else {
+              for (int ks = 0; ks < D / 8; ++ks)
+                mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_t, ks > 0 ? 1u : 0u);
+            } else {
 #pragma unroll
-            for (int ks = 0; ks < D / 8; ++ks)
-              mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_s, ks > 0 ? 1u : 0u);
+              for (int ks = 0; ks < D / 8; ++ks)
+                mma_tf32_ss(dst, dq0 + kstep_kmajor(ks), dk + kstep_kmajor(ks), idesc_s, ks > 0 ? 1u : 0u);
+            }
+            tc_commit(&bar.s_full[r]);
+            if (last_half) tc_commit(&bar.k_empty[s]);
           }
-          tc_commit(&bar.s_full[r]);
-          if (!sweep2 || h == 1) {
-            tc_commit(&bar.k_empty[s]);
-            ++kc;
-          }
+          __syncwarp();
+          if (last_half) ++kc;
         }
-        if (!failed) tc_commit(&bar.q_empty);    // Q free once these MMAs are done
+        if (!failed) {
+          if (elect_one()) tc_commit(&bar.q_empty);    // Q free once these MMAs are done
+          __syncwarp();
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------- accumulating-MMA issuer
-    if (lane == 0) {
+    // (whole warp, one elected lane issuing; see the score issuer)
+    {
       const uint32_t idesc_o = idesc_tf32(128, D, 0, 1);
       const uint64_t dv0 = desc_mnmajor(smem_u32(sV), 0);
       int vc = 0, n = 0, G = 0;
@@ -264,34 +273,38 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         G += item_nkt(it);                // this item's sweep-1 units (whole tiles)
         for (int u = 0; u < nunits; ++u, ++G) {
           const int r = G % R, h = u & 1;
-          if (!mbar_wait(&bar.p_ready[r], (pr_par >> r) & 1u, abort)) { failed = true; break; }
+          if (!warp_wait(&bar.p_ready[r], (pr_par >> r) & 1u, abort)) { failed = true; break; }
           pr_par ^= 1u << r;
           const int s = vc % NSV, nn = vc / NSV;
-          if (h == 0 && !mbar_wait(&bar.v_full[s], nn & 1, abort)) { failed = true; break; }
+          if (h == 0 && !warp_wait(&bar.v_full[s], nn & 1, abort)) { failed = true; break; }
           // the accumulators restart with this item: the previous item's
           // epilogue must have read them
-          if (u == 0 && n > 0 && !mbar_wait(&bar.o_free, (n - 1) & 1, abort)) { failed = true; break; }
-          tc_fence_after();
+          if (u == 0 && n > 0 && !warp_wait(&bar.o_free, (n - 1) & 1, abort)) { failed = true; break; }
           const uint64_t dv = dv0 + desc_step((uint32_t)s * Cfg::kTileBytes) + kstep_mnmajor(8 * h);
           const uint32_t pa = tmem + 128u * r;
           const uint32_t acc0 = u > 0 ? 1u : 0u;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + col_o, pa + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
-                        kk > 0 ? 1u : acc0);
-          if constexpr (PROB) {
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_tf32_ts(tmem + col_ol, pa + 64u + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
+              mma_tf32_ts(tmem + col_o, pa + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
                           kk > 0 ? 1u : acc0);
+            if constexpr (PROB) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_tf32_ts(tmem + col_ol, pa + 64u + 8u * kk, dv + kstep_mnmajor(kk), idesc_o,
+                            kk > 0 ? 1u : acc0);
+            }
+            tc_commit(&bar.pv_done[r]);
+            if (h == 1) tc_commit(&bar.v_empty[s]);
           }
-          tc_commit(&bar.pv_done[r]);
-          if (h == 1) {
-            tc_commit(&bar.v_empty[s]);
-            ++vc;
-          }
+          __syncwarp();
+          if (h == 1) ++vc;
         }
-        if (!failed) tc_commit(&bar.o_full);
+        if (!failed) {
+          if (elect_one()) tc_commit(&bar.o_full);
+          __syncwarp();
+        }
       }
     }
   } else if (warp < kScoreWarp) {
@@ -406,7 +419,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       } else if constexpr (!V::SOFTMAX) {
         // one grid for every row and item: pairs (G_k, G_{k+1}), k = 0..K-1,
-        // computed with the CTA's first item and kept
+        // and the tail's zero pair at K, computed with the CTA's first item and
+        // kept
+        if (n == 0 && threadIdx.x == 64) sPair[p.K] = make_float2(0.0f, 0.0f);
         for (int k = (int)threadIdx.x - 64; k < p.K; k += kElemThreads) {
           if (n == 0) {
             const float G0 = grid_value(k, p.fwm_h), G1 = grid_value(k + 1, p.fwm_h);
@@ -480,7 +495,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (tab_in_smem) sweep2(GridF{sTab + r, KIA_TILE});
         else sweep2(GridF{st.table + grow * (p.K + 1), 1});
       } else {
-        sweep2(GridP{sPair});
+        sweep2(make_gridz(sPair, p.K));
       }
       if (failed) break;
       gbase += nkt + nunits;

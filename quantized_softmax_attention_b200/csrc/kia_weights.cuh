@@ -22,14 +22,16 @@ weights_from_S_kernel(const float* __restrict__ S, int rows, int cols,
                       const int* __restrict__ row_len, OpParams p, float* __restrict__ w,
                       int* __restrict__ bin, float* __restrict__ tout, float* __restrict__ row_m,
                       float* __restrict__ row_n) {
-  // FWM and the fixed step: the forward's per-CTA pairs (G_k, G_{k+1})
-  __shared__ float2 sPair[V::FWM ? KIA_MAX_KCAP : 1];
+  // FWM and the fixed step: the forward's per-CTA pairs (G_k, G_{k+1}) and
+  // the tail's zero pair at K
+  __shared__ float2 sPair[V::FWM ? KIA_MAX_KCAP + 1 : 1];
   // MinMax: one grid per row, as the forward's per-row table
   __shared__ float sTab[kWeightsWarps][V::MINMAX ? KIA_MAX_K + 1 : 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if constexpr (V::FWM) {
-    for (int k = (int)threadIdx.x; k < p.K; k += (int)blockDim.x)
-      sPair[k] = make_float2(grid_value(k, p.fwm_h), grid_value(k + 1, p.fwm_h));
+    for (int k = (int)threadIdx.x; k <= p.K; k += (int)blockDim.x)
+      sPair[k] = k < p.K ? make_float2(grid_value(k, p.fwm_h), grid_value(k + 1, p.fwm_h))
+                         : make_float2(0.0f, 0.0f);
     __syncthreads();
   }
   const int row = blockIdx.x * kWeightsWarps + warp;
@@ -80,7 +82,7 @@ weights_from_S_kernel(const float* __restrict__ S, int rows, int cols,
     }
   };
   if constexpr (V::MINMAX) run(GridF{sTab[warp], 1});
-  else run(GridP{sPair});
+  else run(make_gridz(sPair, p.K));
 }
 
 }  // namespace kia
