@@ -72,6 +72,50 @@ inline bool make_tmap(CUtensorMap* m, const float* base, int BH, int T, int d,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output map for the epilogues' TMA stores: [BH, T, d] fp32, box = 8
+// columns x 32 rows, no swizzle (a warp's staged block, row-major).  Rows past
+// T are not written.
+inline bool make_tmap_out(CUtensorMap* m, const float* base, int BH, int T, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)T * d * 4};
+  cuuint32_t box[3] = {8, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// One warp writes 32 rows x 8 columns of an output: each lane puts its row's
+// eight values (times `scale`) into the warp's 1 KB staging block, and one
+// elected lane stores the block with TMA at (x, y, z) -- the copy engine
+// writes whole lines, and no thread waits on global memory.  The block is
+// rewritten only after the previous store has read it.  The elected lane is
+// the same on every call (all lanes active), so its bulk groups cover every
+// store of the warp; epilogue_store_drain() waits for them before exit.
+__device__ __forceinline__ void epilogue_store8(float* stg, const CUtensorMap* tm,
+                                                const float* src8, float scale, int lane, int x,
+                                                int y, int z) {
+  if (elect_one()) tma_store_wait_read();
+  __syncwarp();
+  *reinterpret_cast<float4*>(stg + lane * 8) =
+      make_float4(src8[0] * scale, src8[1] * scale, src8[2] * scale, src8[3] * scale);
+  *reinterpret_cast<float4*>(stg + lane * 8 + 4) =
+      make_float4(src8[4] * scale, src8[5] * scale, src8[6] * scale, src8[7] * scale);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (elect_one()) {
+    tma_store_3d(tm, stg, x, y, z);
+    tma_store_commit();
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ void epilogue_store_drain() {
+  if (elect_one()) tma_store_wait_all();
+  __syncwarp();
+}
+
 // ------------------------------------------------------ descriptor helpers
 
 // K-major operand, 8-element (32-byte) K step ks of a tile at smem address

@@ -80,9 +80,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKmn,
                 const __grid_constant__ CUtensorMap tmV, const float* __restrict__ Kt,
-                const float* __restrict__ O, const float* __restrict__ dO, StatsView st,
-                WorkView wk, float* __restrict__ dQ, float* __restrict__ dS_dbg, OpParams p, int B,
-                int H, int T, int tab_in_smem) {
+                const float* __restrict__ O, const float* __restrict__ dO,
+                const __grid_constant__ CUtensorMap tmdQ, StatsView st, WorkView wk,
+                float* __restrict__ dS_dbg, OpParams p, int B, int H, int T, int tab_in_smem) {
   static_assert(D == 64, "tensor-core backward tiles are laid out for d = 64");
   constexpr uint32_t kTile = D * KIA_TILE * 4;
   // the stats must come from a forward of this shape and configuration
@@ -507,28 +507,14 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-      // this warp's 32 rows x 16 columns of dQ, 8 columns at a time through
-      // its staging block, so that each store writes 16 rows x 32 bytes
+      // this warp's 32 rows x 16 columns of dQ, 8 columns per TMA store
+      // through its staging block
       {
         float* stg = sStage + (warp - 2) * 256;
         const int row0 = qt * KIA_TILE + quad * 32;
 #pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-          const float* src = o + 8 * pass;
-          *reinterpret_cast<float4*>(stg + lane * 8) = make_float4(src[0], src[1], src[2], src[3]);
-          *reinterpret_cast<float4*>(stg + lane * 8 + 4) =
-              make_float4(src[4], src[5], src[6], src[7]);
-          __syncwarp();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int rl = 16 * h + (lane >> 1);
-            const float4 val = *reinterpret_cast<const float4*>(stg + rl * 8 + (lane & 1) * 4);
-            if (row0 + rl < T)
-              *reinterpret_cast<float4*>(dQ + (rowbase + row0 + rl) * D + col + 8 * pass +
-                                         (lane & 1) * 4) = val;
-          }
-          __syncwarp();
-        }
+        for (int pass = 0; pass < 2; ++pass)
+          epilogue_store8(stg, &tmdQ, o + 8 * pass, 1.0f, lane, (int)col + 8 * pass, row0, bh);
       }
       if (q < T && part == 0) {
         wk.gm[rowbase + q] = gm;
@@ -546,6 +532,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
     }
+    epilogue_store_drain();
   }
   if (failed || *abort) drain_in_flight();
   tc_fence_before();
@@ -560,8 +547,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQmn,
                  const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmGmn,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                 StatsView st, WorkView wk, float* __restrict__ dK, float* __restrict__ dV,
-                 OpParams p, int BH, int T, int tab_in_smem) {
+                 const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                 StatsView st, WorkView wk, OpParams p, int BH, int T, int tab_in_smem) {
   static_assert(D == 64, "tensor-core backward tiles are laid out for d = 64");
   constexpr uint32_t kTile = D * KIA_TILE * 4;
   if (*wk.status != 0) return;
@@ -1064,29 +1051,16 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_ld_wait_regs(v, g);
       tc_fence_before();
       mbar_arrive(&bar.acc_free);            // the accumulators are free for the next item
-      // this warp's 32 rows x 16 columns of dV and dK, 8 columns at a time
-      // through its staging block: each store instruction then writes 16
-      // rows x 32 contiguous bytes (whole sectors) instead of 32 rows x 16
+      // this warp's 32 rows x 16 columns of dV and dK, 8 columns per TMA
+      // store through its staging block
       float* stg = sStage + (warp - 2) * 256;
       const int row0 = kt * KIA_TILE + quad * 32;
 #pragma unroll
-      for (int pass = 0; pass < 4; ++pass) {
-        const float* src = (pass < 2 ? v : g) + 8 * (pass & 1);
-        float* out = pass < 2 ? dV : dK;
-        *reinterpret_cast<float4*>(stg + lane * 8) = make_float4(src[0], src[1], src[2], src[3]);
-        *reinterpret_cast<float4*>(stg + lane * 8 + 4) = make_float4(src[4], src[5], src[6], src[7]);
-        __syncwarp();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int rl = 16 * h + (lane >> 1);
-          const float4 val = *reinterpret_cast<const float4*>(stg + rl * 8 + (lane & 1) * 4);
-          if (row0 + rl < T)
-            *reinterpret_cast<float4*>(out + (rowbase + row0 + rl) * D + col + 8 * (pass & 1) +
-                                       (lane & 1) * 4) = val;
-        }
-        __syncwarp();
-      }
+      for (int pass = 0; pass < 4; ++pass)
+        epilogue_store8(stg, pass < 2 ? &tmdV : &tmdK, (pass < 2 ? v : g) + 8 * (pass & 1), 1.0f,
+                        lane, (int)col + 8 * (pass & 1), row0, item_bh(it));
     }
+    epilogue_store_drain();
   }
   if (failed || *abort) drain_in_flight();
   tc_fence_before();
@@ -1120,13 +1094,14 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
                   float* dV, float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
                   void (*mark)(int, cudaStream_t)) {
   const int BH = B * H;
-  CUtensorMap tq, tg, tk, tv, tqh, tqmh, tgh, tgmh, tkh, tkmh, tvh;
+  CUtensorMap tq, tg, tk, tv, tqh, tqmh, tgh, tgmh, tkh, tkmh, tvh, tdq, tdk, tdv;
   if (!make_tmap(&tq, Q, BH, T, D) || !make_tmap(&tg, dO, BH, T, D) ||
       !make_tmap(&tk, Kt, BH, T, D) || !make_tmap(&tv, Vv, BH, T, D) ||
       !make_tmap(&tqh, Q, BH, T, D, false, 64) || !make_tmap(&tqmh, Q, BH, T, D, true, 64) ||
       !make_tmap(&tgh, dO, BH, T, D, false, 64) || !make_tmap(&tgmh, dO, BH, T, D, true, 64) ||
       !make_tmap(&tkh, Kt, BH, T, D, false, 64) || !make_tmap(&tkmh, Kt, BH, T, D, true, 64) ||
-      !make_tmap(&tvh, Vv, BH, T, D, false, 64))
+      !make_tmap(&tvh, Vv, BH, T, D, false, 64) || !make_tmap_out(&tdq, dQ, BH, T, D) ||
+      !make_tmap_out(&tdk, dK, BH, T, D) || !make_tmap_out(&tdv, dV, BH, T, D))
     return KIA_ERR_CUDA;
   const bool q_tab_smem = tc_bwd_q_smem<D>(p, true) <= 232448;
   const size_t smq = tc_bwd_q_smem<D>(p, q_tab_smem);
@@ -1145,14 +1120,14 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
     tc_bwd_q_kernel<D, V, true><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
-                                                              st, wk, dQ, dS_dbg, p, B, H, T,
+                                                              tdq, st, wk, dS_dbg, p, B, H, T,
                                                               q_tab_smem ? 1 : 0);
   } else {
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
     tc_bwd_q_kernel<D, V, false><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
-                                                               st, wk, dQ, dS_dbg, p, B, H, T,
+                                                               tdq, st, wk, dS_dbg, p, B, H, T,
                                                                q_tab_smem ? 1 : 0);
   }
   if (cudaGetLastError() != cudaSuccess) return KIA_ERR_CUDA;
@@ -1161,7 +1136,7 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk) !=
         cudaSuccess)
       return KIA_ERR_CUDA;
-    kern<<<qgrid, kTcThreads, smk, s>>>(tqh, tqmh, tgh, tgmh, tk, tv, st, wk, dK, dV, p, BH, T,
+    kern<<<qgrid, kTcThreads, smk, s>>>(tqh, tqmh, tgh, tgmh, tk, tv, tdk, tdv, st, wk, p, BH, T,
                                         kv_tab_smem ? 1 : 0);
     return KIA_OK;
   };

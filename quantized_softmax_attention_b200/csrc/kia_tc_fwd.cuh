@@ -86,8 +86,9 @@ struct FwdRowX {
 template <int D, class V>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, StatsView st,
-              OpParams p, int B, int H, int T, int tab_in_smem) {
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const __grid_constant__ CUtensorMap tmOL, StatsView st, OpParams p, int B, int H,
+              int T, int tab_in_smem) {
   constexpr bool PROB = V::PROB;
   using Cfg = FwdCfg<D, PROB>;
   constexpr int NSK = Cfg::kKStages, NSV = Cfg::kVStages, R = Cfg::kRegions;
@@ -525,9 +526,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_before();
       mbar_arrive(&bar.o_free);
       {
+        // this warp's 32 rows x D/4 columns of O (and O_L), 8 columns per TMA
+        // store through its staging block
         float* stg = sStage + (warp - 2) * 256;
         const int row0 = qt * KIA_TILE + quad * 32;
-        const long long rb = (long long)bh * T;
         const float rw = __frcp_rn(Wrow), rwl = __frcp_rn(WLrow);
 #pragma unroll
         for (int pass = 0; pass < (PROB ? 2 : 1) * kCols / 8; ++pass) {
@@ -535,22 +537,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           const bool second = PROB && pass >= kPer;
           const int cp = second ? pass - kPer : pass;
           const float* src = ((PROB && second) ? ol : o) + 8 * cp;
-          const float sc = second ? rwl : rw;
-          float* out = second ? st.OL : O;
-          *reinterpret_cast<float4*>(stg + lane * 8) =
-              make_float4(src[0] * sc, src[1] * sc, src[2] * sc, src[3] * sc);
-          *reinterpret_cast<float4*>(stg + lane * 8 + 4) =
-              make_float4(src[4] * sc, src[5] * sc, src[6] * sc, src[7] * sc);
-          __syncwarp();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int rl = 16 * h + (lane >> 1);
-            const float4 val = *reinterpret_cast<const float4*>(stg + rl * 8 + (lane & 1) * 4);
-            if (row0 + rl < T)
-              *reinterpret_cast<float4*>(out + (rb + row0 + rl) * D + col + 8 * cp +
-                                         (lane & 1) * 4) = val;
-          }
-          __syncwarp();
+          epilogue_store8(stg, second ? &tmOL : &tmO, src, second ? rwl : rw, lane,
+                          (int)col + 8 * cp, row0, bh);
         }
       }
       if (qrow < T && part == 0) {
@@ -565,6 +553,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       if (bh == 0 && qt == nt - 1 && threadIdx.x == 64) write_header(st.header, B, H, T, D, p);
     }
+    epilogue_store_drain();
   }
   if (failed || *abort) drain_in_flight();
   tc_fence_before();
@@ -583,8 +572,9 @@ size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem) {
 }
 
 template <int D, class V>
-int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, float* O,
-                 const StatsView& st, int B, int H, int T, const OpParams& p, cudaStream_t s) {
+int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const CUtensorMap& to, const CUtensorMap& tol, const StatsView& st, int B, int H,
+                 int T, const OpParams& p, cudaStream_t s) {
   bool tab_in_smem = true;
   size_t smem = tc_fwd_smem<D, V::PROB>(p, true);
   if (smem > 232448) {
@@ -600,7 +590,7 @@ int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   const int sms = num_sms();
   if (sms <= 0) return KIA_ERR_CUDA;
   const dim3 grid(std::min(sms, B * H * nt));
-  tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, O, st, p, B, H, T,
+  tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, to, tol, st, p, B, H, T,
                                                      tab_in_smem ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
 }
@@ -633,12 +623,13 @@ int tc_forward(const float* Q, const float* Kt, const float* V, float* O, void* 
                int H, int T, const OpParams& p, cudaStream_t s) {
   const long long rows = (long long)B * H * T;
   StatsView st = stats_view(stats, rows, D, p);
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to, tol;
   if (!make_tmap(&tq, Q, B * H, T, D) || !make_tmap(&tk, Kt, B * H, T, D) ||
-      !make_tmap(&tv, V, B * H, T, D, /*mn_major=*/true))
+      !make_tmap(&tv, V, B * H, T, D, /*mn_major=*/true) || !make_tmap_out(&to, O, B * H, T, D) ||
+      !make_tmap_out(&tol, st.OL ? st.OL : O, B * H, T, D))
     return KIA_ERR_CUDA;
   return dispatch_variant(p, [&]<class Vt>() {
-    return tc_forward_v<D, Vt>(tq, tk, tv, O, st, B, H, T, p, s);
+    return tc_forward_v<D, Vt>(tq, tk, tv, to, tol, st, B, H, T, p, s);
   });
 }
 
