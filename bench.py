@@ -56,10 +56,11 @@ def parse():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--diag", default=None, choices=["geometry", "decomposition"],
                     help="time one of the diagnostic row kernels instead of the step")
-    ap.add_argument("--matrix", default=None, choices=["variants", "sweep"],
+    ap.add_argument("--matrix", default=None, choices=["variants", "sweep", "one_b"],
                     help="one JSON line per operator variant (every calibration x "
-                         "reconstruction x surrogate x gradient mode at the 124M shape) or per "
-                         "point of the B16 H12 T 1024-4096 throughput sweep")
+                         "reconstruction x surrogate x gradient mode at the 124M shape), per "
+                         "point of the B16 H12 T 1024-4096 throughput sweep, or per gradient "
+                         "mode of the 1B-style shape from one shared forward (FWM and MinMax)")
     return ap.parse_args()
 
 
@@ -469,6 +470,62 @@ def diag_main(args):
 
 # ------------------------------------------------------ variant matrices
 
+def one_b_main(args):
+    """The 1B-style configuration B4 H16 T2048 d128, LERP K = 32: for FWM and
+    for MinMax one forward, timed on its own, then the five backward modes
+    from that forward's stats, each timed on its own; one JSON line per
+    (calibration, mode) with the step rate (forward + that backward, 8U)."""
+    import torch
+    from quantized_softmax_attention_b200 import kiattn as K
+    from quantized_softmax_attention_b200 import workloads as W
+    torch.cuda.set_device(0)
+    peak, (src, _, _) = tf32_peak()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        err = K.kiattn_device_error(True)
+        if err != 0:
+            raise RuntimeError(f"device error word {err}")
+        return sum(a.elapsed_time(b) for a, b in ev) / args.steps
+
+    for cal in (W.CAL_FWM, W.CAL_MINMAX):
+        w = W.one_b(cal=cal)
+        q, k, v, g = (x.cuda() for x in W.make_inputs(w))
+        cfg = lib_config(w, K)
+        bufs = K.Buffers(w.B, w.H, w.T, w.d, cfg)
+        t_fwd = timed(lambda: K.kiattn_fwd(q, k, v, bufs.O, bufs.stats, cfg))
+        K.kiattn_fwd(q, k, v, bufs.O, bufs.stats, cfg)
+        U = gemm_units(w)
+        for grad in range(5):
+            c = cfg.replace(grad=grad)
+            t_bwd = timed(lambda: K.kiattn_bwd(q, k, v, bufs.O, g, bufs.stats, bufs.dQ, bufs.dK,
+                                               bufs.dV, bufs.work, c))
+            tf = algorithmic_flops(w) / ((t_fwd + t_bwd) * 1e-3) / 1e12
+            cd = {**config_dict(W.Workload(**{**w.__dict__, "grad": grad}), 1),
+                  "forward": "one forward shared by the five modes"}
+            print(json.dumps({"matrix": "one_b", "config": cd, "value": tf, "unit": "TFLOP/s",
+                              "ms_fwd": t_fwd, "ms_bwd": t_bwd, "ms_per_step": t_fwd + t_bwd,
+                              "fwd_tflops": 3 * U / (t_fwd * 1e-3) / 1e12,
+                              "bwd_tflops": 5 * U / (t_bwd * 1e-3) / 1e12,
+                              "frac_of_tf32_roofline": tf / peak, "peak": peak,
+                              "peak_source": src, "steps": args.steps, "warmup": args.warmup}),
+                  flush=True)
+        del bufs, q, k, v, g
+
+
 def matrix_main(args):
     """Fwd+bwd throughput over a matrix of operator variants: `variants` runs
     the 124M span-ladder inputs under every calibration x reconstruction x
@@ -548,6 +605,9 @@ def main():
     if args.diag:
         diag_main(args)
         return
+    if args.matrix == "one_b":
+        one_b_main(args)
+        return
     if args.matrix:
         matrix_main(args)
         return
@@ -579,9 +639,8 @@ def main():
         K.kiattn_bwd(q, k, v, bufs.O, g, bufs.stats, bufs.dQ, bufs.dK, bufs.dV, bufs.work, cfg)
 
     # our kernels per step: the forward, then the tensor-core backward's query
-    # and key passes (d = 64) or the exact backward's four row and tile
-    # kernels (d = 128), plus the projection's scan
-    launches_per_step = 1 + (2 if w.d == 64 else 4) + (1 if w.grad == K.GRAD_PROJECT else 0)
+    # and key passes, plus the projection's scan
+    launches_per_step = 3 + (1 if w.grad == K.GRAD_PROJECT else 0)
     for _ in range(args.warmup):
         flush.zero_()
         step()

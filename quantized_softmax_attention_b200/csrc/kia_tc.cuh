@@ -300,3 +300,4 @@ int tc_backward(const float* Q, const float* Kt, const float* V, const float* O,
 
 #include "kia_tc_fwd.cuh"
 #include "kia_tc_bwd.cuh"
+#include "kia_tc_bwd128.cuh"

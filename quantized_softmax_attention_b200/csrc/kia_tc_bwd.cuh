@@ -1147,19 +1147,4 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
   return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
 }
 
-template <int D>
-int tc_backward(const float* Q, const float* Kt, const float* V, const float* O, const float* dO,
-                const StatsView& st, const WorkView& wk, float* dQ, float* dK, float* dV,
-                float* dS_dbg, int B, int H, int T, const OpParams& p, cudaStream_t s,
-                void (*mark)(int, cudaStream_t)) {
-  if constexpr (D != 64) {
-    return KIA_ERR_UNSUPPORTED;
-  } else {
-    return dispatch_variant(p, [&]<class Vt>() {
-      return tc_backward_v<D, Vt>(Q, Kt, V, O, dO, st, wk, dQ, dK, dV, dS_dbg, B, H, T, p, s,
-                                  mark);
-    });
-  }
-}
-
 }  // namespace kia

@@ -209,7 +209,7 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
   const bool tc = gemm == KIA_GEMM_TF32;
   prof_mark(2, s);
   int rc;
-  if (tc && D == 64) {
+  if (tc) {
     // query pass (checks the stats, centering, dQ with its calibration terms),
     // key pass (dK with the calibration terms folded into dS, dV)
     prof_mark(3, s);
@@ -224,8 +224,7 @@ int backward(const float* Q, const float* Kt, const float* V, const float* O, co
     prof_mark(6, s);
     return KIA_OK;
   }
-  // exact-fp32 kernels (and the d = 128 backward in TF32 mode, with the
-  // tensor cores' operand truncation so it sees the TF32 forward's arithmetic)
+  // exact-fp32 kernels
   rc = backward_rows<D>(Q, Kt, O, dO, st, wk, dQ, dK, dS_dbg, B, H, T, p, s, true, nullptr);
   if (rc) return rc;
   prof_mark(3, s);

@@ -252,15 +252,19 @@ def test_tc_forward_bitwise_identical_across_modes_and_surrogates():
             np.testing.assert_array_equal(o.view(np.uint32), outs[0].view(np.uint32))
 
 
-def test_tc_d128_forward_and_backward():
-    Q, Kt, V, dO = _inputs(1, 2, 256, 128, 43)
-    for cal, (rec, ste) in itertools.product((K.CAL_MINMAX, K.CAL_FWM), RECSTE):
-        cfg = K.Config(K=32, cal=cal, rec=rec, ste=ste)
+@pytest.mark.parametrize("T", [256, 200])
+def test_tc_d128_forward_and_backward(T):
+    """d = 128 on the tensor cores, forward and both backward passes: every
+    calibration x reconstruction x surrogate, every gradient mode, a ragged
+    tail; per-row zero sums for the zero-sum modes."""
+    Q, Kt, V, dO = _inputs(1, 2, T, 128, 43)
+    for cal, (rec, ste), grad in itertools.product((K.CAL_MINMAX, K.CAL_FWM, K.CAL_FIXED), RECSTE, MODES):
+        cfg = K.Config(K=32 if cal != K.CAL_FIXED else 4, cal=cal, rec=rec, ste=ste, grad=grad)
         errs, _, _ = compare(Q, Kt, V, dO, cfg, TF32_RULE, 2e-3, 1e-4)
-        assert errs["O"] < 2e-3, errs
-        # the d = 128 backward runs the exact-fp32 kernels on the TF32 forward
-        for name in ("dQ", "dK", "dV"):
-            assert errs[name] < 2e-3, (cal, rec, ste, errs)
+        for name in ("O", "dQ", "dK", "dV", "dS"):
+            assert errs[name] < 2e-3, (cal, rec, ste, grad, errs)
+        if grad in (K.GRAD_FULL, K.GRAD_PROJECT):
+            assert errs["zero_sum"] < 1e-5, errs
 
 
 # ---------------------------------------- fixed-upstream decomposition
