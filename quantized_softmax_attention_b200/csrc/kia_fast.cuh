@@ -122,12 +122,18 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return upk(r);
 }
 
-// Forward weights of two neighbouring scores at once (same arithmetic as
-// fwd_weights, paired).  wf2 / wl2 as in fwd_weights.
+// Forward weights of two scores at once: the same arithmetic as fwd_weights,
+// each half of every packed operation an ordinary IEEE operation, so the
+// weights, bins and t are bit-identical to fwd_weights' on each score.
+// wf2 / wl2 as in fwd_weights; returns both grid positions.
+struct Pos2 {
+  Pos a, b;
+};
 template <class V, bool CLAMP0, class G>
-__device__ __forceinline__ void fwd_weights2(const G& grid, float m, float rh, float Kf,
+__device__ __forceinline__ Pos2 fwd_weights2(const G& grid, float m, float rh, float Kf,
                                              float Km1f, float s0, float s1, float2& wf2,
                                              float2& wl2) {
+  Pos2 ps{};
   if constexpr (V::SOFTMAX) {
     wf2 = make_float2(round_exp<V::EXPR>(expf(s0 - m)), round_exp<V::EXPR>(expf(s1 - m)));
     wl2 = wf2;
@@ -140,8 +146,15 @@ __device__ __forceinline__ void fwd_weights2(const G& grid, float m, float rh, f
     const float2 tmp = add2_rd(uc, mg);
     const float2 kf = sub2(tmp, mg);
     const float2 t = sub2(u, kf);
-    const float2 g0 = grid.pair(__float_as_int(tmp.x) - kMagicBits);
-    const float2 g1 = grid.pair(__float_as_int(tmp.y) - kMagicBits);
+    const int k0 = __float_as_int(tmp.x) - kMagicBits, k1 = __float_as_int(tmp.y) - kMagicBits;
+    float2 g0, g1;
+    if constexpr (kZeroTail<G>) {
+      g0 = grid.at(k0, V::FWM && u.x > Kf);
+      g1 = grid.at(k1, V::FWM && u.y > Kf);
+    } else {
+      g0 = grid.pair(k0);
+      g1 = grid.pair(k1);
+    }
     const float2 lo = make_float2(g0.x, g1.x), hi = make_float2(g0.y, g1.y);
     const float2 lerp = fma2(t, sub2(hi, lo), lo);
     if constexpr (V::NEAREST) {
@@ -151,12 +164,15 @@ __device__ __forceinline__ void fwd_weights2(const G& grid, float m, float rh, f
       wf2 = lerp;
       wl2 = lerp;
     }
-    if constexpr (V::FWM) {
+    if constexpr (V::FWM && !kZeroTail<G>) {
       const bool t0 = u.x > Kf, t1 = u.y > Kf;
       wf2 = make_float2(t0 ? 0.0f : wf2.x, t1 ? 0.0f : wf2.y);
       wl2 = make_float2(t0 ? 0.0f : wl2.x, t1 ? 0.0f : wl2.y);
     }
+    ps.a = Pos{u.x, t.x, kf.x, k0};
+    ps.b = Pos{u.y, t.y, kf.y, k1};
   }
+  return ps;
 }
 
 // Forward weights: wf (forward probabilities' numerator) and wl (LERP

@@ -178,7 +178,7 @@ tc_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   ScoresSmem<D>& sm = *reinterpret_cast<ScoresSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int qt = blockIdx.x, kt = blockIdx.y, bh = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int row = qt * KIA_TILE + threadIdx.x;
   const bool skip = p.causal && kt > qt;
   if (skip) {

@@ -12,21 +12,23 @@
 //    S^T, dP^T recomputed; P = w_fwd / W_fwd; dS^T as above
 //    dV_j += P^T dO_i,  dK_j += dS^T Q_i          (A operands from TMEM)
 //
-// Both passes stream the other side in half tiles of 64 rows through two
-// TMEM buffers, so the MMAs of the next half tile run while the element
-// warps work on the current one.  Each output row is owned by one CTA and
-// written once: no atomics.  The query pass also computes the centering D
-// of its rows and, once its row sums are complete, the calibration terms
-// (section 3, Calibration gradients; Appendix B): g_m at the argmax key and
-// g_n at the argmin key (or the zero-sum projection's shift), added to dQ
-// there and folded into dS^T by the key pass before its dK contraction.
+// Both passes stream the other side in half tiles of 64 rows through three
+// rotating TMEM regions, so the MMAs of the next half tiles run while the
+// element warps work on the current one.  Each output row is owned by one
+// CTA and written once: no atomics.  The query pass also computes the
+// centering D of its rows and, once its row sums are complete, the
+// calibration terms (section 3, Calibration gradients; Appendix B): g_m at
+// the argmax key and g_n at the argmin key (or the zero-sum projection's
+// shift), added to dQ there and folded into dS^T by the key pass before its
+// dK contraction.
 // Warp roles (20 warps): 0 = TMA producer, 1 = issuer of the accumulating
 // MMAs (dQ, or dV and dK) and TMEM owner, 18 = issuer of the score MMAs
-// (S and dP), 19 = spare, 2..17 = element warps in two groups of eight: group g works on the half
-// tiles u with u % 2 == g (TMEM buffer g), so the two groups run out of
-// phase and one computes while the other waits for its operands.  Warp w
-// reaches TMEM lanes 32*(w%4)..+31; the two warps of a group that share
-// those lanes split a half tile's 64 columns.
+// (S and dP), 19 = spare (query pass) or the per-query constant producer
+// (key pass), 2..17 = element warps, all sixteen on every half tile: warp w
+// reaches TMEM lanes 32*(w%4)..+31, and the four warps that share those
+// lanes take 16 of the half tile's 64 columns each.  (Two groups taking
+// alternate half tiles left one group idle at the end of every item while
+// the other finished its last half tile.)
 #pragma once
 #include <algorithm>
 #include <type_traits>
@@ -69,6 +71,7 @@ struct BwdKBars {
   uint64_t st_free[3];            // dV, dK MMAs of region r done
   uint64_t acc_full;              // all dV, dK MMAs of an item done
   uint64_t acc_free;              // the item's dV, dK read out of TMEM
+  uint64_t acc_issued;            // the item's last dV, dK MMAs issued
   uint32_t tmem_base;
   int abort;
 };
@@ -136,7 +139,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&bar.sp_full[b], 1);
-      mbar_init(&bar.elem_done[b], kGroupThreads);
+      mbar_init(&bar.elem_done[b], kElemThreads);
       mbar_init(&bar.st_free[b], 1);
     }
     mbar_init(&bar.dq_full, 1);
@@ -309,9 +312,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;       // 0..3: (group, half of a unit)
-    const int grp = part >> 1;              // half tiles u with u % 2 == grp
-    const int sub = part & 1;               // columns 32 sub .. 32 sub + 31 of a unit
+    const int part = (warp - 2) >> 2;       // 0..3: columns 16 part .. +15 of every unit
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
@@ -381,19 +382,18 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // loads of the element loop are shared-memory loads when the grid is
       // in shared memory (a runtime choice of pointer makes them generic)
       auto unit_loop = [&](const auto& grid) {
-      for (int u = grp; u < nunits && !failed; u += 2) {
+      for (int u = 0; u < nunits && !failed; ++u) {
         const int j = u >> 1, gu = gbase + u, rg = gu % R;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (gu / R) & 1, abort))) { failed = true; break; }
         tc_fence_after();
         const bool edge = (p.causal && j == qt) || (j + 1) * KIA_TILE > T;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        {
           float v[16], g[16];
-          const uint32_t cs = 128u * rg + 32u * sub + 16u * c;    // 16 columns of S
+          const uint32_t cs = 128u * rg + 16u * part;    // this thread's 16 columns of S
           tmem_ld16(tmem + lane_addr + cs, v);
           tmem_ld16(tmem + lane_addr + cs + 64u, g);
           tmem_ld_wait_regs(v, g);
-          const int key0 = j * KIA_TILE + 64 * grp + 32 * sub + 16 * c;
+          const int key0 = 64 * u + 16 * part;
           if (!edge) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -457,6 +457,22 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
+      // this thread's columns of the key rows of the row's calibration terms
+      // (argmax, argmin), loaded now so that their latency passes during the
+      // waits below
+      constexpr int kCols = D / kRowSplit;   // 16
+      const uint32_t col = (uint32_t)(part * kCols);
+      float4 ka4[kCols / 4], kn4[V::MINMAX ? kCols / 4 : 1];
+      {
+        const float4* k4 = reinterpret_cast<const float4*>(Kt + (rowbase + am) * D + col);
+#pragma unroll
+        for (int i = 0; i < kCols / 4; ++i) ka4[i] = k4[i];
+        if constexpr (V::MINMAX) {
+          const float4* n4 = reinterpret_cast<const float4*>(Kt + (rowbase + an) * D + col);
+#pragma unroll
+          for (int i = 0; i < kCols / 4; ++i) kn4[i] = n4[i];
+        }
+      }
       // row sums of the four column groups
       sAC[(part * 2 + 0) * KIA_TILE + r] = A;
       sAC[(part * 2 + 1) * KIA_TILE + r] = C;
@@ -466,8 +482,6 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tc_fence_after();
       // this thread's 16 columns of dQ, then the accumulator is free for the
       // next item
-      constexpr int kCols = D / kRowSplit;   // 16
-      const uint32_t col = (uint32_t)(part * kCols);
       float o[kCols];
       tmem_ld16(tmem + lane_addr + kColDQ + col, o);
       tmem_ld_wait_regs(o);
@@ -485,10 +499,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float gmq = proj ? 0.0f : gm;   // the projection shift is applied by the scan pass
       if (q < T) {
         if (gmq != 0.0f) {
-          const float4* k4 = reinterpret_cast<const float4*>(Kt + (rowbase + am) * D + col);
 #pragma unroll
           for (int i = 0; i < kCols / 4; ++i) {
-            const float4 kk = k4[i];
+            const float4 kk = ka4[i];
             o[4 * i] = fmaf(gmq, kk.x, o[4 * i]);
             o[4 * i + 1] = fmaf(gmq, kk.y, o[4 * i + 1]);
             o[4 * i + 2] = fmaf(gmq, kk.z, o[4 * i + 2]);
@@ -496,10 +509,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
         if (V::MINMAX && gn != 0.0f) {
-          const float4* k4 = reinterpret_cast<const float4*>(Kt + (rowbase + an) * D + col);
 #pragma unroll
           for (int i = 0; i < kCols / 4; ++i) {
-            const float4 kk = k4[i];
+            const float4 kk = kn4[V::MINMAX ? i : 0];
             o[4 * i] = fmaf(gn, kk.x, o[4 * i]);
             o[4 * i + 1] = fmaf(gn, kk.y, o[4 * i + 1]);
             o[4 * i + 2] = fmaf(gn, kk.z, o[4 * i + 2]);
@@ -607,15 +619,16 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&bar.sp_full[b], 1);
-      mbar_init(&bar.elem_done[b], kGroupThreads);
+      mbar_init(&bar.elem_done[b], kElemThreads);
       mbar_init(&bar.st_free[b], 1);
     }
     for (int sl = 0; sl < 4; ++sl) {
       mbar_init(&bar.qc_ready[sl], 32);
-      mbar_init(&bar.qc_free[sl], kGroupThreads);
+      mbar_init(&bar.qc_free[sl], kElemThreads);
     }
     mbar_init(&bar.acc_full, 1);
     mbar_init(&bar.acc_free, kElemThreads);
+    mbar_init(&bar.acc_issued, 1);
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -711,6 +724,10 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       ItemSeq seq(nitems);
       for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
         if (!warp_wait(&bar.kv_full, n & 1, abort)) { failed = true; break; }
+        // the previous item's last dV / dK MMAs go into the tensor pipe ahead
+        // of this item's: the element warps wait for them before their
+        // epilogue, while this item's first scores can wait
+        if (n > 0 && !warp_wait(&bar.acc_issued, (n - 1) & 1, abort)) { failed = true; break; }
         // S^T, dP^T of half tile u (queries 64 (2 q0 + u)..) into region
         // g % R, once the dV / dK MMAs of half tile g - R have released it
         const int nunits = item_units(it);
@@ -783,7 +800,10 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           __syncwarp();
         }
         if (!failed) {
-          if (elect_one()) tc_commit(&bar.acc_full);
+          if (elect_one()) {
+            tc_commit(&bar.acc_full);
+            mbar_arrive(&bar.acc_issued);
+          }
           __syncwarp();
         }
       }
@@ -805,7 +825,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // raw per-query values of one unit (lane l: queries l and l + 32), loaded
     // one unit ahead so that their latency overlaps the wait for a free slot
     struct Raw {
-      float m[2], rh[2], D[2], Wb[2], Wf[2], gm[2], gn[2];
+      float m[2], rh[2], dl[2], Wb[2], Wf[2], gm[2], gn[2];   // dl: the row's D
       int am[2], an[2];
     };
     auto load_raw = [&](int it, int u, Raw& x) {
@@ -816,7 +836,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const long long qr = rowbase + (q < T ? q : T - 1);
         x.m[hq] = st.m[qr];
         x.rh[hq] = st.rh[qr];
-        x.D[hq] = wk.D[qr];
+        x.dl[hq] = wk.D[qr];
         x.Wb[hq] = st.Wb[qr];
         x.Wf[hq] = st.Wf[qr];
         x.gm[hq] = wk.gm[qr];
@@ -830,7 +850,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     int it = cseq.next(), u = 0;
     if (it >= 0) load_raw(it, 0, cur);
     for (int g = 0; it >= 0 && !failed; ++g) {
-      const int sl = 2 * (g & 1) + ((g >> 1) & 1);
+      const int sl = g & 3;
       // the next half tile (possibly of the next item)
       int it2 = it, u2 = u + 1;
       if (u2 == item_units(it)) { u2 = 0; it2 = cseq.next(); }
@@ -848,7 +868,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int e = sl * kSlotQ + 32 * hq + lane;          // its slot entry
         const int Lq = p.causal ? q + 1 : T;
         const float rWb = Lq == 1 ? 0.0f : __fdiv_rn(1.0f, cur.Wb[hq]);
-        const float nD = -cur.D[hq] * rWb;       // dw = dP rWb + nD
+        const float nD = -cur.dl[hq] * rWb;       // dw = dP rWb + nD
         const float nrh = V::SOFTMAX ? 1.0f : -cur.rh[hq];
         sC4[e] = make_float4(cur.m[hq], rWb * nrh, nD * nrh, __fdiv_rn(1.0f, cur.Wf[hq]));
         // calibration terms of the query's row, added to dS^T before dK:
@@ -913,9 +933,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;        // 0..3: (group, half of a unit)
-    const int grp = part >> 1;               // half tiles u with u % 2 == grp
-    const int sub = part & 1;                // query columns 32 sub .. 32 sub + 31 of a unit
+    const int part = (warp - 2) >> 2;        // 0..3: query columns 16 part .. +15 of every unit
+    const int grp = part >> 1;               // which copy of the FWM grid pairs this warp reads
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
@@ -931,29 +950,28 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const int kt = item_kt(it), q0 = item_q0(it), nunits = item_units(it);
       const int kj = kt * KIA_TILE + r;
       const long long rowbase = (long long)item_bh(it) * T;
-      for (int u = grp; u < nunits && !failed; u += 2) {
+      for (int u = 0; u < nunits && !failed; ++u) {
         const int gu = gbase + u;
         const int qi = q0 + (u >> 1);
         const int rg = gu % R;
-        const int sl = 2 * grp + ((gu >> 1) & 1);           // this unit's constant slot
+        const int sl = gu & 3;                               // this unit's constant slot
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[sl], (gu >> 2) & 1, abort))) { failed = true; break; }
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (gu / R) & 1, abort))) { failed = true; break; }
         tc_fence_after();
         const bool edge =
             (p.causal && qi == kt) || (qi + 1) * KIA_TILE > T || (kt + 1) * KIA_TILE > T;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        {
           float v[16], g[16];
-          const uint32_t cs = 128u * rg + 32u * sub + 16u * c;
+          const uint32_t cs = 128u * rg + 16u * part;        // this thread's 16 query columns
           tmem_ld16(tmem + lane_addr + cs, v);
           tmem_ld16(tmem + lane_addr + cs + 64u, g);
           tmem_ld_wait_regs(v, g);
-          const int ql0 = 64 * (u & 1) + 32 * sub + 16 * c;   // first query (in the tile) of the chunk
-          const int e0 = sl * kSlotQ + 32 * sub + 16 * c;     // its slot entry
+          const int ql0 = 64 * (u & 1) + 16 * part;   // first query (in the tile) of the chunk
+          const int e0 = sl * kSlotQ + 16 * part;     // its slot entry
           // the element loop, without the mask test on units with no masked pair
           auto body = [&](auto edge_c, auto tabs_c) {
             constexpr bool EDGE = decltype(edge_c)::value;
-            constexpr bool TABS = decltype(tabs_c)::value;   // per-query grids in shared memory
+            [[maybe_unused]] constexpr bool TABS = decltype(tabs_c)::value;   // per-query grids in shared memory
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int ql = ql0 + i;
@@ -1015,10 +1033,10 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           if constexpr (!PROJ && !V::SOFTMAX) {
             // the chunk's queries whose argmax (argmin) key lies in this warp's
             // 32 keys: a warp-uniform test, the per-element work only for them
-            const int sh = 16 * c;
-            const uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu;
+            const int hq = part >> 1, sh = 16 * (part & 1);
+            const uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
             const uint32_t bn =
-                V::MINMAX ? (sMask[((sl * 2 + 1) * 4 + quad) * 2 + sub] >> sh) & 0xFFFFu : 0u;
+                V::MINMAX ? (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu : 0u;
             if ((bm | bn) != 0u) {
 #pragma unroll
               for (int i = 0; i < 16; ++i) {

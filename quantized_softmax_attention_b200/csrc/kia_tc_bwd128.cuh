@@ -454,6 +454,7 @@ struct BwdKV128Bars {
   uint64_t elem_done;              // P^T, dS^T written over S^T, dP^T
   uint64_t st_free;                // the unit's dV, dK MMAs done: region free
   uint64_t acc_full, acc_free;
+  uint64_t acc_issued;             // the item's last dV, dK MMAs issued
   uint32_t tmem_base;
   int abort;
 };
@@ -513,6 +514,7 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     mbar_init(&bar.st_free, 1);
     mbar_init(&bar.acc_full, 1);
     mbar_init(&bar.acc_free, kElemThreads);
+    mbar_init(&bar.acc_issued, 1);
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -595,6 +597,8 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       if (!warp_wait(&bar.k_ready, n & 1, abort)) { failed = true; break; }
       if (!warp_wait(&bar.v_full, n & 1, abort)) { failed = true; break; }
+      // the previous item's last dV / dK MMAs ahead of this item's scores
+      if (n > 0 && !warp_wait(&bar.acc_issued, (n - 1) & 1, abort)) { failed = true; break; }
       const int nunits = item_units(it);
       for (int u = 0; u < nunits; ++u, ++g) {
         if (g > 0 && !warp_wait(&bar.st_free, (g - 1) & 1, abort)) { failed = true; break; }
@@ -651,7 +655,10 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncwarp();
       }
       if (failed) break;
-      if (elect_one()) tc_commit(&bar.acc_full);
+      if (elect_one()) {
+        tc_commit(&bar.acc_full);
+        mbar_arrive(&bar.acc_issued);
+      }
       __syncwarp();
     }
   } else if (warp == kScoreWarp + 1) {

@@ -13,23 +13,21 @@
 //            operand of O += P V (and P_L for Prob-STE, O_L += P_L V);
 //   epilogue: O = O_acc / W (and O_L = O_L_acc / W_L), per-row statistics.
 //
-// Both sweeps walk the keys in units of 64 (half key tiles), numbered
-// across the two sweeps.  Unit U lives in TMEM region U % R (S / P in its
-// first 64 columns, P_L in the next 64; R = 3 regions where the
-// accumulators leave room), so the scores of the next units are computed
-// while the current ones are turned into weights and multiplied into O.
+// Sweep 1 walks the keys in whole key tiles (N = 128 MMAs), sweep 2 in
+// units of 64 (half key tiles); units are numbered across both sweeps, and
+// unit U lives in TMEM region U % R (S / P in its first 64 columns, P_L in
+// the next 64; R = 3 regions where the accumulators leave room), so the
+// scores of the next units are computed while the current ones are turned
+// into weights and multiplied into O.
 // Warp roles (20 warps): 0 = TMA producer, 1 = issuer of the accumulating
 // MMAs (O += P V, O_L += P_L V) and TMEM owner, 18 = issuer of the score
-// MMAs (S = Q K^T) -- two issuing threads on different SM sub-partitions,
-// because one thread alone spends more time on commits and waits than the
-// tensor core spends on the MMAs -- 19 = spare, 2..17 = element warps in two
-// groups of eight; group g takes the units with U % 2 == g, so the two
-// groups run half a unit out of phase.  Element warp
-// w reaches TMEM lanes 32*(w%4)..+31 (query rows); in each group two warps
-// share those rows and split a unit's 64 columns, so each query row is
-// served by four threads (two per group) whose row statistics are merged
-// through shared memory.  O and O_L leave through shared memory and TMA
-// stores.
+// MMAs (S = Q K^T) -- two issuing warps, each running its loop converged
+// with one elected lane issuing -- 19 = spare, 2..17 = element warps, all
+// sixteen on every unit: warp w reaches TMEM lanes 32*(w%4)..+31 (query
+// rows), and the four warps that share those rows take a quarter of each
+// unit's columns, so each query row is served by four threads whose row
+// statistics are merged through shared memory.  O and O_L leave through
+// shared memory and TMA stores.
 #pragma once
 #include <algorithm>
 
@@ -40,7 +38,6 @@ namespace kia {
 
 constexpr int kRowSplit = 4;        // element threads per TMEM lane (row)
 constexpr int kElemThreads = 128 * kRowSplit;   // 16 element warps (warps 2..17)
-constexpr int kGroupThreads = kElemThreads / 2; // element threads of one group
 constexpr int kScoreWarp = 2 + kElemThreads / 32;   // warp 18: issues the score MMAs
 // + TMA producer (warp 0), accumulating-MMA issuer (warp 1), score-MMA issuer
 // (warp 18) and one spare warp, so that every SM sub-partition holds five
@@ -63,7 +60,7 @@ struct FwdBars {
   uint64_t k_full[3], k_empty[3];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[3];    // S of a unit ready in region r (tcgen05.commit)
-  uint64_t s_free[3];    // sweep 1: the unit's group done reading region r
+  uint64_t s_free[3];    // sweep 1: the element warps done reading region r
   uint64_t p_ready[3];   // sweep 2: P (and P_L) written into region r
   uint64_t pv_done[3];   // sweep 2: P V of region r finished (tcgen05.commit)
   uint64_t o_full;       // all P V of an item done
@@ -126,8 +123,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(&bar.k_full[s], 1);
       mbar_init(&bar.k_empty[s], 1);
       mbar_init(&bar.s_full[s], 1);
-      mbar_init(&bar.s_free[s], kGroupThreads);
-      mbar_init(&bar.p_ready[s], kGroupThreads);
+      mbar_init(&bar.s_free[s], kElemThreads);
+      mbar_init(&bar.p_ready[s], kElemThreads);
       mbar_init(&bar.pv_done[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -311,9 +308,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------ element warps
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;          // 0..3: (group, half of the unit)
-    const int grp = part >> 1;                 // units U with U % 2 == grp
-    const int sub = part & 1;                  // columns 32 sub .. 32 sub + 31 of a unit
+    const int part = (warp - 2) >> 2;          // 0..3: this warp's quarter of every unit
     const int r = quad * 32 + lane;            // query row in the tile
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
@@ -330,24 +325,20 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // row extrema and the keys of their first occurrences
       float m = -INFINITY, n_ = INFINITY;
       int am = 0, an = 0;
-      // sweep 1: statistics of this thread's 64 columns of each of its key
-      // tiles (group g takes the tiles j with j % 2 == g)
+      // sweep 1: statistics of this thread's 32 columns of every key tile
       const int nkt = nunits / 2;
-      for (int j = grp; j < nkt; j += 2) {
+      for (int j = 0; j < nkt; ++j) {
         const int U = gbase + j, rg = U % R;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[rg], (U / R) & 1, abort))) { failed = true; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        {
           float v[32];
-          tmem_ld32(tmem + lane_addr + 128u * rg + 64u * sub + 32u * c, v);
+          tmem_ld32(tmem + lane_addr + 128u * rg + 32u * part, v);
           tmem_ld_wait_regs(v);
-          if (c == 1) {
-            tc_fence_before();
-            mbar_arrive(&bar.s_free[rg]);
-          }
-          const int key0 = KIA_TILE * j + 64 * sub + 32 * c;
-          if (!is_edge(2 * j + sub)) {
+          tc_fence_before();
+          mbar_arrive(&bar.s_free[rg]);
+          const int key0 = KIA_TILE * j + 32 * part;
+          if (!is_edge(2 * j + (part >> 1))) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               // strict comparisons keep the lowest index on ties
@@ -437,50 +428,58 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       mbar_arrive(&bar.row_sync);
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n + 1) & 1, abort))) { failed = true; break; }
-      // sweep 2: weights -> P (and P_L) in TMEM, normalisers
-      float W = 0.0f, WL = 0.0f;
+      // sweep 2: weights -> P (and P_L) in TMEM, normalisers (even and odd
+      // columns summed separately, as packed pairs)
+      float2 W2 = make_float2(0.0f, 0.0f), WL2 = make_float2(0.0f, 0.0f);
       auto sweep2 = [&](auto grid) {
-        for (int u = grp; u < nunits && !failed; u += 2) {
+        for (int u = 0; u < nunits && !failed; ++u) {
           const int U = gbase + nkt + u, rg = U % R;
           if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[rg], (U / R) & 1, abort))) { failed = true; break; }
           tc_fence_after();
           const bool edge = is_edge(u);
-          const uint32_t col_s = 128u * rg + 32u * sub;   // this thread's S / P columns
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            float w16[16], vl[16];
-            tmem_ld16(tmem + lane_addr + col_s + 16u * c, w16);
+          const uint32_t col_s = 128u * rg + 16u * part;  // this thread's 16 S / P columns
+          {
+            constexpr int c = 0;
+            float w16[16];
+            [[maybe_unused]] float vl[16];
+            tmem_ld16(tmem + lane_addr + col_s, w16);
             tmem_ld_wait_regs(w16);
-            const int key0 = 64 * u + 32 * sub + 16 * c;
+            const int key0 = 64 * u + 16 * part;
             if (!edge) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                // clamped like the edge tiles: these scores come from other
-                // MMAs than the ones the row max was taken from, and nothing
-                // makes the two bit-identical
-                float wf, wl;
-                fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
-                W += wf;
-                w16[i] = wf;
+              for (int i = 0; i < 16; i += 2) {
+                // two scores at a time (packed fp32 pairs); clamped like the
+                // edge tiles: these scores come from other MMAs than the ones
+                // the row max was taken from, and nothing makes the two
+                // bit-identical
+                float2 wf, wl;
+                fwd_weights2<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], w16[i + 1], wf, wl);
+                W2 = add2(W2, wf);
+                w16[i] = wf.x;
+                w16[i + 1] = wf.y;
                 if constexpr (PROB) {
-                  WL += wl;
-                  vl[i] = wl;
+                  WL2 = add2(WL2, wl);
+                  vl[i] = wl.x;
+                  vl[i + 1] = wl.y;
                 }
               }
             } else {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                float wf, wl;
-                fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], wf, wl);
+              for (int i = 0; i < 16; i += 2) {
+                float2 wf, wl;
+                fwd_weights2<V, true>(grid, rc.m, rc.rh, Kf, Km1f, w16[i], w16[i + 1], wf, wl);
                 const int key = key0 + i;
-                const bool ok = key < T && (!p.causal || key <= qrow);
-                wf = ok ? wf : 0.0f;
-                wl = ok ? wl : 0.0f;
-                W += wf;
-                w16[i] = wf;
+                const bool ok0 = key < T && (!p.causal || key <= qrow);
+                const bool ok1 = key + 1 < T && (!p.causal || key + 1 <= qrow);
+                wf = make_float2(ok0 ? wf.x : 0.0f, ok1 ? wf.y : 0.0f);
+                wl = make_float2(ok0 ? wl.x : 0.0f, ok1 ? wl.y : 0.0f);
+                W2 = add2(W2, wf);
+                w16[i] = wf.x;
+                w16[i + 1] = wf.y;
                 if constexpr (PROB) {
-                  WL += wl;
-                  vl[i] = wl;
+                  WL2 = add2(WL2, wl);
+                  vl[i] = wl.x;
+                  vl[i + 1] = wl.y;
                 }
               }
             }
@@ -501,8 +500,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (failed) break;
       gbase += nkt + nunits;
       // normalisers of the whole row
-      rx.W[part][r] = W;
-      rx.WL[part][r] = WL;
+      rx.W[part][r] = W2.x + W2.y;
+      rx.WL[part][r] = WL2.x + WL2.y;
       mbar_arrive(&bar.row_sync);
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n + 2) & 1, abort))) { failed = true; break; }
       const float Wrow = (rx.W[0][r] + rx.W[1][r]) + (rx.W[2][r] + rx.W[3][r]);

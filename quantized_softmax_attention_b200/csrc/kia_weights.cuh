@@ -3,12 +3,13 @@
 // scores: the per-row calibration (row_calibration), the grid tables in the
 // forward's form (one pair table (G_k, G_{k+1}) per CTA for FWM and the fixed
 // step, one table per row for MinMax, both from grid_value), and the element
-// function fwd_weights<V, true> that the forward's sweep 2 calls on every
-// unit, compiled for the same operator variant V; keys past the row's last
-// visible one go through it too and are zeroed afterwards, as the forward's
-// masked keys are.  The bins and t written out are the grid position
-// fwd_weights returns, so a bit-exact match against the oracle's fp32
-// definition pins the forward's weights, bins and t themselves.
+// function fwd_weights2<V, true> (two scores at a time, as packed fp32
+// pairs) that the forward's sweep 2 calls on every unit, compiled for the
+// same operator variant V; keys past the row's last visible one go through it
+// too and are zeroed afterwards, as the forward's masked keys are.  The bins
+// and t written out are the grid positions fwd_weights2 returns, so a
+// bit-exact match against the oracle's fp32 definition pins the forward's
+// weights, bins and t themselves.
 #pragma once
 #include "kia_fast.cuh"
 
@@ -66,19 +67,27 @@ weights_from_S_kernel(const float* __restrict__ S, int rows, int cols,
     __syncwarp();
   }
   const float Kf = p.Kf, Km1f = (float)(p.K - 1);
+  // one key's outputs from its grid position and weights
+  auto put = [&](int j, const Pos& pos, float wf) {
+    const bool vis = j < L;
+    const bool tail = V::FWM && pos.u > Kf;
+    const bool live = vis && !tail;
+    int b = pos.k;
+    if constexpr (V::NEAREST) b += pos.t >= 0.5f ? 1 : 0;
+    w[(size_t)row * cols + j] = vis ? wf : 0.0f;
+    if (bin) bin[(size_t)row * cols + j] = live ? b : -1;
+    if (tout) tout[(size_t)row * cols + j] = live ? pos.t : 0.0f;
+  };
+  // keys j and j + 32 as one packed pair, as the forward's sweep 2 computes
+  // its scores
   auto run = [&](const auto& grid) {
-    for (int j = lane; j < cols; j += 32) {
-      const float x = s[j];
-      const bool vis = j < L;
-      float wf, wl;
-      const Pos pos = fwd_weights<V, true>(grid, rc.m, rc.rh, Kf, Km1f, x, wf, wl);
-      const bool tail = V::FWM && pos.u > Kf;
-      const bool live = vis && !tail;
-      int b = pos.k;
-      if constexpr (V::NEAREST) b += pos.t >= 0.5f ? 1 : 0;
-      w[(size_t)row * cols + j] = vis ? wf : 0.0f;
-      if (bin) bin[(size_t)row * cols + j] = live ? b : -1;
-      if (tout) tout[(size_t)row * cols + j] = live ? pos.t : 0.0f;
+    for (int j = lane; j < cols; j += 64) {
+      const int j1 = j + 32;
+      const float x0 = s[j], x1 = j1 < cols ? s[j1] : x0;
+      float2 wf, wl;
+      const Pos2 ps = fwd_weights2<V, true>(grid, rc.m, rc.rh, Kf, Km1f, x0, x1, wf, wl);
+      put(j, ps.a, wf.x);
+      if (j1 < cols) put(j1, ps.b, wf.y);
     }
   };
   if constexpr (V::MINMAX) run(GridF{sTab[warp], 1});
