@@ -28,6 +28,29 @@ struct Var {
   static constexpr bool MINMAX = (CAL_ == KIA_CAL_MINMAX) && !SOFTMAX_;
 };
 
+// x added to element i of a 16-register array, i known only at run time (a
+// jump on i instead of a loop over the 16 candidates)
+__device__ __forceinline__ void add_at16(float (&a)[16], int i, float x) {
+  switch (i) {
+    case 0: a[0] += x; break;
+    case 1: a[1] += x; break;
+    case 2: a[2] += x; break;
+    case 3: a[3] += x; break;
+    case 4: a[4] += x; break;
+    case 5: a[5] += x; break;
+    case 6: a[6] += x; break;
+    case 7: a[7] += x; break;
+    case 8: a[8] += x; break;
+    case 9: a[9] += x; break;
+    case 10: a[10] += x; break;
+    case 11: a[11] += x; break;
+    case 12: a[12] += x; break;
+    case 13: a[13] += x; break;
+    case 14: a[14] += x; break;
+    default: a[15] += x; break;
+  }
+}
+
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 

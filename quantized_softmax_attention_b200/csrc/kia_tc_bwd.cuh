@@ -582,13 +582,13 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   constexpr int kSlots = 4, kSlotQ = 64;
   float4* sC4 = reinterpret_cast<float4*>(sQDmn + kKvSlots * kHalfPair);
   float4* sX4 = sC4 + kSlots * kSlotQ;
-  // calibration terms, read only where a query's argmax (argmin) key is this
-  // thread's key: key - tile start, and the coefficient
-  int2* sCI = reinterpret_cast<int2*>(sX4 + kSlots * kSlotQ);  // (argmax, argmin) - kt * 128
-  float2* sCG = reinterpret_cast<float2*>(sCI + kSlots * kSlotQ);  // (g_m, g_n)
+  // calibration terms, read only where a query's argmax (argmin) key lies in
+  // a warp's 32 keys: (key - tile start, coefficient bits)
+  int2* sCM = reinterpret_cast<int2*>(sX4 + kSlots * kSlotQ);   // argmax key, g_m
+  int2* sCN = sCM + kSlots * kSlotQ;                            // argmin key, g_n
   // which queries of a unit have their argmax (argmin) key in lanes
   // 32 quad..32 quad + 31: [slot][argmax / argmin][quad][query half]
-  uint32_t* sMask = reinterpret_cast<uint32_t*>(sCG + kSlots * kSlotQ);
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sCN + kSlots * kSlotQ);
   // epilogue: 1 KB per element warp to turn its rows into full-sector stores
   float* sStage = reinterpret_cast<float*>(sMask + kSlots * 2 * 4 * 2);   // [16 warps][32][8]
   float* sTab = sStage + kElemThreads / 32 * 256;   // [slot][64][K + 1]
@@ -884,8 +884,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if constexpr (!PROJ && !V::SOFTMAX) {
           const int ka = cur.am[hq] - kt * KIA_TILE;
           const int kn = V::MINMAX ? cur.an[hq] - kt * KIA_TILE : -1;
-          sCI[e] = make_int2(ka, kn);
-          sCG[e] = make_float2(gm, gn);
+          sCM[e] = make_int2(ka, __float_as_int(gm));
+          sCN[e] = make_int2(kn, __float_as_int(gn));
           const bool hit_m = gm != 0.0f && ka >= 0 && ka < KIA_TILE;
           const bool hit_n = V::MINMAX && gn != 0.0f && kn >= 0 && kn < KIA_TILE;
 #pragma unroll
@@ -968,13 +968,14 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           tmem_ld_wait_regs(v, g);
           const int ql0 = 64 * (u & 1) + 16 * part;   // first query (in the tile) of the chunk
           const int e0 = sl * kSlotQ + 16 * part;     // its slot entry
-          // the element loop, without the mask test on units with no masked pair
-          auto body = [&](auto edge_c, auto tabs_c) {
-            constexpr bool EDGE = decltype(edge_c)::value;
+          // the element loop, one body for every unit; the masked pairs of an
+          // edge unit are zeroed afterwards (their scores are finite, so the
+          // body's clamped grid index stays inside the table)
+          auto body = [&](auto tabs_c) {
             [[maybe_unused]] constexpr bool TABS = decltype(tabs_c)::value;   // per-query grids in shared memory
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const int ql = ql0 + i;
+              [[maybe_unused]] const int ql = ql0 + i;
               const float4 cq = sC4[e0 + i];
               float4 xq = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
               if constexpr (V::MINMAX || PROJ) xq = sX4[e0 + i];
@@ -1009,43 +1010,46 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 if constexpr (V::MINMAX) dS = fmaf(dP, xq.y, dS + xq.z);   // degenerate rows: dw
               }
               if constexpr (PROJ) dS += xq.w;
-              if constexpr (EDGE) {
-                const int q = qi * KIA_TILE + ql;
-                if (!(kj < T && q < T && (!p.causal || kj <= q))) {
-                  P = 0.0f;
-                  dS = 0.0f;
-                }
-              }
               v[i] = P;
               g[i] = dS;
             }
           };
-          auto run = [&](auto tabs_c) {
-            if (edge) body(std::true_type{}, tabs_c);
-            else body(std::false_type{}, tabs_c);
-          };
           if constexpr (V::MINMAX) {
-            if (tab_in_smem) run(std::true_type{});
-            else run(std::false_type{});
+            if (tab_in_smem) body(std::true_type{});
+            else body(std::false_type{});
           } else {
-            run(std::true_type{});
+            body(std::true_type{});
+          }
+          if (edge) {
+            // future keys, and rows or keys past T: no weight, no gradient
+            const int qb = qi * KIA_TILE + ql0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (!(kj < T && qb + i < T && (!p.causal || kj <= qb + i))) {
+                v[i] = 0.0f;
+                g[i] = 0.0f;
+              }
+            }
           }
           if constexpr (!PROJ && !V::SOFTMAX) {
             // the chunk's queries whose argmax (argmin) key lies in this warp's
-            // 32 keys: a warp-uniform test, the per-element work only for them
+            // 32 keys (visible pairs: the edge zeroing above never meets
+            // them); the loops run over the set bits only, warp-uniformly
             const int hq = part >> 1, sh = 16 * (part & 1);
-            const uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
-            const uint32_t bn =
-                V::MINMAX ? (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu : 0u;
-            if ((bm | bn) != 0u) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                if ((bm | bn) & (1u << i)) {
-                  const int2 ci = sCI[e0 + i];
-                  const float2 cg = sCG[e0 + i];
-                  if ((bm >> i) & 1u) g[i] += (ci.x == r) ? cg.x : 0.0f;
-                  if (V::MINMAX && ((bn >> i) & 1u)) g[i] += (ci.y == r) ? cg.y : 0.0f;
-                }
+            uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
+            while (bm != 0u) {
+              const int i = __ffs(bm) - 1;
+              bm &= bm - 1u;
+              const int2 c = sCM[e0 + i];
+              if (c.x == r) add_at16(g, i, __int_as_float(c.y));
+            }
+            if constexpr (V::MINMAX) {
+              uint32_t bn = (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
+              while (bn != 0u) {
+                const int i = __ffs(bn) - 1;
+                bn &= bn - 1u;
+                const int2 c = sCN[e0 + i];
+                if (c.x == r) add_at16(g, i, __int_as_float(c.y));
               }
             }
           }

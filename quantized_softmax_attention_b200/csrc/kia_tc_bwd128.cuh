@@ -478,9 +478,9 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   constexpr int kSlots = 2, kSlotQ = 64;
   float4* sC4 = reinterpret_cast<float4*>(sQDmn + 2 * kHalf128);
   float4* sX4 = sC4 + kSlots * kSlotQ;
-  int2* sCI = reinterpret_cast<int2*>(sX4 + kSlots * kSlotQ);
-  float2* sCG = reinterpret_cast<float2*>(sCI + kSlots * kSlotQ);
-  uint32_t* sMask = reinterpret_cast<uint32_t*>(sCG + kSlots * kSlotQ);   // [slot][max/min][quad][half]
+  int2* sCM = reinterpret_cast<int2*>(sX4 + kSlots * kSlotQ);   // argmax key, g_m bits
+  int2* sCN = sCM + kSlots * kSlotQ;                            // argmin key, g_n bits
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sCN + kSlots * kSlotQ);   // [slot][max/min][quad][half]
   float* sStage = reinterpret_cast<float*>(sMask + kSlots * 2 * 4 * 2);   // [16 warps][32][8]
   float2* sPair = reinterpret_cast<float2*>(sStage + kElemThreads / 32 * 256);
   const int pair_floats = (!V::SOFTMAX && !V::MINMAX) ? 2 * (p.K + 1) : 0;
@@ -721,8 +721,8 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if constexpr (!PROJ && !V::SOFTMAX) {
           const int ka = cur.am[hq] - kt * KIA_TILE;
           const int kn = V::MINMAX ? cur.an[hq] - kt * KIA_TILE : -1;
-          sCI[e] = make_int2(ka, kn);
-          sCG[e] = make_float2(gm, gn);
+          sCM[e] = make_int2(ka, __float_as_int(gm));
+          sCN[e] = make_int2(kn, __float_as_int(gn));
           const bool hit_m = gm != 0.0f && ka >= 0 && ka < KIA_TILE;
           const bool hit_n = V::MINMAX && gn != 0.0f && kn >= 0 && kn < KIA_TILE;
 #pragma unroll
@@ -779,11 +779,13 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tmem_ld_wait_regs(v, gg);
         const int ql0 = 64 * (u & 1) + 16 * part;   // first query (in the tile) of the chunk
         const int e0 = sl * kSlotQ + 16 * part;     // its slot entry
-        auto body = [&](auto edge_c) {
-          constexpr bool EDGE = decltype(edge_c)::value;
+        // one body for every unit; the masked pairs of an edge unit are
+        // zeroed afterwards (finite scores: the clamped grid index stays in
+        // the table)
+        auto body = [&]() {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int ql = ql0 + i;
+            [[maybe_unused]] const int ql = ql0 + i;
             const float4 cq = sC4[e0 + i];
             float4 xq = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             if constexpr (V::MINMAX || PROJ) xq = sX4[e0 + i];
@@ -815,35 +817,39 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
               if constexpr (V::MINMAX) dS = fmaf(dP, xq.y, dS + xq.z);
             }
             if constexpr (PROJ) dS += xq.w;
-            if constexpr (EDGE) {
-              const int q = qi * KIA_TILE + ql;
-              if (!(kj < T && q < T && (!p.causal || kj <= q))) {
-                P = 0.0f;
-                dS = 0.0f;
-              }
-            }
             v[i] = P;
             gg[i] = dS;
           }
         };
-        if (edge) body(std::true_type{});
-        else body(std::false_type{});
+        body();
+        if (edge) {
+          const int qb = qi * KIA_TILE + ql0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (!(kj < T && qb + i < T && (!p.causal || kj <= qb + i))) {
+              v[i] = 0.0f;
+              gg[i] = 0.0f;
+            }
+          }
+        }
         if constexpr (!PROJ && !V::SOFTMAX) {
           // calibration terms for the chunk's queries whose argmax (argmin) key
           // lies in this warp's 32 keys
           const int hq = part >> 1, sh = 16 * (part & 1);
-          const uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
-          const uint32_t bn =
-              V::MINMAX ? (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu : 0u;
-          if ((bm | bn) != 0u) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              if ((bm | bn) & (1u << i)) {
-                const int2 ci = sCI[e0 + i];
-                const float2 cg = sCG[e0 + i];
-                if ((bm >> i) & 1u) gg[i] += (ci.x == r) ? cg.x : 0.0f;
-                if (V::MINMAX && ((bn >> i) & 1u)) gg[i] += (ci.y == r) ? cg.y : 0.0f;
-              }
+          uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
+          while (bm != 0u) {
+            const int i = __ffs(bm) - 1;
+            bm &= bm - 1u;
+            const int2 c = sCM[e0 + i];
+            if (c.x == r) add_at16(gg, i, __int_as_float(c.y));
+          }
+          if constexpr (V::MINMAX) {
+            uint32_t bn = (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
+            while (bn != 0u) {
+              const int i = __ffs(bn) - 1;
+              bn &= bn - 1u;
+              const int2 c = sCN[e0 + i];
+              if (c.x == r) add_at16(gg, i, __int_as_float(c.y));
             }
           }
         }
