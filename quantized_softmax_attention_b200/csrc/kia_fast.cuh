@@ -28,6 +28,21 @@ struct Var {
   static constexpr bool MINMAX = (CAL_ == KIA_CAL_MINMAX) && !SOFTMAX_;
 };
 
+// Which of the 16 consecutive queries q0..q0+15 may attend key kj: key and
+// query inside [0, T), and kj <= q under the causal mask (bit i for q0 + i).
+__device__ __forceinline__ uint32_t visible16(int kj, int q0, int T, bool causal) {
+  if (kj >= T) return 0u;
+  uint32_t vis = 0xFFFFu;
+  const int nq = T - q0;                        // queries left before T
+  if (nq < 16) vis = nq <= 0 ? 0u : (1u << nq) - 1u;
+  if (causal) {
+    const int d = kj - q0;                      // first visible query offset
+    if (d >= 16) return 0u;
+    if (d > 0) vis &= 0xFFFFu << d;
+  }
+  return vis;
+}
+
 // x added to element i of a 16-register array, i known only at run time (a
 // jump on i instead of a loop over the 16 candidates)
 __device__ __forceinline__ void add_at16(float (&a)[16], int i, float x) {

@@ -1022,13 +1022,12 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
           if (edge) {
             // future keys, and rows or keys past T: no weight, no gradient
-            const int qb = qi * KIA_TILE + ql0;
+            const uint32_t vis = visible16(kj, qi * KIA_TILE + ql0, T, p.causal != 0);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              if (!(kj < T && qb + i < T && (!p.causal || kj <= qb + i))) {
-                v[i] = 0.0f;
-                g[i] = 0.0f;
-              }
+              const bool keep = (vis >> i) & 1u;
+              v[i] = keep ? v[i] : 0.0f;
+              g[i] = keep ? g[i] : 0.0f;
             }
           }
           if constexpr (!PROJ && !V::SOFTMAX) {

@@ -823,13 +823,12 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         };
         body();
         if (edge) {
-          const int qb = qi * KIA_TILE + ql0;
+          const uint32_t vis = visible16(kj, qi * KIA_TILE + ql0, T, p.causal != 0);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            if (!(kj < T && qb + i < T && (!p.causal || kj <= qb + i))) {
-              v[i] = 0.0f;
-              gg[i] = 0.0f;
-            }
+            const bool keep = (vis >> i) & 1u;
+            v[i] = keep ? v[i] : 0.0f;
+            gg[i] = keep ? gg[i] : 0.0f;
           }
         }
         if constexpr (!PROJ && !V::SOFTMAX) {
