@@ -38,7 +38,10 @@
 
 namespace kia {
 
-constexpr int kBwdSmemTabK = 16;  // key pass: per-query grids up to K = 16 in shared memory
+// key pass: slots of per-query constants (MinMax keeps two, so that the
+// slots' per-query grids fit in shared memory up to K = 22)
+template <class V>
+__host__ __device__ constexpr int kv_const_slots() { return V::MINMAX ? 2 : 4; }
 constexpr int kBwdRegions = 3;    // TMEM regions of 128 columns (S | dP) in rotation
 constexpr int kBwdSlots = 3;      // query pass: slots of the K / V half-tile ring
 constexpr int kKmnSlots = 2;      // query pass: slots of the K MN-major half-tile ring
@@ -573,13 +576,14 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float* sV = reinterpret_cast<float*>(base + kTile);
   uint8_t* sQD = base + 2 * kTile;                            // [2][Q half | dO half]
   uint8_t* sQDmn = sQD + kKvSlots * kHalfPair;                // [2][Q half | dO half], MN-major
-  // Per-query constants of a unit (64 queries) in four slots, filled ahead of
-  // the element groups by the constant warp: half tile g (numbered across the
-  // CTA's items) uses slot 2 (g % 2) + (g / 2) % 2.
+  // Per-query constants of a unit (64 queries) in kSlots slots (four, or two
+  // under MinMax, whose slots also hold the queries' grids), filled ahead of
+  // the element warps by the constant warp: half tile g (numbered across the
+  // CTA's items) uses slot g % kSlots.
   // sC4 = (m, k1, k0, 1/W_fwd): the score-gradient factor -dw/h = dP k1 + k0
   // (softmax: dw itself); sX4 (MinMax or projection) = (1/h, the degenerate
   // row's dw = dP x.y + x.z, 0 elsewhere, the projection shift c)
-  constexpr int kSlots = 4, kSlotQ = 64;
+  constexpr int kSlots = kv_const_slots<V>(), kSlotQ = 64;
   float4* sC4 = reinterpret_cast<float4*>(sQDmn + kKvSlots * kHalfPair);
   float4* sX4 = sC4 + kSlots * kSlotQ;
   // calibration terms, read only where a query's argmax (argmin) key lies in
@@ -850,18 +854,32 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     int it = cseq.next(), u = 0;
     if (it >= 0) load_raw(it, 0, cur);
     for (int g = 0; it >= 0 && !failed; ++g) {
-      const int sl = g & 3;
+      const int sl = g % kSlots;
       // the next half tile (possibly of the next item)
       int it2 = it, u2 = u + 1;
       if (u2 == item_units(it)) { u2 = 0; it2 = cseq.next(); }
       Raw nxt;
       if (it2 >= 0) load_raw(it2, u2, nxt);
-      if (g >= kSlots && !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[sl], ((g >> 2) - 1) & 1, abort))) {
+      if (g >= kSlots && !__all_sync(0xffffffffu, mbar_wait(&bar.qc_free[sl], ((g / kSlots) - 1) & 1, abort))) {
         failed = true;
         break;
       }
       const int kt = item_kt(it);
       const long long rowbase = (long long)item_bh(it) * T;
+      if (V::MINMAX && tab_in_smem) {
+        // the unit's 64 per-query grids are consecutive rows of the stats
+        // table: asynchronous copies into the slot, issued before the
+        // constants below so that their latency passes meanwhile (rows past
+        // T are filled with ones; their queries are masked)
+        const int qf = 64 * (2 * item_q0(it) + u);
+        const int nvalid = max(0, min(kSlotQ, T - qf)) * K1, ntot = kSlotQ * K1;
+        const float* src = st.table + (rowbase + qf) * K1;
+        float* dst = sTab + (size_t)sl * kSlotQ * K1;
+        for (int x = lane; x < ntot; x += 32) {
+          if (x < nvalid) cp_async4(dst + x, src + x);
+          else dst[x] = 1.0f;
+        }
+      }
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
         const int q = 64 * (2 * item_q0(it) + u) + 32 * hq + lane;
@@ -899,31 +917,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
         }
       }
-      if (V::MINMAX && tab_in_smem) {
-        // the unit's 64 per-query grids are consecutive rows of the stats
-        // table: one coalesced copy, its loads issued together in four batches
-        // (rows past T are filled with ones; their queries are masked)
-        const int qf = 64 * (2 * item_q0(it) + u);
-        const int nvalid = max(0, min(kSlotQ, T - qf)) * K1, ntot = kSlotQ * K1;
-        const float* src = st.table + (rowbase + qf) * K1;
-        float* dst = sTab + (size_t)sl * kSlotQ * K1;
-        constexpr int kBatches = 4;
-        constexpr int kBatch = (kSlotQ * (kBwdSmemTabK + 1) + 32 * kBatches - 1) / (32 * kBatches);
-#pragma unroll
-        for (int b = 0; b < kBatches; ++b) {
-          float buf[kBatch];
-#pragma unroll
-          for (int i = 0; i < kBatch; ++i) {
-            const int x = lane + 32 * (b * kBatch + i);
-            buf[i] = x < nvalid ? src[x] : 1.0f;
-          }
-#pragma unroll
-          for (int i = 0; i < kBatch; ++i) {
-            const int x = lane + 32 * (b * kBatch + i);
-            if (x < ntot) dst[x] = buf[i];
-          }
-        }
-      }
+      if (V::MINMAX && tab_in_smem) cp_async_wait_all();   // the unit's grids have landed
       __syncwarp();
       mbar_arrive(&bar.qc_ready[sl]);
       cur = nxt;
@@ -954,8 +948,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int gu = gbase + u;
         const int qi = q0 + (u >> 1);
         const int rg = gu % R;
-        const int sl = gu & 3;                               // this unit's constant slot
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[sl], (gu >> 2) & 1, abort))) { failed = true; break; }
+        const int sl = gu % kSlots;                          // this unit's constant slot
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[sl], (gu / kSlots) & 1, abort))) { failed = true; break; }
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (gu / R) & 1, abort))) { failed = true; break; }
         tc_fence_after();
         const bool edge =
@@ -1102,11 +1096,12 @@ size_t tc_bwd_q_smem(const OpParams& p, bool tab_in_smem) {
 template <int D>
 size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
-  const int tab =
-      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? 4 * 64 * (p.K + 1) : 0) : 4 * (p.K + 1));
+  const size_t slots = minmax_tab ? 2 : 4;   // kv_const_slots
+  const size_t tab =
+      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? slots * 64 * (p.K + 1) : 0) : 4 * (p.K + 1));
   return 1024 + 2 * (size_t)D * KIA_TILE * 4 + 2 * kKvSlots * (size_t)kHalfPair +
-         4 * 64 * (16 + 16 + 8 + 8) + 4 * 2 * 4 * 2 * 4 + kElemThreads / 32 * 1024 +
-         (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdKBars);
+         slots * 64 * (16 + 16 + 8 + 8) + slots * 2 * 4 * 2 * 4 + kElemThreads / 32 * 1024 +
+         ((tab + 31) & ~(size_t)31) * 4 + sizeof(BwdKBars);
 }
 
 template <int D, class V>
@@ -1126,7 +1121,7 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
     return KIA_ERR_CUDA;
   const bool q_tab_smem = tc_bwd_q_smem<D>(p, true) <= 232448;
   const size_t smq = tc_bwd_q_smem<D>(p, q_tab_smem);
-  const bool kv_tab_smem = p.K <= kBwdSmemTabK && tc_bwd_kv_smem<D>(p, true) <= 232448;
+  const bool kv_tab_smem = tc_bwd_kv_smem<D>(p, true) <= 232448;
   const size_t smk = tc_bwd_kv_smem<D>(p, kv_tab_smem);
   if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
   const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
