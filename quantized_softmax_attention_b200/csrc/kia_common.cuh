@@ -279,13 +279,17 @@ constexpr uint32_t kSuspendHintNs = 1000000u;     // 1 ms per sleep, then re-che
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (;;) {
+  for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > g_kia_wait_limit_ns) {
-      *abort = 1;
-      atomicExch(&g_kia_device_error, KIA_ERR_TIMEOUT);
-      return false;
+    // the abort flag and the time limit (a global load) only every 16th
+    // pass, so that nothing slow sits between two probes of the barrier
+    if ((n & 15u) == 0u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > g_kia_wait_limit_ns) {
+        *abort = 1;
+        atomicExch(&g_kia_device_error, KIA_ERR_TIMEOUT);
+        return false;
+      }
     }
   }
 }
