@@ -88,7 +88,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmV, const float* __restrict__ Kt,
                 const float* __restrict__ O, const float* __restrict__ dO,
                 const __grid_constant__ CUtensorMap tmdQ, StatsView st, WorkView wk,
-                float* __restrict__ dS_dbg, OpParams p, int B, int H, int T, int tab_in_smem) {
+                float* __restrict__ dS_dbg, OpParams p, int B, int H, int T, int tab_in_smem,
+                int nkv) {
   static_assert(D == 64, "tensor-core backward tiles are laid out for d = 64");
   constexpr uint32_t kTile = D * KIA_TILE * 4;
   // the stats must come from a forward of this shape and configuration
@@ -108,8 +109,10 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // slots each, so that a slot refills while the next two are in use.
   float* sQ = reinterpret_cast<float*>(base);
   float* sG = reinterpret_cast<float*>(base + kTile);
-  uint8_t* sKV = base + 2 * kTile;                           // [3][K half | V half]
-  uint8_t* sKmn = sKV + kBwdSlots * kHalfPair;                // [2][K half, MN-major]
+  // the K / V ring has kBwdSlots slots, one less when a MinMax grid table
+  // needs the room (only the producer and the score issuer use the ring)
+  const int NKV = V::MINMAX ? nkv : kBwdSlots;   // a constant for the other variants
+  uint8_t* sKmn = base + 2 * kTile;                          // [2][K half, MN-major]
   // epilogue: 1 KB per element warp to turn its rows into full-sector stores
   float* sStage = reinterpret_cast<float*>(sKmn + kKmnSlots * kHalfTile);   // [16 warps][32][8]
   float* sAC = sStage + kElemThreads / 32 * 256;              // [kRowSplit][2][128]
@@ -118,6 +121,9 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int tab_floats =
       V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   BwdQBars& bar = *reinterpret_cast<BwdQBars*>(sTab + ((tab_floats + 31) & ~31));
+  // the K / V ring last (1024-aligned), so that its depth moves no other buffer
+  uint8_t* sKV =
+      base + ((reinterpret_cast<uint8_t*>(&bar + 1) - base + 1023) & ~(ptrdiff_t)1023);  // [NKV][K | V]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = B * H;
@@ -193,8 +199,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           moved = true;
         }
         if (ik >= 0) {
-          const int sl = gk % kBwdSlots;
-          if (mbar_test(&bar.kv_empty[sl], ((gk / kBwdSlots) & 1) ^ 1)) {
+          const int sl = gk % NKV;
+          if (mbar_test(&bar.kv_empty[sl], ((gk / NKV) & 1) ^ 1)) {
             uint8_t* dst = sKV + sl * kHalfPair;
             mbar_arrive_expect_tx(&bar.kv_full[sl], kHalfPair);
             for (int b = 0; b < D / 32; ++b) {
@@ -248,8 +254,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (!warp_wait(&bar.st_free[r], (sf_par >> r) & 1u, abort)) { failed = true; break; }
             sf_par ^= 1u << r;
           }
-          const int sl = g % kBwdSlots;
-          if (!warp_wait(&bar.kv_full[sl], (g / kBwdSlots) & 1, abort)) { failed = true; break; }
+          const int sl = g % NKV;
+          if (!warp_wait(&bar.kv_full[sl], (g / NKV) & 1, abort)) { failed = true; break; }
           const uint64_t dk = dkv + desc_step((uint32_t)sl * kHalfPair);   // K half, V half after it
           const uint64_t dv = dk + desc_step(kHalfTile);
           const uint32_t dst = tmem + 128u * r;
@@ -563,7 +569,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmGmn,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                 StatsView st, WorkView wk, OpParams p, int BH, int T, int tab_in_smem) {
+                 StatsView st, WorkView wk, OpParams p, int BH, int T, int tab_in_smem,
+                 int nmn) {
   static_assert(D == 64, "tensor-core backward tiles are laid out for d = 64");
   constexpr uint32_t kTile = D * KIA_TILE * 4;
   if (*wk.status != 0) return;
@@ -575,7 +582,10 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float* sK = reinterpret_cast<float*>(base);
   float* sV = reinterpret_cast<float*>(base + kTile);
   uint8_t* sQD = base + 2 * kTile;                            // [2][Q half | dO half]
-  uint8_t* sQDmn = sQD + kKvSlots * kHalfPair;                // [2][Q half | dO half], MN-major
+  // the MN-major ring has kKvSlots slots, one when a MinMax grid table needs
+  // the room (only the producer and the dV / dK issuer use it); it sits last
+  // in shared memory (below), so that its depth moves no other buffer
+  const int NMN = V::MINMAX ? nmn : kKvSlots;   // a constant for the other variants
   // Per-query constants of a unit (64 queries) in kSlots slots (four, or two
   // under MinMax, whose slots also hold the queries' grids), filled ahead of
   // the element warps by the constant warp: half tile g (numbered across the
@@ -584,7 +594,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   // (softmax: dw itself); sX4 (MinMax or projection) = (1/h, the degenerate
   // row's dw = dP x.y + x.z, 0 elsewhere, the projection shift c)
   constexpr int kSlots = kv_const_slots<V>(), kSlotQ = 64;
-  float4* sC4 = reinterpret_cast<float4*>(sQDmn + kKvSlots * kHalfPair);
+  float4* sC4 = reinterpret_cast<float4*>(sQD + kKvSlots * kHalfPair);
   float4* sX4 = sC4 + kSlots * kSlotQ;
   // calibration terms, read only where a query's argmax (argmin) key lies in
   // a warp's 32 keys: (key - tile start, coefficient bits)
@@ -599,6 +609,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int K1 = p.K + 1;
   const int tab_floats = V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? kSlots * kSlotQ * K1 : 0) : 4 * K1);
   BwdKBars& bar = *reinterpret_cast<BwdKBars*>(sTab + ((tab_floats + 31) & ~31));
+  uint8_t* sQDmn =    // [NMN][Q half | dO half], MN-major, 1024-aligned
+      base + ((reinterpret_cast<uint8_t*>(&bar + 1) - base + 1023) & ~(ptrdiff_t)1023);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
@@ -695,8 +707,8 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
         }
         if (im >= 0) {
-          const int sl = gm % kKvSlots;
-          if (mbar_test(&bar.mn_empty[sl], ((gm / kKvSlots) & 1) ^ 1)) {
+          const int sl = gm % NMN;
+          if (mbar_test(&bar.mn_empty[sl], ((gm / NMN) & 1) ^ 1)) {
             uint8_t* dst = sQDmn + sl * kHalfPair;
             const int row = 64 * (2 * item_q0(im) + um);
             mbar_arrive_expect_tx(&bar.mn_full[sl], kHalfPair);
@@ -777,10 +789,10 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int nunits = item_units(it);
         // dV += P^T dO, dK += dS^T Q for half tile u (A operands in region g % R)
         for (int u = 0; u < nunits; ++u, ++g) {
-          const int r = g % R, sl = g % kKvSlots;
+          const int r = g % R, sl = g % NMN;
           if (!warp_wait(&bar.elem_done[r], (ed_par >> r) & 1u, abort)) { failed = true; break; }
           ed_par ^= 1u << r;
-          if (!warp_wait(&bar.mn_full[sl], (g / kKvSlots) & 1, abort)) { failed = true; break; }
+          if (!warp_wait(&bar.mn_full[sl], (g / NMN) & 1, abort)) { failed = true; break; }
           // the accumulators restart with this item: the previous item's
           // epilogue must have read them
           if (u == 0 && n > 0 && !warp_wait(&bar.acc_free, (n - 1) & 1, abort)) { failed = true; break; }
@@ -1084,24 +1096,26 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 template <int D>
-size_t tc_bwd_q_smem(const OpParams& p, bool tab_in_smem) {
+size_t tc_bwd_q_smem(const OpParams& p, bool tab_in_smem, int nkv) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
-  return 1024 + 2 * (size_t)D * KIA_TILE * 4 + kBwdSlots * (size_t)kHalfPair +
-         kKmnSlots * (size_t)kHalfTile + kElemThreads / 32 * 1024 +
-         (2 * kRowSplit + 1) * KIA_TILE * 4 + (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdQBars);
+  const size_t head = 2 * (size_t)D * KIA_TILE * 4 + kKmnSlots * (size_t)kHalfTile +
+                      kElemThreads / 32 * 1024 + (2 * kRowSplit + 1) * KIA_TILE * 4 +
+                      (size_t)((tab + 31) & ~31) * 4 + sizeof(BwdQBars);
+  return 1024 + ((head + 1023) & ~(size_t)1023) + nkv * (size_t)kHalfPair;
 }
 
 template <int D>
-size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem) {
+size_t tc_bwd_kv_smem(const OpParams& p, bool tab_in_smem, int nmn) {
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const size_t slots = minmax_tab ? 2 : 4;   // kv_const_slots
   const size_t tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? slots * 64 * (p.K + 1) : 0) : 4 * (p.K + 1));
-  return 1024 + 2 * (size_t)D * KIA_TILE * 4 + 2 * kKvSlots * (size_t)kHalfPair +
-         slots * 64 * (16 + 16 + 8 + 8) + slots * 2 * 4 * 2 * 4 + kElemThreads / 32 * 1024 +
-         ((tab + 31) & ~(size_t)31) * 4 + sizeof(BwdKBars);
+  const size_t head = 2 * (size_t)D * KIA_TILE * 4 + kKvSlots * (size_t)kHalfPair +
+                      slots * 64 * (16 + 16 + 8 + 8) + slots * 2 * 4 * 2 * 4 +
+                      kElemThreads / 32 * 1024 + ((tab + 31) & ~(size_t)31) * 4 + sizeof(BwdKBars);
+  return 1024 + ((head + 1023) & ~(size_t)1023) + nmn * (size_t)kHalfPair;
 }
 
 template <int D, class V>
@@ -1119,10 +1133,25 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
       !make_tmap(&tvh, Vv, BH, T, D, false, 64) || !make_tmap_out(&tdq, dQ, BH, T, D) ||
       !make_tmap_out(&tdk, dK, BH, T, D) || !make_tmap_out(&tdv, dV, BH, T, D))
     return KIA_ERR_CUDA;
-  const bool q_tab_smem = tc_bwd_q_smem<D>(p, true) <= 232448;
-  const size_t smq = tc_bwd_q_smem<D>(p, q_tab_smem);
-  const bool kv_tab_smem = tc_bwd_kv_smem<D>(p, true) <= 232448;
-  const size_t smk = tc_bwd_kv_smem<D>(p, kv_tab_smem);
+  // MinMax grid tables in shared memory where they fit, with one ring a slot
+  // shallower if that is what makes them fit; else read from global memory
+  constexpr size_t kMax = 232448;
+  bool q_tab_smem = true;
+  int nkv = kBwdSlots;
+  if (tc_bwd_q_smem<D>(p, true, nkv) > kMax) nkv = kBwdSlots - 1;
+  if (tc_bwd_q_smem<D>(p, true, nkv) > kMax) {
+    q_tab_smem = false;
+    nkv = kBwdSlots;
+  }
+  const size_t smq = tc_bwd_q_smem<D>(p, q_tab_smem, nkv);
+  bool kv_tab_smem = true;
+  int nmn = kKvSlots;
+  if (tc_bwd_kv_smem<D>(p, true, nmn) > kMax) nmn = kKvSlots - 1;
+  if (tc_bwd_kv_smem<D>(p, true, nmn) > kMax) {
+    kv_tab_smem = false;
+    nmn = kKvSlots;
+  }
+  const size_t smk = tc_bwd_kv_smem<D>(p, kv_tab_smem, nmn);
   if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
   const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
                                     p.grad == KIA_GRAD_MIN_ONLY);
@@ -1137,14 +1166,14 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
       return KIA_ERR_CUDA;
     tc_bwd_q_kernel<D, V, true><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
                                                               tdq, st, wk, dS_dbg, p, B, H, T,
-                                                              q_tab_smem ? 1 : 0);
+                                                              q_tab_smem ? 1 : 0, nkv);
   } else {
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
     tc_bwd_q_kernel<D, V, false><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
                                                                tdq, st, wk, dS_dbg, p, B, H, T,
-                                                               q_tab_smem ? 1 : 0);
+                                                               q_tab_smem ? 1 : 0, nkv);
   }
   if (cudaGetLastError() != cudaSuccess) return KIA_ERR_CUDA;
   mark(4, s);
@@ -1153,7 +1182,7 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
         cudaSuccess)
       return KIA_ERR_CUDA;
     kern<<<qgrid, kTcThreads, smk, s>>>(tqh, tqmh, tgh, tgmh, tk, tv, tdk, tdv, st, wk, p, BH, T,
-                                        kv_tab_smem ? 1 : 0);
+                                        kv_tab_smem ? 1 : 0, nmn);
     return KIA_OK;
   };
   const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;

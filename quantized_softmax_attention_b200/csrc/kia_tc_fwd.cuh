@@ -85,16 +85,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
               const __grid_constant__ CUtensorMap tmOL, StatsView st, OpParams p, int B, int H,
-              int T, int tab_in_smem) {
+              int T, int tab_in_smem, int nsk) {
   constexpr bool PROB = V::PROB;
   using Cfg = FwdCfg<D, PROB>;
-  constexpr int NSK = Cfg::kKStages, NSV = Cfg::kVStages, R = Cfg::kRegions;
+  // K ring depth: Cfg::kKStages, one less when a MinMax grid table needs the
+  // room (the producer and the score issuer are the only users of the ring)
+  const int NSK = V::MINMAX ? nsk : Cfg::kKStages;   // a constant for the other variants
+  constexpr int NSV = Cfg::kVStages, R = Cfg::kRegions;
   constexpr uint32_t kTileF = Cfg::kTileBytes / 4;     // floats per operand tile
   extern __shared__ uint8_t smraw[];
   uint8_t* base = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
   float* sQ = reinterpret_cast<float*>(base);
-  float* sK = sQ + kTileF;
-  float* sV = sK + NSK * kTileF;
+  float* sV = sQ + kTileF;
   FwdRowX& rx = *reinterpret_cast<FwdRowX*>(sV + NSV * kTileF);
   // epilogue: 1 KB per element warp to turn its rows into full-sector stores
   float* sStage = reinterpret_cast<float*>(&rx + 1);      // [16 warps][32][8]
@@ -102,6 +104,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int tab_floats =
       V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   FwdBars& bar = *reinterpret_cast<FwdBars*>(sTab + ((tab_floats + 31) & ~31));
+  // the K ring last (1024-aligned), so that its depth moves no other buffer
+  float* sK = reinterpret_cast<float*>(
+      base + ((reinterpret_cast<uint8_t*>(&bar + 1) - base + 1023) & ~(ptrdiff_t)1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = B * H;
@@ -561,24 +566,35 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 }
 
 template <int D, bool PROB>
-size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem) {
+size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem, int nsk) {
   using Cfg = FwdCfg<D, PROB>;
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
   const int tab =
       p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
-  return 1024 + (size_t)(1 + Cfg::kKStages + Cfg::kVStages) * Cfg::kTileBytes + sizeof(FwdRowX) +
-         kElemThreads / 32 * 1024 + (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
+  const size_t head = (size_t)(1 + Cfg::kVStages) * Cfg::kTileBytes + sizeof(FwdRowX) +
+                      kElemThreads / 32 * 1024 + (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
+  return 1024 + ((head + 1023) & ~(size_t)1023) + (size_t)nsk * Cfg::kTileBytes;
 }
 
 template <int D, class V>
 int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const CUtensorMap& tol, const StatsView& st, int B, int H,
                  int T, const OpParams& p, cudaStream_t s) {
+  // a MinMax grid table in shared memory if it fits, with a K ring one stage
+  // shallower if that is what makes it fit; else the grids are read from
+  // global memory
+  constexpr int kNsk = FwdCfg<D, V::PROB>::kKStages;
   bool tab_in_smem = true;
-  size_t smem = tc_fwd_smem<D, V::PROB>(p, true);
+  int nsk = kNsk;
+  size_t smem = tc_fwd_smem<D, V::PROB>(p, true, nsk);
+  if (smem > 232448 && kNsk > 2) {
+    nsk = kNsk - 1;
+    smem = tc_fwd_smem<D, V::PROB>(p, true, nsk);
+  }
   if (smem > 232448) {
     tab_in_smem = false;
-    smem = tc_fwd_smem<D, V::PROB>(p, false);
+    nsk = kNsk;
+    smem = tc_fwd_smem<D, V::PROB>(p, false, nsk);
   }
   if (smem > 232448) return KIA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(tc_fwd_kernel<D, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -590,7 +606,7 @@ int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   if (sms <= 0) return KIA_ERR_CUDA;
   const dim3 grid(std::min(sms, B * H * nt));
   tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, to, tol, st, p, B, H, T,
-                                                     tab_in_smem ? 1 : 0);
+                                                     tab_in_smem ? 1 : 0, nsk);
   return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
 }
 
