@@ -338,37 +338,48 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int q = qt * KIA_TILE + r;
       const long long rowbase = (long long)bh * T;
       const long long qr = rowbase + (q < T ? q : T - 1);
-      // this row's calibration and centering (written by the forward)
+      // Every global load of the item's prologue is issued before the first
+      // use of any of them (a warp stalls at its first use of a pending load,
+      // so loads behind it would wait a round trip more): this row's
+      // calibration (written by the forward), then the operands of the
+      // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE), which four
+      // consecutive element threads read for one row (coalesced) and add by
+      // shuffles, leaving the row's D in shared memory.
       const float m = st.m[qr];
       const int am = st.am[qr], an = V::MINMAX ? st.an[qr] : am;
       const float rh = st.rh[qr];
+      const float Wb = st.Wb[qr];
+      const int e = (int)threadIdx.x - 64;
+      const int rr = e >> 2, cc = e & 3;       // row of the tile, quarter of the row
+      const int qq = qt * KIA_TILE + rr;
+      const long long qrr = rowbase + (qq < T ? qq : T - 1);
+      float4 ga[D / 16], ob[D / 16];
+      {
+        const float4* g4 = reinterpret_cast<const float4*>(dO + qrr * D) + cc * (D / 16);
+        const float4* o4 =
+            reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qrr * D) + cc * (D / 16);
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          ga[c] = g4[c];
+          ob[c] = o4[c];
+        }
+      }
       const float nrh = -rh;
       const float dg = (V::MINMAX && rh == 0.0f) ? 1.0f : 0.0f;
       const int L = p.causal ? q + 1 : T;
       // a one-key row has P = 1 whatever its score: zero gradient
-      const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]);
+      const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, Wb);
       // the key rows this row's epilogue gathers (argmax, argmin) into L2 now
       prefetch_l2(Kt + (rowbase + am) * D + part * (D / kRowSplit));
       if constexpr (V::MINMAX) prefetch_l2(Kt + (rowbase + an) * D + part * (D / kRowSplit));
-      // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE): four
-      // consecutive element threads read one row's D values (coalesced), add
-      // their partial sums by shuffles and leave the row's D in shared memory
       {
-        const int e = (int)threadIdx.x - 64;
-        const int rr = e >> 2, cc = e & 3;     // row of the tile, quarter of the row
-        const int qq = qt * KIA_TILE + rr;
-        const long long qrr = rowbase + (qq < T ? qq : T - 1);
-        const float4* g4 = reinterpret_cast<const float4*>(dO + qrr * D) + cc * (D / 16);
-        const float4* o4 =
-            reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qrr * D) + cc * (D / 16);
         float acc = 0.0f;
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
-          const float4 a = g4[c], b4 = o4[c];
-          acc = fmaf(a.x, b4.x, acc);
-          acc = fmaf(a.y, b4.y, acc);
-          acc = fmaf(a.z, b4.z, acc);
-          acc = fmaf(a.w, b4.w, acc);
+          acc = fmaf(ga[c].x, ob[c].x, acc);
+          acc = fmaf(ga[c].y, ob[c].y, acc);
+          acc = fmaf(ga[c].z, ob[c].z, acc);
+          acc = fmaf(ga[c].w, ob[c].w, acc);
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
