@@ -6,7 +6,6 @@
 //             and the gradient mode (section 3 Calibration gradients;
 //             Appendix B), applied as the 2-sparse update at the argmax /
 //             argmin keys;
-//   scatter - (tensor-core path) the dK side of that update, per key tile;
 //   scan    - the zero-sum projection's common-mode shift c_i, which adds
 //             c_i to every visible score gradient of row i: dQ_i += c_i sum_J k_j
 //             and dK_j += sum_{i sees j} c_i q_i (prefix / suffix sums).
@@ -106,47 +105,6 @@ bwd_calib_kernel(const float* __restrict__ Q, const float* __restrict__ Kt, Stat
     if (gm != 0.0f) atomicAdd(dK + base + (size_t)am * D + c, gm * q[c]);
     if (gn != 0.0f) atomicAdd(dK + base + (size_t)an * D + c, gn * q[c]);
   }
-}
-
-// Calibration terms into dK without global atomics: one CTA per (batch*head,
-// 128-key tile) collects g_m q_i for every row i whose argmax key lies in the
-// tile (and g_n q_i for the argmin), in shared memory, then adds the tile to
-// dK.  Rows i can only point at keys j <= i under the causal mask.
-template <int D>
-__global__ void __launch_bounds__(256)
-bwd_scatter_kernel(const float* __restrict__ Q, WorkView wk, float* __restrict__ dK, OpParams p,
-                   int T) {
-  if (*wk.status != 0) return;
-  extern __shared__ float acc[];   // [128][D]
-  const int bh = blockIdx.x;
-  const int base = blockIdx.y * KIA_TILE;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = threadIdx.x; e < KIA_TILE * D; e += blockDim.x) acc[e] = 0.0f;
-  __syncthreads();
-  const long long rowbase = (long long)bh * T;
-  const int i0 = p.causal ? base : 0;
-  // each thread serves one row: if its argmax (argmin) key lies in the tile it
-  // adds g q_i into that key's row, walking the columns from a lane-dependent
-  // start so that the 32 lanes of a warp hit 32 different banks
-  for (int i = i0 + (int)threadIdx.x; i < T; i += blockDim.x) {
-    const float gm = wk.gm[rowbase + i], gn = wk.gn[rowbase + i];
-    const int am = wk.am[rowbase + i] - base, an = wk.an[rowbase + i] - base;
-    const bool hm = gm != 0.0f && am >= 0 && am < KIA_TILE;
-    const bool hn = gn != 0.0f && an >= 0 && an < KIA_TILE;
-    if (!hm && !hn) continue;
-    const float* q = Q + (rowbase + i) * D;
-    for (int cc = 0; cc < D; ++cc) {
-      const int c = (cc + lane) & (D - 1);
-      const float qc = q[c];
-      if (hm) atomicAdd(&acc[am * D + c], gm * qc);
-      if (hn) atomicAdd(&acc[an * D + c], gn * qc);
-    }
-  }
-  (void)warp;
-  __syncthreads();
-  const int nrows = min(KIA_TILE, T - base);
-  for (int e = threadIdx.x; e < nrows * D; e += blockDim.x)
-    dK[(rowbase + base) * D + e] += acc[e];
 }
 
 // Zero-sum projection, common-mode part: dQ_i += c_i sum_{j in J_i} k_j and

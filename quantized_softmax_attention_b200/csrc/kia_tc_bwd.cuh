@@ -838,7 +838,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else if (warp == kScoreWarp + 1) {
     // -------------------------------------------- query-constant producer
     // Loads the per-query constants of each unit into its slot while the
-    // element groups work on earlier units (lane l: queries l and l + 32).
+    // element warps work on earlier units (lane l: queries l and l + 32).
     // FWM: each group's copy of the shared grid's pairs, published with the
     // first units' constants
     if (!V::SOFTMAX && !V::MINMAX) {
