@@ -8,8 +8,10 @@
 //             argmin keys;
 //   scan    - the zero-sum projection's common-mode shift c_i, which adds
 //             c_i to every visible score gradient of row i: dQ_i += c_i sum_J k_j
-//             and dK_j += sum_{i sees j} c_i q_i (prefix / suffix sums).
-// All are O(B H T d) and bandwidth-bound.
+//             and dK_j += sum_{i sees j} c_i q_i (prefix / suffix sums);
+//   decomp  - the fixed-upstream gradient decomposition per row over a dS
+//             dump (Appendix F).
+// All are bandwidth-bound row passes.
 #pragma once
 #include "kia_elem.cuh"
 #include "kia_stats.cuh"
