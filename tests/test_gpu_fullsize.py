@@ -167,6 +167,9 @@ def test_1B_shape_five_gradient_modes_from_one_forward():
     (1024, 64, K.CAL_FWM, K.REC_NEAREST, K.STE_PROB),
     (2048, 16, K.CAL_MINMAX, K.REC_NEAREST, K.STE_WEIGHT),
     (4096, 32, K.CAL_FWM, K.REC_LERP, K.STE_WEIGHT),
+    # MinMax grids kept in shared memory with one ring slot fewer
+    (1024, 64, K.CAL_MINMAX, K.REC_NEAREST, K.STE_PROB),
+    (2048, 32, K.CAL_MINMAX, K.REC_LERP, K.STE_WEIGHT),
 ])
 def test_throughput_sweep_shapes(T, Kint, cal, rec, ste):
     """Points of the B16 H12 d64 sweep (T up to 4096, K from 2 to 64)."""
