@@ -7,17 +7,19 @@
 // probe), section 5.4 and Appendix D.6 (Figure S4).
 //
 // One warp per row, specialised at compile time on calibration and
-// reconstruction.  Rows of at most kGeoRegKeys keys (T a multiple of 4) are
-// read from HBM once into registers, four keys per lane per 128-key chunk,
-// and only the chunks the row reaches are touched; the third sweep
-// recomputes e and w from the held scores rather than keeping them, for
-// occupancy.  Other rows take three sweeps over global memory, the later two
-// served by L1/L2.  The operator
+// reconstruction.  Rows of at most kGeoRowKeys keys are copied from HBM once
+// into the warp's shared-memory buffer (asynchronous copies, all in flight
+// together); the three sweeps run as rolled loops over it, and the second
+// leaves e and w there for the third.  (An earlier form held the row in
+// registers, unrolled over eight 128-key chunks: its code overflowed the
+// instruction cache.)  Longer rows take three sweeps over global memory, the
+// later two served by L1/L2.  The operator
 // weights are the fused kernels' paired fp32 weight stage (kia_fast.cuh), so
 // the grid decisions are the forward's; a key is in the top bucket iff its
 // grid coordinate u = (m - s) / h is below 1/2 (nearest node 0).
 #pragma once
 #include <cfloat>
+#include <type_traits>
 
 #include "kia_common.cuh"
 #include "kia_fast.cuh"
@@ -25,8 +27,8 @@
 namespace kia {
 
 constexpr int kGeoWarps = 8;
-constexpr int kGeoChunks = 8;                     // float4 chunks per lane
-constexpr int kGeoRegKeys = 4 * 32 * kGeoChunks;  // 1024 keys held in registers
+constexpr int kGeoRowKeys = 1024;                 // rows up to this length are staged
+constexpr size_t kGeoSmemBytes = (size_t)kGeoWarps * 2 * kGeoRowKeys * 4;   // 64 KB
 
 // out fields per row (include/kiattn.h: KIA_GEO_*)
 enum { kGeoSpan = 0, kGeoH, kGeoQNorm, kGeoEntSoftmax, kGeoEntOp, kGeoTV, kGeoTopSoftmax,
@@ -66,14 +68,8 @@ __device__ __forceinline__ void geo_pair(const GeoRow& r, float& s0, float& s1, 
   a.Ex = fmaf(e0, x.x, fmaf(e1, x.y, a.Ex));
   a.W += wf.x + wf.y;
   a.Wlw = fmaf(wf.x, __logf(fmaxf(wf.x, FLT_MIN)), fmaf(wf.y, __logf(fmaxf(wf.y, FLT_MIN)), a.Wlw));
-  if (u.x < 0.5f) {
-    a.Tsm += e0;
-    a.Top += wf.x;
-  }
-  if (u.y < 0.5f) {
-    a.Tsm += e1;
-    a.Top += wf.y;
-  }
+  a.Tsm += (u.x < 0.5f ? e0 : 0.0f) + (u.y < 0.5f ? e1 : 0.0f);
+  a.Top += (u.x < 0.5f ? wf.x : 0.0f) + (u.y < 0.5f ? wf.y : 0.0f);
   s0 = e0;
   s1 = e1;
   w0 = wf.x;
@@ -87,12 +83,15 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <class V>
-__global__ void __launch_bounds__(32 * kGeoWarps, 4)
+__global__ void __launch_bounds__(32 * kGeoWarps)
 geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long long rows, int T,
                 int d, int causal, OpParams p, float* __restrict__ out) {
   // (G_k, G_{k+1}) pairs: one per warp under MinMax (the grid follows the
   // row), one per block under FWM (the grid is the same for every row)
   __shared__ float2 sPair[V::MINMAX ? kGeoWarps : 1][V::MINMAX ? KIA_MAX_K : KIA_MAX_KCAP];
+  // per warp: the row's scores, overwritten by e = e^{s - m}, and the
+  // operator's weights w (rows of at most kGeoRowKeys keys)
+  extern __shared__ float sRows[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if constexpr (V::FWM) {
     for (int k = threadIdx.x; k < p.K; k += blockDim.x)
@@ -104,36 +103,39 @@ geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long l
   const int i = (int)(row % T);
   const int L = causal ? i + 1 : T;
   const float* s = S + row * (long long)T;
-  const bool in_regs = (T & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&
-                       L <= kGeoRegKeys;
-  const int nch = (L + 127) >> 7;   // chunks the row reaches (warp-uniform)
-  // the query's squared norm, loaded up front so that its latency overlaps
-  // the score loads
+  const bool staged = L <= kGeoRowKeys;
+  float* se = sRows + (size_t)warp * 2 * kGeoRowKeys;   // scores, then e
+  float* sw = se + kGeoRowKeys;                          // w
+  // the row into shared memory, all copies in flight together: 16 bytes at a
+  // time where the row starts on a 16-byte boundary, else 4
+  if (staged) {
+    if ((reinterpret_cast<uintptr_t>(s) & 15) == 0) {
+      const int L4 = L & ~3;
+      for (int j = 4 * lane; j < L4; j += 128) cp_async16(se + j, s + j);
+      if (lane < L - L4) cp_async4(se + L4 + lane, s + L4 + lane);
+    } else {
+      for (int j = lane; j < L; j += 32) cp_async4(se + j, s + j);
+    }
+  }
+  // the query's squared norm while the copies land
   float qn = 0.0f;
   if (Q) {
     const float* q = Q + row * (long long)d;
     for (int k = lane; k < d; k += 32) qn = fmaf(q[k], q[k], qn);
   }
+  if (staged) {
+    cp_async_wait_all();
+    __syncwarp();
+  }
 
   // sweep 1: row extrema (section 3, calibration statistics)
-  float4 v[kGeoChunks];
   float m = -INFINITY, n = INFINITY;
-  if (in_regs) {
-#pragma unroll
-    for (int c = 0; c < kGeoChunks; ++c) {
-      if (c < nch) {
-        const int j = 4 * lane + 128 * c;
-        if (j + 3 < L) {
-          v[c] = __ldg(reinterpret_cast<const float4*>(s + j));
-          m = fmaxf(m, fmaxf(fmaxf(v[c].x, v[c].y), fmaxf(v[c].z, v[c].w)));
-          n = fminf(n, fminf(fminf(v[c].x, v[c].y), fminf(v[c].z, v[c].w)));
-        } else {
-          v[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (j < L) { v[c].x = s[j]; m = fmaxf(m, v[c].x); n = fminf(n, v[c].x); }
-          if (j + 1 < L) { v[c].y = s[j + 1]; m = fmaxf(m, v[c].y); n = fminf(n, v[c].y); }
-          if (j + 2 < L) { v[c].z = s[j + 2]; m = fmaxf(m, v[c].z); n = fminf(n, v[c].z); }
-        }
-      }
+  if (staged) {
+#pragma unroll 4
+    for (int j = lane; j < L; j += 32) {
+      const float x = se[j];
+      m = fmaxf(m, x);
+      n = fminf(n, x);
     }
   } else {
     for (int j = lane; j < L; j += 32) {
@@ -164,50 +166,38 @@ geometry_kernel(const float* __restrict__ S, const float* __restrict__ Q, long l
     r.g.q = sPair[0];
   }
 
-  // sweep 2: normalisers, entropy sums and top-bucket masses (the scores
-  // stay in registers; sweep 3 recomputes e and w from them, which keeps the
-  // register count low enough for more resident warps)
+  // sweep 2: normalisers, entropy sums and top-bucket masses, two keys
+  // (j, j + 32) at a time; a staged row keeps e and w for sweep 3
   GeoSums a = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (in_regs) {
-#pragma unroll
-    for (int cc = 0; cc < kGeoChunks; ++cc) {
-      if (cc < nch) {
-        const int j = 4 * lane + 128 * cc;
-        float x0 = v[cc].x, x1 = v[cc].y, x2 = v[cc].z, x3 = v[cc].w, w0, w1, w2, w3;
-        if (128 * cc + 128 <= L) {
-          geo_pair<V, false>(r, x0, x1, w0, w1, true, true, a);
-          geo_pair<V, false>(r, x2, x3, w2, w3, true, true, a);
-        } else {
-          geo_pair<V, true>(r, x0, x1, w0, w1, j < L, j + 1 < L, a);
-          geo_pair<V, true>(r, x2, x3, w2, w3, j + 2 < L, j + 3 < L, a);
+  auto sweep2 = [&](auto* src, auto keep_c) {
+    constexpr bool KEEP = decltype(keep_c)::value;
+    for (int j = lane; j < L; j += 64) {
+      const bool ok1 = j + 32 < L;
+      float x0 = src[j], x1 = ok1 ? src[j + 32] : m, w0, w1;
+      if (ok1) geo_pair<V, false>(r, x0, x1, w0, w1, true, true, a);
+      else geo_pair<V, true>(r, x0, x1, w0, w1, true, false, a);
+      if constexpr (KEEP) {
+        se[j] = x0;
+        sw[j] = w0;
+        if (ok1) {
+          se[j + 32] = x1;
+          sw[j + 32] = w1;
         }
       }
     }
-  } else {
-    for (int j = lane; j < L; j += 32) {
-      float x = s[j], y = m, w0, w1;
-      geo_pair<V, true>(r, x, y, w0, w1, true, false, a);
-    }
-  }
+  };
+  if (staged) sweep2(se, std::true_type{});
+  else sweep2(s, std::false_type{});
   const float Z = warp_sum(a.Z), Ex = warp_sum(a.Ex), W = warp_sum(a.W),
               Wlw = warp_sum(a.Wlw), Tsm = warp_sum(a.Tsm), Top = warp_sum(a.Top);
   const float rZ = 1.0f / Z, rW = 1.0f / W;
 
-  // sweep 3: total variation 1/2 sum_j |P_op,j - P_softmax,j|
+  // sweep 3: total variation 1/2 sum_j |P_op,j - P_softmax,j| (a long row
+  // recomputes e and w from its scores)
   float tv = 0.0f;
-  if (in_regs) {
-    GeoSums dummy = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int cc = 0; cc < kGeoChunks; ++cc) {
-      if (cc < nch) {
-        const int j = 4 * lane + 128 * cc;
-        float x0 = v[cc].x, x1 = v[cc].y, x2 = v[cc].z, x3 = v[cc].w, w0, w1, w2, w3;
-        geo_pair<V, true>(r, x0, x1, w0, w1, j < L, j + 1 < L, dummy);
-        geo_pair<V, true>(r, x2, x3, w2, w3, j + 2 < L, j + 3 < L, dummy);
-        tv += fabsf(fmaf(w0, rW, -x0 * rZ)) + fabsf(fmaf(w1, rW, -x1 * rZ)) +
-              fabsf(fmaf(w2, rW, -x2 * rZ)) + fabsf(fmaf(w3, rW, -x3 * rZ));
-      }
-    }
+  if (staged) {
+#pragma unroll 4
+    for (int j = lane; j < L; j += 32) tv += fabsf(fmaf(sw[j], rW, -se[j] * rZ));
   } else {
     GeoSums dummy = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = lane; j < L; j += 32) {

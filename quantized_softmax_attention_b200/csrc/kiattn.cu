@@ -446,8 +446,11 @@ int kiattn_geometry(const float* S, const float* Q, int B, int H, int T, int d,
   const int dq = Q ? d : 0;
   auto launch = [&](auto var) {
     using V = decltype(var);
-    geometry_kernel<V><<<(unsigned)blocks, 32 * kGeoWarps, 0, s>>>(S, Q, rows, T, dq,
-                                                                  cfg->causal, p, out);
+    if (cudaFuncSetAttribute(geometry_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kGeoSmemBytes) != cudaSuccess)
+      return;
+    geometry_kernel<V><<<(unsigned)blocks, 32 * kGeoWarps, kGeoSmemBytes, s>>>(
+        S, Q, rows, T, dq, cfg->causal, p, out);
   };
   const bool lerp = p.rec == KIA_REC_LERP;
   if (p.cal == KIA_CAL_MINMAX) {
