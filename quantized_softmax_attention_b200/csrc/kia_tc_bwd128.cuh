@@ -68,7 +68,8 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdQ,
                    const float* __restrict__ Q, const float* __restrict__ Kt,
                    const float* __restrict__ O, const float* __restrict__ dO, StatsView st,
-                   WorkView wk, float* __restrict__ dS_dbg, OpParams p, int B, int H, int T) {
+                   WorkView wk, float* __restrict__ dS_dbg, OpParams p, int B, int H, int T,
+                   int tab_in_smem, int nkmn) {
   constexpr int D = 128;
   __shared__ int s_hdr_ok;
   if (threadIdx.x == 0) {
@@ -82,14 +83,22 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   extern __shared__ uint8_t smraw[];
   uint8_t* base = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
   uint8_t* sKV = base;                                  // [2][K half | V half]
-  uint8_t* sKmn = sKV + 2 * 2 * kHalf128;               // [2][K half, MN-major]
-  float* sStage = reinterpret_cast<float*>(sKmn + 2 * kHalf128);   // [16 warps][32][8]
+  float* sStage = reinterpret_cast<float*>(sKV + 2 * 2 * kHalf128);   // [16 warps][32][8]
   float* sAC = sStage + kElemThreads / 32 * 256;        // [kRowSplit][2][128]
   float* sDc = sAC + 2 * kRowSplit * KIA_TILE;          // [128] centering D
-  float2* sPair = reinterpret_cast<float2*>(sDc + KIA_TILE);   // FWM grid pairs (+ zero pair)
-  const int pair_floats = (!V::SOFTMAX && !V::MINMAX) ? 2 * (p.K + 1) : 0;
+  // FWM grid pairs (+ the tail's zero pair), or under MinMax the rows' own
+  // grids [K + 1][128] when they fit
+  float2* sPair = reinterpret_cast<float2*>(sDc + KIA_TILE);
+  float* sTab = reinterpret_cast<float*>(sPair);
+  const int pair_floats = V::SOFTMAX ? 0
+                        : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
   BwdQ128Bars& bar =
       *reinterpret_cast<BwdQ128Bars*>(reinterpret_cast<float*>(sPair) + ((pair_floats + 31) & ~31));
+  // the MN-major K ring last (1024-aligned): two slots, one when a MinMax
+  // grid table needs the room (only the producer and the dQ issuer use it)
+  const int NKM = V::MINMAX ? nkmn : 2;
+  uint8_t* sKmn =
+      base + ((reinterpret_cast<uint8_t*>(&bar + 1) - base + 1023) & ~(ptrdiff_t)1023);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = B * H;
@@ -160,8 +169,8 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
           }
         }
         if (im >= 0) {
-          const int sl = gm & 1;
-          if (mbar_test(&bar.kmn_empty[sl], ((gm >> 1) & 1) ^ 1)) {
+          const int sl = gm % NKM;
+          if (mbar_test(&bar.kmn_empty[sl], ((gm / NKM) & 1) ^ 1)) {
             uint8_t* dst = sKmn + sl * kHalf128;
             mbar_arrive_expect_tx(&bar.kmn_full[sl], kHalf128);
             for (int b = 0; b < D / 32; ++b)
@@ -222,9 +231,9 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       const int nunits = item_units(it);
       for (int u = 0; u < nunits; ++u, ++g) {
-        const int sl = g & 1;
+        const int sl = g % NKM;
         if (!warp_wait(&bar.elem_done, g & 1, abort)) { failed = true; break; }
-        if (!warp_wait(&bar.kmn_full[sl], (g >> 1) & 1, abort)) { failed = true; break; }
+        if (!warp_wait(&bar.kmn_full[sl], (g / NKM) & 1, abort)) { failed = true; break; }
         // the accumulator restarts with this item: the previous item's
         // epilogue must have read it
         if (u == 0 && n > 0 && !warp_wait(&bar.dq_free, (n - 1) & 1, abort)) { failed = true; break; }
@@ -307,6 +316,12 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
           if (qq < T) wk.D[qrr] = acc;
         }
       }
+      if constexpr (V::MINMAX) {
+        // the row's grid, column r of [K + 1][128] (four threads per row)
+        if (tab_in_smem)
+          for (int k = part; k <= p.K; k += kRowSplit)
+            sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
+      }
       mbar_arrive(&bar.row_sync);
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (2 * n) & 1, abort))) { failed = true; break; }
       const float Dc = sDc[r];
@@ -350,7 +365,8 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         }
       };
       if constexpr (V::MINMAX) {
-        unit_loop(GridF{st.table + qr * (p.K + 1), 1});
+        if (tab_in_smem) unit_loop(GridF{sTab + r, KIA_TILE});
+        else unit_loop(GridF{st.table + qr * (p.K + 1), 1});
       } else if constexpr (V::SOFTMAX) {
         unit_loop(GridP{sPair});
       } else {
@@ -433,11 +449,14 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-inline size_t tc_bwd_q128_smem(const OpParams& p) {
-  const int pair_floats = (!p.softmax && p.cal != KIA_CAL_MINMAX) ? 2 * (p.K + 1) : 0;
-  return 1024 + 2 * 2 * (size_t)kHalf128 + 2 * (size_t)kHalf128 + kElemThreads / 32 * 1024 +
-         (2 * kRowSplit + 1) * KIA_TILE * 4 + (size_t)((pair_floats + 31) & ~31) * 4 +
-         sizeof(BwdQ128Bars);
+inline size_t tc_bwd_q128_smem(const OpParams& p, bool tab_in_smem, int nkmn) {
+  const bool minmax = !p.softmax && p.cal == KIA_CAL_MINMAX;
+  const size_t tab = p.softmax ? 0 : (minmax ? (tab_in_smem ? (size_t)(p.K + 1) * KIA_TILE : 0)
+                                              : 2 * (size_t)(p.K + 1));
+  const size_t head = 2 * 2 * (size_t)kHalf128 + kElemThreads / 32 * 1024 +
+                      (2 * kRowSplit + 1) * KIA_TILE * 4 + ((tab + 31) & ~(size_t)31) * 4 +
+                      sizeof(BwdQ128Bars);
+  return 1024 + ((head + 1023) & ~(size_t)1023) + (size_t)nkmn * kHalf128;
 }
 
 
@@ -914,7 +933,17 @@ int tc_backward128_v(const float* Q, const float* Kt, const float* Vv, const flo
       !make_tmap_out(&tdq, dQ, BH, T, D) || !make_tmap_out(&tdk, dK, BH, T, D) ||
       !make_tmap_out(&tdv, dV, BH, T, D))
     return KIA_ERR_CUDA;
-  const size_t smq = tc_bwd_q128_smem(p), smk = tc_bwd_kv128_smem(p);
+  // the rows' MinMax grids in shared memory where they fit, with the
+  // MN-major K ring one slot shallower if that is what makes them fit
+  constexpr size_t kMax = 232448;
+  bool q_tab = true;
+  int nkmn = 2;
+  if (tc_bwd_q128_smem(p, true, nkmn) > kMax) nkmn = 1;
+  if (tc_bwd_q128_smem(p, true, nkmn) > kMax) {
+    q_tab = false;
+    nkmn = 2;
+  }
+  const size_t smq = tc_bwd_q128_smem(p, q_tab, nkmn), smk = tc_bwd_kv128_smem(p);
   if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
   const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
                                     p.grad == KIA_GRAD_MIN_ONLY);
@@ -927,7 +956,7 @@ int tc_backward128_v(const float* Q, const float* Kt, const float* Vv, const flo
         cudaSuccess)
       return KIA_ERR_CUDA;
     kern<<<grid, kTcThreads, smq, s>>>(tkh, tkmh, tvh, tdq, Q, Kt, O, dO, st, wk, dS_dbg, p, B, H,
-                                       T);
+                                       T, q_tab ? 1 : 0, nkmn);
     return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
   };
   int rc = need_c ? launch_q(tc_bwd_q128_kernel<V, true>) : launch_q(tc_bwd_q128_kernel<V, false>);
