@@ -51,6 +51,7 @@ constexpr int kKvSlots = 2;       // key pass: slots of each half-tile query rin
 
 struct BwdQBars {
   uint64_t qd_full, qd_empty;     // Q_i, dO_i (K-major), per item
+  uint64_t d_read;                // the element warps done reading dO_i for the centering D
   uint64_t kv_full[3], kv_empty[3];     // half tiles of K, V K-major (for S, dP)
   uint64_t kmn_full[3], kmn_empty[3];   // half tiles of K MN-major (for dQ)
   uint64_t sp_full[3];            // S and dP of a half tile in TMEM region r
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKmn,
                 const __grid_constant__ CUtensorMap tmV, const float* __restrict__ Kt,
-                const float* __restrict__ O, const float* __restrict__ dO,
+                const float* __restrict__ O,
                 const __grid_constant__ CUtensorMap tmdQ, StatsView st, WorkView wk,
                 float* __restrict__ dS_dbg, OpParams p, int B, int H, int T, int tab_in_smem,
                 int nkv) {
@@ -140,6 +141,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(&bar.qd_full, 1);
     mbar_init(&bar.qd_empty, 1);
+    mbar_init(&bar.d_read, kElemThreads);
     for (int sl = 0; sl < kBwdSlots; ++sl) {
       mbar_init(&bar.kv_full[sl], 1);
       mbar_init(&bar.kv_empty[sl], 1);
@@ -186,7 +188,11 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       PollGuard guard;
       while ((iq >= 0 || ik >= 0 || im >= 0) && !failed) {
         bool moved = false;
-        if (iq >= 0 && mbar_test(&bar.qd_empty, (nq & 1) ^ 1)) {
+        // Q_i and dO_i replace the previous item's once its S and dP MMAs are
+        // done and the element warps have read its dO for D (an item of two
+        // half tiles can finish its MMAs before that)
+        if (iq >= 0 && mbar_test(&bar.qd_empty, (nq & 1) ^ 1) &&
+            (nq == 0 || mbar_test(&bar.d_read, (nq - 1) & 1))) {
           mbar_arrive_expect_tx(&bar.qd_full, 2 * kTile);
           for (int b = 0; b < D / 32; ++b) {
             tma_load_3d(sQ + b * 32 * KIA_TILE, &tmQ, &bar.qd_full, b * 32, item_qt(iq) * KIA_TILE,
@@ -331,39 +337,50 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int k = (int)threadIdx.x - 64; k <= p.K; k += kElemThreads)
         sPair[k] = k < p.K ? make_float2(st.table[k], st.table[k + 1]) : make_float2(0.0f, 0.0f);
     }
+    // An item's prologue operands from global memory: this row's
+    // calibration (written by the forward), and a quarter of a row of O_bar
+    // (O, or O_L for Prob-STE) for the centering D = dO . O_bar, which four
+    // consecutive element threads form for one row, with dO from the item's
+    // tile in shared memory, and add by shuffles.  They are loaded during the
+    // previous item's epilogue, so that their DRAM latency passes during its
+    // stores.
+    const int e = (int)threadIdx.x - 64;
+    const int rr = e >> 2, cc = e & 3;         // row of the tile, quarter of the row
+    struct Pro {
+      float m, rh, Wb;
+      int am, an;
+      float4 ob[D / 16];
+    };
+    auto load_pro = [&](int it, Pro& x) {
+      const long long rb = (long long)item_bh(it) * T;
+      const int q = item_qt(it) * KIA_TILE + r, qq = item_qt(it) * KIA_TILE + rr;
+      const long long qr = rb + (q < T ? q : T - 1), qrr = rb + (qq < T ? qq : T - 1);
+      x.m = st.m[qr];
+      x.am = st.am[qr];
+      x.an = V::MINMAX ? st.an[qr] : x.am;
+      x.rh = st.rh[qr];
+      x.Wb = st.Wb[qr];
+      const float4* o4 =
+          reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qrr * D) + cc * (D / 16);
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) x.ob[c] = o4[c];
+    };
+    Pro pro;
     int gbase = 0, n = 0;
     ItemSeq seq(nitems);
-    for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
+    int it0 = seq.next();
+    if (it0 >= 0) load_pro(it0, pro);
+    for (int it = it0; it >= 0 && !failed; it = seq.next(), ++n) {
       const int qt = item_qt(it), bh = item_bh(it), nunits = item_units(it);
       const int q = qt * KIA_TILE + r;
       const long long rowbase = (long long)bh * T;
       const long long qr = rowbase + (q < T ? q : T - 1);
-      // Every global load of the item's prologue is issued before the first
-      // use of any of them (a warp stalls at its first use of a pending load,
-      // so loads behind it would wait a round trip more): this row's
-      // calibration (written by the forward), then the operands of the
-      // centering D = dO . O_bar (O_bar = O, or O_L for Prob-STE), which four
-      // consecutive element threads read for one row (coalesced) and add by
-      // shuffles, leaving the row's D in shared memory.
-      const float m = st.m[qr];
-      const int am = st.am[qr], an = V::MINMAX ? st.an[qr] : am;
-      const float rh = st.rh[qr];
-      const float Wb = st.Wb[qr];
-      const int e = (int)threadIdx.x - 64;
-      const int rr = e >> 2, cc = e & 3;       // row of the tile, quarter of the row
+      const float m = pro.m;
+      const int am = pro.am, an = pro.an;
+      const float rh = pro.rh;
+      const float Wb = pro.Wb;
       const int qq = qt * KIA_TILE + rr;
       const long long qrr = rowbase + (qq < T ? qq : T - 1);
-      float4 ga[D / 16], ob[D / 16];
-      {
-        const float4* g4 = reinterpret_cast<const float4*>(dO + qrr * D) + cc * (D / 16);
-        const float4* o4 =
-            reinterpret_cast<const float4*>((V::PROB ? st.OL : O) + qrr * D) + cc * (D / 16);
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          ga[c] = g4[c];
-          ob[c] = o4[c];
-        }
-      }
       const float nrh = -rh;
       const float dg = (V::MINMAX && rh == 0.0f) ? 1.0f : 0.0f;
       const int L = p.causal ? q + 1 : T;
@@ -373,14 +390,21 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       prefetch_l2(Kt + (rowbase + am) * D + part * (D / kRowSplit));
       if constexpr (V::MINMAX) prefetch_l2(Kt + (rowbase + an) * D + part * (D / kRowSplit));
       {
+        // dO_i's row rr, columns 16 cc .. 16 cc + 15: column block cc / 2 of
+        // the tile, 16-byte chunks (cc % 2) 4 + c, stored at chunk position
+        // chunk ^ (row % 8) of the row's 128 bytes (the 128-byte swizzle)
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.qd_full, n & 1, abort))) { failed = true; break; }
+        const uint8_t* grow = reinterpret_cast<const uint8_t*>(sG) + (cc >> 1) * (KIA_TILE * 128) + rr * 128;
         float acc = 0.0f;
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
-          acc = fmaf(ga[c].x, ob[c].x, acc);
-          acc = fmaf(ga[c].y, ob[c].y, acc);
-          acc = fmaf(ga[c].z, ob[c].z, acc);
-          acc = fmaf(ga[c].w, ob[c].w, acc);
+          const float4 ga = *reinterpret_cast<const float4*>(grow + ((((cc & 1) * 4 + c) ^ (rr & 7)) * 16));
+          acc = fmaf(ga.x, pro.ob[c].x, acc);
+          acc = fmaf(ga.y, pro.ob[c].y, acc);
+          acc = fmaf(ga.z, pro.ob[c].z, acc);
+          acc = fmaf(ga.w, pro.ob[c].w, acc);
         }
+        mbar_arrive(&bar.d_read);
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
         if (cc == 0) {
@@ -452,31 +476,6 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (failed) break;
       gbase += nunits;
-      {
-        // the next item's rows (statistics, dO and O_bar for its centering)
-        // into L2 while this item's epilogue runs
-        ItemSeq peek = seq;
-        const int nx = peek.next();
-        if (nx >= 0) {
-          const int e = (int)threadIdx.x - 64;
-          const int qn = item_qt(nx) * KIA_TILE + (e >> 2);
-          const long long rn = (long long)item_bh(nx) * T + (qn < T ? qn : T - 1);
-          prefetch_l2(dO + rn * D + (e & 3) * (D / 4));
-          prefetch_l2((V::PROB ? st.OL : O) + rn * D + (e & 3) * (D / 4));
-          if (e < 5 * 4) {
-            // 128 rows of one per-row array = four 128-byte lines
-            const long long r0 = (long long)item_bh(nx) * T + item_qt(nx) * KIA_TILE +
-                                 32 * (e & 3);
-            const int a = e >> 2;
-            const void* ptr = a == 0 ? (const void*)(st.m + r0)
-                            : a == 1 ? (const void*)(st.am + r0)
-                            : a == 2 ? (const void*)(st.an + r0)
-                            : a == 3 ? (const void*)(st.rh + r0)
-                                     : (const void*)(st.Wb + r0);
-            if (item_qt(nx) * KIA_TILE + 32 * (e & 3) < T) prefetch_l2(ptr);
-          }
-        }
-      }
       // this thread's columns of the key rows of the row's calibration terms
       // (argmax, argmin), loaded now so that their latency passes during the
       // waits below
@@ -536,6 +535,21 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             o[4 * i + 1] = fmaf(gn, kk.y, o[4 * i + 1]);
             o[4 * i + 2] = fmaf(gn, kk.z, o[4 * i + 2]);
             o[4 * i + 3] = fmaf(gn, kk.w, o[4 * i + 3]);
+          }
+        }
+      }
+      {
+        // the next item's prologue operands: their latency passes during the
+        // stores below
+        ItemSeq peek = seq;
+        const int nx = peek.next();
+        if (nx >= 0) {
+          load_pro(nx, pro);
+          if constexpr (V::MINMAX) {
+            // and its rows of the grid table into L2 (copied in its prologue)
+            const int qn = item_qt(nx) * KIA_TILE + r;
+            if (tab_in_smem && part == 0)
+              prefetch_l2(st.table + ((long long)item_bh(nx) * T + (qn < T ? qn : T - 1)) * (p.K + 1));
           }
         }
       }
@@ -1175,14 +1189,14 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
-    tc_bwd_q_kernel<D, V, true><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
+    tc_bwd_q_kernel<D, V, true><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O,
                                                               tdq, st, wk, dS_dbg, p, B, H, T,
                                                               q_tab_smem ? 1 : 0, nkv);
   } else {
     if (cudaFuncSetAttribute(tc_bwd_q_kernel<D, V, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq) != cudaSuccess)
       return KIA_ERR_CUDA;
-    tc_bwd_q_kernel<D, V, false><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O, dO,
+    tc_bwd_q_kernel<D, V, false><<<qgrid, kTcThreads, smq, s>>>(tq, tg, tkh, tkmh, tvh, Kt, O,
                                                                tdq, st, wk, dS_dbg, p, B, H, T,
                                                                q_tab_smem ? 1 : 0, nkv);
   }
