@@ -65,7 +65,7 @@ struct FwdBars {
   uint64_t pv_done[3];   // sweep 2: P V of region r finished (tcgen05.commit)
   uint64_t o_full;       // all P V of an item done
   uint64_t o_free;       // the item's O (and O_L) read out of TMEM
-  uint64_t row_sync;     // element-thread rendezvous, three times per item
+  uint64_t row_sync;     // element-thread rendezvous, two or three times per item
   uint32_t tmem_base;
   int abort;
 };
@@ -317,7 +317,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int r = quad * 32 + lane;            // query row in the tile
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const float Kf = p.Kf, Km1f = (float)(p.K - 1);
-    int gbase = 0, n = 0;
+    int gbase = 0, n = 0, rs = 0;   // rs: row_sync phases passed
     ItemSeq seq(nitems);
     for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       const int qt = item_qt(it), bh = item_bh(it), nunits = 2 * item_nkt(it);
@@ -378,7 +378,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       rx.am[part][r] = am;
       rx.an[part][r] = an;
       mbar_arrive(&bar.row_sync);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n) & 1, abort))) { failed = true; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, rs++ & 1, abort))) { failed = true; break; }
       m = rx.m[0][r];
       am = rx.am[0][r];
       n_ = rx.n[0][r];
@@ -431,8 +431,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
         }
       }
-      mbar_arrive(&bar.row_sync);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n + 1) & 1, abort))) { failed = true; break; }
+      // the grid in place before sweep 2: per row under MinMax; FWM's shared
+      // grid is built with the CTA's first item only (softmax has none)
+      if (V::MINMAX || (!V::SOFTMAX && n == 0)) {
+        mbar_arrive(&bar.row_sync);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, rs++ & 1, abort))) { failed = true; break; }
+      }
       // sweep 2: weights -> P (and P_L) in TMEM, normalisers (even and odd
       // columns summed separately, as packed pairs)
       float2 W2 = make_float2(0.0f, 0.0f), WL2 = make_float2(0.0f, 0.0f);
@@ -508,7 +512,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       rx.W[part][r] = W2.x + W2.y;
       rx.WL[part][r] = WL2.x + WL2.y;
       mbar_arrive(&bar.row_sync);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (3 * n + 2) & 1, abort))) { failed = true; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, rs++ & 1, abort))) { failed = true; break; }
       const float Wrow = (rx.W[0][r] + rx.W[1][r]) + (rx.W[2][r] + rx.W[3][r]);
       const float WLrow =
           PROB ? (rx.WL[0][r] + rx.WL[1][r]) + (rx.WL[2][r] + rx.WL[3][r]) : Wrow;
