@@ -43,26 +43,29 @@ __device__ __forceinline__ uint32_t visible16(int kj, int q0, int T, bool causal
   return vis;
 }
 
-// x added to element i of a 16-register array, i known only at run time (a
-// jump on i instead of a loop over the 16 candidates)
-__device__ __forceinline__ void add_at16(float (&a)[16], int i, float x) {
-  switch (i) {
-    case 0: a[0] += x; break;
-    case 1: a[1] += x; break;
-    case 2: a[2] += x; break;
-    case 3: a[3] += x; break;
-    case 4: a[4] += x; break;
-    case 5: a[5] += x; break;
-    case 6: a[6] += x; break;
-    case 7: a[7] += x; break;
-    case 8: a[8] += x; break;
-    case 9: a[9] += x; break;
-    case 10: a[10] += x; break;
-    case 11: a[11] += x; break;
-    case 12: a[12] += x; break;
-    case 13: a[13] += x; break;
-    case 14: a[14] += x; break;
-    default: a[15] += x; break;
+// Calibration terms of a chunk of 16 query columns: bm (bn) marks, the same
+// in every lane of the warp, the columns whose argmax (argmin) key lies among
+// the warp's 32 keys; cm[i] (cn[i]) holds column i's (key offset in the tile,
+// coefficient bits), and the thread holding that key adds the coefficient to
+// column i's score gradient.  Unrolled over the columns with compile-time
+// indices: a loop over the set bits with a jump on a run-time index into the
+// register array cost many times its instruction count.
+template <bool MINMAX>
+__device__ __forceinline__ void add_calibration16(float (&g)[16], uint32_t bm, uint32_t bn,
+                                                  const int2* cm, const int2* cn, int r) {
+  if ((bm | bn) == 0u) return;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if ((bm >> i) & 1u) {
+      const int2 c = cm[i];
+      g[i] += c.x == r ? __int_as_float(c.y) : 0.0f;
+    }
+    if constexpr (MINMAX) {
+      if ((bn >> i) & 1u) {
+        const int2 c = cn[i];
+        g[i] += c.x == r ? __int_as_float(c.y) : 0.0f;
+      }
+    }
   }
 }
 

@@ -852,24 +852,14 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         if constexpr (!PROJ && !V::SOFTMAX) {
           // calibration terms for the chunk's queries whose argmax (argmin) key
-          // lies in this warp's 32 keys
+          // lies in this warp's 32 keys (masks made visibly warp-uniform)
           const int hq = part >> 1, sh = 16 * (part & 1);
-          uint32_t bm = (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
-          while (bm != 0u) {
-            const int i = __ffs(bm) - 1;
-            bm &= bm - 1u;
-            const int2 c = sCM[e0 + i];
-            if (c.x == r) add_at16(gg, i, __int_as_float(c.y));
-          }
-          if constexpr (V::MINMAX) {
-            uint32_t bn = (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu;
-            while (bn != 0u) {
-              const int i = __ffs(bn) - 1;
-              bn &= bn - 1u;
-              const int2 c = sCN[e0 + i];
-              if (c.x == r) add_at16(gg, i, __int_as_float(c.y));
-            }
-          }
+          const uint32_t bm =
+              __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu, 0);
+          const uint32_t bn = V::MINMAX
+              ? __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu, 0)
+              : 0u;
+          add_calibration16<V::MINMAX>(gg, bm, bn, sCM + e0, sCN + e0, r);
         }
         tmem_st16(tmem + lane_addr + kColS + 16u * part, v);
         tmem_st16(tmem + lane_addr + kColP + 16u * part, gg);
