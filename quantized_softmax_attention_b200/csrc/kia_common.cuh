@@ -589,6 +589,22 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+// One column of the warp's 32 TMEM lanes: read (waiting for it), and write.
+__device__ __forceinline__ float tmem_ld1_sync(uint32_t taddr) {
+  uint32_t x;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(x)
+      : "r"(taddr)
+      : "memory");
+  return __uint_as_float(x);
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr),
+               "r"(__float_as_uint(v))
+               : "memory");
+}
 
 // Named barrier among `count` threads (multiple of 32), id 1..15.
 __device__ __forceinline__ void named_bar_sync(int id, int count) {

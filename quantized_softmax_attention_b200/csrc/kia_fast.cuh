@@ -43,29 +43,30 @@ __device__ __forceinline__ uint32_t visible16(int kj, int q0, int T, bool causal
   return vis;
 }
 
-// Calibration terms of a chunk of 16 query columns: bm (bn) marks, the same
-// in every lane of the warp, the columns whose argmax (argmin) key lies among
-// the warp's 32 keys; cm[i] (cn[i]) holds column i's (key offset in the tile,
-// coefficient bits), and the thread holding that key adds the coefficient to
-// column i's score gradient.  Unrolled over the columns with compile-time
-// indices: a loop over the set bits with a jump on a run-time index into the
-// register array cost many times its instruction count.
-template <bool MINMAX>
-__device__ __forceinline__ void add_calibration16(float (&g)[16], uint32_t bm, uint32_t bn,
-                                                  const int2* cm, const int2* cn, int r) {
+// Calibration terms of a chunk of 16 query columns, added in tensor memory
+// once the chunk's score gradients are stored there, column i at TMEM address
+// col0 + i for this warp's 32 lanes: bm (bn) marks, the same in every lane,
+// the columns whose argmax (argmin) key lies among the warp's 32 keys; cm[i]
+// (cn[i]) holds column i's (key offset in the tile, coefficient bits).  Per
+// marked column the warp reads the column, the thread holding that key adds
+// the coefficient, and the warp writes the column back, argmax terms before
+// argmin terms.  A few instructions per term: adding into the registers
+// instead needs a jump on a run-time index into the array or a test per
+// column, and either cost many times that.
+__device__ __forceinline__ void add_calibration_tmem(uint32_t col0, uint32_t bm, uint32_t bn,
+                                                     const int2* cm, const int2* cn, int r) {
   if ((bm | bn) == 0u) return;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if ((bm >> i) & 1u) {
-      const int2 c = cm[i];
-      g[i] += c.x == r ? __int_as_float(c.y) : 0.0f;
-    }
-    if constexpr (MINMAX) {
-      if ((bn >> i) & 1u) {
-        const int2 c = cn[i];
-        g[i] += c.x == r ? __int_as_float(c.y) : 0.0f;
-      }
-    }
+  tmem_st_wait();   // the chunk's own stores have landed
+  while ((bm | bn) != 0u) {
+    const bool fm = bm != 0u;
+    const int i = __ffs(fm ? bm : bn) - 1;
+    if (fm) bm &= bm - 1u;
+    else bn &= bn - 1u;
+    const int2 c = (fm ? cm : cn)[i];
+    const uint32_t ta = col0 + (uint32_t)i;
+    const float x = tmem_ld1_sync(ta);
+    tmem_st1(ta, c.x == r ? x + __int_as_float(c.y) : x);
+    tmem_st_wait();   // before a later term of the same column reads it
   }
 }
 

@@ -1072,10 +1072,13 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const uint32_t bn = V::MINMAX
                 ? __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu, 0)
                 : 0u;
-            add_calibration16<V::MINMAX>(g, bm, bn, sCM + e0, sCN + e0, r);
+            tmem_st16(tmem + lane_addr + cs, v);
+            tmem_st16(tmem + lane_addr + cs + 64u, g);
+            add_calibration_tmem(tmem + lane_addr + cs + 64u, bm, bn, sCM + e0, sCN + e0, r);
+          } else {
+            tmem_st16(tmem + lane_addr + cs, v);
+            tmem_st16(tmem + lane_addr + cs + 64u, g);
           }
-          tmem_st16(tmem + lane_addr + cs, v);
-          tmem_st16(tmem + lane_addr + cs + 64u, g);
         }
         tmem_st_wait();
         tc_fence_before();

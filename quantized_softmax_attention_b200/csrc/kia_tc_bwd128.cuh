@@ -859,10 +859,13 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           const uint32_t bn = V::MINMAX
               ? __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu, 0)
               : 0u;
-          add_calibration16<V::MINMAX>(gg, bm, bn, sCM + e0, sCN + e0, r);
+          tmem_st16(tmem + lane_addr + kColS + 16u * part, v);
+          tmem_st16(tmem + lane_addr + kColP + 16u * part, gg);
+          add_calibration_tmem(tmem + lane_addr + kColP + 16u * part, bm, bn, sCM + e0, sCN + e0, r);
+        } else {
+          tmem_st16(tmem + lane_addr + kColS + 16u * part, v);
+          tmem_st16(tmem + lane_addr + kColP + 16u * part, gg);
         }
-        tmem_st16(tmem + lane_addr + kColS + 16u * part, v);
-        tmem_st16(tmem + lane_addr + kColP + 16u * part, gg);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bar.elem_done);
