@@ -462,16 +462,45 @@ inline size_t tc_bwd_q128_smem(const OpParams& p, bool tab_in_smem, int nkmn) {
 
 // ------------------------------------------------------------------ key pass
 
+// Eight columns of the warp's 32 TMEM lanes (the key pass's half units).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t x[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]),
+                 "=r"(x[6]), "=r"(x[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(x[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait_regs8(float (&v)[8], float (&w)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                 "+f"(v[6]), "+f"(v[7]), "+f"(w[0]), "+f"(w[1]), "+f"(w[2]), "+f"(w[3]),
+                 "+f"(w[4]), "+f"(w[5]), "+f"(w[6]), "+f"(w[7])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+
 struct BwdKV128Bars {
   uint64_t k_ready;                // K of the item written into TMEM (element threads)
   uint64_t k_free;                 // the item's S^T MMAs are done with it
   uint64_t v_full, v_empty;        // V of the item (shared memory, K-major)
   uint64_t qd_full, qd_empty;      // Q and dO half tiles, K-major (for S^T, dP^T)
   uint64_t mn_full, mn_empty;      // Q and dO half tiles, MN-major (for dK, dV)
-  uint64_t sp_full;                // S^T, dP^T of a unit in the region
+  // the region holds a unit's two halves of 32 queries side by side
+  // (columns S [32 h, 32 h + 32), dP the same 64 further), each with its own
+  // barriers, so that one half's MMAs overlap the other half's element work
+  uint64_t sp_full[2];             // S^T, dP^T of half h in the region
   uint64_t qc_ready[2], qc_free[2];   // per-query constants of a unit in slot s
-  uint64_t elem_done;              // P^T, dS^T written over S^T, dP^T
-  uint64_t st_free;                // the unit's dV, dK MMAs done: region free
+  uint64_t elem_done[2];           // P^T, dS^T of half h written over S^T, dP^T
+  uint64_t st_free[2];             // half h's dV, dK MMAs done: its columns free
   uint64_t acc_full, acc_free;
   uint64_t acc_issued;             // the item's last dV, dK MMAs issued
   uint32_t tmem_base;
@@ -524,13 +553,15 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     mbar_init(&bar.qd_empty, 1);
     mbar_init(&bar.mn_full, 1);
     mbar_init(&bar.mn_empty, 1);
-    mbar_init(&bar.sp_full, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bar.sp_full[h], 1);
+      mbar_init(&bar.elem_done[h], kElemThreads);
+      mbar_init(&bar.st_free[h], 1);
+    }
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bar.qc_ready[s], 32);
       mbar_init(&bar.qc_free[s], kElemThreads);
     }
-    mbar_init(&bar.elem_done, kElemThreads);
-    mbar_init(&bar.st_free, 1);
     mbar_init(&bar.acc_full, 1);
     mbar_init(&bar.acc_free, kElemThreads);
     mbar_init(&bar.acc_issued, 1);
@@ -606,8 +637,10 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------- score-MMA issuer
-    // S^T = K Q^T (A = K from TMEM), dP^T = V dO^T (A = V from shared memory)
-    const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
+    // S^T = K Q^T (A = K from TMEM), dP^T = V dO^T (A = V from shared memory),
+    // one half of 32 queries at a time (N = 32; the half's rows start 4 KB
+    // into each 128-byte-swizzled column block of the half tile)
+    const uint32_t id_s = idesc_tf32(128, 32, 0, 0);
     const uint64_t dva = desc_kmajor(smem_u32(sV), 0);
     const uint64_t dqd = desc_kmajor_half(smem_u32(sQD));
     const uint64_t dgd = dqd + desc_step(kHalf128);
@@ -619,23 +652,29 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       // the previous item's last dV / dK MMAs ahead of this item's scores
       if (n > 0 && !warp_wait(&bar.acc_issued, (n - 1) & 1, abort)) { failed = true; break; }
       const int nunits = item_units(it);
-      for (int u = 0; u < nunits; ++u, ++g) {
-        if (g > 0 && !warp_wait(&bar.st_free, (g - 1) & 1, abort)) { failed = true; break; }
+      for (int u = 0; u < nunits && !failed; ++u, ++g) {
         if (!warp_wait(&bar.qd_full, g & 1, abort)) { failed = true; break; }
-        if (elect_one()) {
-          tc_fence_after();
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          // half h's columns are free once the previous unit's half-h dV, dK
+          // MMAs are done
+          if (g > 0 && !warp_wait(&bar.st_free[h], (g - 1) & 1, abort)) { failed = true; break; }
+          const uint64_t hq = desc_step(4096u * (uint32_t)h);
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ts(tmem + kColS, tmem + kColK + 8u * ks, dqd + kstep_kmajor_half(ks), id_s,
-                        ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ts(tmem + kColS + 32u * h, tmem + kColK + 8u * ks,
+                          dqd + hq + kstep_kmajor_half(ks), id_s, ks > 0 ? 1u : 0u);
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ss(tmem + kColP, dva + kstep_kmajor(ks), dgd + kstep_kmajor_half(ks), id_s,
-                        ks > 0 ? 1u : 0u);
-          tc_commit(&bar.sp_full);
-          tc_commit(&bar.qd_empty);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ss(tmem + kColP + 32u * h, dva + kstep_kmajor(ks),
+                          dgd + hq + kstep_kmajor_half(ks), id_s, ks > 0 ? 1u : 0u);
+            tc_commit(&bar.sp_full[h]);
+            if (h == 1) tc_commit(&bar.qd_empty);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
       if (failed) break;
       if (elect_one()) {
@@ -653,25 +692,30 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     ItemSeq seq(nitems);
     for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       const int nunits = item_units(it);
-      for (int u = 0; u < nunits; ++u, ++g) {
-        if (!warp_wait(&bar.elem_done, g & 1, abort)) { failed = true; break; }
-        if (!warp_wait(&bar.mn_full, g & 1, abort)) { failed = true; break; }
-        if (u == 0 && n > 0 && !warp_wait(&bar.acc_free, (n - 1) & 1, abort)) { failed = true; break; }
-        const uint32_t acc0 = u > 0 ? 1u : 0u;
-        if (elect_one()) {
-          tc_fence_after();
+      for (int u = 0; u < nunits && !failed; ++u, ++g) {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          // half h: queries 32 h .. 32 h + 31 of the unit, the MN-major
+          // k-steps 4 h .. 4 h + 3 of the half tile
+          if (!warp_wait(&bar.elem_done[h], g & 1, abort)) { failed = true; break; }
+          if (h == 0 && !warp_wait(&bar.mn_full, g & 1, abort)) { failed = true; break; }
+          if (u == 0 && h == 0 && n > 0 && !warp_wait(&bar.acc_free, (n - 1) & 1, abort)) { failed = true; break; }
+          const uint32_t acc0 = (u > 0 || h > 0) ? 1u : 0u;
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + kColDV, tmem + kColS + 8u * kk, dgm + kstep_mnmajor(kk), id_acc,
-                        kk > 0 ? 1u : acc0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_tf32_ts(tmem + kColDV, tmem + kColS + 32u * h + 8u * kk,
+                          dgm + kstep_mnmajor(4 * h + kk), id_acc, kk > 0 ? 1u : acc0);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + kColDK, tmem + kColP + 8u * kk, dqm + kstep_mnmajor(kk), id_acc,
-                        kk > 0 ? 1u : acc0);
-          tc_commit(&bar.st_free);
-          tc_commit(&bar.mn_empty);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_tf32_ts(tmem + kColDK, tmem + kColP + 32u * h + 8u * kk,
+                          dqm + kstep_mnmajor(4 * h + kk), id_acc, kk > 0 ? 1u : acc0);
+            tc_commit(&bar.st_free[h]);
+            if (h == 1) tc_commit(&bar.mn_empty);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
       if (failed) break;
       if (elect_one()) {
@@ -788,22 +832,26 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int qi = q0 + (u >> 1);
         const int sl = g & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.qc_ready[sl], (g >> 1) & 1, abort))) { failed = true; break; }
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full, g & 1, abort))) { failed = true; break; }
-        tc_fence_after();
         const bool edge =
             (p.causal && qi == kt) || (qi + 1) * KIA_TILE > T || (kt + 1) * KIA_TILE > T;
-        float v[16], gg[16];
-        tmem_ld16(tmem + lane_addr + kColS + 16u * part, v);
-        tmem_ld16(tmem + lane_addr + kColP + 16u * part, gg);
-        tmem_ld_wait_regs(v, gg);
-        const int ql0 = 64 * (u & 1) + 16 * part;   // first query (in the tile) of the chunk
-        const int e0 = sl * kSlotQ + 16 * part;     // its slot entry
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+        // half h: this thread's 8 query columns 32 h + 8 part .. + 7
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[h], g & 1, abort))) { failed = true; break; }
+        tc_fence_after();
+        const uint32_t cS = kColS + 32u * h + 8u * part, cP = kColP + 32u * h + 8u * part;
+        float v[8], gg[8];
+        tmem_ld8(tmem + lane_addr + cS, v);
+        tmem_ld8(tmem + lane_addr + cP, gg);
+        tmem_ld_wait_regs8(v, gg);
+        const int ql0 = 64 * (u & 1) + 32 * h + 8 * part;   // first query (in the tile) of the chunk
+        const int e0 = sl * kSlotQ + 32 * h + 8 * part;     // its slot entry
         // one body for every unit; the masked pairs of an edge unit are
         // zeroed afterwards (finite scores: the clamped grid index stays in
         // the table)
         auto body = [&]() {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             [[maybe_unused]] const int ql = ql0 + i;
             const float4 cq = sC4[e0 + i];
             float4 xq = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -842,9 +890,10 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         };
         body();
         if (edge) {
+          // bits 0..7 of the mask of the 16 queries from ql0
           const uint32_t vis = visible16(kj, qi * KIA_TILE + ql0, T, p.causal != 0);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             const bool keep = (vis >> i) & 1u;
             v[i] = keep ? v[i] : 0.0f;
             gg[i] = keep ? gg[i] : 0.0f;
@@ -852,23 +901,26 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         if constexpr (!PROJ && !V::SOFTMAX) {
           // calibration terms for the chunk's queries whose argmax (argmin) key
-          // lies in this warp's 32 keys (masks made visibly warp-uniform)
-          const int hq = part >> 1, sh = 16 * (part & 1);
+          // lies in this warp's 32 keys (masks of the half's 32 queries, made
+          // visibly warp-uniform; this thread's 8 bits)
+          const int sh = 8 * part;
           const uint32_t bm =
-              __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 0) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu, 0);
+              __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 0) * 4 + quad) * 2 + h] >> sh) & 0xFFu, 0);
           const uint32_t bn = V::MINMAX
-              ? __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 1) * 4 + quad) * 2 + hq] >> sh) & 0xFFFFu, 0)
+              ? __shfl_sync(0xffffffffu, (sMask[((sl * 2 + 1) * 4 + quad) * 2 + h] >> sh) & 0xFFu, 0)
               : 0u;
-          tmem_st16(tmem + lane_addr + kColS + 16u * part, v);
-          tmem_st16(tmem + lane_addr + kColP + 16u * part, gg);
-          add_calibration_tmem(tmem + lane_addr + kColP + 16u * part, bm, bn, sCM + e0, sCN + e0, r);
+          tmem_st8(tmem + lane_addr + cS, v);
+          tmem_st8(tmem + lane_addr + cP, gg);
+          add_calibration_tmem(tmem + lane_addr + cP, bm, bn, sCM + e0, sCN + e0, r);
         } else {
-          tmem_st16(tmem + lane_addr + kColS + 16u * part, v);
-          tmem_st16(tmem + lane_addr + kColP + 16u * part, gg);
+          tmem_st8(tmem + lane_addr + cS, v);
+          tmem_st8(tmem + lane_addr + cP, gg);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bar.elem_done);
+        mbar_arrive(&bar.elem_done[h]);
+        }
+        if (failed) break;
         mbar_arrive(&bar.qc_free[sl]);
       }
       if (failed) break;
