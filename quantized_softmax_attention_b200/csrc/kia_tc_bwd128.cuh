@@ -48,14 +48,43 @@ __device__ __forceinline__ void row_to_tmem32(uint32_t taddr, const float* row) 
 
 // ---------------------------------------------------------------- query pass
 
+// Eight columns of the warp's 32 TMEM lanes (the passes' half units).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t x[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]),
+                 "=r"(x[6]), "=r"(x[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(x[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait_regs8(float (&v)[8], float (&w)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                 "+f"(v[6]), "+f"(v[7]), "+f"(w[0]), "+f"(w[1]), "+f"(w[2]), "+f"(w[3]),
+                 "+f"(w[4]), "+f"(w[5]), "+f"(w[6]), "+f"(w[7])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+
 struct BwdQ128Bars {
   uint64_t qd_ready;               // Q, dO of the item written into TMEM (element threads)
   uint64_t qd_free;                // the item's S / dP MMAs are done with them
   uint64_t kv_full[2], kv_empty[2];    // K | V half tiles (K-major)
   uint64_t kmn_full[2], kmn_empty[2];  // K half tiles (MN-major)
-  uint64_t sp_full;                // S, dP of a unit in the region
-  uint64_t elem_done;              // dS written over S
-  uint64_t st_free;                // the unit's dQ MMAs done: region free
+  // the region holds a unit's two halves of 32 keys side by side (columns
+  // S [32 h, 32 h + 32), dP the same 64 further), each with its own barriers,
+  // so that one half's MMAs overlap the other half's element work
+  uint64_t sp_full[2];             // S, dP of half h in the region
+  uint64_t elem_done[2];           // dS of half h written over S
+  uint64_t st_free[2];             // half h's dQ MMAs done: its columns free
   uint64_t dq_full, dq_free;
   uint64_t row_sync;
   uint32_t tmem_base;
@@ -118,9 +147,11 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       mbar_init(&bar.kmn_full[s], 1);
       mbar_init(&bar.kmn_empty[s], 1);
     }
-    mbar_init(&bar.sp_full, 1);
-    mbar_init(&bar.elem_done, kElemThreads);
-    mbar_init(&bar.st_free, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bar.sp_full[h], 1);
+      mbar_init(&bar.elem_done[h], kElemThreads);
+      mbar_init(&bar.st_free[h], 1);
+    }
     mbar_init(&bar.dq_full, 1);
     mbar_init(&bar.dq_free, kElemThreads);
     mbar_init(&bar.row_sync, kElemThreads);
@@ -187,36 +218,42 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     }
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------- score-MMA issuer
-    // S = Q K^T and dP = dO V^T with A from TMEM; whole warp in the loop, one
-    // elected lane issuing
-    const uint32_t id_s = idesc_tf32(128, 64, 0, 0);
+    // S = Q K^T and dP = dO V^T with A from TMEM, one half of 32 keys at a
+    // time (N = 32; the half's rows start 4 KB into each 128-byte-swizzled
+    // column block of the half tile); whole warp in the loop, one elected
+    // lane issuing
+    const uint32_t id_s = idesc_tf32(128, 32, 0, 0);
     const uint64_t dkv = desc_kmajor_half(smem_u32(sKV));
     int g = 0, n = 0;
     ItemSeq seq(nitems);
     for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       if (!warp_wait(&bar.qd_ready, n & 1, abort)) { failed = true; break; }
       const int nunits = item_units(it);
-      for (int u = 0; u < nunits; ++u, ++g) {
-        // the region is free once the previous unit's dQ MMAs are done
-        if (g > 0 && !warp_wait(&bar.st_free, (g - 1) & 1, abort)) { failed = true; break; }
+      for (int u = 0; u < nunits && !failed; ++u, ++g) {
         const int sl = g & 1;
         if (!warp_wait(&bar.kv_full[sl], (g >> 1) & 1, abort)) { failed = true; break; }
-        const uint64_t dk = dkv + desc_step((uint32_t)sl * 2 * kHalf128);
-        const uint64_t dv = dk + desc_step(kHalf128);
-        if (elect_one()) {
-          tc_fence_after();
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          // half h's columns are free once the previous unit's half-h dQ MMAs
+          // are done
+          if (g > 0 && !warp_wait(&bar.st_free[h], (g - 1) & 1, abort)) { failed = true; break; }
+          const uint64_t dk = dkv + desc_step((uint32_t)sl * 2 * kHalf128 + 4096u * (uint32_t)h);
+          const uint64_t dv = dk + desc_step(kHalf128);
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ts(tmem + kColS, tmem + kColQ + 8u * ks, dk + kstep_kmajor_half(ks), id_s,
-                        ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ts(tmem + kColS + 32u * h, tmem + kColQ + 8u * ks,
+                          dk + kstep_kmajor_half(ks), id_s, ks > 0 ? 1u : 0u);
 #pragma unroll
-          for (int ks = 0; ks < D / 8; ++ks)
-            mma_tf32_ts(tmem + kColP, tmem + kColG + 8u * ks, dv + kstep_kmajor_half(ks), id_s,
-                        ks > 0 ? 1u : 0u);
-          tc_commit(&bar.sp_full);
-          tc_commit(&bar.kv_empty[sl]);
+            for (int ks = 0; ks < D / 8; ++ks)
+              mma_tf32_ts(tmem + kColP + 32u * h, tmem + kColG + 8u * ks,
+                          dv + kstep_kmajor_half(ks), id_s, ks > 0 ? 1u : 0u);
+            tc_commit(&bar.sp_full[h]);
+            if (h == 1) tc_commit(&bar.kv_empty[sl]);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
       if (failed) break;
       if (elect_one()) tc_commit(&bar.qd_free);   // Q, dO in TMEM free once these MMAs are done
@@ -230,25 +267,30 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     ItemSeq seq(nitems);
     for (int it = seq.next(); it >= 0 && !failed; it = seq.next(), ++n) {
       const int nunits = item_units(it);
-      for (int u = 0; u < nunits; ++u, ++g) {
+      for (int u = 0; u < nunits && !failed; ++u, ++g) {
         const int sl = g % NKM;
-        if (!warp_wait(&bar.elem_done, g & 1, abort)) { failed = true; break; }
-        if (!warp_wait(&bar.kmn_full[sl], (g / NKM) & 1, abort)) { failed = true; break; }
-        // the accumulator restarts with this item: the previous item's
-        // epilogue must have read it
-        if (u == 0 && n > 0 && !warp_wait(&bar.dq_free, (n - 1) & 1, abort)) { failed = true; break; }
         const uint64_t db = dkm + desc_step((uint32_t)sl * kHalf128);
-        const uint32_t acc0 = u > 0 ? 1u : 0u;
-        if (elect_one()) {
-          tc_fence_after();
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          // half h: keys 32 h .. 32 h + 31 of the unit, the MN-major k-steps
+          // 4 h .. 4 h + 3 of the half tile
+          if (!warp_wait(&bar.elem_done[h], g & 1, abort)) { failed = true; break; }
+          if (h == 0 && !warp_wait(&bar.kmn_full[sl], (g / NKM) & 1, abort)) { failed = true; break; }
+          // the accumulator restarts with this item: the previous item's
+          // epilogue must have read it
+          if (u == 0 && h == 0 && n > 0 && !warp_wait(&bar.dq_free, (n - 1) & 1, abort)) { failed = true; break; }
+          const uint32_t acc0 = (u > 0 || h > 0) ? 1u : 0u;
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ts(tmem + kColDQ, tmem + kColS + 8u * kk, db + kstep_mnmajor(kk), id_dq,
-                        kk > 0 ? 1u : acc0);
-          tc_commit(&bar.st_free);
-          tc_commit(&bar.kmn_empty[sl]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_tf32_ts(tmem + kColDQ, tmem + kColS + 32u * h + 8u * kk,
+                          db + kstep_mnmajor(4 * h + kk), id_dq, kk > 0 ? 1u : acc0);
+            tc_commit(&bar.st_free[h]);
+            if (h == 1) tc_commit(&bar.kmn_empty[sl]);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
       if (failed) break;
       if (elect_one()) tc_commit(&bar.dq_full);
@@ -329,39 +371,44 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       float A = 0.0f, C = 0.0f;
       auto unit_loop = [&](const auto& grid) {
         for (int u = 0; u < nunits && !failed; ++u, ++g) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full, g & 1, abort))) { failed = true; break; }
-          tc_fence_after();
-          const int key0 = 64 * u + 16 * part;
           const bool edge = (p.causal && (u >> 1) == qt) || 64 * u + 64 > T;
-          float v[16], gg[16];
-          tmem_ld16(tmem + lane_addr + kColS + 16u * part, v);
-          tmem_ld16(tmem + lane_addr + kColP + 16u * part, gg);
-          tmem_ld_wait_regs(v, gg);
-          if (!edge) {
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            // half h: this thread's 8 key columns 32 h + 8 part .. + 7
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[h], g & 1, abort))) { failed = true; break; }
+            tc_fence_after();
+            const int key0 = 64 * u + 32 * h + 8 * part;
+            const uint32_t cS = kColS + 32u * h + 8u * part, cP = kColP + 32u * h + 8u * part;
+            float v[8], gg[8];
+            tmem_ld8(tmem + lane_addr + cS, v);
+            tmem_ld8(tmem + lane_addr + cP, gg);
+            tmem_ld_wait_regs8(v, gg);
+            if (!edge) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float dw = fmaf(gg[i], rWb, nDr);
-              v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+              for (int i = 0; i < 8; ++i) {
+                const float dw = fmaf(gg[i], rWb, nDr);
+                v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int key = key0 + i;
+                const bool ok = key < T && (!p.causal || key <= q);
+                const float dw = ok ? fmaf(gg[i], rWb, nDr) : 0.0f;
+                v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+              }
             }
-          } else {
+            tmem_st8(tmem + lane_addr + cS, v);
+            if (dS_dbg && q < T) {
+              float* dst = dS_dbg + (rowbase + q) * T + key0;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int key = key0 + i;
-              const bool ok = key < T && (!p.causal || key <= q);
-              const float dw = ok ? fmaf(gg[i], rWb, nDr) : 0.0f;
-              v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+              for (int i = 0; i < 8; ++i)
+                if (key0 + i < T) dst[i] = v[i];
             }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bar.elem_done[h]);
           }
-          tmem_st16(tmem + lane_addr + kColS + 16u * part, v);
-          if (dS_dbg && q < T) {
-            float* dst = dS_dbg + (rowbase + q) * T + key0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (key0 + i < T) dst[i] = v[i];
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&bar.elem_done);
         }
       };
       if constexpr (V::MINMAX) {
@@ -461,32 +508,6 @@ inline size_t tc_bwd_q128_smem(const OpParams& p, bool tab_in_smem, int nkmn) {
 
 
 // ------------------------------------------------------------------ key pass
-
-// Eight columns of the warp's 32 TMEM lanes (the key pass's half units).
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t x[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]),
-                 "=r"(x[6]), "=r"(x[7])
-               : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(x[i]);
-}
-__device__ __forceinline__ void tmem_ld_wait_regs8(float (&v)[8], float (&w)[8]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
-                 "+f"(v[6]), "+f"(v[7]), "+f"(w[0]), "+f"(w[1]), "+f"(w[2]), "+f"(w[3]),
-                 "+f"(w[4]), "+f"(w[5]), "+f"(w[6]), "+f"(w[7])
-               :
-               : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
-               : "memory");
-}
 
 struct BwdKV128Bars {
   uint64_t k_ready;                // K of the item written into TMEM (element threads)
