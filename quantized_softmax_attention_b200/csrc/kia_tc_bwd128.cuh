@@ -524,6 +524,10 @@ struct BwdKV128Bars {
   uint64_t st_free[2];             // half h's dV, dK MMAs done: its columns free
   uint64_t acc_full, acc_free;
   uint64_t acc_issued;             // the item's last dV, dK MMAs issued
+  // MinMax with the queries' grids in shared memory: table slot h holds the
+  // 32 grids of the current unit's half h
+  uint64_t tab_ready[2];           // half h's grids copied into slot h (constant warp)
+  uint64_t tab_free[2];            // the element warps done with slot h
   uint32_t tmem_base;
   int abort;
 };
@@ -534,7 +538,7 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmGmn,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdK,
                     const __grid_constant__ CUtensorMap tmdV, const float* __restrict__ Kt,
-                    StatsView st, WorkView wk, OpParams p, int BH, int T) {
+                    StatsView st, WorkView wk, OpParams p, int BH, int T, int tab_in_smem) {
   constexpr int D = 128;
   if (*wk.status != 0) return;
   extern __shared__ uint8_t smraw[];
@@ -555,6 +559,10 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int pair_floats = (!V::SOFTMAX && !V::MINMAX) ? 2 * (p.K + 1) : 0;
   BwdKV128Bars& bar =
       *reinterpret_cast<BwdKV128Bars*>(reinterpret_cast<float*>(sPair) + ((pair_floats + 31) & ~31));
+  // MinMax: two slots of 32 queries' grids ([slot][32][K + 1]) after the barriers
+  const int K1 = p.K + 1;
+  const bool tabs = V::MINMAX && tab_in_smem;
+  float* sTabH = reinterpret_cast<float*>(&bar + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
@@ -586,6 +594,10 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     mbar_init(&bar.acc_full, 1);
     mbar_init(&bar.acc_free, kElemThreads);
     mbar_init(&bar.acc_issued, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bar.tab_ready[h], 32);
+      mbar_init(&bar.tab_free[h], kElemThreads);
+    }
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -822,6 +834,31 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       }
       __syncwarp();
       mbar_arrive(&bar.qc_ready[sl]);
+      if (tabs) {
+        // the unit's grids, half h into slot h once the element warps are
+        // done with the previous unit's half h (asynchronous copies; rows
+        // past T are filled with ones, their queries are masked)
+        const long long rowbase = (long long)item_bh(it) * T;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          if (g > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar.tab_free[h], (g - 1) & 1, abort))) {
+            failed = true;
+            break;
+          }
+          const int qf = 64 * (2 * item_q0(it) + u) + 32 * h;
+          const int nvalid = max(0, min(32, T - qf)) * K1, ntot = 32 * K1;
+          const float* src = st.table + (rowbase + qf) * K1;
+          float* dst = sTabH + h * 32 * K1;
+          for (int x = lane; x < ntot; x += 32) {
+            if (x < nvalid) cp_async4(dst + x, src + x);
+            else dst[x] = 1.0f;
+          }
+          cp_async_wait_all();
+          __syncwarp();
+          mbar_arrive(&bar.tab_ready[h]);
+        }
+        if (failed) break;
+      }
       cur = nxt;
       it = it2;
       u = u2;
@@ -858,6 +895,7 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
         // half h: this thread's 8 query columns 32 h + 8 part .. + 7
+        if (tabs && !__all_sync(0xffffffffu, mbar_wait(&bar.tab_ready[h], g & 1, abort))) { failed = true; break; }
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[h], g & 1, abort))) { failed = true; break; }
         tc_fence_after();
         const uint32_t cS = kColS + 32u * h + 8u * part, cP = kColP + 32u * h + 8u * part;
@@ -870,7 +908,8 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // one body for every unit; the masked pairs of an edge unit are
         // zeroed afterwards (finite scores: the clamped grid index stays in
         // the table)
-        auto body = [&]() {
+        auto body = [&](auto tabs_c) {
+          [[maybe_unused]] constexpr bool TABS = decltype(tabs_c)::value;   // grids in shared memory
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             [[maybe_unused]] const int ql = ql0 + i;
@@ -893,7 +932,9 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
               const float t = __fsub_rn(uu, __fsub_rn(tmp, kMagic));
               float2 gp;
               if constexpr (V::MINMAX) {
-                const float* gq = st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * (p.K + 1);
+                const float* gq;
+                if constexpr (TABS) gq = sTabH + (h * 32 + 8 * part + i) * K1;
+                else gq = st.table + (rowbase + min(qi * KIA_TILE + ql, T - 1)) * (p.K + 1);
                 gp = GridF{gq, 1}.pair(__float_as_int(tmp) - kMagicBits);
               } else {
                 gp = gridz.at(__float_as_int(tmp) - kMagicBits, uu > Kf);
@@ -909,7 +950,9 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             gg[i] = dS;
           }
         };
-        body();
+        if (tabs) body(std::true_type{});
+        else body(std::false_type{});
+        if (tabs) mbar_arrive(&bar.tab_free[h]);   // the half's grids have been read
         if (edge) {
           // bits 0..7 of the mask of the 16 queries from ql0
           const uint32_t vis = visible16(kj, qi * KIA_TILE + ql0, T, p.causal != 0);
@@ -975,11 +1018,12 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-inline size_t tc_bwd_kv128_smem(const OpParams& p) {
+inline size_t tc_bwd_kv128_smem(const OpParams& p, bool tab_in_smem) {
   const int pair_floats = (!p.softmax && p.cal != KIA_CAL_MINMAX) ? 2 * (p.K + 1) : 0;
+  const size_t tab = tab_in_smem ? 2 * 32 * (size_t)(p.K + 1) * 4 : 0;
   return 1024 + 128 * KIA_TILE * 4 + 4 * (size_t)kHalf128 + 2 * 64 * (16 + 16 + 8 + 8) +
          2 * 2 * 4 * 2 * 4 + kElemThreads / 32 * 1024 + (size_t)((pair_floats + 31) & ~31) * 4 +
-         sizeof(BwdKV128Bars);
+         sizeof(BwdKV128Bars) + tab;
 }
 
 // The d = 128 backward: query pass, then key pass (the projection's scan
@@ -1009,7 +1053,9 @@ int tc_backward128_v(const float* Q, const float* Kt, const float* Vv, const flo
     q_tab = false;
     nkmn = 2;
   }
-  const size_t smq = tc_bwd_q128_smem(p, q_tab, nkmn), smk = tc_bwd_kv128_smem(p);
+  // the key pass holds two halves' query grids where they fit
+  const bool kv_tab = !p.softmax && p.cal == KIA_CAL_MINMAX && tc_bwd_kv128_smem(p, true) <= kMax;
+  const size_t smq = tc_bwd_q128_smem(p, q_tab, nkmn), smk = tc_bwd_kv128_smem(p, kv_tab);
   if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
   const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
                                     p.grad == KIA_GRAD_MIN_ONLY);
@@ -1032,7 +1078,8 @@ int tc_backward128_v(const float* Q, const float* Kt, const float* Vv, const flo
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk) !=
         cudaSuccess)
       return KIA_ERR_CUDA;
-    kern<<<grid, kTcThreads, smk, s>>>(tqh, tqmh, tgh, tgmh, tv, tdk, tdv, Kt, st, wk, p, BH, T);
+    kern<<<grid, kTcThreads, smk, s>>>(tqh, tqmh, tgh, tgmh, tv, tdk, tdv, Kt, st, wk, p, BH, T,
+                                       kv_tab ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
   };
   const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;
