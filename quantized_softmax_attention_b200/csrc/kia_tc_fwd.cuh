@@ -100,10 +100,20 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   FwdRowX& rx = *reinterpret_cast<FwdRowX*>(sV + NSV * kTileF);
   // epilogue: 1 KB per element warp to turn its rows into full-sector stores
   float* sStage = reinterpret_cast<float*>(&rx + 1);      // [16 warps][32][8]
-  float* sTab = sStage + kElemThreads / 32 * 256;
-  const int tab_floats =
-      V::SOFTMAX ? 0 : (V::MINMAX ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
-  FwdBars& bar = *reinterpret_cast<FwdBars*>(sTab + ((tab_floats + 31) & ~31));
+  // the grid table: FWM's pairs, or MinMax's rows [K + 1][128] when
+  // tab_in_smem is 1 (after the staging block) or 2 (over it: the table is
+  // written after sweep 1 and read in sweep 2, the staging block written in
+  // the epilogue, so each warp lets its stores read their staging before the
+  // rendezvous that precedes the table's writes)
+  constexpr int kStageF = kElemThreads / 32 * 256;
+  float* sTab = (V::MINMAX && tab_in_smem == 2) ? sStage : sStage + kStageF;
+  const int tab_end =
+      V::SOFTMAX ? kStageF
+                 : (V::MINMAX ? (tab_in_smem == 1   ? kStageF + (p.K + 1) * KIA_TILE
+                                 : tab_in_smem == 2 ? max(kStageF, (p.K + 1) * KIA_TILE)
+                                                    : kStageF)
+                              : kStageF + 2 * (p.K + 1));
+  FwdBars& bar = *reinterpret_cast<FwdBars*>(sStage + ((tab_end + 31) & ~31));
   // the K ring last (1024-aligned), so that its depth moves no other buffer
   float* sK = reinterpret_cast<float*>(
       base + ((reinterpret_cast<uint8_t*>(&bar + 1) - base + 1023) & ~(ptrdiff_t)1023));
@@ -372,6 +382,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
       if (failed) break;
+      if (V::MINMAX && tab_in_smem == 2) {
+        // the table overlays the staging block: this warp's epilogue stores
+        // of the previous item have read it before the rendezvous below
+        if (elect_one()) tma_store_wait_read();
+        __syncwarp();
+      }
       // merge the four threads of the row (lowest index on ties)
       rx.m[part][r] = m;
       rx.n[part][r] = n_;
@@ -569,14 +585,21 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// tab_in_smem: 0 MinMax grids in global memory, 1 in their own region, 2 over
+// the epilogue's staging block
 template <int D, bool PROB>
-size_t tc_fwd_smem(const OpParams& p, bool tab_in_smem, int nsk) {
+size_t tc_fwd_smem(const OpParams& p, int tab_in_smem, int nsk) {
   using Cfg = FwdCfg<D, PROB>;
   const bool minmax_tab = !p.softmax && p.cal == KIA_CAL_MINMAX;
-  const int tab =
-      p.softmax ? 0 : (minmax_tab ? (tab_in_smem ? (p.K + 1) * KIA_TILE : 0) : 2 * (p.K + 1));
+  const int stage_f = kElemThreads / 32 * 256;
+  const int tab_end =
+      p.softmax ? stage_f
+                : (minmax_tab ? (tab_in_smem == 1   ? stage_f + (p.K + 1) * KIA_TILE
+                                 : tab_in_smem == 2 ? std::max(stage_f, (p.K + 1) * KIA_TILE)
+                                                    : stage_f)
+                              : stage_f + 2 * (p.K + 1));
   const size_t head = (size_t)(1 + Cfg::kVStages) * Cfg::kTileBytes + sizeof(FwdRowX) +
-                      kElemThreads / 32 * 1024 + (size_t)((tab + 31) & ~31) * 4 + sizeof(FwdBars);
+                      (size_t)((tab_end + 31) & ~31) * 4 + sizeof(FwdBars);
   return 1024 + ((head + 1023) & ~(size_t)1023) + (size_t)nsk * Cfg::kTileBytes;
 }
 
@@ -588,17 +611,23 @@ int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   // shallower if that is what makes it fit; else the grids are read from
   // global memory
   constexpr int kNsk = FwdCfg<D, V::PROB>::kKStages;
-  bool tab_in_smem = true;
+  int tab_in_smem = 1;
   int nsk = kNsk;
-  size_t smem = tc_fwd_smem<D, V::PROB>(p, true, nsk);
+  size_t smem = tc_fwd_smem<D, V::PROB>(p, 1, nsk);
   if (smem > 232448 && kNsk > 2) {
     nsk = kNsk - 1;
-    smem = tc_fwd_smem<D, V::PROB>(p, true, nsk);
+    smem = tc_fwd_smem<D, V::PROB>(p, 1, nsk);
+  }
+  if (smem > 232448 && V::MINMAX) {
+    // over the staging block, with the full K ring
+    tab_in_smem = 2;
+    nsk = kNsk;
+    smem = tc_fwd_smem<D, V::PROB>(p, 2, nsk);
   }
   if (smem > 232448) {
-    tab_in_smem = false;
+    tab_in_smem = 0;
     nsk = kNsk;
-    smem = tc_fwd_smem<D, V::PROB>(p, false, nsk);
+    smem = tc_fwd_smem<D, V::PROB>(p, 0, nsk);
   }
   if (smem > 232448) return KIA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(tc_fwd_kernel<D, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -610,7 +639,7 @@ int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   if (sms <= 0) return KIA_ERR_CUDA;
   const dim3 grid(std::min(sms, B * H * nt));
   tc_fwd_kernel<D, V><<<grid, kTcThreads, smem, s>>>(tq, tk, tv, to, tol, st, p, B, H, T,
-                                                     tab_in_smem ? 1 : 0, nsk);
+                                                     tab_in_smem, nsk);
   return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
 }
 
