@@ -18,11 +18,15 @@
 //    S^T = K Q^T (TS), dP^T = V dO^T (SS: V stays in shared memory)
 //    P^T and dS^T over S^T and dP^T, dV += P^T dO, dK += dS^T Q (TS, N = 128)
 //
-// With one region per pass the units run one after another (MMAs of a unit,
-// then its element stage, then its accumulating MMAs); all sixteen element
-// warps work on every unit, four threads per row, 16 columns each.  The
-// stationary rows are copied into tensor memory by the element threads at
-// the start of each item, once the previous item's MMAs are done with them.
+// With one region per pass, each unit runs as two halves of 32 keys (query
+// pass) or 32 queries (key pass) side by side in the region, each with its
+// own barriers: a half's N = 32 score MMAs, its element stage and its
+// accumulating MMAs overlap the other half's.  All sixteen element warps work
+// on every half, four threads per row, 8 columns each.  The stationary rows
+// are copied into tensor memory by the element threads at the start of each
+// item, once the previous item's MMAs are done with them.  Under MinMax the
+// key pass keeps each half's 32 query grids in one of two shared-memory
+// slots, refilled by the constant warp as the element warps release them.
 #pragma once
 #include "kia_tc_bwd.cuh"
 
