@@ -42,6 +42,21 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // Number of SMs of the current device (cached per device; 0 on error).
+// Dynamic shared memory a launch of `kern` may request: the device's opt-in
+// per-block maximum less the kernel's own static shared memory (0 if either
+// cannot be read).  Sizes are checked against this rather than the device
+// maximum alone, which a kernel with static shared variables cannot reach.
+template <class F>
+inline size_t dyn_smem_budget(F* kern) {
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return 0;
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, kern) != cudaSuccess) return 0;
+  return optin > (int)a.sharedSizeBytes ? (size_t)optin - a.sharedSizeBytes : 0;
+}
+
 inline int num_sms() {
   static int cache[64] = {0};
   int dev = 0;

@@ -1154,26 +1154,30 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
     return KIA_ERR_CUDA;
   // MinMax grid tables in shared memory where they fit, with one ring a slot
   // shallower if that is what makes them fit; else read from global memory
-  constexpr size_t kMax = 232448;
+  const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
+                                    p.grad == KIA_GRAD_MIN_ONLY);
+  const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;
+  const size_t kMaxQ = need_c ? dyn_smem_budget(tc_bwd_q_kernel<D, V, true>)
+                              : dyn_smem_budget(tc_bwd_q_kernel<D, V, false>);
+  const size_t kMaxK = proj ? dyn_smem_budget(tc_bwd_kv_kernel<D, V, true>)
+                            : dyn_smem_budget(tc_bwd_kv_kernel<D, V, false>);
   bool q_tab_smem = true;
   int nkv = kBwdSlots;
-  if (tc_bwd_q_smem<D>(p, true, nkv) > kMax) nkv = kBwdSlots - 1;
-  if (tc_bwd_q_smem<D>(p, true, nkv) > kMax) {
+  if (tc_bwd_q_smem<D>(p, true, nkv) > kMaxQ) nkv = kBwdSlots - 1;
+  if (tc_bwd_q_smem<D>(p, true, nkv) > kMaxQ) {
     q_tab_smem = false;
     nkv = kBwdSlots;
   }
   const size_t smq = tc_bwd_q_smem<D>(p, q_tab_smem, nkv);
   bool kv_tab_smem = true;
   int nmn = kKvSlots;
-  if (tc_bwd_kv_smem<D>(p, true, nmn) > kMax) nmn = kKvSlots - 1;
-  if (tc_bwd_kv_smem<D>(p, true, nmn) > kMax) {
+  if (tc_bwd_kv_smem<D>(p, true, nmn) > kMaxK) nmn = kKvSlots - 1;
+  if (tc_bwd_kv_smem<D>(p, true, nmn) > kMaxK) {
     kv_tab_smem = false;
     nmn = kKvSlots;
   }
   const size_t smk = tc_bwd_kv_smem<D>(p, kv_tab_smem, nmn);
-  if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
-  const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
-                                    p.grad == KIA_GRAD_MIN_ONLY);
+  if (smq > kMaxQ || smk > kMaxK) return KIA_ERR_UNSUPPORTED;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   // both passes are persistent: one CTA per SM walks the items
   const int sms = num_sms();
@@ -1204,7 +1208,6 @@ int tc_backward_v(const float* Q, const float* Kt, const float* Vv, const float*
                                         kv_tab_smem ? 1 : 0, nmn);
     return KIA_OK;
   };
-  const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;
   if ((proj ? launch_kv(tc_bwd_kv_kernel<D, V, true>) : launch_kv(tc_bwd_kv_kernel<D, V, false>)))
     return KIA_ERR_CUDA;
   mark(5, s);

@@ -1049,20 +1049,24 @@ int tc_backward128_v(const float* Q, const float* Kt, const float* Vv, const flo
     return KIA_ERR_CUDA;
   // the rows' MinMax grids in shared memory where they fit, with the
   // MN-major K ring one slot shallower if that is what makes them fit
-  constexpr size_t kMax = 232448;
+  const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
+                                    p.grad == KIA_GRAD_MIN_ONLY);
+  const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;
+  const size_t kMaxQ = need_c ? dyn_smem_budget(tc_bwd_q128_kernel<V, true>)
+                              : dyn_smem_budget(tc_bwd_q128_kernel<V, false>);
+  const size_t kMaxK = proj ? dyn_smem_budget(tc_bwd_kv128_kernel<V, true>)
+                            : dyn_smem_budget(tc_bwd_kv128_kernel<V, false>);
   bool q_tab = true;
   int nkmn = 2;
-  if (tc_bwd_q128_smem(p, true, nkmn) > kMax) nkmn = 1;
-  if (tc_bwd_q128_smem(p, true, nkmn) > kMax) {
+  if (tc_bwd_q128_smem(p, true, nkmn) > kMaxQ) nkmn = 1;
+  if (tc_bwd_q128_smem(p, true, nkmn) > kMaxQ) {
     q_tab = false;
     nkmn = 2;
   }
   // the key pass holds two halves' query grids where they fit
-  const bool kv_tab = !p.softmax && p.cal == KIA_CAL_MINMAX && tc_bwd_kv128_smem(p, true) <= kMax;
+  const bool kv_tab = !p.softmax && p.cal == KIA_CAL_MINMAX && tc_bwd_kv128_smem(p, true) <= kMaxK;
   const size_t smq = tc_bwd_q128_smem(p, q_tab, nkmn), smk = tc_bwd_kv128_smem(p, kv_tab);
-  if (smq > 232448 || smk > 232448) return KIA_ERR_UNSUPPORTED;
-  const bool need_c = V::MINMAX && (p.grad == KIA_GRAD_FULL || p.grad == KIA_GRAD_MAX_ONLY ||
-                                    p.grad == KIA_GRAD_MIN_ONLY);
+  if (smq > kMaxQ || smk > kMaxK) return KIA_ERR_UNSUPPORTED;
   const int nt = (T + KIA_TILE - 1) / KIA_TILE;
   const int sms = num_sms();
   if (sms <= 0) return KIA_ERR_CUDA;
@@ -1086,7 +1090,6 @@ int tc_backward128_v(const float* Q, const float* Kt, const float* Vv, const flo
                                        kv_tab ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? KIA_OK : KIA_ERR_CUDA;
   };
-  const bool proj = !V::SOFTMAX && p.grad == KIA_GRAD_PROJECT;
   rc = proj ? launch_kv(tc_bwd_kv128_kernel<V, true>) : launch_kv(tc_bwd_kv128_kernel<V, false>);
   if (rc) return rc;
   mark(5, s);

@@ -611,25 +611,26 @@ int tc_forward_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   // shallower if that is what makes it fit; else the grids are read from
   // global memory
   constexpr int kNsk = FwdCfg<D, V::PROB>::kKStages;
+  const size_t kMax = dyn_smem_budget(tc_fwd_kernel<D, V>);
   int tab_in_smem = 1;
   int nsk = kNsk;
   size_t smem = tc_fwd_smem<D, V::PROB>(p, 1, nsk);
-  if (smem > 232448 && kNsk > 2) {
+  if (smem > kMax && kNsk > 2) {
     nsk = kNsk - 1;
     smem = tc_fwd_smem<D, V::PROB>(p, 1, nsk);
   }
-  if (smem > 232448 && V::MINMAX) {
+  if (smem > kMax && V::MINMAX) {
     // over the staging block, with the full K ring
     tab_in_smem = 2;
     nsk = kNsk;
     smem = tc_fwd_smem<D, V::PROB>(p, 2, nsk);
   }
-  if (smem > 232448) {
+  if (smem > kMax) {
     tab_in_smem = 0;
     nsk = kNsk;
     smem = tc_fwd_smem<D, V::PROB>(p, 0, nsk);
   }
-  if (smem > 232448) return KIA_ERR_UNSUPPORTED;
+  if (smem > kMax) return KIA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(tc_fwd_kernel<D, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return KIA_ERR_CUDA;
