@@ -327,6 +327,18 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar.qd_ready);
+      {
+        // the next item's Q and dO rows into L2 now, so that their copy into
+        // tensor memory at its start waits for L2 rather than DRAM
+        ItemSeq peek = seq;
+        const int nx = peek.next();
+        if (nx >= 0) {
+          const int qn = item_qt(nx) * KIA_TILE + r;
+          const long long qrn = (long long)item_bh(nx) * T + (qn < T ? qn : T - 1);
+          prefetch_l2(Q + qrn * D + 32 * part);
+          prefetch_l2(dO + qrn * D + 32 * part);
+        }
+      }
       // this row's calibration and centering (written by the forward)
       const float m = st.m[qr];
       const int am = st.am[qr], an = V::MINMAX ? st.an[qr] : am;
@@ -890,6 +902,16 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar.k_ready);
+      {
+        // the next item's K row into L2 now (its copy into tensor memory then
+        // waits for L2 rather than DRAM)
+        ItemSeq peek = seq;
+        const int nx = peek.next();
+        if (nx >= 0) {
+          const int kn = item_kt(nx) * KIA_TILE + r;
+          prefetch_l2(Kt + ((long long)item_bh(nx) * T + (kn < T ? kn : T - 1)) * D + 32 * part);
+        }
+      }
       for (int u = 0; u < nunits && !failed; ++u, ++g) {
         const int qi = q0 + (u >> 1);
         const int sl = g & 1;
