@@ -538,29 +538,29 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-      {
-        // the next item's prologue operands: their latency passes during the
-        // stores below
-        ItemSeq peek = seq;
-        const int nx = peek.next();
-        if (nx >= 0) {
-          load_pro(nx, pro);
-          if constexpr (V::MINMAX) {
-            // and its rows of the grid table into L2 (copied in its prologue)
-            const int qn = item_qt(nx) * KIA_TILE + r;
-            if (tab_in_smem && part == 0)
-              prefetch_l2(st.table + ((long long)item_bh(nx) * T + (qn < T ? qn : T - 1)) * (p.K + 1));
-          }
-        }
-      }
       // this warp's 32 rows x 16 columns of dQ, 8 columns per TMA store
       // through its staging block
       {
         float* stg = sStage + (warp - 2) * 256;
         const int row0 = qt * KIA_TILE + quad * 32;
-#pragma unroll
-        for (int pass = 0; pass < 2; ++pass)
-          epilogue_store8(stg, &tmdQ, o + 8 * pass, 1.0f, lane, (int)col + 8 * pass, row0, bh);
+        epilogue_store8(stg, &tmdQ, o, 1.0f, lane, (int)col, row0, bh);
+        {
+          // the next item's prologue operands: issued between the two
+          // stores (their latency passes during the second and the next
+          // item's start)
+          ItemSeq peek = seq;
+          const int nx = peek.next();
+          if (nx >= 0) {
+            load_pro(nx, pro);
+            if constexpr (V::MINMAX) {
+              // and its rows of the grid table into L2 (copied in its prologue)
+              const int qn = item_qt(nx) * KIA_TILE + r;
+              if (tab_in_smem && part == 0)
+                prefetch_l2(st.table + ((long long)item_bh(nx) * T + (qn < T ? qn : T - 1)) * (p.K + 1));
+            }
+          }
+        }
+        epilogue_store8(stg, &tmdQ, o + 8, 1.0f, lane, (int)col + 8, row0, bh);
       }
       if (q < T && part == 0) {
         wk.gm[rowbase + q] = gm;
