@@ -924,7 +924,11 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int Lq = p.causal ? q + 1 : T;
         const float rWb = Lq == 1 ? 0.0f : __fdiv_rn(1.0f, cur.Wb[hq]);
         const float nD = -cur.dl[hq] * rWb;       // dw = dP rWb + nD
-        const float nrh = V::SOFTMAX ? 1.0f : -cur.rh[hq];
+        // a degenerate MinMax row (1/h = 0) has dS = dw (uniform P): with its
+        // grid in shared memory that comes through the slope of a patched
+        // grid (below) and the factor 1 here, else through x.y, x.z
+        const bool fold = V::MINMAX && tab_in_smem && cur.rh[hq] == 0.0f;
+        const float nrh = (V::SOFTMAX || fold) ? 1.0f : -cur.rh[hq];
         sC4[e] = make_float4(cur.m[hq], rWb * nrh, nD * nrh, __fdiv_rn(1.0f, cur.Wf[hq]));
         // calibration terms of the query's row, added to dS^T before dK:
         // g_m at the argmax key, g_n at the argmin key, or the projection
@@ -932,8 +936,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const bool live = q < T;
         const float gm = live ? cur.gm[hq] : 0.0f, gn = live ? cur.gn[hq] : 0.0f;
         if constexpr (V::MINMAX || PROJ) {
-          // a degenerate MinMax row (1/h = 0) has dS = dw: uniform P
-          const float dg = (V::MINMAX && cur.rh[hq] == 0.0f) ? 1.0f : 0.0f;
+          const float dg = (V::MINMAX && !tab_in_smem && cur.rh[hq] == 0.0f) ? 1.0f : 0.0f;
           sX4[e] = make_float4(cur.rh[hq], dg * rWb, dg * nD, PROJ ? gm : 0.0f);
         }
         if constexpr (!PROJ && !V::SOFTMAX) {
@@ -956,6 +959,15 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       if (V::MINMAX && tab_in_smem) cp_async_wait_all();   // the unit's grids have landed
       __syncwarp();
+      if (V::MINMAX && tab_in_smem) {
+        // a degenerate row's grid gets G_1 = 2 in the slot: its scores all sit
+        // at node 0 (u = 0), so the slope G_1 - G_0 = 1 makes the score
+        // gradient dw; its weight G_0 = 1 is unchanged
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq)
+          if (cur.rh[hq] == 0.0f) sTab[(size_t)(sl * kSlotQ + 32 * hq + lane) * K1 + 1] = 2.0f;
+        __syncwarp();
+      }
       mbar_arrive(&bar.qc_ready[sl]);
       cur = nxt;
       it = it2;
@@ -1038,7 +1050,7 @@ tc_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const float wf = V::NEAREST ? (t >= 0.5f ? gp.y : gp.x) : __fmaf_rn(t, a, gp.x);
                 P = wf * cq.w;
                 dS = a * dSn;
-                if constexpr (V::MINMAX) dS = fmaf(dP, xq.y, dS + xq.z);   // degenerate rows: dw
+                if constexpr (V::MINMAX && !TABS) dS = fmaf(dP, xq.y, dS + xq.z);   // degenerate rows: dw
               }
               if constexpr (PROJ) dS += xq.w;
               v[i] = P;
