@@ -256,7 +256,9 @@ __device__ __forceinline__ Pos fwd_weights(const G& grid, float m, float rh, flo
 // normalisation Jacobian at the surrogate's point).  Returns the detached
 // dS; accumulates A += dw a_k and, when NEED_C, C += dw (b - a_k u / h) with
 // b = -(1-t) k G_k - t (k+1) G_{k+1}.  nrh = -rh; dg = 1 on degenerate rows.
-template <class V, bool NEED_C, class G>
+// FOLD: degenerate rows come with nrh = 1 and a grid whose first slope is 1
+// (the caller's copy patched to G_1 = 2), so dS = dw needs no dg term.
+template <class V, bool NEED_C, bool FOLD = false, class G>
 __device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, float nrh, float dg,
                                            float Kf, float Km1f, float s, float dw, float& A,
                                            float& C) {
@@ -281,7 +283,7 @@ __device__ __forceinline__ float bwd_delta(const G& grid, float m, float rh, flo
     A += da;
     float delta;
     if constexpr (V::MINMAX) {
-      delta = fmaf(dw, dg, da * nrh);
+      delta = FOLD ? da * nrh : fmaf(dw, dg, da * nrh);
       if constexpr (NEED_C) {
         const float kg0 = p.kf * g.x;
         const float bpos = fmaf(p.t, fmaf(p.kf + 1.0f, g.y, -kg0), kg0);  // -b

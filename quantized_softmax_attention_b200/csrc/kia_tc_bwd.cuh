@@ -381,8 +381,12 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float Wb = pro.Wb;
       const int qq = qt * KIA_TILE + rr;
       const long long qrr = rowbase + (qq < T ? qq : T - 1);
-      const float nrh = -rh;
-      const float dg = (V::MINMAX && rh == 0.0f) ? 1.0f : 0.0f;
+      // a degenerate MinMax row (1/h = 0) has dS = dw: with its grid in shared
+      // memory through the copy patched to G_1 = 2 (below) and the factor 1,
+      // else through dg
+      const bool fold = V::MINMAX && tab_in_smem && rh == 0.0f;
+      const float nrh = fold ? 1.0f : -rh;
+      const float dg = (V::MINMAX && !tab_in_smem && rh == 0.0f) ? 1.0f : 0.0f;
       const int L = p.causal ? q + 1 : T;
       // a one-key row has P = 1 whatever its score: zero gradient
       const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, Wb);
@@ -415,7 +419,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if constexpr (V::MINMAX) {
         if (tab_in_smem)
           for (int k = part; k <= p.K; k += kRowSplit)
-            sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
+            sTab[k * KIA_TILE + r] = (fold && k == 1) ? 2.0f : st.table[qr * (p.K + 1) + k];
       }
       mbar_arrive(&bar.row_sync);
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (2 * n) & 1, abort))) { failed = true; break; }
@@ -425,7 +429,8 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // the unit loop, instantiated per grid placement so that the grid
       // loads of the element loop are shared-memory loads when the grid is
       // in shared memory (a runtime choice of pointer makes them generic)
-      auto unit_loop = [&](const auto& grid) {
+      auto unit_loop = [&](const auto& grid, auto fold_c) {
+      constexpr bool FOLD = decltype(fold_c)::value;
       for (int u = 0; u < nunits && !failed; ++u) {
         const int j = u >> 1, gu = gbase + u, rg = gu % R;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar.sp_full[rg], (gu / R) & 1, abort))) { failed = true; break; }
@@ -442,7 +447,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float dw = fmaf(g[i], rWb, nDr);
-              v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+              v[i] = bwd_delta<V, NEED_C, FOLD>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
             }
           } else {
 #pragma unroll
@@ -450,7 +455,7 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               const int key = key0 + i;
               const bool ok = key < T && (!p.causal || key <= q);
               const float dw = ok ? fmaf(g[i], rWb, nDr) : 0.0f;
-              v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+              v[i] = bwd_delta<V, NEED_C, FOLD>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
             }
           }
           tmem_st16(tmem + lane_addr + cs, v);
@@ -467,12 +472,12 @@ tc_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       };
       if constexpr (V::MINMAX) {
-        if (tab_in_smem) unit_loop(GridF{sTab + r, KIA_TILE});
-        else unit_loop(GridF{st.table + qr * (p.K + 1), 1});
+        if (tab_in_smem) unit_loop(GridF{sTab + r, KIA_TILE}, std::true_type{});
+        else unit_loop(GridF{st.table + qr * (p.K + 1), 1}, std::false_type{});
       } else if constexpr (V::SOFTMAX) {
-        unit_loop(GridP{sPair});
+        unit_loop(GridP{sPair}, std::false_type{});
       } else {
-        unit_loop(make_gridz(sPair, p.K));
+        unit_loop(make_gridz(sPair, p.K), std::false_type{});
       }
       if (failed) break;
       gbase += nunits;
