@@ -343,8 +343,12 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       const float m = st.m[qr];
       const int am = st.am[qr], an = V::MINMAX ? st.an[qr] : am;
       const float rh = st.rh[qr];
-      const float nrh = -rh;
-      const float dg = (V::MINMAX && rh == 0.0f) ? 1.0f : 0.0f;
+      // a degenerate MinMax row (1/h = 0) has dS = dw: with its grid in shared
+      // memory through the copy patched to G_1 = 2 (below) and the factor 1,
+      // else through dg
+      const bool fold = V::MINMAX && tab_in_smem && rh == 0.0f;
+      const float nrh = fold ? 1.0f : -rh;
+      const float dg = (V::MINMAX && !tab_in_smem && rh == 0.0f) ? 1.0f : 0.0f;
       const int L = p.causal ? q + 1 : T;
       const float rWb = (L == 1) ? 0.0f : __fdiv_rn(1.0f, st.Wb[qr]);
       prefetch_l2(Kt + (rowbase + am) * D + part * 32);
@@ -378,14 +382,15 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         // the row's grid, column r of [K + 1][128] (four threads per row)
         if (tab_in_smem)
           for (int k = part; k <= p.K; k += kRowSplit)
-            sTab[k * KIA_TILE + r] = st.table[qr * (p.K + 1) + k];
+            sTab[k * KIA_TILE + r] = (fold && k == 1) ? 2.0f : st.table[qr * (p.K + 1) + k];
       }
       mbar_arrive(&bar.row_sync);
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.row_sync, (2 * n) & 1, abort))) { failed = true; break; }
       const float Dc = sDc[r];
       const float nDr = -Dc * rWb;
       float A = 0.0f, C = 0.0f;
-      auto unit_loop = [&](const auto& grid) {
+      auto unit_loop = [&](const auto& grid, auto fold_c) {
+        constexpr bool FOLD = decltype(fold_c)::value;
         for (int u = 0; u < nunits && !failed; ++u, ++g) {
           const bool edge = (p.causal && (u >> 1) == qt) || 64 * u + 64 > T;
 #pragma unroll 1
@@ -403,7 +408,7 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const float dw = fmaf(gg[i], rWb, nDr);
-                v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+                v[i] = bwd_delta<V, NEED_C, FOLD>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
               }
             } else {
 #pragma unroll
@@ -411,7 +416,7 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 const int key = key0 + i;
                 const bool ok = key < T && (!p.causal || key <= q);
                 const float dw = ok ? fmaf(gg[i], rWb, nDr) : 0.0f;
-                v[i] = bwd_delta<V, NEED_C>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
+                v[i] = bwd_delta<V, NEED_C, FOLD>(grid, m, rh, nrh, dg, Kf, Km1f, v[i], dw, A, C);
               }
             }
             tmem_st8(tmem + lane_addr + cS, v);
@@ -428,12 +433,12 @@ tc_bwd_q128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         }
       };
       if constexpr (V::MINMAX) {
-        if (tab_in_smem) unit_loop(GridF{sTab + r, KIA_TILE});
-        else unit_loop(GridF{st.table + qr * (p.K + 1), 1});
+        if (tab_in_smem) unit_loop(GridF{sTab + r, KIA_TILE}, std::true_type{});
+        else unit_loop(GridF{st.table + qr * (p.K + 1), 1}, std::false_type{});
       } else if constexpr (V::SOFTMAX) {
-        unit_loop(GridP{sPair});
+        unit_loop(GridP{sPair}, std::false_type{});
       } else {
-        unit_loop(make_gridz(sPair, p.K));
+        unit_loop(make_gridz(sPair, p.K), std::false_type{});
       }
       if (failed) break;
       sAC[(part * 2 + 0) * KIA_TILE + r] = A;
@@ -822,12 +827,16 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int Lq = p.causal ? q + 1 : T;
         const float rWb = Lq == 1 ? 0.0f : __fdiv_rn(1.0f, cur.Wb[hq]);
         const float nD = -cur.D[hq] * rWb;
-        const float nrh = V::SOFTMAX ? 1.0f : -cur.rh[hq];
+        // a degenerate MinMax row (1/h = 0) has dS = dw (uniform P): with the
+        // grids in shared memory through its slot copy patched to G_1 = 2 and
+        // the factor 1 here, else through x.y, x.z
+        const bool fold = tabs && cur.rh[hq] == 0.0f;
+        const float nrh = (V::SOFTMAX || fold) ? 1.0f : -cur.rh[hq];
         sC4[e] = make_float4(cur.m[hq], rWb * nrh, nD * nrh, __fdiv_rn(1.0f, cur.Wf[hq]));
         const bool live = q < T;
         const float gm = live ? cur.gm[hq] : 0.0f, gn = live ? cur.gn[hq] : 0.0f;
         if constexpr (V::MINMAX || PROJ) {
-          const float dg = (V::MINMAX && cur.rh[hq] == 0.0f) ? 1.0f : 0.0f;
+          const float dg = (V::MINMAX && !tabs && cur.rh[hq] == 0.0f) ? 1.0f : 0.0f;
           sX4[e] = make_float4(cur.rh[hq], dg * rWb, dg * nD, PROJ ? gm : 0.0f);
         }
         if constexpr (!PROJ && !V::SOFTMAX) {
@@ -870,6 +879,10 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             else dst[x] = 1.0f;
           }
           cp_async_wait_all();
+          __syncwarp();
+          // a degenerate row (this lane's query of the half) gets G_1 = 2:
+          // its scores all sit at node 0, the slope 1 carries dw
+          if (cur.rh[h] == 0.0f) dst[lane * K1 + 1] = 2.0f;
           __syncwarp();
           mbar_arrive(&bar.tab_ready[h]);
         }
@@ -969,7 +982,7 @@ tc_bwd_kv128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
               const float wf = V::NEAREST ? (t >= 0.5f ? gp.y : gp.x) : __fmaf_rn(t, a, gp.x);
               P = wf * cq.w;
               dS = a * dSn;
-              if constexpr (V::MINMAX) dS = fmaf(dP, xq.y, dS + xq.z);
+              if constexpr (V::MINMAX && !TABS) dS = fmaf(dP, xq.y, dS + xq.z);
             }
             if constexpr (PROJ) dS += xq.w;
             v[i] = P;
